@@ -1,0 +1,553 @@
+#!/usr/bin/env python3
+"""Benchmark of the SAS gated block-sparse attention hot path on B200.
+
+One step = one pass of the whole prefill/training path over the workload's inputs
+(already resident in HBM): key pooling -> gate keys -> gate scores -> Top-K -> gated
+attention forward -> gated attention backward. A decode step of the batch-64 decode
+workload is measured beside it and reported in the same line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl sas|reference]
+
+For N > 1 (torchrun, one rank per GPU) every rank runs its own replica of the workload
+(the path shards into independent problems; no collective touches the data), the
+timing is the max over ranks, and `value` counts the work of all ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import sas_inputs as si  # noqa: E402
+
+METRIC = "gated sparse attn TFLOP/s (attended, fwd/bwd) + decode tok/s; % of B200 roofline"
+TRAIN_WORKLOAD = "qwen3-4b-train-32k"
+DECODE_WORKLOAD = "qwen3-8b-decode-b64"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="sas", choices=["sas", "reference"])
+    ap.add_argument("--workload", default=TRAIN_WORKLOAD)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=6, help="oracle rows per CPU-baseline sample")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------------------------------
+# distributed plumbing
+# ------------------------------------------------------------------------------------------
+
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                              device_id=torch.device("cuda", local))
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, ws: int, dev) -> float:
+    if ws == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ------------------------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return None
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        hi = max(sm)
+        loaded = [x for x in sm if x >= 0.5 * hi] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------------
+# helpers
+# ------------------------------------------------------------------------------------------
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained", d["bf16_tflops"]), \
+            "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def source_sha(files) -> str:
+    h = hashlib.sha256()
+    for f in files:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(op: str):
+    """dram bytes per launch of `op` from the committed ncu summary, if its sources match."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(op)
+    if not d:
+        return None
+    try:
+        if source_sha(d["sources"]) != d["source_sha"]:
+            return None
+    except OSError:
+        return None
+    return d["bytes_per_launch"]
+
+
+def attended_pairs_gpu(idx: torch.Tensor, cu: torch.Tensor, block: int) -> int:
+    """(token, kv, key) pairs with a finite logit, counted on the device from the selection."""
+    T = idx.shape[0]
+    cu64 = cu.long()
+    tok = torch.arange(T, device=idx.device)
+    seq = torch.searchsorted(cu64[1:], tok, right=True)
+    pos = tok - cu64[seq]
+    j = idx.long()
+    lo = j * block
+    hi = torch.minimum((j + 1) * block, pos[:, None, None] + 1)
+    n = torch.where(j >= 0, (hi - lo).clamp(min=0), torch.zeros_like(j))
+    return int(n.sum().item())
+
+
+class Timer:
+    """CUDA events around each op of a step, on the stream the library launches on."""
+
+    def __init__(self):
+        self.ops = {}
+
+    def run(self, name, fn):
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        r = fn()
+        e.record()
+        self.ops.setdefault(name, []).append((s, e))
+        return r
+
+    def mean_ms(self):
+        return {k: sum(a.elapsed_time(b) for a, b in v) / len(v) for k, v in self.ops.items()}
+
+
+# ------------------------------------------------------------------------------------------
+# the prefill / training step
+# ------------------------------------------------------------------------------------------
+
+def train_step(sas, prob, g, backward: bool, timer: Timer | None = None):
+    run = timer.run if timer is not None else (lambda name, fn: fn())
+    pooled = run("sas_pool_keys", lambda: sas.sas_pool_keys(prob, g["k_nope"], pooled=g["_pooled"]))
+    gk = run("sas_gate_keys", lambda: sas.sas_gate_keys(prob, pooled, g["wk"], g["knorm_w"],
+                                                        gate_keys=g["_gk"]))
+    scores, lse = run("sas_gate_scores", lambda: sas.sas_gate_scores(
+        prob, g["q_nope"], g["k_nope"], gk, g["wq"], g["qnorm_w"], g["wk"], g["knorm_w"],
+        scores=g["_scores"], lse=g["_glse"]))
+    idx, logg = run("sas_topk", lambda: sas.sas_topk(prob, scores, lse, idx=g["_idx"],
+                                                     logg=g["_logg"]))
+    o, alse = run("sas_attn_fwd", lambda: sas.sas_attn_fwd(prob, g["q"], g["k"], g["v"], idx, logg,
+                                                           o=g["_o"], lse=g["_alse"],
+                                                           workspace=g["_wsf"]))
+    out = [o, alse, idx, logg]
+    if backward:
+        grads = run("sas_attn_bwd", lambda: sas.sas_attn_bwd(
+            prob, g["q"], g["k"], g["v"], o, g["dout"], alse, idx, logg, dq=g["_dq"], dk=g["_dk"],
+            dv=g["_dv"], dlogg=g["_dlogg"], workspace=g["_wsb"]))
+        out += list(grads)
+    return out
+
+
+def alloc_outputs(sas, prob, g, backward):
+    import ctypes
+    dev = prob.device
+    T, Hq, Hkv, d, K, NB, h = (prob.total_tokens, prob.num_q_heads, prob.num_kv_heads,
+                               prob.head_dim, prob.topk, prob.max_blocks, prob.gate_hidden)
+    g["_pooled"] = torch.empty((prob.batch, NB, Hkv, 3 * d), dtype=torch.float32, device=dev)
+    g["_gk"] = torch.empty((prob.batch, NB, Hkv, h), dtype=torch.float32, device=dev)
+    g["_scores"] = torch.empty((T, Hkv, NB), dtype=torch.float32, device=dev)
+    g["_glse"] = torch.empty((T, Hkv), dtype=torch.float32, device=dev)
+    g["_idx"] = torch.empty((T, Hkv, K + 1), dtype=torch.int32, device=dev)
+    g["_logg"] = torch.empty((T, Hkv, K + 1), dtype=torch.float32, device=dev)
+    g["_o"] = torch.empty((T, Hq, d), dtype=prob.dtype, device=dev)
+    g["_alse"] = torch.empty((T, Hq), dtype=torch.float32, device=dev)
+    lib = sas.lib_handle()
+    n = ctypes.c_size_t(0)
+    lib.sas_attn_fwd_workspace_size(prob.ref, ctypes.byref(n))
+    g["_wsf"] = torch.empty(max(256, n.value), dtype=torch.uint8, device=dev)
+    if backward:
+        g["_dq"] = torch.empty_like(g["q"])
+        g["_dk"] = torch.empty_like(g["k"])
+        g["_dv"] = torch.empty_like(g["v"])
+        g["_dlogg"] = torch.empty((T, Hkv, K + 1), dtype=torch.float32, device=dev)
+        lib.sas_attn_bwd_workspace_size(prob.ref, ctypes.byref(n))
+        g["_wsb"] = torch.empty(max(256, n.value), dtype=torch.uint8, device=dev)
+
+
+# ------------------------------------------------------------------------------------------
+# oracle sample (CPU baseline and the reference arm)
+# ------------------------------------------------------------------------------------------
+
+def oracle_sample(cpu_inp, shape, rows, backward):
+    """Oracle gate + Top-K + attention (fwd, and bwd rows) on some query rows; returns the
+    attended FLOPs those rows represent (fwd 4*pairs*d per head, row-bwd 6*pairs*d per head:
+    recompute, dP, dQ)."""
+    from oracle import sas_oracle as orc
+    B, K, d, G = shape.block, shape.topk, shape.head_dim, shape.group
+    sel = orc.prefill_selection(cpu_inp["q_nope"], cpu_inp["k_nope"], cpu_inp["wq"],
+                                cpu_inp["qnorm_w"], cpu_inp["wk"], cpu_inp["knorm_w"],
+                                shape.cu_seqlens, B, K, shape.rms_eps, shape.gate_rope_base, rows)
+    idx = np.full((shape.total_tokens, shape.num_kv_heads, K + 1), -1, dtype=np.int32)
+    logg = np.zeros(idx.shape)
+    idx[rows], logg[rows] = sel["idx"], sel["logg"]
+    orc.attention_fwd(cpu_inp["q"], cpu_inp["k"], cpu_inp["v"], idx, logg, shape.cu_seqlens, B,
+                      rows=rows)
+    if backward:
+        orc.attention_bwd_rows(cpu_inp["q"], cpu_inp["k"], cpu_inp["v"], cpu_inp["dout"], idx, logg,
+                               shape.cu_seqlens, B, rows)
+    pos = shape.positions()[rows]
+    j = sel["idx"].astype(np.int64)
+    lo = j * B
+    hi = np.minimum((j + 1) * B, pos[:, None, None] + 1)
+    pairs = int(np.where(j >= 0, np.maximum(hi - lo, 0), 0).sum())
+    return pairs * G * d * (4 + (6 if backward else 0))
+
+
+def cpu_inputs_from(g):
+    keys = ("q_nope", "k_nope", "q", "k", "v", "dout", "wq", "wk", "qnorm_w", "knorm_w")
+    return {k: g[k].float().cpu().numpy().astype(np.float64) for k in keys if k in g}
+
+
+def sample_rows(shape, n, seed):
+    r = np.random.Generator(np.random.PCG64(seed))
+    return np.sort(r.choice(shape.total_tokens, size=n, replace=False))
+
+
+# ------------------------------------------------------------------------------------------
+# decode
+# ------------------------------------------------------------------------------------------
+
+def bench_decode(sas, dev, steps, warmup, flush, hbm_peak):
+    shp = si.decode_workload(DECODE_WORKLOAD)
+    inp = si.decode_inputs(shp, device=dev)
+    prob = sas.DecodeProblem(seqlens=inp["lengths"], capacity=shp.capacity,
+                             num_q_heads=shp.num_q_heads, num_kv_heads=shp.num_kv_heads,
+                             head_dim=shp.head_dim, block=shp.block, topk=shp.topk,
+                             gate_hidden=shp.gate_hidden, dtype=torch.bfloat16)
+    import ctypes
+    n = ctypes.c_size_t(0)
+    sas.lib_handle().sas_decode_workspace_size(prob.ref, ctypes.byref(n))
+    ws = torch.empty(max(256, n.value), dtype=torch.uint8, device=dev)
+    o = torch.empty((shp.batch, shp.num_q_heads, shp.head_dim), dtype=torch.bfloat16, device=dev)
+    idx = torch.empty((shp.batch, shp.num_kv_heads, shp.topk + 1), dtype=torch.int32, device=dev)
+    logg = torch.empty(idx.shape, dtype=torch.float32, device=dev)
+
+    def step():
+        return sas.sas_decode(prob, inp["q"], inp["q_nope"], inp["k_cache"], inp["v_cache"],
+                              inp["gate_key_cache"], inp["cur_pool"], inp["wq"], inp["qnorm_w"],
+                              inp["wk"], inp["knorm_w"], o=o, idx_out=idx, logg_out=logg,
+                              workspace=ws)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(steps):
+        flush.zero_()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        step()
+        e.record()
+        ts.append((s, e))
+    torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in ts) / len(ts)
+    # algorithmic bytes: the selected K/V rows, every cached gate key of the complete blocks,
+    # q, q_nope, pool state, gate weights, O
+    L = inp["lengths"].long()
+    B = shp.block
+    j = idx.long()
+    pos = (L - 1)[:, None, None]
+    keys = torch.where(j >= 0, (torch.minimum((j + 1) * B, pos + 1) - j * B).clamp(min=0),
+                       torch.zeros_like(j)).sum().item()
+    kv_bytes = keys * shp.head_dim * 2 * 2
+    c = ((L - 1) // B)
+    gk_bytes = int(c.sum().item()) * shp.num_kv_heads * shp.gate_hidden * 2
+    other = (2 * shp.batch * shp.num_q_heads * shp.head_dim * 2 + shp.batch * shp.num_kv_heads * 3
+             * shp.head_dim * 4 + inp["wq"].numel() * 2 + inp["wk"].numel() * 2
+             + shp.batch * shp.num_q_heads * shp.head_dim * 2)
+    total = kv_bytes + gk_bytes + other
+    gbs = total / (ms * 1e-3) / 1e9
+    return {
+        "metric": "decode tok/s", "value": shp.batch / (ms * 1e-3), "unit": "tok/s",
+        "ms_per_step": ms, "config": {"workload": DECODE_WORKLOAD, "batch": shp.batch,
+                                      "context_min": int(L.min()), "context_max": int(L.max()),
+                                      "budget_tokens": (shp.topk + 1) * B},
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": gbs / hbm_peak, "traffic": ncu_traffic("sas_decode"),
+                     "algorithmic_bytes": total, "selected_kv_bytes": kv_bytes,
+                     "gate_key_bytes": gk_bytes, "peak_source": "measured copy, of measured"},
+        "selected_kv_gbs": kv_bytes / (ms * 1e-3) / 1e9,
+    }
+
+
+# ------------------------------------------------------------------------------------------
+# main
+# ------------------------------------------------------------------------------------------
+
+def main():
+    a = parse()
+    ws, rank, local = dist_setup()
+    if a.impl == "reference":
+        return reference_arm(a, ws, rank)
+    import gated_block_sparse_sas_b200 as sas
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    hbm_peak, tc_peak, tc_sust, peak_src = measured_peaks()
+
+    shape = si.workload(a.workload)
+    backward = "train" in a.workload or "varlen" in a.workload
+    g = si.prefill_inputs(shape, device=dev, with_dout=backward)
+    prob = sas.Problem.from_lengths(shape.lengths, dev, num_q_heads=shape.num_q_heads,
+                                    num_kv_heads=shape.num_kv_heads, head_dim=shape.head_dim,
+                                    block=shape.block, topk=shape.topk,
+                                    gate_hidden=shape.gate_hidden, dtype=shape.torch_dtype)
+    alloc_outputs(sas, prob, g, backward)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    for _ in range(max(3, a.warmup)):
+        out = train_step(sas, prob, g, backward)
+    torch.cuda.synchronize()
+    pairs = attended_pairs_gpu(out[2], prob.cu_seqlens, shape.block)
+    G, d = shape.group, shape.head_dim
+    fwd_flops = 4.0 * pairs * G * d
+    bwd_flops = 2.5 * fwd_flops if backward else 0.0
+
+    timer = Timer()
+    steps = []
+    barrier(ws)
+    torch.cuda.synchronize()
+    n0 = sas.kernel_launches()
+    with ClockSampler(dev.index) as clk:
+        for _ in range(a.steps):
+            flush.zero_()
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record()
+            train_step(sas, prob, g, backward, timer)
+            e.record()
+            steps.append((s, e))
+        torch.cuda.synchronize()
+    barrier(ws)
+    launches = sas.kernel_launches() - n0
+    ms = sum(x.elapsed_time(y) for x, y in steps) / len(steps)
+    ms = max_over_ranks(ms, ws, dev)
+    ops = timer.mean_ms()
+    work = fwd_flops + bwd_flops
+    value = work * ws / (ms * 1e-3) / 1e12
+
+    # dominant kernel roofline (tensor-bound attention; peak: sustained, timed inside a long step)
+    dom = max(("sas_attn_fwd", "sas_attn_bwd") if backward else ("sas_attn_fwd",),
+              key=lambda k: ops[k])
+    dflops = fwd_flops if dom == "sas_attn_fwd" else bwd_flops
+    ach = dflops / (ops[dom] * 1e-3) / 1e12
+    roof = {"bound": "tensor", "kernel": dom, "achieved": ach, "peak": tc_sust, "unit": "TFLOP/s",
+            "frac": ach / tc_sust, "traffic": ncu_traffic(dom),
+            "peak_source": f"bf16 dense sustained, of {peak_src}",
+            "algorithmic_flops_per_launch": dflops}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws, "steps": a.steps,
+        "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if shape.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded counter-based generator, approx. N(0,1))",
+        "config": {"workload": a.workload, "batch": shape.batch, "seq_len": shape.max_seqlen,
+                   "num_q_heads": shape.num_q_heads, "num_kv_heads": shape.num_kv_heads,
+                   "head_dim": d, "block": shape.block, "topk": shape.topk,
+                   "gate_hidden": shape.gate_hidden, "passes": "fwd+bwd" if backward else "fwd",
+                   "parallelism": f"replicas x{ws}", "l2": "flushed (256 MiB write) between steps"},
+        "attended": {"pairs_per_kv_head_total": pairs, "fwd_tflop": fwd_flops / 1e12,
+                     "bwd_tflop": bwd_flops / 1e12,
+                     "dense_causal_fraction": pairs / (shape.num_kv_heads * sum(
+                         L * (L + 1) / 2 for L in shape.lengths))},
+        "ops_ms": ops,
+        "roofline": roof,
+        "gpu_launches": launches,
+    }
+    cs = clk.summary()
+    if cs:
+        line["clocks"] = cs
+
+    if not a.no_decode:
+        try:
+            line["decode"] = bench_decode(sas, dev, max(3, a.steps), max(3, a.warmup), flush, hbm_peak)
+        except torch.OutOfMemoryError as ex:   # pragma: no cover
+            line["decode"] = {"error": f"out of memory: {ex}"[:200]}
+
+    if not a.no_e2e:
+        line["e2e"] = e2e(sas, prob, g, backward, work, dev, a, ws)
+
+    if rank == 0 and ws == 1 and not a.no_cpu_baseline:
+        cpu = cpu_inputs_from(g)
+        rows = sample_rows(shape, a.cpu_rows, 7)
+        threads = torch.get_num_threads()
+        t0 = time.perf_counter()
+        fl = oracle_sample(cpu, shape, rows, backward)
+        dt = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads,
+                                "kind": "oracle", "seconds": dt,
+                                "sample": f"{len(rows)} random query rows of {a.workload} "
+                                          "(gate, Top-K, attention fwd" +
+                                          (" + dQ/dlogg rows" if backward else "") +
+                                          ") at full sequence length, fp64 numpy"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        torch.distributed.destroy_process_group()
+
+
+def e2e(sas, prob, g, backward, work, dev, a, ws):
+    """Same step through the public API with host buffers: pinned H2D of every input, the
+    step, D2H of every result; timed on the device stream."""
+    names = ["q_nope", "k_nope", "q", "k", "v", "wq", "wk", "qnorm_w", "knorm_w"] + \
+        (["dout"] if backward else [])
+    host = {k: g[k].cpu().pin_memory() for k in names}
+    dg = dict(g)
+    outs_host = None
+    steps = max(2, min(a.steps, 3))
+    ts = []
+    for it in range(steps + 1):
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for k in names:
+            dg[k].copy_(host[k], non_blocking=True)
+        out = train_step(sas, prob, dg, backward)
+        res = [out[0], out[1]] + (out[4:] if backward else [])
+        if outs_host is None:
+            outs_host = [torch.empty(r.shape, dtype=r.dtype, pin_memory=True) for r in res]
+        for hdst, r in zip(outs_host, res):
+            hdst.copy_(r, non_blocking=True)
+        e.record()
+        if it > 0:
+            ts.append((s, e))
+    torch.cuda.synchronize()
+    ms = sum(x.elapsed_time(y) for x, y in ts) / len(ts)
+    ms = max_over_ranks(ms, ws, dev)
+    h2d = sum(host[k].numel() * host[k].element_size() for k in names)
+    d2h = sum(o.numel() * o.element_size() for o in outs_host)
+    return {"value": work * ws / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def reference_arm(a, ws, rank):
+    """The oracle, as it stands, on the machine's host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    shape = si.workload(a.workload)
+    backward = "train" in a.workload or "varlen" in a.workload
+    inp = si.prefill_inputs(shape, device="cpu", with_dout=backward)
+    cpu = {k: v.float().numpy().astype(np.float64) for k, v in inp.items() if k != "cu_seqlens"}
+    for i in range(a.warmup):
+        oracle_sample(cpu, shape, sample_rows(shape, 1, 100 + i), backward)
+    t = []
+    fl = 0.0
+    for i in range(a.steps):
+        rows = sample_rows(shape, 2, 1000 + i)
+        t0 = time.perf_counter()
+        fl += oracle_sample(cpu, shape, rows, backward)
+        t.append(time.perf_counter() - t0)
+    tot = sum(t)
+    val = fl / tot / 1e12
+    threads = torch.get_num_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": ws,
+            "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * tot / a.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded counter-based generator, approx. N(0,1))",
+            "config": {"workload": a.workload, "batch": shape.batch, "seq_len": shape.max_seqlen,
+                       "passes": "fwd+bwd" if backward else "fwd", "parallelism": "cpu oracle"},
+            "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                             "sample": f"2 random query rows per step of {a.workload} (gate, "
+                                       "Top-K, attention fwd + dQ/dlogg rows), fp64 numpy"},
+            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

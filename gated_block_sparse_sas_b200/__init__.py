@@ -1,0 +1,309 @@
+"""Python binding of libsas_b200.so -- SAS gated block-sparse attention on B200 (sm_100a).
+
+Argument marshalling only: every step runs in the library's CUDA kernels; PyTorch
+provides device memory and the current stream. The entry points carry the C names
+(see include/sas.h for the operator, layouts and error behaviour). There is no CPU
+path: without the compiled library, importing this package fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsas_b200.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with "
+                      "`python -m gated_block_sparse_sas_b200.build` (nvcc, sm_100a)")
+_lib = ctypes.CDLL(LIB_PATH)
+
+SAS_OK, SAS_ERR_INVALID_ARG, SAS_ERR_UNSUPPORTED, SAS_ERR_CUDA, SAS_ERR_WORKSPACE = 0, -1, -2, -3, -4
+SAS_BF16, SAS_FP32 = 0, 1
+_vp, _i32, _f32, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+
+
+class SasProblem(ctypes.Structure):
+    _fields_ = [("batch", _i32), ("total_tokens", _i32), ("max_seqlen", _i32),
+                ("num_q_heads", _i32), ("num_kv_heads", _i32), ("head_dim", _i32),
+                ("block", _i32), ("topk", _i32), ("gate_hidden", _i32), ("rms_eps", _f32),
+                ("dtype", ctypes.c_int), ("cu_seqlens", _vp), ("gate_rope_cos", _vp),
+                ("gate_rope_sin", _vp)]
+
+
+class SasDecodeProblem(ctypes.Structure):
+    _fields_ = [("batch", _i32), ("capacity", _i32), ("num_q_heads", _i32),
+                ("num_kv_heads", _i32), ("head_dim", _i32), ("block", _i32), ("topk", _i32),
+                ("gate_hidden", _i32), ("rms_eps", _f32), ("dtype", ctypes.c_int),
+                ("seqlens", _vp), ("gate_rope_cos", _vp), ("gate_rope_sin", _vp)]
+
+
+_P = ctypes.POINTER(SasProblem)
+_DP = ctypes.POINTER(SasDecodeProblem)
+_SIGS = {
+    "sas_last_error": ([], ctypes.c_char_p),
+    "sas_kernel_launches": ([], ctypes.c_uint64),
+    "sas_rope_tables": ([_i32, _i32, ctypes.c_double, _vp, _vp], ctypes.c_int),
+    "sas_pool_keys": ([_P, _vp, _vp, _vp], ctypes.c_int),
+    "sas_gate_keys": ([_P, _vp, _vp, _vp, _vp, _vp], ctypes.c_int),
+    "sas_gate_scores": ([_P] + [_vp] * 10, ctypes.c_int),
+    "sas_topk": ([_P, _vp, _vp, _vp, _vp, _vp], ctypes.c_int),
+    "sas_attn_fwd_workspace_size": ([_P, ctypes.POINTER(_sz)], ctypes.c_int),
+    "sas_attn_fwd": ([_P] + [_vp] * 8 + [_sz, _vp], ctypes.c_int),
+    "sas_attn_bwd_workspace_size": ([_P, ctypes.POINTER(_sz)], ctypes.c_int),
+    "sas_attn_bwd": ([_P] + [_vp] * 13 + [_sz, _vp], ctypes.c_int),
+    "sas_decode_workspace_size": ([_DP, ctypes.POINTER(_sz)], ctypes.c_int),
+    "sas_decode": ([_DP] + [_vp] * 14 + [_sz, _vp], ctypes.c_int),
+}
+for _name, (_args, _res) in _SIGS.items():
+    _fn = getattr(_lib, _name)
+    _fn.argtypes = _args
+    _fn.restype = _res
+
+
+class SasError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: status {status}: {_lib.sas_last_error().decode()}")
+
+
+def _check(status: int, where: str):
+    if status != SAS_OK:
+        raise SasError(status, where)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("expected a torch.Tensor")
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to the library must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def rope_tables(positions: int, rot_dim: int, base: float = 1e6):
+    """Host fp32 cos/sin tables [positions, rot_dim/2] built by the library in double."""
+    c = np.empty((positions, rot_dim // 2), dtype=np.float32)
+    s = np.empty_like(c)
+    _check(_lib.sas_rope_tables(positions, rot_dim, base, c.ctypes.data, s.ctypes.data),
+           "sas_rope_tables")
+    return c, s
+
+
+def _dtype_code(dt) -> int:
+    if dt == torch.bfloat16:
+        return SAS_BF16
+    if dt == torch.float32:
+        return SAS_FP32
+    raise ValueError(f"unsupported dtype {dt}")
+
+
+@dataclasses.dataclass
+class Problem:
+    """A packed prefill/training problem plus the device buffers it points at."""
+    cu_seqlens: torch.Tensor        # int32 [batch+1], device
+    max_seqlen: int
+    total_tokens: int
+    num_q_heads: int
+    num_kv_heads: int
+    head_dim: int
+    block: int
+    topk: int
+    gate_hidden: int
+    dtype: torch.dtype
+    rms_eps: float = 1e-6
+    gate_rope_base: float = 1e6
+    rope_cos: torch.Tensor | None = None
+    rope_sin: torch.Tensor | None = None
+
+    def __post_init__(self):
+        if self.rope_cos is None:
+            c, s = rope_tables(self.max_seqlen, self.gate_hidden, self.gate_rope_base)
+            dev = self.cu_seqlens.device
+            self.rope_cos = torch.from_numpy(c).to(dev)
+            self.rope_sin = torch.from_numpy(s).to(dev)
+        self._c = SasProblem(len(self.cu_seqlens) - 1, self.total_tokens, self.max_seqlen,
+                             self.num_q_heads, self.num_kv_heads, self.head_dim, self.block,
+                             self.topk, self.gate_hidden, self.rms_eps, _dtype_code(self.dtype),
+                             _ptr(self.cu_seqlens), _ptr(self.rope_cos), _ptr(self.rope_sin))
+
+    @property
+    def batch(self) -> int:
+        return len(self.cu_seqlens) - 1
+
+    @property
+    def max_blocks(self) -> int:
+        return (self.max_seqlen + self.block - 1) // self.block
+
+    @property
+    def device(self):
+        return self.cu_seqlens.device
+
+    @property
+    def ref(self):
+        return ctypes.byref(self._c)
+
+    @classmethod
+    def from_lengths(cls, lengths, device, **kw):
+        cu = torch.tensor(np.concatenate([[0], np.cumsum(lengths)]), dtype=torch.int32,
+                          device=device)
+        return cls(cu_seqlens=cu, max_seqlen=int(max(lengths)), total_tokens=int(sum(lengths)), **kw)
+
+
+def sas_pool_keys(p: Problem, k_nope, pooled=None, stream=None):
+    if pooled is None:
+        pooled = torch.empty((p.batch, p.max_blocks, p.num_kv_heads, 3 * p.head_dim),
+                             dtype=torch.float32, device=p.device)
+    _check(_lib.sas_pool_keys(p.ref, _ptr(k_nope), _ptr(pooled), _stream(stream)), "sas_pool_keys")
+    return pooled
+
+
+def sas_gate_keys(p: Problem, pooled, wk, knorm_w, gate_keys=None, stream=None):
+    if gate_keys is None:
+        gate_keys = torch.empty((p.batch, p.max_blocks, p.num_kv_heads, p.gate_hidden),
+                                dtype=torch.float32, device=p.device)
+    _check(_lib.sas_gate_keys(p.ref, _ptr(pooled), _ptr(wk), _ptr(knorm_w), _ptr(gate_keys),
+                              _stream(stream)), "sas_gate_keys")
+    return gate_keys
+
+
+def sas_gate_scores(p: Problem, q_nope, k_nope, gate_keys, wq, qnorm_w, wk, knorm_w,
+                    scores=None, lse=None, stream=None):
+    if scores is None:
+        scores = torch.empty((p.total_tokens, p.num_kv_heads, p.max_blocks), dtype=torch.float32,
+                             device=p.device)
+    if lse is None:
+        lse = torch.empty((p.total_tokens, p.num_kv_heads), dtype=torch.float32, device=p.device)
+    _check(_lib.sas_gate_scores(p.ref, _ptr(q_nope), _ptr(k_nope), _ptr(gate_keys), _ptr(wq),
+                                _ptr(qnorm_w), _ptr(wk), _ptr(knorm_w), _ptr(scores), _ptr(lse),
+                                _stream(stream)), "sas_gate_scores")
+    return scores, lse
+
+
+def sas_topk(p: Problem, scores, lse, idx=None, logg=None, stream=None):
+    shape = (p.total_tokens, p.num_kv_heads, p.topk + 1)
+    if idx is None:
+        idx = torch.empty(shape, dtype=torch.int32, device=p.device)
+    if logg is None:
+        logg = torch.empty(shape, dtype=torch.float32, device=p.device)
+    _check(_lib.sas_topk(p.ref, _ptr(scores), _ptr(lse), _ptr(idx), _ptr(logg), _stream(stream)),
+           "sas_topk")
+    return idx, logg
+
+
+def _workspace(fn, prob_ref, device):
+    """A fresh workspace of the size the library asks for (torch's stream-ordered allocator)."""
+    n = _sz(0)
+    _check(fn(prob_ref, ctypes.byref(n)), fn.__name__)
+    return torch.empty(max(int(n.value), 256), dtype=torch.uint8, device=device)
+
+
+def sas_attn_fwd(p: Problem, q, k, v, idx, logg, o=None, lse=None, workspace=None, stream=None):
+    if o is None:
+        o = torch.empty((p.total_tokens, p.num_q_heads, p.head_dim), dtype=p.dtype, device=p.device)
+    if lse is None:
+        lse = torch.empty((p.total_tokens, p.num_q_heads), dtype=torch.float32, device=p.device)
+    ws = workspace if workspace is not None else _workspace(_lib.sas_attn_fwd_workspace_size, p.ref, p.device)
+    _check(_lib.sas_attn_fwd(p.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(logg), _ptr(o),
+                             _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)), "sas_attn_fwd")
+    return o, lse
+
+
+def sas_attn_bwd(p: Problem, q, k, v, o, dout, lse, idx, logg, dq=None, dk=None, dv=None,
+                 dlogg=None, workspace=None, stream=None):
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if dlogg is None:
+        dlogg = torch.empty((p.total_tokens, p.num_kv_heads, p.topk + 1), dtype=torch.float32,
+                            device=p.device)
+    ws = workspace if workspace is not None else _workspace(_lib.sas_attn_bwd_workspace_size, p.ref, p.device)
+    _check(_lib.sas_attn_bwd(p.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
+                             _ptr(idx), _ptr(logg), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dlogg),
+                             _ptr(ws), ws.numel(), _stream(stream)), "sas_attn_bwd")
+    return dq, dk, dv, dlogg
+
+
+def prefill_selection(p: Problem, q_nope, k_nope, wq, qnorm_w, wk, knorm_w, stream=None):
+    """A1..A4 in order: pool -> gate keys -> scores -> Top-K. Returns (idx, logg)."""
+    pooled = sas_pool_keys(p, k_nope, stream=stream)
+    gk = sas_gate_keys(p, pooled, wk, knorm_w, stream=stream)
+    scores, lse = sas_gate_scores(p, q_nope, k_nope, gk, wq, qnorm_w, wk, knorm_w, stream=stream)
+    return sas_topk(p, scores, lse, stream=stream)
+
+
+@dataclasses.dataclass
+class DecodeProblem:
+    seqlens: torch.Tensor           # int32 [batch], device
+    capacity: int
+    num_q_heads: int
+    num_kv_heads: int
+    head_dim: int
+    block: int
+    topk: int
+    gate_hidden: int
+    dtype: torch.dtype
+    rms_eps: float = 1e-6
+    gate_rope_base: float = 1e6
+    rope_cos: torch.Tensor | None = None
+    rope_sin: torch.Tensor | None = None
+
+    def __post_init__(self):
+        if self.rope_cos is None:
+            c, s = rope_tables(self.capacity, self.gate_hidden, self.gate_rope_base)
+            dev = self.seqlens.device
+            self.rope_cos = torch.from_numpy(c).to(dev)
+            self.rope_sin = torch.from_numpy(s).to(dev)
+        self._c = SasDecodeProblem(len(self.seqlens), self.capacity, self.num_q_heads,
+                                   self.num_kv_heads, self.head_dim, self.block, self.topk,
+                                   self.gate_hidden, self.rms_eps, _dtype_code(self.dtype),
+                                   _ptr(self.seqlens), _ptr(self.rope_cos), _ptr(self.rope_sin))
+
+    @property
+    def batch(self) -> int:
+        return len(self.seqlens)
+
+    @property
+    def device(self):
+        return self.seqlens.device
+
+    @property
+    def ref(self):
+        return ctypes.byref(self._c)
+
+
+def sas_decode(p: DecodeProblem, q, q_nope, k_cache, v_cache, gate_key_cache, cur_pool, wq,
+               qnorm_w, wk, knorm_w, o=None, idx_out=None, logg_out=None, workspace=None,
+               stream=None, want_selection: bool = False):
+    if o is None:
+        o = torch.empty((p.batch, p.num_q_heads, p.head_dim), dtype=p.dtype, device=p.device)
+    if want_selection and idx_out is None:
+        idx_out = torch.empty((p.batch, p.num_kv_heads, p.topk + 1), dtype=torch.int32,
+                              device=p.device)
+        logg_out = torch.empty((p.batch, p.num_kv_heads, p.topk + 1), dtype=torch.float32,
+                               device=p.device)
+    ws = workspace if workspace is not None else _workspace(_lib.sas_decode_workspace_size, p.ref, p.device)
+    _check(_lib.sas_decode(p.ref, _ptr(q), _ptr(q_nope), _ptr(k_cache), _ptr(v_cache),
+                           _ptr(gate_key_cache), _ptr(cur_pool), _ptr(wq), _ptr(qnorm_w), _ptr(wk),
+                           _ptr(knorm_w), _ptr(o), _ptr(idx_out), _ptr(logg_out), _ptr(ws),
+                           ws.numel(), _stream(stream)), "sas_decode")
+    return (o, idx_out, logg_out) if want_selection else o
+
+
+def lib_handle():
+    return _lib
+
+
+def kernel_launches() -> int:
+    """Kernels the library has launched from this thread so far."""
+    return int(_lib.sas_kernel_launches())

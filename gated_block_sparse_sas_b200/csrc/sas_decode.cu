@@ -1,0 +1,462 @@
+// Sparse decode step (A7). Model card "tencent/Simple-Attention-Sparsification": the
+// released setup decodes with a 2,048-token budget (1,024 / 4,096 also usable), i.e.
+// Top-K historical blocks plus the current block; Chinese guide, caveat 3: the budget
+// caps the tokens each query attends to, not the KV cache.
+//
+// Three launches: (1) gate + Top-K per (sequence, kv head) -> selection in workspace;
+// (2) split-K gated attention over the selected blocks -> per-split (m, l, acc);
+// (3) merge of the splits -> O. The attention only ever reads the selected blocks.
+#include <math.h>
+
+#include "sas_common.cuh"
+#include "sas_kernels.h"
+
+namespace sas {
+
+constexpr int kDecThreads = 256;
+constexpr int kDecWarps = kDecThreads / 32;
+
+__device__ __forceinline__ float block_reduce_sum(float v, float* red) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  v = warp_sum(v);
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float r = 0.f;
+  for (int w = 0; w < kDecWarps; ++w) r += red[w];
+  return r;
+}
+
+__device__ __forceinline__ float block_reduce_max(float v, float* red) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  v = warp_max(v);
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float r = -INFINITY;
+  for (int w = 0; w < kDecWarps; ++w) r = fmaxf(r, red[w]);
+  return r;
+}
+
+// ---------------------------------------------------------------------------------------
+// (1) gate: q~ (Qproj over the G concatenated pre-rotary heads, RMSNorm, rotary at L-1),
+// current-block key from the running pool state (max, min, sum/n; Kproj, RMSNorm, rotary
+// at c*B), scores against the cached block keys, logsumexp over j <= c, Top-K over j < c.
+// ---------------------------------------------------------------------------------------
+template <typename T, int H, int NPT>
+__global__ void __launch_bounds__(kDecThreads) decode_gate_kernel(
+    const T* __restrict__ q_nope, const __nv_bfloat16* __restrict__ gkc,
+    const float* __restrict__ cur_pool, const T* __restrict__ wq, const float* __restrict__ qnorm_w,
+    const T* __restrict__ wk, const float* __restrict__ knorm_w, const int32_t* __restrict__ seqlens,
+    const float* __restrict__ rc, const float* __restrict__ rs, int Hq, int Hkv, int d, int B, int K,
+    int NBmax, int capacity, float eps, int32_t* __restrict__ sel_idx, float* __restrict__ sel_logg,
+    int32_t* __restrict__ idx_out, float* __restrict__ logg_out) {
+  extern __shared__ float smem[];
+  const int G = Hq / Hkv, GD = G * d, C = 3 * d;
+  float* qcat = smem;                  // [GD]
+  float* P = qcat + GD;                // [C]
+  float* xq = P + C;                   // [H]
+  float* xk = xq + H;                  // [H]
+  float* s = xk + H;                   // [NBmax + 1]
+  float* red = s + NBmax + 1;          // [kDecWarps]
+  int* cnt_red = reinterpret_cast<int*>(red + kDecWarps);  // [kDecWarps]
+
+  const int kv = blockIdx.x, b = blockIdx.y;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int L = seqlens[b];
+  const int t = L - 1, c = t / B, n = L - c * B;
+  const size_t orow = ((size_t)b * Hkv + kv) * (K + 1);
+  if (L < 1 || L > capacity) {   // invalid length: empty selection, the merge writes 0
+    for (int sl = tid; sl <= K; sl += kDecThreads) {
+      sel_idx[orow + sl] = -1;
+      sel_logg[orow + sl] = 0.f;
+      if (idx_out) idx_out[orow + sl] = -1;
+      if (logg_out) logg_out[orow + sl] = 0.f;
+    }
+    return;
+  }
+
+  for (int e = tid; e < GD; e += kDecThreads)
+    qcat[e] = to_f(q_nope[((size_t)b * Hq + (size_t)kv * G) * d + e]);
+  for (int e = tid; e < C; e += kDecThreads) {
+    const int part = e / d, ch = e - part * d;
+    const float x = cur_pool[(((size_t)b * Hkv + kv) * 3 + part) * d + ch];
+    P[e] = (part == 2) ? x / (float)n : x;
+  }
+  __syncthreads();
+  // projections: 2 threads per output channel for each of q and k (H <= 128 -> <= 512 jobs)
+  for (int job = tid; job < 2 * H; job += kDecThreads) {
+    const bool isq = job < H;
+    const int i = isq ? job : job - H;
+    const T* w = isq ? wq + ((size_t)kv * H + i) * GD : wk + ((size_t)kv * H + i) * C;
+    const float* x = isq ? qcat : P;
+    const int n_in = isq ? GD : C;
+    float acc = 0.f;
+    for (int e = 0; e < n_in; ++e) acc = fmaf(to_f(w[e]), x[e], acc);
+    (isq ? xq : xk)[i] = acc;
+  }
+  __syncthreads();
+  if (warp == 0 || warp == 1) {
+    float* x = warp == 0 ? xq : xk;
+    const float* w = warp == 0 ? qnorm_w : knorm_w;
+    const int pos = warp == 0 ? t : c * B;
+    float ss = 0.f;
+    for (int e = lane; e < H; e += 32) ss += x[e] * x[e];
+    ss = warp_sum(ss);
+    const float rn = sqrtf(ss / (float)H + eps);
+    float lo[H / 64 > 0 ? H / 64 : 1], hi[H / 64 > 0 ? H / 64 : 1];
+    int u = 0;
+    for (int e = lane; e < H / 2; e += 32, ++u) {
+      const float a = x[e] / rn * w[e], bb = x[e + H / 2] / rn * w[e + H / 2];
+      const float cs = rc[(size_t)pos * (H / 2) + e], sn = rs[(size_t)pos * (H / 2) + e];
+      lo[u] = a * cs - bb * sn;
+      hi[u] = bb * cs + a * sn;
+    }
+    __syncwarp();
+    u = 0;
+    for (int e = lane; e < H / 2; e += 32, ++u) { x[e] = lo[u]; x[e + H / 2] = hi[u]; }
+  }
+  __syncthreads();
+  const float sqrt_h = sqrtf((float)H);
+  // historical scores: 4 lanes per block, 8 blocks per warp pass
+  {
+    const int sub = lane & 3, grp = lane >> 2;
+    constexpr int PER = H / 4;   // channels per lane
+    const __nv_bfloat16* base = gkc + ((size_t)b * Hkv + kv) * (size_t)NBmax * H;
+    for (int jb = warp * 8; jb < c; jb += 8 * kDecWarps) {   // warp-uniform trip count
+      const int j = jb + grp;
+      float acc = 0.f;
+      if (j < c) {
+        const __nv_bfloat16* kr = base + (size_t)j * H + sub * PER;
+#pragma unroll
+        for (int e0 = 0; e0 < PER; e0 += 8) {
+          const uint4 uv = *reinterpret_cast<const uint4*>(kr + e0);
+          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&uv);
+#pragma unroll
+          for (int w2 = 0; w2 < 4; ++w2) {
+            const float2 f = __bfloat1622float2(h2[w2]);
+            acc = fmaf(xq[sub * PER + e0 + 2 * w2], f.x, acc);
+            acc = fmaf(xq[sub * PER + e0 + 2 * w2 + 1], f.y, acc);
+          }
+        }
+      }
+      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+      if (sub == 0 && j < c) s[j] = acc / sqrt_h;
+    }
+    if (warp == 0) {
+      float dot = 0.f;
+      for (int e = lane; e < H; e += 32) dot += xq[e] * xk[e];
+      dot = warp_sum(dot);
+      if (lane == 0) s[c] = dot / sqrt_h;
+    }
+  }
+  __syncthreads();
+  // logsumexp over j <= c
+  float mx = -INFINITY;
+  for (int j = tid; j <= c; j += kDecThreads) mx = fmaxf(mx, s[j]);
+  mx = block_reduce_max(mx, red);
+  float se = 0.f;
+  for (int j = tid; j <= c; j += kDecThreads) se += expf(s[j] - mx);
+  se = block_reduce_sum(se, red);
+  const float lse = mx + logf(se);
+  if (c <= K) {
+    for (int sl = tid; sl <= K; sl += kDecThreads) {
+      const int jj = sl <= c ? sl : -1;
+      const float lg = sl <= c ? s[sl] - lse : 0.f;
+      sel_idx[orow + sl] = jj;
+      sel_logg[orow + sl] = lg;
+      if (idx_out) idx_out[orow + sl] = jj;
+      if (logg_out) logg_out[orow + sl] = lg;
+    }
+    return;
+  }
+  // exact K-th largest of s[0..c-1] by a bitwise search over order-preserving keys
+  uint32_t key[NPT];
+#pragma unroll
+  for (int r = 0; r < NPT; ++r) {
+    const int j = tid + r * kDecThreads;
+    key[r] = (j < c) ? order_key(s[j]) : 0u;
+  }
+  uint32_t thr = 0;
+#pragma unroll 1
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t cand = thr | (1u << bit);
+    int cn = 0;
+#pragma unroll
+    for (int r = 0; r < NPT; ++r) cn += key[r] >= cand;
+    cn = __reduce_add_sync(0xffffffffu, cn);
+    __syncthreads();
+    if (lane == 0) cnt_red[warp] = cn;
+    __syncthreads();
+    int tot = 0;
+    for (int w = 0; w < kDecWarps; ++w) tot += cnt_red[w];
+    if (tot >= K) thr = cand;
+  }
+  int gt = 0;
+#pragma unroll
+  for (int r = 0; r < NPT; ++r) gt += key[r] > thr;
+  gt = __reduce_add_sync(0xffffffffu, gt);
+  __syncthreads();
+  if (lane == 0) cnt_red[warp] = gt;
+  __syncthreads();
+  int gtot = 0;
+  for (int w = 0; w < kDecWarps; ++w) gtot += cnt_red[w];
+  const int need_eq = K - gtot;
+  if (warp == 0) {   // ordered emission by one warp
+    const unsigned below = (1u << lane) - 1u;
+    int out = 0, eq_seen = 0;
+    for (int j0 = 0; j0 < c; j0 += 32) {
+      const int j = j0 + lane;
+      const uint32_t kk = (j < c) ? order_key(s[j]) : 0u;
+      const bool is_gt = kk > thr, is_eq = kk == thr;
+      const unsigned eqm = __ballot_sync(0xffffffffu, is_eq);
+      const int eq_rank = eq_seen + __popc(eqm & below);
+      const bool sel = is_gt || (is_eq && eq_rank < need_eq);
+      const unsigned selm = __ballot_sync(0xffffffffu, sel);
+      if (sel) {
+        const int pos = out + __popc(selm & below);
+        const float lg = s[j] - lse;
+        sel_idx[orow + pos] = j;
+        sel_logg[orow + pos] = lg;
+        if (idx_out) idx_out[orow + pos] = j;
+        if (logg_out) logg_out[orow + pos] = lg;
+      }
+      out += __popc(selm);
+      eq_seen += __popc(eqm);
+    }
+    if (lane == 0) {
+      const float lg = s[c] - lse;
+      sel_idx[orow + K] = c;
+      sel_logg[orow + K] = lg;
+      if (idx_out) idx_out[orow + K] = c;
+      if (logg_out) logg_out[orow + K] = lg;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// (2) split-K attention over the selected blocks. CTA = (kv, sequence, split); each warp
+// streams every 8th key of the CTA's blocks (one 2*d-byte row of K and of V per key, lane
+// slices of d/32 channels) and keeps an online softmax for the G heads.
+// ---------------------------------------------------------------------------------------
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(
+    const T* __restrict__ q, const T* __restrict__ kc, const T* __restrict__ vc,
+    const int32_t* __restrict__ seqlens, const int32_t* __restrict__ sel_idx,
+    const float* __restrict__ sel_logg, int Hkv, int capacity, int B, int K, int nsplit,
+    float scale_log2, float* __restrict__ part_ml, float* __restrict__ part_acc) {
+  constexpr int E = D / 32;
+  __shared__ float sm_m[kDecWarps][G], sm_l[kDecWarps][G];
+  __shared__ float sm_acc[kDecWarps][G][D];
+  const int kv = blockIdx.x, b = blockIdx.y, split = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int L = min(seqlens[b], capacity);
+  const int Hq = Hkv * G;
+  const int slots = K + 1;
+  const int per = (slots + nsplit - 1) / nsplit;
+  const int sl0 = split * per, sl1 = min(slots, sl0 + per);
+  const size_t srow = ((size_t)b * Hkv + kv) * (K + 1);
+  float qr[G][E], acc[G][E], m[G], l[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      qr[g][e] = to_f(q[((size_t)b * Hq + kv * G + g) * D + lane * E + e]);
+      acc[g][e] = 0.f;
+    }
+    m[g] = -INFINITY;
+    l[g] = 0.f;
+  }
+  const T* kbase = kc + ((size_t)b * Hkv + kv) * (size_t)capacity * D + lane * E;
+  const T* vbase = vc + ((size_t)b * Hkv + kv) * (size_t)capacity * D + lane * E;
+  for (int sl = sl0; sl < sl1; ++sl) {
+    const int j = sel_idx[srow + sl];
+    if (j < 0) continue;
+    const float bias = sel_logg[srow + sl] * kLog2e;
+    const int i0 = j * B, i1 = min(i0 + B, L);
+    for (int i = i0 + warp; i < i1; i += kDecWarps) {
+      float kk[E], vv[E];
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        kk[e] = to_f(kbase[(size_t)i * D + e]);
+        vv[e] = to_f(vbase[(size_t)i * D + e]);
+      }
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        float p = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) p = fmaf(qr[g][e], kk[e], p);
+        p = warp_sum(p) * scale_log2 + bias;
+        const float mn = fmaxf(m[g], p);
+        const float a = exp2f(m[g] - mn), pe = exp2f(p - mn);
+        l[g] = l[g] * a + pe;
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[g][e] = fmaf(acc[g][e], a, pe * vv[e]);
+        m[g] = mn;
+      }
+    }
+  }
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    if (lane == 0) { sm_m[warp][g] = m[g]; sm_l[warp][g] = l[g]; }
+#pragma unroll
+    for (int e = 0; e < E; ++e) sm_acc[warp][g][lane * E + e] = acc[g][e];
+  }
+  __syncthreads();
+  const size_t prow = (((size_t)b * Hkv + kv) * nsplit + split) * G;
+  for (int e = threadIdx.x; e < G * D; e += kDecThreads) {
+    const int g = e / D, ch = e - g * D;
+    float M = -INFINITY;
+    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, sm_m[w][g]);
+    float ls = 0.f, as = 0.f;
+    if (M != -INFINITY) {
+      for (int w = 0; w < kDecWarps; ++w) {
+        const float f = exp2f(sm_m[w][g] - M);
+        ls += sm_l[w][g] * f;
+        as += sm_acc[w][g][ch] * f;
+      }
+    }
+    part_acc[(prow + g) * D + ch] = as;
+    if (ch == 0) {
+      part_ml[(prow + g) * 2] = M;
+      part_ml[(prow + g) * 2 + 1] = ls;
+    }
+  }
+}
+
+// (3) merge the splits (log2-domain maxima) and normalise.
+template <typename T, int D, int G>
+__global__ void decode_merge_kernel(const float* __restrict__ part_ml, const float* __restrict__ part_acc,
+                                    int Hkv, int nsplit, T* __restrict__ o) {
+  const int kv = blockIdx.x, b = blockIdx.y;
+  const int Hq = Hkv * G;
+  for (int e = threadIdx.x; e < G * D; e += blockDim.x) {
+    const int g = e / D, ch = e - g * D;
+    float M = -INFINITY;
+    for (int sp = 0; sp < nsplit; ++sp)
+      M = fmaxf(M, part_ml[((((size_t)b * Hkv + kv) * nsplit + sp) * G + g) * 2]);
+    float ls = 0.f, as = 0.f;
+    for (int sp = 0; sp < nsplit; ++sp) {
+      const size_t pr = (((size_t)b * Hkv + kv) * nsplit + sp) * G + g;
+      const float mm = part_ml[pr * 2];
+      if (mm == -INFINITY) continue;
+      const float f = exp2f(mm - M);
+      ls += part_ml[pr * 2 + 1] * f;
+      as += part_acc[pr * D + ch] * f;
+    }
+    o[((size_t)b * Hq + kv * G + g) * D + ch] = from_f<T>(ls > 0.f ? as / ls : 0.f);
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+int decode_nsplit(const sas_decode_problem& p) {
+  const int pairs = p.batch * p.num_kv_heads;
+  int ns = (8 * 148 + pairs - 1) / pairs;
+  if (ns < 1) ns = 1;
+  if (ns > p.topk + 1) ns = p.topk + 1;
+  return ns;
+}
+
+size_t decode_workspace_bytes(const sas_decode_problem& p) {
+  const int G = p.num_q_heads / p.num_kv_heads;
+  const size_t pairs = (size_t)p.batch * p.num_kv_heads;
+  const size_t ns = decode_nsplit(p);
+  auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  return al(pairs * (p.topk + 1) * 4) * 2 + al(pairs * ns * G * 2 * 4) +
+         al(pairs * ns * G * p.head_dim * 4);
+}
+
+template <typename T, int D, int G>
+static void decode_attn_launch(const sas_decode_problem& p, const void* q, const void* kc,
+                               const void* vc, int32_t* sel_idx, float* sel_logg, float* part_ml,
+                               float* part_acc, void* o, int ns, cudaStream_t st) {
+  dim3 grid(p.num_kv_heads, p.batch, ns);
+  decode_attn_kernel<T, D, G><<<grid, kDecThreads, 0, st>>>(
+      (const T*)q, (const T*)kc, (const T*)vc, p.seqlens, sel_idx, sel_logg, p.num_kv_heads,
+      p.capacity, p.block, p.topk, ns, kLog2e / sqrtf((float)D), part_ml, part_acc);
+  decode_merge_kernel<T, D, G><<<dim3(p.num_kv_heads, p.batch), 256, 0, st>>>(
+      part_ml, part_acc, p.num_kv_heads, ns, (T*)o);
+}
+
+template <typename T>
+static void decode_gate_launch(const sas_decode_problem& p, const void* q_nope, const void* gkc,
+                               const float* cur_pool, const void* wq, const float* qnorm_w,
+                               const void* wk, const float* knorm_w, int32_t* sel_idx,
+                               float* sel_logg, int32_t* idx_out, float* logg_out, cudaStream_t st) {
+  const int NBmax = (p.capacity + p.block - 1) / p.block;
+  const int G = p.num_q_heads / p.num_kv_heads;
+  const size_t smem = (size_t)(G * p.head_dim + 3 * p.head_dim + 2 * p.gate_hidden + NBmax + 1 +
+                               2 * kDecWarps) * sizeof(float);
+  dim3 grid(p.num_kv_heads, p.batch);
+#define SAS_DG(H, NPT)                                                                           \
+  {                                                                                              \
+    cudaFuncSetAttribute(decode_gate_kernel<T, H, NPT>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                         (int)smem);                                                             \
+    decode_gate_kernel<T, H, NPT><<<grid, kDecThreads, smem, st>>>(                              \
+        (const T*)q_nope, (const __nv_bfloat16*)gkc, cur_pool, (const T*)wq, qnorm_w, (const T*)wk, \
+        knorm_w, p.seqlens, p.gate_rope_cos, p.gate_rope_sin, p.num_q_heads, p.num_kv_heads,      \
+        p.head_dim, p.block, p.topk, NBmax, p.capacity, p.rms_eps, sel_idx, sel_logg, idx_out,   \
+        logg_out);                                                                               \
+  }
+#define SAS_DG_H(NPT)                              \
+  switch (p.gate_hidden) {                         \
+    case 32: SAS_DG(32, NPT); break;               \
+    case 64: SAS_DG(64, NPT); break;               \
+    default: SAS_DG(128, NPT); break;              \
+  }
+  if (NBmax <= 256) { SAS_DG_H(1) }
+  else if (NBmax <= 1024) { SAS_DG_H(4) }
+  else if (NBmax <= 2048) { SAS_DG_H(8) }
+  else { SAS_DG_H(16) }
+#undef SAS_DG_H
+#undef SAS_DG
+}
+
+sas_status launch_decode(const sas_decode_problem& p, const void* q, const void* q_nope,
+                         const void* k_cache, const void* v_cache, const void* gkc,
+                         const float* cur_pool, const void* wq, const float* qnorm_w,
+                         const void* wk, const float* knorm_w, void* o, int32_t* idx_out,
+                         float* logg_out, void* ws, cudaStream_t st) {
+  const int G = p.num_q_heads / p.num_kv_heads;
+  const size_t pairs = (size_t)p.batch * p.num_kv_heads;
+  const int ns = decode_nsplit(p);
+  auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  char* w = (char*)ws;
+  int32_t* sel_idx = (int32_t*)w;
+  w += al(pairs * (p.topk + 1) * 4);
+  float* sel_logg = (float*)w;
+  w += al(pairs * (p.topk + 1) * 4);
+  float* part_ml = (float*)w;
+  w += al(pairs * ns * G * 2 * 4);
+  float* part_acc = (float*)w;
+  if (p.dtype == SAS_BF16)
+    decode_gate_launch<__nv_bfloat16>(p, q_nope, gkc, cur_pool, wq, qnorm_w, wk, knorm_w, sel_idx,
+                                      sel_logg, idx_out, logg_out, st);
+  else
+    decode_gate_launch<float>(p, q_nope, gkc, cur_pool, wq, qnorm_w, wk, knorm_w, sel_idx, sel_logg,
+                              idx_out, logg_out, st);
+  sas_status s = launch_status("decode gate", 1);
+  if (s != SAS_OK) return s;
+#define SAS_DA(T, D, G)                                                                      \
+  decode_attn_launch<T, D, G>(p, q, k_cache, v_cache, sel_idx, sel_logg, part_ml, part_acc, o, \
+                              ns, st)
+#define SAS_DA_G(T, D)                   \
+  switch (G) {                           \
+    case 1: SAS_DA(T, D, 1); break;      \
+    case 2: SAS_DA(T, D, 2); break;      \
+    case 4: SAS_DA(T, D, 4); break;      \
+    case 5: SAS_DA(T, D, 5); break;      \
+    default: SAS_DA(T, D, 8); break;     \
+  }
+  if (p.dtype == SAS_BF16) {
+    if (p.head_dim == 64) { SAS_DA_G(__nv_bfloat16, 64) } else { SAS_DA_G(__nv_bfloat16, 128) }
+  } else {
+    if (p.head_dim == 64) { SAS_DA_G(float, 64) } else { SAS_DA_G(float, 128) }
+  }
+#undef SAS_DA_G
+#undef SAS_DA
+  return launch_status("decode attention", 2);
+}
+
+}  // namespace sas

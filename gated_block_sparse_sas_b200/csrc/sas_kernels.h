@@ -1,0 +1,37 @@
+// Internal launcher declarations (host side) shared by the C ABI implementation.
+#pragma once
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include "sas.h"
+
+namespace sas {
+
+sas_status launch_pool_keys(const sas_problem& p, const void* k_nope, float* pooled, cudaStream_t st);
+sas_status launch_gate_keys(const sas_problem& p, const float* pooled, const void* wk,
+                            const float* knorm_w, float* gkeys, cudaStream_t st);
+sas_status launch_gate_scores(const sas_problem& p, const void* q_nope, const void* k_nope,
+                              const float* gkeys, const void* wq, const float* qnorm_w,
+                              const void* wk, const float* knorm_w, float* scores, float* lse,
+                              cudaStream_t st);
+sas_status launch_topk(const sas_problem& p, const float* scores, const float* lse, int32_t* idx,
+                       float* logg, cudaStream_t st);
+
+sas_status launch_attn_fwd_simt(const sas_problem& p, const void* q, const void* k, const void* v,
+                                const int32_t* idx, const float* logg, void* o, float* lse,
+                                cudaStream_t st);
+sas_status launch_attn_bwd_simt(const sas_problem& p, const void* q, const void* k, const void* v,
+                                const void* o, const void* dout, const float* lse,
+                                const int32_t* idx, const float* logg, void* dq, void* dk, void* dv,
+                                float* dlogg, float* drow, cudaStream_t st);
+
+int decode_nsplit(const sas_decode_problem& p);
+size_t decode_workspace_bytes(const sas_decode_problem& p);
+sas_status launch_decode(const sas_decode_problem& p, const void* q, const void* q_nope,
+                         const void* k_cache, const void* v_cache, const void* gkc,
+                         const float* cur_pool, const void* wq, const float* qnorm_w,
+                         const void* wk, const float* knorm_w, void* o, int32_t* idx_out,
+                         float* logg_out, void* ws, cudaStream_t st);
+
+}  // namespace sas

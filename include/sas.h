@@ -1,0 +1,203 @@
+/*
+ * sas.h -- C ABI of the B200 (sm_100a) gated block-sparse attention library.
+ *
+ * The operator is SAS gated sparse attention as described on the SAS pages:
+ *   - project README "SAS: Simple Attention Sparsification via End-to-End
+ *     Optimization of Context Ranking", intro items (a) and (b): discrete Top-K
+ *     block selection, each selected block carrying a continuous gate that is
+ *     added to the attention logits;
+ *   - model card "tencent/Simple-Attention-Sparsification", table "Checkpoint
+ *     configuration": KV block 64, Top-K 31 historical blocks, gate hidden 128,
+ *     query projection Qproj, key-block pooling max + min + average, Q/K
+ *     normalisation, gate RoPE; and its decode-budget paragraph (2,048 tokens,
+ *     1,024 / 4,096 also usable);
+ *   - the paper's abstract: gates inside the attention softmax in log form,
+ *     normalised softmax gates that weigh history against the always-retained
+ *     current block, FlashAttention-style memory-efficient kernel.
+ *
+ * Readings of points the pages leave open (the same ones the test oracle uses):
+ *   one gate per (token, KV head), shared by the G = Hq/Hkv query heads; Qproj
+ *   reads the G pre-rotary query heads concatenated (G*d -> h); pooled block key
+ *   = concat(max, min, mean) (3d -> h); RMSNorm (eps, weight) after each
+ *   projection, then rotate-half rotary over h at position t (query) or j*B
+ *   (block start); score s = q~.k~/sqrt(h); softmax over every causally visible
+ *   block j <= c_t (current block included), log g = s - logsumexp; the current
+ *   block's key pools only tokens c_t*B..t; Top-K over historical blocks j < c_t
+ *   (all if c_t <= K), ties to the lower index; attention logit
+ *   z = q.k/sqrt(d) + log g(block of key) for selected blocks and keys <= t.
+ *
+ * Conventions (every entry point):
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *     never allocates, frees or synchronises. Every launch is asynchronous on
+ *     `stream`. Caller-provided workspace must be at least the size the matching
+ *     *_workspace_size call reports and 256-byte aligned.
+ *   - Tensors are dense, row-major, in the shapes written below; tokens of all
+ *     sequences are packed back to back (cu_seqlens). Device pointers must be
+ *     16-byte aligned.
+ *   - T = total_tokens, Hq/Hkv = query/KV heads, G = Hq/Hkv, d = head_dim,
+ *     B = block, K = topk, h = gate_hidden, NBmax = ceil(max_seqlen / B).
+ *   - "dtype" tensors are bf16 (SAS_BF16) or fp32 (SAS_FP32); fp32 tensors are
+ *     always fp32.
+ *   - Errors: invalid or unsupported arguments are detected before any launch
+ *     and return a negative status; sas_last_error() (thread-local) then holds
+ *     the reason. A failed launch returns SAS_ERR_CUDA. Nothing is launched
+ *     after the first error of a call.
+ *   - Supported: d in {64, 128}; B in {16, 32, 64}; 1 <= K <= 127;
+ *     h in {32, 64, 128}; G in {1, 2, 4, 5, 8}; NBmax <= 2048 (prefill) or
+ *     ceil(capacity / B) <= 4096 (decode). Anything else returns
+ *     SAS_ERR_UNSUPPORTED.
+ */
+#ifndef SAS_H
+#define SAS_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum sas_status {
+  SAS_OK = 0,
+  SAS_ERR_INVALID_ARG = -1,
+  SAS_ERR_UNSUPPORTED = -2,
+  SAS_ERR_CUDA = -3,
+  SAS_ERR_WORKSPACE = -4
+} sas_status;
+
+typedef enum sas_dtype { SAS_BF16 = 0, SAS_FP32 = 1 } sas_dtype;
+
+/* A packed prefill / training problem. */
+typedef struct sas_problem {
+  int32_t batch;          /* number of sequences                                   */
+  int32_t total_tokens;   /* T = cu_seqlens[batch]                                 */
+  int32_t max_seqlen;     /* longest sequence                                      */
+  int32_t num_q_heads;    /* Hq                                                    */
+  int32_t num_kv_heads;   /* Hkv                                                   */
+  int32_t head_dim;       /* d                                                     */
+  int32_t block;          /* B, tokens per KV block                                */
+  int32_t topk;           /* K, historical blocks kept per query                   */
+  int32_t gate_hidden;    /* h                                                     */
+  float rms_eps;          /* RMSNorm epsilon of the gate                           */
+  sas_dtype dtype;        /* element type of Q/K/V/O/dO/dQ/dK/dV and gate weights  */
+  const int32_t* cu_seqlens;   /* device [batch+1], cu_seqlens[0] = 0              */
+  const float* gate_rope_cos;  /* device [max_seqlen, h/2] (sas_rope_tables)        */
+  const float* gate_rope_sin;  /* device [max_seqlen, h/2]                          */
+} sas_problem;
+
+/* One decode step over a batch of contiguous KV caches. */
+typedef struct sas_decode_problem {
+  int32_t batch;
+  int32_t capacity;       /* cache capacity in tokens, Lmax; NBmax = ceil(Lmax/B)  */
+  int32_t num_q_heads;
+  int32_t num_kv_heads;
+  int32_t head_dim;
+  int32_t block;
+  int32_t topk;           /* budget = (K + 1) * B tokens                           */
+  int32_t gate_hidden;
+  float rms_eps;
+  sas_dtype dtype;        /* q / caches / gate weights                              */
+  const int32_t* seqlens;      /* device [batch]: L_b in 1..capacity, newest token at L_b-1 */
+  const float* gate_rope_cos;  /* device [capacity, h/2]                           */
+  const float* gate_rope_sin;
+} sas_decode_problem;
+
+/* Reason for the last non-OK status returned on this thread ("" if none). */
+const char* sas_last_error(void);
+
+/* Diagnostic: number of kernels this library has launched from the calling thread
+ * since the library was loaded (every entry point adds the launches it issued). */
+uint64_t sas_kernel_launches(void);
+
+/* Host helper: cos/sin tables of the gate's rotate-half rotary embedding,
+ * theta(p, i) = p * base^(-2i/rot_dim), computed in double and rounded once to
+ * float. cos_out/sin_out are HOST buffers of positions * rot_dim/2 floats,
+ * row p = position p. Model card "Checkpoint configuration": Gate RoPE enabled. */
+sas_status sas_rope_tables(int32_t positions, int32_t rot_dim, double base,
+                           float* cos_out, float* sin_out);
+
+/* A1 -- key-block pooling (model card "Checkpoint configuration": key block pooling
+ * max + min + average). k_nope: dtype [T, Hkv, d], keys before the backbone's
+ * rotary embedding. pooled: fp32 [batch, NBmax, Hkv, 3d] = (max | min | mean) over
+ * each block's tokens (a sequence's last block may be partial); blocks past a
+ * sequence's end are written as 0. */
+sas_status sas_pool_keys(const sas_problem* p, const void* k_nope, float* pooled,
+                         cudaStream_t stream);
+
+/* A2 -- gate block keys (model card: Q/K normalization, Gate RoPE).
+ * k~_j = rope(RMSNorm(Wk . pooled_j) * knorm_w, pos = j*B).
+ * pooled fp32 [batch, NBmax, Hkv, 3d]; wk dtype [Hkv, h, 3d]; knorm_w fp32 [h];
+ * gate_keys fp32 [batch, NBmax, Hkv, h] (0 past a sequence's end). */
+sas_status sas_gate_keys(const sas_problem* p, const float* pooled, const void* wk,
+                         const float* knorm_w, float* gate_keys, cudaStream_t stream);
+
+/* A3 -- gate scores (model card: Query projection Qproj; abstract: normalised
+ * softmax gates calibrated against the always-retained current block).
+ * q~_t = rope(RMSNorm(Wq . concat_g q_nope[t, kv*G+g]) * qnorm_w, pos = t);
+ * s[t, kv, j] = q~_t . k~_j / sqrt(h) for j < c_t from gate_keys, and for j = c_t
+ * with the current block's key pooled over its tokens c_t*B..t (computed here from
+ * k_nope, wk, knorm_w); s = -inf for j > c_t. lse[t, kv] = logsumexp_{j<=c_t} s.
+ * q_nope dtype [T, Hq, d]; k_nope dtype [T, Hkv, d]; gate_keys fp32 [batch, NBmax,
+ * Hkv, h]; wq dtype [Hkv, h, G*d]; wk dtype [Hkv, h, 3d]; qnorm_w, knorm_w fp32 [h];
+ * scores fp32 [T, Hkv, NBmax]; lse fp32 [T, Hkv]. */
+sas_status sas_gate_scores(const sas_problem* p, const void* q_nope, const void* k_nope,
+                           const float* gate_keys, const void* wq, const float* qnorm_w,
+                           const void* wk, const float* knorm_w, float* scores, float* lse,
+                           cudaStream_t stream);
+
+/* A4 -- Top-K selection (README (b); model card: Training Top-K 31 historical blocks).
+ * Per (t, kv): the min(K, c_t) historical blocks with the highest score (ties to
+ * the lower index), ascending, then the current block c_t, then -1 padding.
+ * idx int32 [T, Hkv, K+1]; logg fp32 [T, Hkv, K+1] = s - lse on kept slots, 0 on
+ * padding. Bit-exact given the scores. */
+sas_status sas_topk(const sas_problem* p, const float* scores, const float* lse,
+                    int32_t* idx, float* logg, cudaStream_t stream);
+
+/* A5 -- gated sparse attention forward (README (b); abstract: gate in the softmax in
+ * log form, FlashAttention-style). For query head hq (kv = hq / G), token t:
+ * z_i = q_t.k_i/sqrt(d) + logg[t, kv, slot] for keys i <= t of block idx[t, kv, slot];
+ * O_t = softmax(z) V; lse_attn = natural-log logsumexp of z.
+ * q dtype [T, Hq, d]; k, v dtype [T, Hkv, d] (rotated); idx/logg as from sas_topk
+ * (any valid selection: ascending historical, current block, -1 padding);
+ * o dtype [T, Hq, d]; lse_attn fp32 [T, Hq]. */
+sas_status sas_attn_fwd_workspace_size(const sas_problem* p, size_t* bytes);
+sas_status sas_attn_fwd(const sas_problem* p, const void* q, const void* k, const void* v,
+                        const int32_t* idx, const float* logg, void* o, float* lse_attn,
+                        void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* A6 -- backward of A5 with the selection held fixed (abstract: the loss reaches the
+ * selector through standard backpropagation). Inputs as A5 plus o, dout (dtype
+ * [T, Hq, d]) and lse_attn. Outputs dq dtype [T, Hq, d]; dk, dv dtype [T, Hkv, d];
+ * dlogg fp32 [T, Hkv, K+1] = sum over the G heads and the keys of block
+ * idx[t, kv, slot] of P (dP - D), 0 on padding. */
+sas_status sas_attn_bwd_workspace_size(const sas_problem* p, size_t* bytes);
+sas_status sas_attn_bwd(const sas_problem* p, const void* q, const void* k, const void* v,
+                        const void* o, const void* dout, const float* lse_attn,
+                        const int32_t* idx, const float* logg, void* dq, void* dk, void* dv,
+                        float* dlogg, void* workspace, size_t workspace_bytes,
+                        cudaStream_t stream);
+
+/* A7 -- one sparse decode step (model card: sparse decode budget; Chinese guide caveat
+ * 3: the budget caps the tokens each query attends to). For sequence b with L_b
+ * cached tokens (newest at L_b-1, c = (L_b-1)/B): gate query at position L_b-1;
+ * historical block keys read from gate_key_cache; the current block's key from the
+ * running pool state (max, min, sum/n, n = L_b - c*B) at position c*B; softmax
+ * gates, Top-K, then the gated attention of the G query heads over the kept blocks.
+ * q dtype [batch, Hq, d] (rotated); q_nope dtype [batch, Hq, d];
+ * k_cache, v_cache dtype [batch, Hkv, capacity, d]; gate_key_cache bf16
+ * [batch, Hkv, NBmax, h] (entries j < c read); cur_pool fp32 [batch, Hkv, 3, d]
+ * (max, min, sum over tokens c*B..L_b-1); wq, wk, qnorm_w, knorm_w as A3;
+ * o dtype [batch, Hq, d]; idx_out int32 / logg_out fp32 [batch, Hkv, K+1] may be NULL. */
+sas_status sas_decode_workspace_size(const sas_decode_problem* p, size_t* bytes);
+sas_status sas_decode(const sas_decode_problem* p, const void* q, const void* q_nope,
+                      const void* k_cache, const void* v_cache, const void* gate_key_cache,
+                      const float* cur_pool, const void* wq, const float* qnorm_w,
+                      const void* wk, const float* knorm_w, void* o, int32_t* idx_out,
+                      float* logg_out, void* workspace, size_t workspace_bytes,
+                      cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SAS_H */

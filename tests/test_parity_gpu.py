@@ -1,0 +1,183 @@
+"""GPU parity: the CUDA library (through its C ABI) against the CPU oracle, element by
+element on the same seeded inputs. Small cases span several tiles and ragged tails;
+tolerances are those stated in tests/parity_utils.py."""
+import numpy as np
+import pytest
+import torch
+
+import sas_inputs as si
+from oracle import sas_oracle as orc
+from parity_utils import (assert_grad_close, assert_out_close, compare_selection, to64,
+                          GATE_ABS)
+
+pytestmark = pytest.mark.gpu
+
+CASES = {
+    # lengths, Hq, Hkv, d, B, K, h, dtype
+    "bf16-d128-B64-ragged": ([300, 64, 1, 130], 8, 2, 128, 64, 3, 128, "bf16"),
+    "bf16-d128-B64-G5": ([513, 77], 10, 2, 128, 64, 4, 128, "bf16"),
+    "bf16-d64-B32": ([257, 33], 8, 4, 64, 32, 5, 64, "bf16"),
+    "fp32-d64-B16-tiny-shape": ([1024], 2, 1, 64, 16, 4, 32, "fp32"),
+    "bf16-d128-B16-K-large": ([200], 4, 1, 128, 16, 20, 32, "bf16"),
+}
+
+
+@pytest.fixture(scope="module")
+def sas():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import gated_block_sparse_sas_b200 as m
+    return m
+
+
+def _setup(sas, name, seed=100):
+    lengths, Hq, Hkv, d, B, K, h, dt = CASES[name]
+    shape = si.Shape(list(lengths), Hq, Hkv, d, B, K, h, dt, seed=seed)
+    inp = si.prefill_inputs(shape, with_dout=True)
+    dev = torch.device("cuda:0")
+    g = {k: v.to(dev) for k, v in inp.items()}
+    prob = sas.Problem.from_lengths(shape.lengths, dev, num_q_heads=Hq, num_kv_heads=Hkv,
+                                    head_dim=d, block=B, topk=K, gate_hidden=h,
+                                    dtype=shape.torch_dtype)
+    return shape, inp, g, prob
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_gate_pipeline(sas, name):
+    shape, inp, g, prob = _setup(sas, name)
+    pooled = sas.sas_pool_keys(prob, g["k_nope"])
+    gk = sas.sas_gate_keys(prob, pooled, g["wk"], g["knorm_w"])
+    scores, lse = sas.sas_gate_scores(prob, g["q_nope"], g["k_nope"], gk, g["wq"], g["qnorm_w"],
+                                      g["wk"], g["knorm_w"])
+    idx, logg = sas.sas_topk(prob, scores, lse)
+    torch.cuda.synchronize()
+    ref = orc.prefill_selection(inp["q_nope"], inp["k_nope"], inp["wq"], inp["qnorm_w"], inp["wk"],
+                                inp["knorm_w"], shape.cu_seqlens, shape.block, shape.topk, 1e-6, 1e6)
+    np.testing.assert_allclose(to64(pooled), ref["pooled"], rtol=2e-6, atol=2e-6)
+    np.testing.assert_allclose(to64(gk), ref["gate_keys"], rtol=0, atol=GATE_ABS)
+    s, sr = to64(scores), ref["scores"]
+    assert (np.isneginf(s) == np.isneginf(sr)).all()
+    fin = np.isfinite(sr)
+    assert np.abs(s[fin] - sr[fin]).max() <= GATE_ABS
+    assert np.abs(to64(lse) - ref["lse"]).max() <= GATE_ABS
+    n, near, flips = compare_selection(idx.cpu().numpy(), logg, ref["idx"], ref["logg"], ref["margin"])
+    assert near <= max(2, 0.01 * n)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_attention_forward(sas, name):
+    shape, inp, g, prob = _setup(sas, name, seed=200)
+    idx, logg = si.random_selection(shape)
+    o, lse = sas.sas_attn_fwd(prob, g["q"], g["k"], g["v"], torch.from_numpy(idx).cuda(),
+                              torch.from_numpy(logg).cuda())
+    torch.cuda.synchronize()
+    O, LSE, _ = orc.attention_fwd(inp["q"], inp["k"], inp["v"], idx, logg, shape.cu_seqlens,
+                                  shape.block)
+    fp32 = shape.dtype == "fp32"
+    assert_out_close(o, O, fp32, "O")
+    assert np.abs(to64(lse) - LSE).max() <= (1e-4 if fp32 else 2e-3)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_attention_backward(sas, name):
+    shape, inp, g, prob = _setup(sas, name, seed=300)
+    idx, logg = si.random_selection(shape)
+    ti, tl = torch.from_numpy(idx).cuda(), torch.from_numpy(logg).cuda()
+    o, lse = sas.sas_attn_fwd(prob, g["q"], g["k"], g["v"], ti, tl)
+    dq, dk, dv, dl = sas.sas_attn_bwd(prob, g["q"], g["k"], g["v"], o, g["dout"], lse, ti, tl)
+    torch.cuda.synchronize()
+    ref = orc.attention_bwd(inp["q"], inp["k"], inp["v"], inp["dout"], idx, logg, shape.cu_seqlens,
+                            shape.block)
+    fp32 = shape.dtype == "fp32"
+    for gpu, r, nm in zip((dq, dk, dv, dl), ref, ("dQ", "dK", "dV", "dlogg")):
+        assert_grad_close(gpu, r, fp32, nm)
+    assert (to64(dl)[idx < 0] == 0).all()
+
+
+def test_tiny_config_end_to_end(sas):
+    """The tiny fp32 workload: gate -> Top-K -> attention fwd/bwd on the GPU against the oracle."""
+    shape = si.workload("tiny-fp32-T1024")
+    inp = si.prefill_inputs(shape, with_dout=True)
+    g = {k: v.cuda() for k, v in inp.items()}
+    prob = sas.Problem.from_lengths(shape.lengths, torch.device("cuda:0"), num_q_heads=2,
+                                    num_kv_heads=1, head_dim=64, block=16, topk=4, gate_hidden=32,
+                                    dtype=torch.float32)
+    idx, logg = sas.prefill_selection(prob, g["q_nope"], g["k_nope"], g["wq"], g["qnorm_w"],
+                                      g["wk"], g["knorm_w"])
+    o, lse = sas.sas_attn_fwd(prob, g["q"], g["k"], g["v"], idx, logg)
+    dq, dk, dv, dl = sas.sas_attn_bwd(prob, g["q"], g["k"], g["v"], o, g["dout"], lse, idx, logg)
+    torch.cuda.synchronize()
+    ref = orc.prefill_selection(inp["q_nope"], inp["k_nope"], inp["wq"], inp["qnorm_w"], inp["wk"],
+                                inp["knorm_w"], shape.cu_seqlens, 16, 4, 1e-6, 1e6)
+    compare_selection(idx.cpu().numpy(), logg, ref["idx"], ref["logg"], ref["margin"])
+    # attention against the oracle on the oracle's own selection (identical except near-ties)
+    ri, rl = ref["idx"], ref["logg"].astype(np.float32)
+    o2, lse2 = sas.sas_attn_fwd(prob, g["q"], g["k"], g["v"], torch.from_numpy(ri).cuda(),
+                                torch.from_numpy(rl).cuda())
+    O, _, _ = orc.attention_fwd(inp["q"], inp["k"], inp["v"], ri, rl, shape.cu_seqlens, 16)
+    assert_out_close(o2, O, True, "O")
+    grads = sas.sas_attn_bwd(prob, g["q"], g["k"], g["v"], o2, g["dout"], lse2,
+                             torch.from_numpy(ri).cuda(), torch.from_numpy(rl).cuda())
+    refg = orc.attention_bwd(inp["q"], inp["k"], inp["v"], inp["dout"], ri, rl, shape.cu_seqlens, 16)
+    for gpu, r, nm in zip(grads, refg, ("dQ", "dK", "dV", "dlogg")):
+        assert_grad_close(gpu, r, True, nm)
+
+
+DEC_CASES = {
+    "bf16-d128-B64": ([1, 64, 65, 700, 2048, 1500], 2048, 8, 2, 128, 64, 7, 128),
+    "bf16-d128-B64-G4-K31": ([4000, 129, 2500], 4096, 16, 4, 128, 64, 31, 128),
+    "bf16-d64-B16": ([30, 17, 300], 512, 4, 2, 64, 16, 5, 32),
+}
+
+
+@pytest.mark.parametrize("name", list(DEC_CASES))
+def test_decode(sas, name):
+    lengths, cap, Hq, Hkv, d, B, K, h = DEC_CASES[name]
+    shp = si.DecodeShape(list(lengths), cap, Hq, Hkv, d, B, K, h, seed=400)
+    inp = si.decode_inputs(shp)
+    g = {k: v.cuda() for k, v in inp.items()}
+    prob = sas.DecodeProblem(seqlens=g["lengths"], capacity=cap, num_q_heads=Hq, num_kv_heads=Hkv,
+                             head_dim=d, block=B, topk=K, gate_hidden=h, dtype=torch.bfloat16)
+    o, idx, logg = sas.sas_decode(prob, g["q"], g["q_nope"], g["k_cache"], g["v_cache"],
+                                  g["gate_key_cache"], g["cur_pool"], g["wq"], g["qnorm_w"], g["wk"],
+                                  g["knorm_w"], want_selection=True)
+    torch.cuda.synchronize()
+    O, ridx, rlogg, margin = orc.decode(inp["q"], inp["q_nope"], inp["k_cache"], inp["v_cache"],
+                                        lengths, inp["gate_key_cache"], inp["cur_pool"], inp["wq"],
+                                        inp["qnorm_w"], inp["wk"], inp["knorm_w"], B, K, 1e-6, 1e6)
+    compare_selection(idx.cpu().numpy(), logg, ridx, rlogg, margin)
+    same = (idx.cpu().numpy() == ridx).all(axis=-1).all(axis=-1)
+    assert_out_close(o[torch.from_numpy(same)], O[same], False, "O")
+
+
+def test_decode_equals_prefill_row(sas):
+    """A decode step over caches written from a prefill equals that prefill's last row."""
+    L, B, K, h = 777, 64, 5, 128
+    shape = si.Shape([L], 8, 2, 128, B, K, h, "bf16", seed=500)
+    inp = si.prefill_inputs(shape)
+    g = {k: v.cuda() for k, v in inp.items()}
+    prob = sas.Problem.from_lengths([L], torch.device("cuda:0"), num_q_heads=8, num_kv_heads=2,
+                                    head_dim=128, block=B, topk=K, gate_hidden=h,
+                                    dtype=torch.bfloat16)
+    pooled = sas.sas_pool_keys(prob, g["k_nope"])
+    gk = sas.sas_gate_keys(prob, pooled, g["wk"], g["knorm_w"])
+    gk_bf = gk.to(torch.bfloat16)
+    scores, lse = sas.sas_gate_scores(prob, g["q_nope"], g["k_nope"], gk_bf.float().contiguous(),
+                                      g["wq"], g["qnorm_w"], g["wk"], g["knorm_w"])
+    idx, logg = sas.sas_topk(prob, scores, lse)
+    o, _ = sas.sas_attn_fwd(prob, g["q"], g["k"], g["v"], idx, logg)
+    c = (L - 1) // B
+    cur = g["k_nope"][c * B:L].float()
+    pool = torch.stack([cur.amax(0), cur.amin(0), cur.sum(0)], dim=1)[None].contiguous()
+    dprob = sas.DecodeProblem(seqlens=torch.tensor([L], dtype=torch.int32, device="cuda"),
+                              capacity=L, num_q_heads=8, num_kv_heads=2, head_dim=128, block=B,
+                              topk=K, gate_hidden=h, dtype=torch.bfloat16)
+    od, di, dl = sas.sas_decode(dprob, g["q"][L - 1:L].contiguous(), g["q_nope"][L - 1:L].contiguous(),
+                                g["k"].transpose(0, 1)[None].contiguous(),
+                                g["v"].transpose(0, 1)[None].contiguous(),
+                                gk_bf[0].transpose(0, 1)[None].contiguous(), pool, g["wq"],
+                                g["qnorm_w"], g["wk"], g["knorm_w"], want_selection=True)
+    torch.cuda.synchronize()
+    assert torch.equal(di[0], idx[L - 1])
+    assert (dl[0] - logg[L - 1]).abs().max().item() <= GATE_ABS
+    assert (od[0].float() - o[L - 1].float()).abs().max().item() <= 2e-2
