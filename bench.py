@@ -49,7 +49,7 @@ def parse():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-rows", type=int, default=6, help="oracle rows per CPU-baseline sample")
+    ap.add_argument("--cpu-rows", type=int, default=64, help="oracle rows per CPU-baseline sample")
     return ap.parse_args()
 
 
@@ -528,7 +528,7 @@ def reference_arm(a, ws, rank):
     t = []
     fl = 0.0
     for i in range(a.steps):
-        rows = sample_rows(shape, 2, 1000 + i)
+        rows = sample_rows(shape, 8, 1000 + i)
         t0 = time.perf_counter()
         fl += oracle_sample(cpu, shape, rows, backward)
         t.append(time.perf_counter() - t0)
@@ -542,7 +542,7 @@ def reference_arm(a, ws, rank):
             "config": {"workload": a.workload, "batch": shape.batch, "seq_len": shape.max_seqlen,
                        "passes": "fwd+bwd" if backward else "fwd", "parallelism": "cpu oracle"},
             "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-                             "sample": f"2 random query rows per step of {a.workload} (gate, "
+                             "sample": f"8 random query rows per step of {a.workload} (gate, "
                                        "Top-K, attention fwd + dQ/dlogg rows), fp64 numpy"},
             "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
