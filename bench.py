@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--impl", default="sas", choices=["sas", "reference"])
     ap.add_argument("--workload", default=TRAIN_WORKLOAD)
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-train", action="store_true", help="decode step only (profiling)")
+    ap.add_argument("--decode-workload", default=DECODE_WORKLOAD)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=64, help="oracle rows per CPU-baseline sample")
@@ -306,8 +308,8 @@ def sample_rows(shape, n, seed):
 # decode
 # ------------------------------------------------------------------------------------------
 
-def bench_decode(sas, dev, steps, warmup, flush, hbm_peak):
-    shp = si.decode_workload(DECODE_WORKLOAD)
+def bench_decode(sas, dev, steps, warmup, flush, hbm_peak, name=DECODE_WORKLOAD):
+    shp = si.decode_workload(name)
     inp = si.decode_inputs(shp, device=dev)
     prob = sas.DecodeProblem(seqlens=inp["lengths"], capacity=shp.capacity,
                              num_q_heads=shp.num_q_heads, num_kv_heads=shp.num_kv_heads,
@@ -357,7 +359,7 @@ def bench_decode(sas, dev, steps, warmup, flush, hbm_peak):
     gbs = total / (ms * 1e-3) / 1e9
     return {
         "metric": "decode tok/s", "value": shp.batch / (ms * 1e-3), "unit": "tok/s",
-        "ms_per_step": ms, "config": {"workload": DECODE_WORKLOAD, "batch": shp.batch,
+        "ms_per_step": ms, "config": {"workload": name, "batch": shp.batch,
                                       "context_min": int(L.min()), "context_max": int(L.max()),
                                       "budget_tokens": (shp.topk + 1) * B},
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
@@ -381,6 +383,11 @@ def main():
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     hbm_peak, tc_peak, tc_sust, peak_src = measured_peaks()
+    if a.no_train:
+        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        print(json.dumps(bench_decode(sas, dev, max(1, a.steps), max(3, a.warmup), flush, hbm_peak,
+                                      a.decode_workload)), flush=True)
+        return
 
     shape = si.workload(a.workload)
     backward = "train" in a.workload or "varlen" in a.workload
@@ -456,7 +463,8 @@ def main():
 
     if not a.no_decode:
         try:
-            line["decode"] = bench_decode(sas, dev, max(3, a.steps), max(3, a.warmup), flush, hbm_peak)
+            line["decode"] = bench_decode(sas, dev, max(3, a.steps), max(3, a.warmup), flush, hbm_peak,
+                                          a.decode_workload)
         except torch.OutOfMemoryError as ex:   # pragma: no cover
             line["decode"] = {"error": f"out of memory: {ex}"[:200]}
 

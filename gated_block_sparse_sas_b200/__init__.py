@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libsas_b200.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with "
-                      "`python -m gated_block_sparse_sas_b200.build` (nvcc, sm_100a)")
+                      "`python gated_block_sparse_sas_b200/build.py` (nvcc, sm_100a)")
 _lib = ctypes.CDLL(LIB_PATH)
 
 SAS_OK, SAS_ERR_INVALID_ARG, SAS_ERR_UNSUPPORTED, SAS_ERR_CUDA, SAS_ERR_WORKSPACE = 0, -1, -2, -3, -4
@@ -58,6 +58,7 @@ _SIGS = {
     "sas_attn_bwd": ([_P] + [_vp] * 13 + [_sz, _vp], ctypes.c_int),
     "sas_decode_workspace_size": ([_DP, ctypes.POINTER(_sz)], ctypes.c_int),
     "sas_decode": ([_DP] + [_vp] * 14 + [_sz, _vp], ctypes.c_int),
+    "sas_decode_noalloc": ([_DP] + [_vp] * 13 + [_vp], ctypes.c_int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(_lib, _name)

@@ -1,6 +1,7 @@
 """Build libsas_b200.so (all CUDA sources, sm_100a) in place with nvcc.
 
-    python -m gated_block_sparse_sas_b200.build
+    python gated_block_sparse_sas_b200/build.py      (run by path: the package itself
+                                                      imports the built library)
 """
 from __future__ import annotations
 

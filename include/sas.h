@@ -197,6 +197,24 @@ sas_status sas_decode(const sas_decode_problem* p, const void* q, const void* q_
                       float* logg_out, void* workspace, size_t workspace_bytes,
                       cudaStream_t stream);
 
+/* Allocation-free variant of sas_decode (no counterpart in the SAS pages; a library
+ * convenience). For callers that cannot allocate device memory around a decode step --
+ * a runtime whose pool has already reserved the device, a plugin inside another
+ * framework's step, a latency-critical loop that must not touch an allocator. Same
+ * arguments and results as sas_decode minus the workspace: the scratch is a fixed 8 MiB
+ * array inside the library, held on every GPU that loads the library until the process
+ * exits. Problems needing more scratch than that (sas_decode_workspace_size) return
+ * SAS_ERR_UNSUPPORTED. The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress); make that first call before any stream capture. Calls whose
+ * kernels overlap on the GPU share the one array and race: serialise them. Nothing in the
+ * scratch needs to start at zero. Allocates nothing (no cudaMalloc/cudaFree). */
+sas_status sas_decode_noalloc(const sas_decode_problem* p, const void* q, const void* q_nope,
+                              const void* k_cache, const void* v_cache,
+                              const void* gate_key_cache, const float* cur_pool,
+                              const void* wq, const float* qnorm_w, const void* wk,
+                              const float* knorm_w, void* o, int32_t* idx_out,
+                              float* logg_out, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

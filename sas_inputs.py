@@ -233,6 +233,8 @@ def workload(name: str) -> Shape:
     if name in ("qwen3-4b-prefill-32k", "qwen3-4b-train-32k"):
         return Shape([32768], 32, 8, 128, 64, 31, 128, "bf16",
                      seed=1 if name.endswith("prefill-32k") else 2)
+    if name == "qwen3-4b-train-16k":      # same layer, half length: profiling captures
+        return Shape([16384], 32, 8, 128, 64, 31, 128, "bf16", seed=5)
     if name == "qwen3-14b-varlen-4seq":
         return Shape(draw_lengths(4, 4, 8192, 65536), 40, 8, 128, 64, 63, 128, "bf16", seed=4)
     raise KeyError(name)
@@ -345,6 +347,9 @@ def decode_workload(name: str) -> DecodeShape:
     if name == "qwen3-8b-decode-b64":
         lengths = draw_lengths(3, 64, 16384, 131072)
         return DecodeShape(lengths, 131072, 32, 8, 128, 64, 31, 128, seed=3)
+    if name == "qwen3-8b-decode-b16-32k":  # a few GB of cache: profiling captures
+        lengths = draw_lengths(6, 16, 8192, 32768)
+        return DecodeShape(lengths, 32768, 32, 8, 128, 64, 31, 128, seed=6)
     raise KeyError(name)
 
 

@@ -25,8 +25,8 @@ def _declared():
 @pytest.fixture(scope="module")
 def sas():
     if not os.path.exists(LIB):
-        from gated_block_sparse_sas_b200 import build
-        build.build()
+        import __graft_entry__
+        __graft_entry__.build()
     import gated_block_sparse_sas_b200 as m
     return m
 
