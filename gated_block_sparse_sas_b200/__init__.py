@@ -206,7 +206,7 @@ def _workspace(fn, prob_ref, device):
     """A fresh workspace of the size the library asks for (torch's stream-ordered allocator)."""
     n = _sz(0)
     _check(fn(prob_ref, ctypes.byref(n)), fn.__name__)
-    return torch.empty(max(int(n.value), 256), dtype=torch.uint8, device=device)
+    return torch.zeros(max(int(n.value), 256), dtype=torch.uint8, device=device)
 
 
 def sas_attn_fwd(p: Problem, q, k, v, idx, logg, o=None, lse=None, workspace=None, stream=None):

@@ -172,7 +172,7 @@ sas_status sas_topk(const sas_problem* p, const float* scores, const float* lse,
 sas_status sas_attn_fwd_workspace_size(const sas_problem* p, size_t* bytes) {
   SAS_TRY(check_problem(p, false));
   SAS_CHECK_ARG(bytes != nullptr, "bytes is NULL");
-  *bytes = 0;
+  *bytes = 256;   // word 0: pipeline error code of the tensor-core kernel (0 = none)
   return SAS_OK;
 }
 
@@ -187,9 +187,14 @@ sas_status sas_attn_fwd(const sas_problem* p, const void* q, const void* k, cons
   SAS_PTR(logg);
   SAS_PTR(o);
   SAS_PTR(lse_attn);
-  (void)workspace;
-  (void)workspace_bytes;
+  SAS_PTR(workspace);
+  if (workspace_bytes < 256) {
+    set_error("workspace too small: %zu < 256 bytes", workspace_bytes);
+    return SAS_ERR_WORKSPACE;
+  }
   if (p->total_tokens == 0) return SAS_OK;
+  if (attn_tc_supported(*p))
+    return launch_attn_fwd_tc(*p, q, k, v, idx, logg, o, lse_attn, (int*)workspace, stream);
   return launch_attn_fwd_simt(*p, q, k, v, idx, logg, o, lse_attn, stream);
 }
 

@@ -26,6 +26,11 @@ sas_status launch_attn_bwd_simt(const sas_problem& p, const void* q, const void*
                                 const int32_t* idx, const float* logg, void* dq, void* dk, void* dv,
                                 float* dlogg, float* drow, cudaStream_t st);
 
+bool attn_tc_supported(const sas_problem& p);
+sas_status launch_attn_fwd_tc(const sas_problem& p, const void* q, const void* k, const void* v,
+                              const int32_t* idx, const float* logg, void* o, float* lse, int* err,
+                              cudaStream_t st);
+
 int decode_nsplit(const sas_decode_problem& p);
 size_t decode_workspace_bytes(const sas_decode_problem& p);
 sas_status launch_decode(const sas_decode_problem& p, const void* q, const void* q_nope,

@@ -113,5 +113,5 @@ def test_empty_problem_is_a_no_op(sas):
     lib = sas.lib_handle()
     p = _prob(sas, total_tokens=0)
     ptrs = [0x10000 + 0x100 * i for i in range(8)]
-    assert lib.sas_attn_fwd(ctypes.byref(p), *ptrs[:7], None, 0, None) == 0
+    assert lib.sas_attn_fwd(ctypes.byref(p), *ptrs[:7], 0x90000, 256, None) == 0
     assert lib.sas_topk(ctypes.byref(p), *ptrs[:4], None) == 0
