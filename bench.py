@@ -51,7 +51,7 @@ def parse():
     ap.add_argument("--decode-workload", default=DECODE_WORKLOAD)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-rows", type=int, default=64, help="oracle rows per CPU-baseline sample")
+    ap.add_argument("--cpu-rows", type=int, default=256, help="oracle rows per CPU-baseline sample")
     return ap.parse_args()
 
 

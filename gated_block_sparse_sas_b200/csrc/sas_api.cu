@@ -201,7 +201,10 @@ sas_status sas_attn_fwd(const sas_problem* p, const void* q, const void* k, cons
 sas_status sas_attn_bwd_workspace_size(const sas_problem* p, size_t* bytes) {
   SAS_TRY(check_problem(p, false));
   SAS_CHECK_ARG(bytes != nullptr, "bytes is NULL");
-  *bytes = (((size_t)p->total_tokens * p->num_q_heads * sizeof(float)) + 255) & ~(size_t)255;
+  // [256 B error word][D = rowsum(dO*O), fp32 T*Hq][per-tile union bitmasks (tensor-core path)]
+  size_t n = 256 + ((((size_t)p->total_tokens * p->num_q_heads * sizeof(float)) + 255) & ~(size_t)255);
+  if (attn_bwd_tc_supported(*p)) n += (attn_bwd_tc_tmask_bytes(*p) + 255) & ~(size_t)255;
+  *bytes = n;
   return SAS_OK;
 }
 
@@ -233,8 +236,18 @@ sas_status sas_attn_bwd(const sas_problem* p, const void* q, const void* k, cons
     }
   }
   if (p->total_tokens == 0) return SAS_OK;
-  return launch_attn_bwd_simt(*p, q, k, v, o, dout, lse_attn, idx, logg, dq, dk, dv, dlogg,
-                              (float*)workspace, stream);
+  char* ws = (char*)workspace;
+  int* err = (int*)ws;
+  float* drow = (float*)(ws + 256);
+  if (attn_bwd_tc_supported(*p)) {
+    uint32_t* tmask = (uint32_t*)(ws + 256 + ((((size_t)p->total_tokens * p->num_q_heads *
+                                                 sizeof(float)) + 255) & ~(size_t)255));
+    SAS_TRY(launch_rowdot(*p, o, dout, drow, stream));
+    return launch_attn_bwd_tc(*p, q, k, v, dout, lse_attn, drow, idx, logg, dq, dk, dv, dlogg,
+                              tmask, err, stream);
+  }
+  return launch_attn_bwd_simt(*p, q, k, v, o, dout, lse_attn, idx, logg, dq, dk, dv, dlogg, drow,
+                              stream);
 }
 
 static sas_status check_decode(const sas_decode_problem* p) {

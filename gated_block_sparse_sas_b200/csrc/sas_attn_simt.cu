@@ -357,6 +357,20 @@ static void bwd_simt_launch(const sas_problem& p, const void* q, const void* k, 
     default: MACRO(T, D, 8); break;      \
   }
 
+sas_status launch_rowdot(const sas_problem& p, const void* o, const void* dout, float* drow,
+                         cudaStream_t st) {
+  const int rows_q = p.total_tokens * p.num_q_heads;
+  const int grid = (int)(((size_t)rows_q * 32 + 255) / 256);
+#define SAS_RD(T, D) attn_bwd_rowdot_kernel<T, D><<<grid, 256, 0, st>>>((const T*)o, (const T*)dout, rows_q, drow)
+  if (p.dtype == SAS_BF16) {
+    if (p.head_dim == 64) SAS_RD(__nv_bfloat16, 64); else SAS_RD(__nv_bfloat16, 128);
+  } else {
+    if (p.head_dim == 64) SAS_RD(float, 64); else SAS_RD(float, 128);
+  }
+#undef SAS_RD
+  return launch_status("attn_bwd row dot", 1);
+}
+
 sas_status launch_attn_fwd_simt(const sas_problem& p, const void* q, const void* k, const void* v,
                                 const int32_t* idx, const float* logg, void* o, float* lse,
                                 cudaStream_t st) {

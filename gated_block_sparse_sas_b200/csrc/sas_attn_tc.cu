@@ -71,26 +71,6 @@ struct TcFwdArgs {
   float scale_log2;
 };
 
-__device__ __forceinline__ void tc_fail(int* err, int code, volatile int* abort_flag) {
-  *abort_flag = 1;
-  atomicCAS(err, 0, code);
-}
-
-// Bounded wait that ignores the abort flag (used to drain in-flight copies / MMAs).
-__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity))
-    if (clock64() - t0 > kWaitCycles) return false;
-  return true;
-}
-
-// Warp-uniform bounded wait: every lane waits, the warp proceeds only if all succeeded.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-  const bool ok = mbar_wait(bar, parity, abort_flag);
-  return __all_sync(0xffffffffu, ok);
-}
-
 __global__ void __launch_bounds__(tcf::kThreads, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const TcFwdArgs a) {

@@ -5,6 +5,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <stdint.h>
 
 namespace sas {
@@ -52,6 +53,32 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (*abort) return false;
     if (clock64() - t0 > kWaitCycles) return false;
   }
+}
+
+// Bounded wait that ignores the abort flag (used to drain in-flight copies / MMAs).
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity))
+    if (clock64() - t0 > kWaitCycles) return false;
+  return true;
+}
+
+// Warp-uniform bounded wait: every lane waits, the warp proceeds only if all succeeded.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  const bool ok = mbar_wait(bar, parity, abort_flag);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Record a pipeline failure (first code wins) and tell the CTA's other roles to stop.
+__device__ __forceinline__ void tc_fail(int* err, int code, volatile int* abort_flag) {
+  *abort_flag = 1;
+  atomicCAS(err, 0, code);
+}
+
+// Named barrier over `nthreads` threads (ids 1..15; 0 is __syncthreads).
+__device__ __forceinline__ void named_bar(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // ---- TMA -----------------------------------------------------------------------------------
