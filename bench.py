@@ -195,6 +195,33 @@ def attended_pairs_gpu(idx: torch.Tensor, cu: torch.Tensor, block: int) -> int:
     return int(n.sum().item())
 
 
+def union_stats(idx: torch.Tensor, cu: torch.Tensor, lengths, Mq: int, Hkv: int, NBmax: int):
+    """Work the tile-union tensor-core kernels actually do on this selection.
+
+    U = sum over (tile of Mq tokens, kv head) of the number of distinct blocks its rows kept
+    (forward and query-major backward visit each once, 128 rows x 64 keys);
+    P = sum over (tile, kv) of the distinct block pairs (key-major backward, 128 x 128).
+    """
+    T = idx.shape[0]
+    dev = idx.device
+    cu64 = cu.long()
+    tok = torch.arange(T, device=dev)
+    seq = torch.searchsorted(cu64[1:], tok, right=True)
+    pos = tok - cu64[seq]
+    n_tiles = (max(lengths) + Mq - 1) // Mq
+    tile = seq * n_tiles + pos // Mq
+    j = idx.long()
+    kvi = torch.arange(Hkv, device=dev)[None, :, None].expand_as(j)
+    nbp = NBmax + (NBmax & 1)
+    lin = (tile[:, None, None] * Hkv + kvi) * nbp + j.clamp(min=0)
+    mark = torch.zeros(len(lengths) * n_tiles * Hkv * nbp, dtype=torch.bool, device=dev)
+    mark[lin[j >= 0]] = True
+    m = mark.view(-1, nbp)
+    U = int(m.sum().item())
+    P = int(m.view(-1, nbp // 2, 2).any(-1).sum().item())
+    return U, P
+
+
 class Timer:
     """CUDA events around each op of a step, on the stream the library launches on."""
 
@@ -406,6 +433,12 @@ def main():
     G, d = shape.group, shape.head_dim
     fwd_flops = 4.0 * pairs * G * d
     bwd_flops = 2.5 * fwd_flops if backward else 0.0
+    Mq = 25 if G == 5 else 128 // G
+    U, P = union_stats(out[2], prob.cu_seqlens, shape.lengths, Mq, shape.num_kv_heads,
+                       prob.max_blocks)
+    mma = 2.0 * 128 * 64 * d                           # one 128 x 64 x d product
+    comp_fwd = U * 2 * mma                             # QK^T + PV per visited block
+    comp_bwd = U * 3 * mma + P * 4 * (2.0 * 128 * 128 * d) if backward else 0.0
 
     timer = Timer()
     steps = []
@@ -453,6 +486,13 @@ def main():
                      "bwd_tflop": bwd_flops / 1e12,
                      "dense_causal_fraction": pairs / (shape.num_kv_heads * sum(
                          L * (L + 1) / 2 for L in shape.lengths))},
+        "computed": {"fwd_tflop": comp_fwd / 1e12, "bwd_tflop": comp_bwd / 1e12,
+                     "union_blocks_per_tile": U / max(1, shape.num_kv_heads * sum(
+                         (L + Mq - 1) // Mq for L in shape.lengths)),
+                     "attended_over_computed": (fwd_flops + bwd_flops) / max(1.0, comp_fwd + comp_bwd),
+                     "fwd_tflops": comp_fwd / (ops["sas_attn_fwd"] * 1e-3) / 1e12,
+                     "bwd_tflops": (comp_bwd / (ops["sas_attn_bwd"] * 1e-3) / 1e12) if backward else None,
+                     "note": "tensor-core work of the tile-union kernels (rows x visited blocks)"},
         "ops_ms": ops,
         "roofline": roof,
         "gpu_launches": launches,
