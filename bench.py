@@ -196,11 +196,12 @@ def attended_pairs_gpu(idx: torch.Tensor, cu: torch.Tensor, block: int) -> int:
 
 
 def union_stats(idx: torch.Tensor, cu: torch.Tensor, lengths, Mq: int, Hkv: int, NBmax: int):
-    """Work the tile-union tensor-core kernels actually do on this selection.
+    """Work the tensor-core kernels actually do on this selection.
 
     U = sum over (tile of Mq tokens, kv head) of the number of distinct blocks its rows kept
     (forward and query-major backward visit each once, 128 rows x 64 keys);
-    P = sum over (tile, kv) of the distinct block pairs (key-major backward, 128 x 128).
+    P = gathered 128-row tiles of the key-major backward: per (sequence, kv, block pair), the
+    tokens that kept a block of the pair, in tiles of Mq tokens (128 keys x 128 rows each).
     """
     T = idx.shape[0]
     dev = idx.device
@@ -218,7 +219,13 @@ def union_stats(idx: torch.Tensor, cu: torch.Tensor, lengths, Mq: int, Hkv: int,
     mark[lin[j >= 0]] = True
     m = mark.view(-1, nbp)
     U = int(m.sum().item())
-    P = int(m.view(-1, nbp // 2, 2).any(-1).sum().item())
+    NP = nbp // 2
+    key = ((tok[:, None, None] * Hkv + kvi) * NP + (j.clamp(min=0) >> 1))[j >= 0]
+    key = torch.unique(key)
+    trow = key // (Hkv * NP)
+    grp = (seq[trow] * Hkv + (key // NP) % Hkv) * NP + key % NP
+    n_tok = torch.bincount(grp, minlength=len(lengths) * Hkv * NP)
+    P = int(((n_tok + Mq - 1) // Mq).sum().item())
     return U, P
 
 

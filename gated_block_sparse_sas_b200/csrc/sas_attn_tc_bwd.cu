@@ -1,20 +1,20 @@
-// Tensor-core (tcgen05 / TMEM / TMA) backward of the gated sparse attention (A6), bf16,
-// head_dim 128, KV block 64. The loss reaches the selector through standard
-// backpropagation (paper abstract): besides dQ, dK, dV the backward returns the gradient
-// of every kept block's log-gate, dlogg = sum over the G heads and the block's keys of
-// dS = P (dP - D).
+// Tensor-core (tcgen05 / TMEM) backward of the gated sparse attention (A6), bf16, head_dim
+// 128, KV block 64. The loss reaches the selector through standard backpropagation (paper
+// abstract): besides dQ, dK, dV the backward returns the gradient of every kept block's
+// log-gate, dlogg = sum over the G heads and the block's keys of dS = P (dP - D).
 //
-// Two passes over the same tile-union decomposition as the forward, so that no output is
-// accumulated with atomics and every sum has a fixed order:
-//   query-major  CTA = (tile of Mq tokens x G heads = 128 rows, kv head). Per union block:
-//                S = Q K^T, dP = dO V^T (TMEM, double-buffered), dS = P (dP - D) in
-//                registers -> bf16 shared tile, dQ += dS K (TMEM). Row sums of dS, reduced
-//                over the G heads of a token, are that token's dlogg for the block.
-//   key-major    CTA = (pair of KV blocks = 128 keys, kv head). For every tile whose union
-//                holds either block (per-tile union bitmasks from a pre-pass): S^T = K Q^T,
-//                dP^T = V dO^T (keys on TMEM lanes, rows on columns, so the per-row softmax
-//                statistics are per-column constants), P^T and dS^T -> bf16 shared tiles,
-//                dV += P^T dO, dK += dS^T Q (TMEM).
+// Two passes, no atomics on any output, every sum in a fixed order:
+//   query-major  CTA = (tile of Mq tokens x G heads = 128 rows, kv head), visiting the union
+//                of the tile rows' blocks (as the forward). Per block: S = Q K^T and
+//                dP = dO V^T (TMEM, double-buffered), dS = P (dP - D) -> bf16 shared tile,
+//                dQ += dS K (TMEM). Row sums of dS over the G heads of a token give dlogg.
+//   key-major    CTA = (pair of KV blocks = 128 keys, kv head), visiting only the tokens
+//                that kept one of the two blocks: a pre-pass writes, per (kv, block pair),
+//                a bitmask over tokens; the CTA walks its row in token order and gathers
+//                128-row tiles (Mq tokens x G heads) of Q and dO with cp.async. Per tile:
+//                S^T = K Q^T, dP^T = V dO^T (keys on TMEM lanes, rows on columns, so the
+//                per-row statistics are per-column constants), P^T and dS^T -> bf16 shared
+//                tiles, dV += P^T dO, dK += dS^T Q (TMEM).
 // D = rowsum(dO * O) comes from the CUDA-core row-dot kernel.
 #include <cuda.h>
 
@@ -50,21 +50,23 @@ constexpr int Q_OFF_BAR = Q_OFF_RS + 2 * 128 * 4;
 constexpr int Q_NBARS = 1 + 2 * kStages + 2 + 2 + 2 + 1;
 constexpr int Q_OFF_MISC = Q_OFF_BAR + Q_NBARS * 8;
 constexpr int Q_SMEM = Q_OFF_MISC + 64 + 1024;
-// key-major pass layout
-constexpr int kMaxTiles = 4096;
-constexpr int K_OFF_K = 0;                       // [128 keys][128 d] as 2 halves
-constexpr int K_OFF_V = K_OFF_K + 2 * kHalf;
-constexpr int K_OFF_Q = K_OFF_V + 2 * kHalf;     // [128 rows][128 d]
-constexpr int K_OFF_DO = K_OFF_Q + 2 * kHalf;
-constexpr int K_OFF_PT = K_OFF_DO + 2 * kHalf;   // P^T  [128 keys][128 rows] as 2 halves
-constexpr int K_OFF_DST = K_OFF_PT + 2 * kHalf;  // dS^T [128 keys][128 rows]
-constexpr int K_OFF_TL = K_OFF_DST + 2 * kHalf;
-constexpr int K_OFF_RC = K_OFF_TL + kMaxTiles * 4;     // 2 x 5 x 128 floats
-constexpr int K_OFF_CNT = K_OFF_RC + 2 * 5 * 128 * 4;
-constexpr int K_OFF_BAR = K_OFF_CNT + 16 * 4;
-constexpr int K_NBARS = 6;
-constexpr int K_OFF_MISC = K_OFF_BAR + K_NBARS * 8;
-constexpr int K_SMEM = K_OFF_MISC + 64 + 1024;
+// gathered key-major pass layout
+constexpr int kGThreads = 384;           // warps 0-3 gather, 4 MMA, 8-11 softmax
+constexpr int kMaxWords = 2048;          // token bitmask words per row (max_seqlen <= 65536)
+constexpr int G_OFF_K = 0;               // [128 keys][128 d] as 2 halves
+constexpr int G_OFF_V = G_OFF_K + 2 * kHalf;
+constexpr int G_OFF_Q = G_OFF_V + 2 * kHalf;     // gathered [128 rows][128 d]
+constexpr int G_OFF_DO = G_OFF_Q + 2 * kHalf;
+constexpr int G_OFF_PT = G_OFF_DO + 2 * kHalf;   // P^T  [128 keys][128 rows] as 2 halves
+constexpr int G_OFF_DST = G_OFF_PT + 2 * kHalf;  // dS^T [128 keys][128 rows]
+constexpr int G_OFF_RC = G_OFF_DST + 2 * kHalf;  // [2][4][128] row constants
+constexpr int G_OFF_WORDS = G_OFF_RC + 2 * 4 * 128 * 4;
+constexpr int G_OFF_PREFIX = G_OFF_WORDS + kMaxWords * 4;
+constexpr int G_OFF_PART = G_OFF_PREFIX + kMaxWords * 4;   // kGThreads partial counts
+constexpr int G_OFF_BAR = G_OFF_PART + kGThreads * 4;
+constexpr int G_NBARS = 6;
+constexpr int G_OFF_MISC = G_OFF_BAR + G_NBARS * 8;
+constexpr int G_SMEM = G_OFF_MISC + 64 + 1024;
 }  // namespace tcb
 
 struct TcBwdArgs {
@@ -73,13 +75,15 @@ struct TcBwdArgs {
   const float* logg;
   const float* lse;
   const float* drow;
-  const uint32_t* tmask;
+  const uint32_t* pmask;      // [batch][Hkv][NP][W] token bitmask per block pair
+  const __nv_bfloat16* q;     // raw pointers for the gathered copies
+  const __nv_bfloat16* dout;
   __nv_bfloat16* dq;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
   float* dlogg;
   int* err;
-  int Hq, Hkv, G, K, Mq, NBmax, n_tiles;
+  int Hq, Hkv, G, K, Mq, NBmax, n_tiles, NP, W;
   float scale_log2, scale;
 };
 
@@ -88,29 +92,35 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
                                     ~static_cast<uintptr_t>(1023));
 }
 
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 // ---------------------------------------------------------------------------------------
-// pre-pass: union bitmask of every (tile, kv head) -> tmask[b][tile][kv][word]
+// pre-pass: bit t of pmask[b][kv][p] = token t of sequence b kept block 2p or 2p+1
 // ---------------------------------------------------------------------------------------
-__global__ void tile_union_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ cu,
-                                  int Hkv, int K, int Mq, int NBmax, int n_tiles,
-                                  uint32_t* __restrict__ tmask) {
-  __shared__ uint32_t words[tcb::kMaxBlocks / 32];
-  const int tile = blockIdx.x, b = blockIdx.y, kv = blockIdx.z;
-  const int nwords = (NBmax + 31) >> 5;
-  for (int w = threadIdx.x; w < nwords; w += blockDim.x) words[w] = 0u;
-  __syncthreads();
-  const int s0 = cu[b], L = cu[b + 1] - s0, t0 = tile * Mq, K1 = K + 1;
-  if (t0 < L) {
-    const int nt = min(Mq, L - t0);
-    for (int e = threadIdx.x; e < nt * K1; e += blockDim.x) {
-      const int tl = e / K1, sl = e - tl * K1;
-      const int j = idx[((size_t)(s0 + t0 + tl) * Hkv + kv) * K1 + sl];
-      if (j >= 0 && j < NBmax) atomicOr(&words[j >> 5], 1u << (j & 31));
-    }
+__global__ void pair_mask_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ cu,
+                                 int batch, int T, int Hkv, int K, int NP, int W,
+                                 uint32_t* __restrict__ pmask) {
+  const int row = (int)(blockIdx.x * (size_t)blockDim.x + threadIdx.x);
+  if (row >= T * Hkv) return;
+  const int tg = row / Hkv, kv = row - tg * Hkv;
+  const int b = seq_of(cu, batch, tg);
+  const int t = tg - cu[b];
+  uint32_t* base = pmask + ((size_t)(b * Hkv + kv) * NP) * W + (t >> 5);
+  const uint32_t bit = 1u << (t & 31);
+  const int32_t* ir = idx + (size_t)row * (K + 1);
+  int prev = -1;
+  for (int s = 0; s <= K; ++s) {
+    const int j = ir[s];
+    if (j < 0) break;
+    const int p = j >> 1;
+    if (p != prev && p < NP) atomicOr(base + (size_t)p * W, bit);
+    prev = p;
   }
-  __syncthreads();
-  uint32_t* out = tmask + (((size_t)b * n_tiles + tile) * Hkv + kv) * nwords;
-  for (int w = threadIdx.x; w < nwords; w += blockDim.x) out[w] = words[w];
 }
 
 // ---------------------------------------------------------------------------------------
@@ -409,12 +419,11 @@ __global__ void __launch_bounds__(tcb::kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------------------
-// key-major pass: dK and dV of a pair of KV blocks
+// key-major pass over gathered rows: dK and dV of a pair of KV blocks
 // ---------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(tcb::kThreads, 1)
-    attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
-                            const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                            const TcBwdArgs a) {
+__global__ void __launch_bounds__(tcb::kGThreads, 1)
+    attn_bwd_dkdv_gather_kernel(const __grid_constant__ CUtensorMap tmK,
+                                const __grid_constant__ CUtensorMap tmV, const TcBwdArgs a) {
   using namespace tcb;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
@@ -425,115 +434,158 @@ __global__ void __launch_bounds__(tcb::kThreads, 1)
   if (key0 >= L) return;
   const int G = a.G, K1 = a.K + 1, Mq = a.Mq;
   const int rows_used = G * Mq;
-  const int nwords = (a.NBmax + 31) >> 5;
 
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + K_OFF_BAR);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + G_OFF_BAR);
   uint64_t* kv_full = bars;
   uint64_t* qd_full = bars + 1;
   uint64_t* st_full = bars + 2;
   uint64_t* pt_full = bars + 3;
   uint64_t* dkv_done = bars + 4;
   uint64_t* dkv_final = bars + 5;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + K_OFF_MISC);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + K_OFF_MISC + 4);
-  int* n_list_s = reinterpret_cast<int*>(sm + K_OFF_MISC + 8);
-  int32_t* tlist = reinterpret_cast<int32_t*>(sm + K_OFF_TL);
-  float* rc = reinterpret_cast<float*>(sm + K_OFF_RC);   // [2][5][128]
-  int* wcnt = reinterpret_cast<int*>(sm + K_OFF_CNT);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + G_OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + G_OFF_MISC + 4);
+  int* n_tok_s = reinterpret_cast<int*>(sm + G_OFF_MISC + 8);
+  float* rc = reinterpret_cast<float*>(sm + G_OFF_RC);          // [2][4][128]
+  uint32_t* words = reinterpret_cast<uint32_t*>(sm + G_OFF_WORDS);
+  int* prefix = reinterpret_cast<int*>(sm + G_OFF_PREFIX);
+  int* part = reinterpret_cast<int*>(sm + G_OFF_PART);
 
+  // ---- token list of this (kv, pair): tokens >= key0 of the pair's bitmask row ----
+  const int w0 = key0 >> 5, w1 = (L + 31) >> 5;
+  const int nw = min(w1 - w0, kMaxWords);
+  const uint32_t* mrow = a.pmask + ((size_t)(b * a.Hkv + kv) * a.NP + pair) * a.W + w0;
+  const int per = (nw + kGThreads - 1) / kGThreads;
+  int cnt = 0;
+  for (int i = tid * per; i < min(nw, (tid + 1) * per); ++i) {
+    const uint32_t w = mrow[i];
+    words[i] = w;
+    cnt += __popc(w);
+  }
+  part[tid] = cnt;
   if (tid == 0) {
-    for (int i = 0; i < K_NBARS; ++i) mbar_init(bars + i, i == 3 ? 128 : 1);
+    for (int i = 0; i < G_NBARS; ++i) mbar_init(bars + i, (i == 1 || i == 3) ? 128 : 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 1) {
+  if (warp == 4) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
-  if (rows_used < kM) {
-    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-    for (int e = tid; e < (kM - rows_used) * 8; e += kThreads) {
-      const int r = rows_used + (e >> 3), c = e & 7;
-      reinterpret_cast<uint4*>(sm + K_OFF_Q + r * 128)[c] = z;
-      reinterpret_cast<uint4*>(sm + K_OFF_Q + kHalf + r * 128)[c] = z;
-      reinterpret_cast<uint4*>(sm + K_OFF_DO + r * 128)[c] = z;
-      reinterpret_cast<uint4*>(sm + K_OFF_DO + kHalf + r * 128)[c] = z;
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0;
+    for (int i = 0; i < kGThreads; ++i) {
+      const int c = part[i];
+      part[i] = run;
+      run += c;
     }
-    fence_async_smem();
+    *n_tok_s = run;
   }
-  // ordered list of the tiles whose union holds block j0 or j0+1 (tiles ending before key0 skipped)
-  const int n_seq_tiles = (L + Mq - 1) / Mq;
-  const int first_tile = key0 / Mq;
-  const uint32_t want = 3u << (j0 & 31);
-  int n_list = 0;
-  for (int c0 = first_tile; c0 < n_seq_tiles; c0 += kThreads) {
-    const int tt = c0 + tid;
-    bool hit = false;
-    if (tt < n_seq_tiles)
-      hit = (a.tmask[(((size_t)b * a.n_tiles + tt) * a.Hkv + kv) * nwords + (j0 >> 5)] & want) != 0u;
-    const unsigned m = __ballot_sync(0xffffffffu, hit);
-    if (lane == 0) wcnt[warp] = __popc(m);
-    __syncthreads();
-    int before = 0, total = 0;
-    for (int w = 0; w < kThreads / 32; ++w) {
-      if (w < warp) before += wcnt[w];
-      total += wcnt[w];
+  __syncthreads();
+  {
+    int run = part[tid];
+    for (int i = tid * per; i < min(nw, (tid + 1) * per); ++i) {
+      prefix[i] = run;
+      run += __popc(words[i]);
     }
-    if (hit) {
-      const int pos = n_list + before + __popc(m & ((1u << lane) - 1u));
-      if (pos < kMaxTiles) tlist[pos] = tt;
-    }
-    n_list += total;
-    __syncthreads();
   }
-  if (tid == 0) *n_list_s = min(n_list, kMaxTiles);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const int ntl = *n_list_s;
+  const int n_tok = *n_tok_s;
+  const int n_tiles = (n_tok + Mq - 1) / Mq;
   const uint32_t tmem = *tmem_slot;
   constexpr int kColDV = 0, kColDK = 128, kColST = 256, kColDPT = 384;
 
-  if (warp == 0) {
-    if (lane == 0 && ntl > 0) {   // producer
-      prefetch_tmap(&tmQ);
-      prefetch_tmap(&tmDO);
+  if (warp < 4) {   // gather: thread r builds row r of every tile
+    const int r = tid;
+    const int tl = r / G, g = r - tl * G;
+    const uint32_t q_dst = smem_u32(sm + G_OFF_Q) + r * 128;
+    const uint32_t do_dst = smem_u32(sm + G_OFF_DO) + r * 128;
+    bool ok = true;
+    for (int i = 0; i < n_tiles && ok; ++i) {
+      const int rank = i * Mq + tl;
+      const bool valid = r < rows_used && rank < n_tok;
+      int t = -1;
+      if (valid) {   // the rank-th set bit of the row
+        int lo = 0, hi = nw - 1;
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (prefix[mid] <= rank) lo = mid; else hi = mid - 1;
+        }
+        uint32_t bits = words[lo];
+        for (int k = rank - prefix[lo]; k > 0; --k) bits &= bits - 1u;
+        t = (w0 + lo) * 32 + (__ffs(bits) - 1);
+      }
+      // row constants: c1 = log-gate - lse (log2 units) per block of the pair, D, position
+      float c10 = -INFINITY, c11 = -INFINITY, dd = 0.f;
+      int pos = -1;
+      size_t qrow = 0;
+      if (valid) {
+        pos = t;
+        qrow = (size_t)(s0 + t) * a.Hq + kv * G + g;
+        const float l2 = a.lse[qrow] * kLog2e;
+        dd = a.drow[qrow];
+        const size_t irow = ((size_t)(s0 + t) * a.Hkv + kv) * K1;
+        for (int s = 0; s < K1; ++s) {
+          const int jj = a.idx[irow + s];
+          if (jj < 0 || jj > j0 + 1) break;
+          if (jj == j0) c10 = a.logg[irow + s] * kLog2e - l2;
+          if (jj == j0 + 1) c11 = a.logg[irow + s] * kLog2e - l2;
+        }
+      }
+      if (i >= 1 && !mbar_wait(dkv_done, (i - 1) & 1, abort_flag)) {   // tiles free again
+        tc_fail(a.err, 31, abort_flag);
+        ok = false;
+        break;
+      }
+      if (r < kM) {
+        if (valid) {
+          const __nv_bfloat16* qs = a.q + qrow * kD;
+          const __nv_bfloat16* ds = a.dout + qrow * kD;
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const uint32_t off = (uint32_t)((c >> 3) * kHalf + (((c & 7) ^ (r & 7)) << 4));
+            cp_async16(q_dst + off, qs + c * 8);
+            cp_async16(do_dst + off, ds + c * 8);
+          }
+        } else {   // rows past the list: finite zeros (0 * garbage could be NaN in the MMAs)
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const uint32_t off = (uint32_t)((c >> 3) * kHalf + (c & 7) * 16);
+            st_shared_v4(q_dst + off, 0u, 0u, 0u, 0u);
+            st_shared_v4(do_dst + off, 0u, 0u, 0u, 0u);
+          }
+        }
+      }
+      float* rcb = rc + (i & 1) * 4 * 128;
+      rcb[r] = c10;
+      rcb[128 + r] = c11;
+      rcb[256 + r] = dd;
+      rcb[384 + r] = __int_as_float(pos);
+      cp_async_wait_all();
+      fence_async_smem();
+      mbar_arrive(qd_full);
+    }
+  } else if (warp == 4) {
+    if (lane == 0 && n_tiles > 0) {   // K/V pair loads + MMA issue
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
       mbar_arrive_expect_tx(kv_full, 8u * kKVHalf);
       for (int h = 0; h < 2; ++h)
         for (int jj = 0; jj < 2; ++jj) {
-          tma_load_3d(sm + K_OFF_K + h * kHalf + jj * kKVHalf, &tmK, kv_full, 64 * h, kv,
+          tma_load_3d(sm + G_OFF_K + h * kHalf + jj * kKVHalf, &tmK, kv_full, 64 * h, kv,
                       s0 + key0 + jj * kB);
-          tma_load_3d(sm + K_OFF_V + h * kHalf + jj * kKVHalf, &tmV, kv_full, 64 * h, kv,
+          tma_load_3d(sm + G_OFF_V + h * kHalf + jj * kKVHalf, &tmV, kv_full, 64 * h, kv,
                       s0 + key0 + jj * kB);
         }
-      int issued = 0;
-      for (int i = 0; i < ntl; ++i) {
-        if (i >= 1 && !mbar_wait(dkv_done, (i - 1) & 1, abort_flag)) {
-          tc_fail(a.err, 21, abort_flag);
-          break;
-        }
-        const int trow = s0 + tlist[i] * Mq;
-        mbar_arrive_expect_tx(qd_full, 4u * rows_used * 128u);
-        tma_load_3d(sm + K_OFF_Q, &tmQ, qd_full, 0, kv * G, trow);
-        tma_load_3d(sm + K_OFF_Q + kHalf, &tmQ, qd_full, 64, kv * G, trow);
-        tma_load_3d(sm + K_OFF_DO, &tmDO, qd_full, 0, kv * G, trow);
-        tma_load_3d(sm + K_OFF_DO + kHalf, &tmDO, qd_full, 64, kv * G, trow);
-        issued = i + 1;
-      }
-      mbar_wait_drain(kv_full, 0);
-      if (issued > 0) mbar_wait_drain(qd_full, (issued - 1) & 1);
-    }
-  } else if (warp == 1) {
-    if (lane == 0 && ntl > 0) {   // MMA issuer
-      constexpr uint32_t kIdT = idesc_bf16_f32(kM, kM, false, false);   // S^T, dP^T: N = 128 rows
+      constexpr uint32_t kIdT = idesc_bf16_f32(kM, kM, false, false);   // S^T, dP^T
       constexpr uint32_t kIdG = idesc_bf16_f32(kM, kD, false, true);    // dV, dK: B MN-major
-      const uint32_t k_addr = smem_u32(sm + K_OFF_K), v_addr = smem_u32(sm + K_OFF_V);
-      const uint32_t q_addr = smem_u32(sm + K_OFF_Q), do_addr = smem_u32(sm + K_OFF_DO);
-      const uint32_t pt_addr = smem_u32(sm + K_OFF_PT), dst_addr = smem_u32(sm + K_OFF_DST);
+      const uint32_t k_addr = smem_u32(sm + G_OFF_K), v_addr = smem_u32(sm + G_OFF_V);
+      const uint32_t q_addr = smem_u32(sm + G_OFF_Q), do_addr = smem_u32(sm + G_OFF_DO);
+      const uint32_t pt_addr = smem_u32(sm + G_OFF_PT), dst_addr = smem_u32(sm + G_OFF_DST);
       bool ok = mbar_wait(kv_full, 0, abort_flag);
-      for (int i = 0; ok && i < ntl; ++i) {
+      for (int i = 0; ok && i < n_tiles; ++i) {
         if (!mbar_wait(qd_full, i & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
@@ -554,7 +606,6 @@ __global__ void __launch_bounds__(tcb::kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t ao = (kk >> 2) * kHalf + (kk & 3) * 32;
-          // dO / Q as MN-major B: 16 rows (K) per step, 64-column halves kHalf apart
           mma_bf16_ss(tmem + kColDV, sdesc_sw128(pt_addr + ao, 16, 1024),
                       sdesc_sw128(do_addr + kk * 2048, kHalf, 1024), kIdG,
                       (i > 0 || kk > 0) ? 1u : 0u);
@@ -568,53 +619,23 @@ __global__ void __launch_bounds__(tcb::kThreads, 1)
         }
         tc_commit(dkv_done);
       }
-      if (!ok) tc_fail(a.err, 22, abort_flag);
+      if (!ok) tc_fail(a.err, 32, abort_flag);
       tc_commit(dkv_final);
       mbar_wait_drain(dkv_final, 0);
+      mbar_wait_drain(kv_full, 0);
     }
-  } else if (warp >= 4) {   // thread k = TMEM lane k = key k of the pair
-    const int k = tid - 128;
+  } else if (warp >= 8) {   // thread k = TMEM lane k = key k of the pair
+    const int k = tid - 256;
     const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
-    const int kp = key0 + k;                       // in-sequence key position
-    const bool second = k >= kB;
+    const int kp = key0 + k;
+    const int coff = (k >= kB) ? 128 : 0;
     bool ok = true;
-    // After a failed wait a warp stops working but keeps iterating, so that every warp
-    // reaches every named barrier.
-    for (int i = 0; i < ntl; ++i) {
-      // per-row constants of tile i (thread k handles row k): bias for j0 / j0+1, lse, D, pos
-      float* rcb = rc + (i & 1) * 5 * 128;
-      {
-        const int r = k, tl = r / G, g = r - tl * G;
-        const int tt0 = tlist[i] * Mq;
-        const int ntt = min(Mq, L - tt0);
-        float b0 = -INFINITY, b1 = -INFINITY, l2 = 0.f, dd = 0.f;
-        int pos = -1;
-        if (r < G * ntt) {
-          const int t = tt0 + tl;
-          pos = t;
-          const size_t qrow = (size_t)(s0 + t) * a.Hq + kv * G + g;
-          l2 = a.lse[qrow] * kLog2e;
-          dd = a.drow[qrow];
-          const size_t irow = ((size_t)(s0 + t) * a.Hkv + kv) * K1;
-          for (int s = 0; s < K1; ++s) {
-            const int jj = a.idx[irow + s];
-            if (jj < 0 || jj > j0 + 1) break;
-            if (jj == j0) b0 = a.logg[irow + s] * kLog2e;
-            if (jj == j0 + 1) b1 = a.logg[irow + s] * kLog2e;
-          }
-        }
-        rcb[r] = b0;
-        rcb[128 + r] = b1;
-        rcb[256 + r] = l2;
-        rcb[384 + r] = dd;
-        rcb[512 + r] = __int_as_float(pos);
-      }
-      named_bar(1, 128);
-      if (ok && !warp_wait(st_full, i & 1, abort_flag)) ok = false;
-      if (ok) tc_fence_after();
-      if (ok && i >= 1 && !warp_wait(dkv_done, (i - 1) & 1, abort_flag)) ok = false;
-      if (!ok) continue;
-      const float* bsel = rcb + (second ? 128 : 0);
+    for (int i = 0; i < n_tiles; ++i) {
+      if (!warp_wait(qd_full, i & 1, abort_flag)) { ok = false; break; }   // row constants ready
+      if (!warp_wait(st_full, i & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      if (i >= 1 && !warp_wait(dkv_done, (i - 1) & 1, abort_flag)) { ok = false; break; }
+      const float* rcb = rc + (i & 1) * 4 * 128;
 #pragma unroll 1
       for (int cc = 0; cc < 4; ++cc) {
         float sv[32], dv[32];
@@ -627,20 +648,17 @@ __global__ void __launch_bounds__(tcb::kThreads, 1)
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
             const int r = cc * 32 + c + u;
-            const float bias = bsel[r];
-            const bool vis = kp <= __float_as_int(rcb[512 + r]);
-            const float x = vis ? fmaf(sv[c + u], a.scale_log2, bias) : -INFINITY;
-            const float p = exp2f(x - rcb[256 + r]);
+            const bool vis = kp <= __float_as_int(rcb[384 + r]);
+            const float p = vis ? exp2f(fmaf(sv[c + u], a.scale_log2, rcb[coff + r])) : 0.f;
             p2[u] = p;
-            d2[u] = p * (dv[c + u] - rcb[384 + r]);
+            d2[u] = vis ? p * (dv[c + u] - rcb[256 + r]) : 0.f;
           }
           pp[c >> 1] = pack_bf16x2(p2[0], p2[1]);
           pd[c >> 1] = pack_bf16x2(d2[0], d2[1]);
         }
-        // element (key k, row r): half r/64, 16-byte chunk (r%64)/8, 128B swizzle by k
         const int half = cc >> 1;
-        const uint32_t rowp = smem_u32(sm + K_OFF_PT + half * kHalf) + k * 128;
-        const uint32_t rowd = smem_u32(sm + K_OFF_DST + half * kHalf) + k * 128;
+        const uint32_t rowp = smem_u32(sm + G_OFF_PT + half * kHalf) + k * 128;
+        const uint32_t rowd = smem_u32(sm + G_OFF_DST + half * kHalf) + k * 128;
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
           const int chunk = (cc & 1) * 4 + q4;
@@ -653,12 +671,12 @@ __global__ void __launch_bounds__(tcb::kThreads, 1)
       tc_fence_before();
       mbar_arrive(pt_full);
     }
-    if (!ok) tc_fail(a.err, 23, abort_flag);
-    const bool have = ok && ntl > 0 && warp_wait(dkv_final, 0, abort_flag);
-    if (ok && ntl > 0 && !have) tc_fail(a.err, 24, abort_flag);
-    // `have` and `ntl` are warp-uniform, so the collective TMEM loads below run on whole
-    // warps; only the stores depend on the lane's key being inside the sequence.
-    if (have || ntl == 0) {
+    if (!ok) tc_fail(a.err, 33, abort_flag);
+    const bool have = ok && n_tiles > 0 && warp_wait(dkv_final, 0, abort_flag);
+    if (ok && n_tiles > 0 && !have) tc_fail(a.err, 34, abort_flag);
+    // `have` and `n_tiles` are warp-uniform: the collective TMEM loads run on whole warps,
+    // only the stores depend on the lane's key being inside the sequence.
+    if (have || n_tiles == 0) {
       const bool store = kp < L;
       __nv_bfloat16* dkr = a.dk + ((size_t)(s0 + kp) * a.Hkv + kv) * kD;
       __nv_bfloat16* dvr = a.dv + ((size_t)(s0 + kp) * a.Hkv + kv) * kD;
@@ -692,7 +710,7 @@ __global__ void __launch_bounds__(tcb::kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 4) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -705,15 +723,14 @@ bool attn_bwd_tc_supported(const sas_problem& p) {
   if (!attn_tc_supported(p)) return false;
   const int G = p.num_q_heads / p.num_kv_heads;
   const int Mq = tc_rows_per_tile(G);
-  return Mq * (p.topk + 1) <= tcb::kMaxSel && (p.max_seqlen + Mq - 1) / Mq <= tcb::kMaxTiles;
+  return Mq * (p.topk + 1) <= tcb::kMaxSel && (p.max_seqlen + 31) / 32 <= tcb::kMaxWords;
 }
 
+// bytes of the per-(kv, block pair) token bitmasks
 size_t attn_bwd_tc_tmask_bytes(const sas_problem& p) {
-  const int G = p.num_q_heads / p.num_kv_heads;
-  const int Mq = tc_rows_per_tile(G);
   const int NBmax = (p.max_seqlen + p.block - 1) / p.block;
-  const size_t n_tiles = (p.max_seqlen + Mq - 1) / Mq;
-  return (size_t)p.batch * n_tiles * p.num_kv_heads * ((NBmax + 31) / 32) * 4;
+  const size_t NP = (NBmax + 1) / 2, W = (p.max_seqlen + 31) / 32;
+  return (size_t)p.batch * p.num_kv_heads * NP * W * 4;
 }
 
 sas_status launch_attn_bwd_tc(const sas_problem& p, const void* q, const void* k, const void* v,
@@ -736,7 +753,9 @@ sas_status launch_attn_bwd_tc(const sas_problem& p, const void* q, const void* k
   a.logg = logg;
   a.lse = lse;
   a.drow = drow;
-  a.tmask = tmask;
+  a.pmask = tmask;
+  a.q = (const __nv_bfloat16*)q;
+  a.dout = (const __nv_bfloat16*)dout;
   a.dq = (__nv_bfloat16*)dq;
   a.dk = (__nv_bfloat16*)dk;
   a.dv = (__nv_bfloat16*)dv;
@@ -749,22 +768,29 @@ sas_status launch_attn_bwd_tc(const sas_problem& p, const void* q, const void* k
   a.Mq = Mq;
   a.NBmax = (p.max_seqlen + p.block - 1) / p.block;
   a.n_tiles = (p.max_seqlen + Mq - 1) / Mq;
+  a.NP = (a.NBmax + 1) / 2;
+  a.W = (p.max_seqlen + 31) / 32;
   a.scale = 1.f / sqrtf(128.f);
   a.scale_log2 = kLog2e * a.scale;
   static std::once_flag attr_once;
   std::call_once(attr_once, [] {
     cudaFuncSetAttribute(attn_bwd_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          tcb::Q_SMEM);
-    cudaFuncSetAttribute(attn_bwd_dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         tcb::K_SMEM);
+    cudaFuncSetAttribute(attn_bwd_dkdv_gather_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         tcb::G_SMEM);
   });
-  tile_union_kernel<<<dim3(a.n_tiles, p.batch, p.num_kv_heads), 128, 0, st>>>(
-      idx, p.cu_seqlens, p.num_kv_heads, p.topk, Mq, a.NBmax, a.n_tiles, tmask);
+  if (cudaMemsetAsync(tmask, 0, attn_bwd_tc_tmask_bytes(p), st) != cudaSuccess) {
+    set_error("attn_bwd: clearing the token bitmasks failed");
+    return SAS_ERR_CUDA;
+  }
+  const int rows = p.total_tokens * p.num_kv_heads;
+  pair_mask_kernel<<<(rows + 255) / 256, 256, 0, st>>>(idx, p.cu_seqlens, p.batch,
+                                                        p.total_tokens, p.num_kv_heads, p.topk,
+                                                        a.NP, a.W, tmask);
   attn_bwd_dq_tc_kernel<<<dim3(a.n_tiles, p.batch, p.num_kv_heads), tcb::kThreads, tcb::Q_SMEM,
                           st>>>(tq, tdo, tk, tv, a);
-  const int n_pairs = (a.NBmax + 1) / 2;
-  attn_bwd_dkdv_tc_kernel<<<dim3(n_pairs, p.batch, p.num_kv_heads), tcb::kThreads, tcb::K_SMEM,
-                            st>>>(tq, tdo, tk, tv, a);
+  attn_bwd_dkdv_gather_kernel<<<dim3(a.NP, p.batch, p.num_kv_heads), tcb::kGThreads, tcb::G_SMEM,
+                                st>>>(tk, tv, a);
   return launch_status("attn_bwd (tensor cores)", 3);
 }
 
