@@ -8,16 +8,20 @@
 // and -inf to the others (abstract: the gate sits inside the softmax in log form). Work per
 // visited block: S = Q K^T (M=128, N=64, K=128) and O += P V (M=128, N=128, K=64).
 //
-// Warp roles (256 threads):
-//   warp 0 lane 0   TMA producer: Q tile once, then K/V blocks of the union through a
-//                   3-stage ring (one 3-D box per 64-row half, block row = s0 + j*64)
-//   warp 1 lane 0   MMA issuer: QK^T into one of two TMEM S buffers, PV into TMEM O
-//   warp 1          TMEM allocation / release (256 columns: O 0..127, S0 128..191,
-//                   S1 192..255)
-//   warps 4..7      softmax: thread r owns TMEM lane r = query row r (token r/G, head r%G);
+// Warp roles (384 threads):
+//   warp 0 lane 0   TMA producer: K/V blocks of the union through a 4-stage ring (one 3-D
+//                   box per 64-column half, block row = s0 + j*64)
+//   warp 1 lane 0   MMA issuer: S = Q K^T with A = Q from TMEM, O += P V with A = P from
+//                   TMEM (only the B operands, K and V, are read from shared memory)
+//   warp 1          TMEM allocation / release (512 columns)
+//   warps 4..11     two softmax warpgroups; warpgroup w stages head-dim half w of the
+//                   tile's Q rows into TMEM, then takes the union blocks n = w, w+2, ... with
+//                   its own O accumulator (O0 0..127, O1 128..255) and S buffer (256..,
+//                   320..). Thread r owns TMEM lane r = query row r (token r/G, head r%G):
 //                   scale, log-gate, causal mask, online max with lazy O rescale (only when
-//                   the row max grows by more than 2^8), P to shared memory (bf16, 128B
-//                   swizzle), epilogue O/l and LSE
+//                   the row max grows by more than 2^8), P as bf16 pairs over the first 32
+//                   columns of its S buffer. The epilogue merges the two partial softmaxes
+//                   (as split-K) and writes O and LSE
 // Every pipeline wait is bounded; a timeout sets the workspace error word and all roles
 // wind down (in-flight TMA drained, MMAs completed, TMEM released) instead of hanging.
 #include <cuda.h>
@@ -36,27 +40,27 @@ namespace tcf {
 constexpr int kD = 128;                 // head dim
 constexpr int kB = 64;                  // keys per block
 constexpr int kM = 128;                 // rows per tile
-constexpr int kStages = 3;
-constexpr int kThreads = 256;
+constexpr int kStages = 4;
+constexpr int kThreads = 384;           // 4 role warps + two softmax warpgroups
 constexpr int kMaxSel = 4096;           // staged (tokens x slots) per tile
 constexpr int kMaxBlocks = 2048;        // NBmax
-constexpr int kHalf = kM * 128;         // one 64-column half of the Q tile: 16 KB
 constexpr int kKVHalf = kB * 128;       // one 64-column half of a K or V block: 8 KB
 constexpr int kStageBytes = 4 * kKVHalf;  // K0 K1 V0 V1
-constexpr int kPBytes = kM * 128;       // P tile: 128 rows x 64 keys bf16
-constexpr int OFF_Q = 0;
-constexpr int OFF_KV = OFF_Q + 2 * kHalf;
-constexpr int OFF_P = OFF_KV + kStages * kStageBytes;
-constexpr int OFF_SEL_IDX = OFF_P + 2 * kPBytes;
+constexpr int OFF_KV = 0;
+constexpr int OFF_SEL_IDX = OFF_KV + kStages * kStageBytes;
 constexpr int OFF_SEL_LG = OFF_SEL_IDX + kMaxSel * 4;
 constexpr int OFF_LIST = OFF_SEL_LG + kMaxSel * 4;
 constexpr int OFF_MASK = OFF_LIST + kMaxBlocks * 4;
-constexpr int OFF_BAR = OFF_MASK + kMaxBlocks / 8;
+constexpr int OFF_XCH = OFF_MASK + kMaxBlocks / 8;   // [2 warpgroups][m, l][128 rows]
+constexpr int OFF_BAR = OFF_XCH + 2 * 2 * 128 * 4;
 constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 2 + 1;
 constexpr int OFF_MISC = OFF_BAR + kNumBars * 8;
 constexpr int kSmemBytes = OFF_MISC + 64 + 1024;   // + slack for 1024-byte alignment
-constexpr uint32_t kTmemCols = 256;
-constexpr int kColS = 128;              // S buffers start column
+// TMEM columns: O0 0..127, O1 128..255, S0 256..319, S1 320..383 (P of a block is written
+// as bf16 pairs over the first 32 columns of its S buffer), Q 384..447 (bf16 pairs)
+constexpr uint32_t kTmemCols = 512;
+constexpr int kColS = 256;
+constexpr int kColQ = 384;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 }  // namespace tcf
 
@@ -64,6 +68,7 @@ struct TcFwdArgs {
   const int32_t* cu;
   const int32_t* idx;
   const float* logg;
+  const __nv_bfloat16* q;
   __nv_bfloat16* o;
   float* lse;
   int* err;
@@ -72,8 +77,8 @@ struct TcFwdArgs {
 };
 
 __global__ void __launch_bounds__(tcf::kThreads, 1)
-    attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                       const __grid_constant__ CUtensorMap tmV, const TcFwdArgs a) {
+    attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                       const TcFwdArgs a) {
   using namespace tcf;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>(
@@ -86,10 +91,9 @@ __global__ void __launch_bounds__(tcf::kThreads, 1)
   if (t0 >= L) return;
   const int nt = min(a.Mq, L - t0);
   const int G = a.G, K1 = a.K + 1;
-  const int rows_used = G * a.Mq;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
-  uint64_t* q_full = bars;
+  uint64_t* q_ready = bars;                  // Q staged in TMEM (256 softmax threads)
   uint64_t* kv_full = bars + 1;
   uint64_t* kv_empty = kv_full + kStages;
   uint64_t* s_full = kv_empty + kStages;
@@ -108,7 +112,7 @@ __global__ void __launch_bounds__(tcf::kThreads, 1)
   const int nwords = (a.NBmax + 31) >> 5;
   for (int w = tid; w < nwords; w += kThreads) mask[w] = 0u;
   if (tid == 0) {
-    mbar_init(q_full, 1);
+    mbar_init(q_ready, 256);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(kv_full + s, 1);
       mbar_init(kv_empty + s, 1);
@@ -125,15 +129,6 @@ __global__ void __launch_bounds__(tcf::kThreads, 1)
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
-  }
-  if (rows_used < kM) {   // rows the Q box leaves untouched must hold zeros, not stale data
-    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-    for (int e = tid; e < (kM - rows_used) * 8; e += kThreads) {
-      const int r = rows_used + (e >> 3), c = e & 7;
-      reinterpret_cast<uint4*>(sm + OFF_Q + r * 128)[c] = z;
-      reinterpret_cast<uint4*>(sm + OFF_Q + kHalf + r * 128)[c] = z;
-    }
-    fence_async_smem();
   }
   __syncthreads();
   for (int e = tid; e < nt * K1; e += kThreads) {
@@ -176,13 +171,9 @@ __global__ void __launch_bounds__(tcf::kThreads, 1)
 
   // ------------------------------ roles ------------------------------
   if (warp == 0) {
-    if (lane == 0) {   // TMA producer
-      prefetch_tmap(&tmQ);
+    if (lane == 0) {   // TMA producer: K/V blocks of the union
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
-      mbar_arrive_expect_tx(q_full, 2u * rows_used * 128u);
-      tma_load_3d(sm + OFF_Q, &tmQ, q_full, 0, kv * G, s0 + t0);
-      tma_load_3d(sm + OFF_Q + kHalf, &tmQ, q_full, 64, kv * G, s0 + t0);
       int issued = 0;
       for (int n = 0; n < nb; ++n) {
         const int st = n % kStages;
@@ -200,7 +191,6 @@ __global__ void __launch_bounds__(tcf::kThreads, 1)
         issued = n + 1;
       }
       // no copy may still be in flight when the CTA exits
-      mbar_wait_drain(q_full, 0);
       for (int n = max(0, issued - kStages); n < issued; ++n)
         mbar_wait_drain(kv_full + n % kStages, (n / kStages) & 1);
     }
@@ -208,8 +198,7 @@ __global__ void __launch_bounds__(tcf::kThreads, 1)
     if (lane == 0) {   // MMA issuer
       constexpr uint32_t kIdescQK = idesc_bf16_f32(kM, kB, false, false);
       constexpr uint32_t kIdescPV = idesc_bf16_f32(kM, kD, false, true);
-      const uint32_t q_addr = smem_u32(sm + OFF_Q);
-      bool ok = mbar_wait(q_full, 0, abort_flag);
+      bool ok = mbar_wait(q_ready, 0, abort_flag);
       if (ok) tc_fence_after();
       for (int n = 0; ok && n <= nb; ++n) {
         if (n < nb) {
@@ -218,10 +207,10 @@ __global__ void __launch_bounds__(tcf::kThreads, 1)
           tc_fence_after();
           const uint32_t k_addr = smem_u32(sm + OFF_KV + st * kStageBytes);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t ad = sdesc_sw128(q_addr + (kk >> 2) * kHalf + (kk & 3) * 32, 16, 1024);
+          for (int kk = 0; kk < 8; ++kk) {   // S = Q K^T: A = Q from TMEM, B = K (K-major smem)
             const uint64_t bd = sdesc_sw128(k_addr + (kk >> 2) * kKVHalf + (kk & 3) * 32, 16, 1024);
-            mma_bf16_ss(tmem + kColS + bb * kB, ad, bd, kIdescQK, kk > 0 ? 1u : 0u);
+            mma_bf16_ts(tmem + kColS + bb * kB, tmem + kColQ + kk * 8, bd, kIdescQK,
+                        kk > 0 ? 1u : 0u);
           }
           tc_commit(s_full + bb);
         }
@@ -229,14 +218,13 @@ __global__ void __launch_bounds__(tcf::kThreads, 1)
           const int m = n - 1, pb = m & 1, st = m % kStages;
           if (!mbar_wait(p_full + pb, (m >> 1) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t p_addr = smem_u32(sm + OFF_P + pb * kPBytes);
           const uint32_t v_addr = smem_u32(sm + OFF_KV + st * kStageBytes + 2 * kKVHalf);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = sdesc_sw128(p_addr + kk * 32, 16, 1024);
-            // V as the MN-major B operand: 64-column halves kKVHalf apart, 8-key groups 1 KB apart
+          for (int kk = 0; kk < 4; ++kk) {   // O += P V: A = P from TMEM, B = V (MN-major smem)
             const uint64_t bd = sdesc_sw128(v_addr + kk * 2048, kKVHalf, 1024);
-            mma_bf16_ss(tmem, ad, bd, kIdescPV, (m > 0 || kk > 0) ? 1u : 0u);
+            // even blocks accumulate into O0, odd blocks into O1 (one per softmax warpgroup)
+            mma_bf16_ts(tmem + pb * kD, tmem + kColS + pb * kB + kk * 8, bd, kIdescPV,
+                        (m > 1 || kk > 0) ? 1u : 0u);
           }
           tc_commit(pv_done + pb);
           tc_commit(kv_empty + st);
@@ -246,98 +234,140 @@ __global__ void __launch_bounds__(tcf::kThreads, 1)
       tc_commit(o_final);
       mbar_wait_drain(o_final, 0);   // all MMAs done before the TMEM is released
     }
-  } else if (warp >= 4) {   // softmax warpgroup
-    const int r = tid - 128;
+  } else if (warp >= 4) {   // softmax: warpgroup wg takes the union blocks n = wg, wg+2, ...
+    const int wg = (warp - 4) >> 2;
+    const int r = tid - 128 - wg * 128;
     const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
     const int tl = r / G;
     const bool valid = r < G * nt;
     const int t = t0 + tl;
     const int ct = t / kB;
+    const int hq = kv * G + (r % G);
     const int32_t* my_idx = sel_idx + tl * K1;
     const float* my_lg = sel_lg + tl * K1;
+    const uint32_t o_col = wg * kD;                    // this warpgroup's O accumulator
+    const uint32_t s_col = kColS + wg * kB;            // and S / P buffer
+    {   // stage this row of Q in TMEM: warpgroup wg writes head-dim half wg (bf16 pairs)
+      uint32_t qw[32];
+      if (valid) {
+        const uint4* src = reinterpret_cast<const uint4*>(a.q + ((size_t)(s0 + t) * a.Hq + hq) * kD + wg * 64);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint4 u = src[i];
+          qw[4 * i] = u.x; qw[4 * i + 1] = u.y; qw[4 * i + 2] = u.z; qw[4 * i + 3] = u.w;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) qw[i] = 0u;
+      }
+      tmem_st32(tmem + lane_addr + kColQ + wg * 32, reinterpret_cast<const float*>(qw));
+      tc_fence_before();
+      mbar_arrive(q_ready);
+    }
     float m_ref = -INFINITY, l_sum = 0.f;
     int sp = 0;
     bool ok = true;
-    for (int n = 0; n < nb; ++n) {
-      const int bb = n & 1;
+    for (int n = wg; n < nb; n += 2) {
       const int j = list[n];
-      if (!warp_wait(s_full + bb, (n >> 1) & 1, abort_flag)) { ok = false; break; }
+      if (!warp_wait(s_full + wg, (n >> 1) & 1, abort_flag)) { ok = false; break; }
+      // PV(n-2), this warpgroup's previous block, was issued before QK(n) and so has already
+      // completed: O and the P columns are free (the wait returns at once)
+      if (n >= 2 && !warp_wait(pv_done + wg, ((n - 2) >> 1) & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      float s[kB];
-      tmem_ld32(tmem + lane_addr + kColS + bb * kB, s);
-      tmem_ld32(tmem + lane_addr + kColS + bb * kB + 32, s + 32);
       float bias = -INFINITY;
       if (valid) {
         while (sp < K1 && my_idx[sp] >= 0 && my_idx[sp] < j) ++sp;
         if (sp < K1 && my_idx[sp] == j) bias = my_lg[sp] * kLog2e;
       }
-      const int limit = (j == ct) ? (t - j * kB) : (kB - 1);   // last visible key column
-      float rmax = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < kB; ++c) {
-        const float x = (c <= limit) ? fmaf(s[c], a.scale_log2, bias) : -INFINITY;
-        s[c] = x;
-        rmax = fmaxf(rmax, x);
-      }
-      const bool grow = rmax > m_ref + kRescaleThreshold;
-      const float m_new = grow ? rmax : m_ref;
-      const float alpha = grow ? exp2f(m_ref - m_new) : 1.f;
-      const bool need_o = grow && (m_ref != -INFINITY);
-      if (__any_sync(0xffffffffu, need_o)) {
-        // O may only be touched once PV(n-1) has completed
-        if (!warp_wait(pv_done + ((n - 1) & 1), ((n - 1) >> 1) & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-#pragma unroll 1
-        for (int c0 = 0; c0 < kD; c0 += 32) {
-          float ov[32];
-          tmem_ld32(tmem + lane_addr + c0, ov);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) ov[i] *= alpha;
-          tmem_st32(tmem + lane_addr + c0, ov);
-        }
-      }
-      l_sum *= alpha;
-      m_ref = m_new;
-      if (n >= 2 && !warp_wait(pv_done + bb, ((n - 2) >> 1) & 1, abort_flag)) { ok = false; break; }
-      const float ref = (m_ref == -INFINITY) ? 0.f : m_ref;
-      float psum = 0.f;
+      const bool has = bias != -INFINITY;
       uint32_t pk[kB / 2];
+      if (__any_sync(0xffffffffu, has)) {
+        float s[kB];
+        tmem_ld32(tmem + lane_addr + s_col, s);
+        tmem_ld32(tmem + lane_addr + s_col + 32, s + 32);
+        const int limit = (j == ct) ? (t - j * kB) : (kB - 1);   // last visible key column
+        float smax = -INFINITY;                                   // max of the raw scores
+        if (limit == kB - 1) {
 #pragma unroll
-      for (int c = 0; c < kB; c += 2) {
-        const float p0 = exp2f(s[c] - ref), p1 = exp2f(s[c + 1] - ref);
-        psum += p0 + p1;
-        pk[c >> 1] = pack_bf16x2(p0, p1);
+          for (int c = 0; c < kB; ++c) smax = fmaxf(smax, s[c]);
+        } else {
+#pragma unroll
+          for (int c = 0; c < kB; ++c)
+            if (c <= limit) smax = fmaxf(smax, s[c]);
+        }
+        const float rmax = has ? fmaf(smax, a.scale_log2, bias) : -INFINITY;
+        const bool grow = rmax > m_ref + kRescaleThreshold;
+        const float m_new = grow ? rmax : m_ref;
+        const float alpha = grow ? ex2_approx(m_ref - m_new) : 1.f;
+        const bool need_o = grow && (m_ref != -INFINITY);
+        if (__any_sync(0xffffffffu, need_o)) {
+#pragma unroll 1
+          for (int c0 = 0; c0 < kD; c0 += 32) {
+            float ov[32];
+            tmem_ld32(tmem + lane_addr + o_col + c0, ov);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ov[i] *= alpha;
+            tmem_st32(tmem + lane_addr + o_col + c0, ov);
+          }
+        }
+        l_sum *= alpha;
+        m_ref = m_new;
+        // p = 2^(s*scale + bias - m): one FMA and one ex2 per score; rows without the
+        // block (bias = -inf) and masked keys give exactly 0
+        const float off = has ? bias - m_ref : -INFINITY;
+        float psum = 0.f;
+#pragma unroll
+        for (int c = 0; c < kB; c += 2) {
+          const float p0 = (c <= limit) ? ex2_approx(fmaf(s[c], a.scale_log2, off)) : 0.f;
+          const float p1 = (c + 1 <= limit) ? ex2_approx(fmaf(s[c + 1], a.scale_log2, off)) : 0.f;
+          psum += p0 + p1;
+          pk[c >> 1] = pack_bf16x2(p0, p1);
+        }
+        l_sum += psum;
+      } else {   // no row of this warp kept block j: its P row is zero, m and l unchanged
+#pragma unroll
+        for (int c = 0; c < kB / 2; ++c) pk[c] = 0u;
       }
-      l_sum += psum;
-      const uint32_t prow = smem_u32(sm + OFF_P + bb * kPBytes) + r * 128;
-#pragma unroll
-      for (int c = 0; c < 8; ++c)
-        st_shared_v4(prow + ((c ^ (r & 7)) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2],
-                     pk[4 * c + 3]);
-      fence_async_smem();
+      tmem_st32(tmem + lane_addr + s_col, reinterpret_cast<const float*>(pk));   // P over S
       tc_fence_before();
-      mbar_arrive(p_full + bb);
+      mbar_arrive(p_full + wg);
     }
+    // merge the two partial softmaxes: O = (O0 2^(m0-M) + O1 2^(m1-M)) / (l0 2^(m0-M) + l1 2^(m1-M))
+    float* xch = reinterpret_cast<float*>(sm + OFF_XCH);
+    xch[wg * 256 + r] = m_ref;
+    xch[wg * 256 + 128 + r] = l_sum;
+    named_bar(1, 256);   // both warpgroups, always reached
+    const float m0 = xch[r], l0 = xch[128 + r], m1 = xch[256 + r], l1 = xch[384 + r];
+    const float M = fmaxf(m0, m1);
+    const float f0 = (m0 == -INFINITY) ? 0.f : ex2_approx(m0 - M);
+    const float f1 = (m1 == -INFINITY) ? 0.f : ex2_approx(m1 - M);
+    const float l = l0 * f0 + l1 * f1;
+    const float inv = (l > 0.f) ? 1.f / l : 0.f;
     if (ok) ok = warp_wait(o_final, 0, abort_flag);
     if (ok) {
       tc_fence_after();
-      const float inv = (l_sum > 0.f) ? 1.f / l_sum : 0.f;
-      const int hq = kv * G + (r % G);
       __nv_bfloat16* orow = a.o + ((size_t)(s0 + t) * a.Hq + hq) * kD;
 #pragma unroll 1
-      for (int c0 = 0; c0 < kD; c0 += 32) {
-        float ov[32];
-        tmem_ld32(tmem + lane_addr + c0, ov);
+      for (int c0 = wg * 64; c0 < wg * 64 + 64; c0 += 32) {   // each warpgroup: half the columns
+        // an accumulator that no PV wrote (union of 0 or 1 blocks) holds garbage: skip it
+        // (nb is CTA-uniform, so the collective loads stay warp-uniform)
+        float o0[32], o1[32];
+        if (nb > 0) tmem_ld32(tmem + lane_addr + c0, o0);
+        else for (int i = 0; i < 32; ++i) o0[i] = 0.f;
+        if (nb > 1) tmem_ld32(tmem + lane_addr + kD + c0, o1);
+        else for (int i = 0; i < 32; ++i) o1[i] = 0.f;
         if (valid) {
           uint32_t pk[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(ov[2 * i] * inv, ov[2 * i + 1] * inv);
+          for (int i = 0; i < 16; ++i)
+            pk[i] = pack_bf16x2((o0[2 * i] * f0 + o1[2 * i] * f1) * inv,
+                                (o0[2 * i + 1] * f0 + o1[2 * i + 1] * f1) * inv);
           uint4* dst = reinterpret_cast<uint4*>(orow + c0);
 #pragma unroll
           for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
         }
       }
-      if (valid) a.lse[(size_t)(s0 + t) * a.Hq + hq] = (m_ref + log2f(l_sum)) * kLn2;
+      if (valid && wg == 0) a.lse[(size_t)(s0 + t) * a.Hq + hq] = (M + log2f(l)) * kLn2;
     } else {
       tc_fail(a.err, 3, abort_flag);
     }
@@ -395,9 +425,8 @@ sas_status launch_attn_fwd_tc(const sas_problem& p, const void* q, const void* k
                               cudaStream_t st) {
   const int G = p.num_q_heads / p.num_kv_heads;
   const int Mq = tc_rows_per_tile(G);
-  CUtensorMap tq, tk, tv;
-  if (!make_tmap_bf16_3d(&tq, q, 128, p.num_q_heads, p.total_tokens, 64, G, Mq) ||
-      !make_tmap_bf16_3d(&tk, k, 128, p.num_kv_heads, p.total_tokens, 64, 1, 64) ||
+  CUtensorMap tk, tv;
+  if (!make_tmap_bf16_3d(&tk, k, 128, p.num_kv_heads, p.total_tokens, 64, 1, 64) ||
       !make_tmap_bf16_3d(&tv, v, 128, p.num_kv_heads, p.total_tokens, 64, 1, 64)) {
     set_error("attn_fwd: TMA descriptor creation failed");
     return SAS_ERR_CUDA;
@@ -406,6 +435,7 @@ sas_status launch_attn_fwd_tc(const sas_problem& p, const void* q, const void* k
   a.cu = p.cu_seqlens;
   a.idx = idx;
   a.logg = logg;
+  a.q = (const __nv_bfloat16*)q;
   a.o = (__nv_bfloat16*)o;
   a.lse = lse;
   a.err = err;
@@ -423,7 +453,7 @@ sas_status launch_attn_fwd_tc(const sas_problem& p, const void* q, const void* k
                          tcf::kSmemBytes);
   });
   dim3 grid(a.n_tiles, p.batch, p.num_kv_heads);
-  attn_fwd_tc_kernel<<<grid, tcf::kThreads, tcf::kSmemBytes, st>>>(tq, tk, tv, a);
+  attn_fwd_tc_kernel<<<grid, tcf::kThreads, tcf::kSmemBytes, st>>>(tk, tv, a);
   return launch_status("attn_fwd (tensor cores)", 1);
 }
 

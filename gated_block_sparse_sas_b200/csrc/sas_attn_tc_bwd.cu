@@ -28,7 +28,7 @@ namespace sas {
 using namespace sm100;
 
 namespace tcb {
-constexpr int kD = 128, kB = 64, kM = 128, kThreads = 256;
+constexpr int kD = 128, kB = 64, kM = 128, kThreads = 384;   // query-major: 4 role warps + 2 dS warpgroups
 constexpr int kHalf = kM * 128;          // 128 rows x 128 B
 constexpr int kKVHalf = kB * 128;        // 64 rows x 128 B
 constexpr int kStageBytes = 4 * kKVHalf; // K0 K1 V0 V1
@@ -45,8 +45,8 @@ constexpr int Q_OFF_SEL_IDX = Q_OFF_DS + 2 * kTileBytes;
 constexpr int Q_OFF_SEL_LG = Q_OFF_SEL_IDX + kMaxSel * 4;
 constexpr int Q_OFF_LIST = Q_OFF_SEL_LG + kMaxSel * 4;
 constexpr int Q_OFF_MASK = Q_OFF_LIST + kMaxBlocks * 4;
-constexpr int Q_OFF_RS = Q_OFF_MASK + kMaxBlocks / 8;          // 2 x 128 floats
-constexpr int Q_OFF_BAR = Q_OFF_RS + 2 * 128 * 4;
+constexpr int Q_OFF_RS = Q_OFF_MASK + kMaxBlocks / 8;          // [2 wg][2][128] floats
+constexpr int Q_OFF_BAR = Q_OFF_RS + 4 * 128 * 4;
 constexpr int Q_NBARS = 1 + 2 * kStages + 2 + 2 + 2 + 1;
 constexpr int Q_OFF_MISC = Q_OFF_BAR + Q_NBARS * 8;
 constexpr int Q_SMEM = Q_OFF_MISC + 64 + 1024;
@@ -312,8 +312,9 @@ __global__ void __launch_bounds__(tcb::kThreads, 1)
       tc_commit(dq_final);
       mbar_wait_drain(dq_final, 0);
     }
-  } else if (warp >= 4) {   // dS warpgroup: thread r = TMEM lane r = query row r
-    const int r = tid - 128;
+  } else if (warp >= 4) {   // dS warpgroup wg takes the union blocks n = wg, wg+2, ...
+    const int wg = (warp - 4) >> 2;
+    const int r = tid - 128 - wg * 128;   // TMEM lane r = query row r
     const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
     const int tl = r / G, g = r - tl * G;
     const bool valid = r < G * nt;
@@ -326,42 +327,47 @@ __global__ void __launch_bounds__(tcb::kThreads, 1)
     const float dd = valid ? a.drow[qrow] : 0.f;
     float* dl_row = a.dlogg + ((size_t)(s0 + t) * a.Hkv + kv) * K1;
     const bool leader = valid && g == 0;
-    if (leader)
+    if (leader && wg == 0)
       for (int s = 0; s < K1; ++s)
         if (my_idx[s] < 0) dl_row[s] = 0.f;
     int sp = 0;
     bool ok = true;
     // After a failed wait a warp stops working but keeps iterating, so that the named
-    // barrier below (G not dividing 32) is always reached by all four warps.
-    for (int n = 0; n < nb; ++n) {
-      const int bb = n & 1;
+    // barrier below (G not dividing 32) is always reached by all four warps of the group.
+    for (int n = wg; n < nb; n += 2) {
+      const int bb = wg;
       const int j = list[n];
       float rsum = 0.f;
       bool hit = false;
       if (ok && !warp_wait(s_full + bb, (n >> 1) & 1, abort_flag)) ok = false;
       if (ok) {
         tc_fence_after();
-        float s[kB], dp[kB];
-        tmem_ld32(tmem + lane_addr + 128 + bb * 128, s);
-        tmem_ld32(tmem + lane_addr + 128 + bb * 128 + 32, s + 32);
-        tmem_ld32(tmem + lane_addr + 128 + bb * 128 + 64, dp);
-        tmem_ld32(tmem + lane_addr + 128 + bb * 128 + 96, dp + 32);
         float bias = -INFINITY;
         if (valid) {
           while (sp < K1 && my_idx[sp] >= 0 && my_idx[sp] < j) ++sp;
           hit = sp < K1 && my_idx[sp] == j;
           if (hit) bias = my_lg[sp] * kLog2e;
         }
-        const int limit = (j == ct) ? (t - j * kB) : (kB - 1);
         uint32_t pk[kB / 2];
+        if (__any_sync(0xffffffffu, hit)) {
+          float s[kB], dp[kB];
+          tmem_ld32(tmem + lane_addr + 128 + bb * 128, s);
+          tmem_ld32(tmem + lane_addr + 128 + bb * 128 + 32, s + 32);
+          tmem_ld32(tmem + lane_addr + 128 + bb * 128 + 64, dp);
+          tmem_ld32(tmem + lane_addr + 128 + bb * 128 + 96, dp + 32);
+          const int limit = (j == ct) ? (t - j * kB) : (kB - 1);
+          const float off = hit ? bias - lse2 : -INFINITY;   // P = 2^(s*scale + bias - lse)
 #pragma unroll
-        for (int c = 0; c < kB; c += 2) {
-          const float x0 = (c <= limit) ? fmaf(s[c], a.scale_log2, bias) : -INFINITY;
-          const float x1 = (c + 1 <= limit) ? fmaf(s[c + 1], a.scale_log2, bias) : -INFINITY;
-          const float p0 = exp2f(x0 - lse2), p1 = exp2f(x1 - lse2);
-          const float d0 = p0 * (dp[c] - dd), d1 = p1 * (dp[c + 1] - dd);
-          rsum += d0 + d1;
-          pk[c >> 1] = pack_bf16x2(d0, d1);
+          for (int c = 0; c < kB; c += 2) {
+            const float p0 = (c <= limit) ? ex2_approx(fmaf(s[c], a.scale_log2, off)) : 0.f;
+            const float p1 = (c + 1 <= limit) ? ex2_approx(fmaf(s[c + 1], a.scale_log2, off)) : 0.f;
+            const float d0 = p0 * (dp[c] - dd), d1 = p1 * (dp[c + 1] - dd);
+            rsum += d0 + d1;
+            pk[c >> 1] = pack_bf16x2(d0, d1);
+          }
+        } else {   // no row of this warp kept block j: its dS rows are zero
+#pragma unroll
+          for (int c = 0; c < kB / 2; ++c) pk[c] = 0u;
         }
         if (n >= 2 && !warp_wait(ds_free + bb, ((n - 2) >> 1) & 1, abort_flag)) ok = false;
         if (ok) {
@@ -380,11 +386,12 @@ __global__ void __launch_bounds__(tcb::kThreads, 1)
         for (int off = 1; off < G; off <<= 1) rsum += __shfl_xor_sync(0xffffffffu, rsum, off);
         if (ok && leader && hit) dl_row[sp] = rsum;
       } else {
-        rs[bb * 128 + r] = rsum;
-        named_bar(1, 128);
+        float* rsb = rs + (wg * 2 + ((n >> 1) & 1)) * 128;   // double-buffered per group
+        rsb[r] = rsum;
+        named_bar(1 + wg, 128);
         if (ok && leader && hit) {
           float tot = 0.f;
-          for (int u = 0; u < G; ++u) tot += rs[bb * 128 + tl * G + u];
+          for (int u = 0; u < G; ++u) tot += rsb[tl * G + u];
           dl_row[sp] = tot;
         }
       }
@@ -394,7 +401,7 @@ __global__ void __launch_bounds__(tcb::kThreads, 1)
       tc_fence_after();
       __nv_bfloat16* orow = a.dq + qrow * kD;
 #pragma unroll 1
-      for (int c0 = 0; c0 < kD; c0 += 32) {
+      for (int c0 = wg * 64; c0 < wg * 64 + 64; c0 += 32) {   // each group: half the columns
         float ov[32];
         tmem_ld32(tmem + lane_addr + c0, ov);
         if (valid) {
@@ -649,7 +656,7 @@ __global__ void __launch_bounds__(tcb::kGThreads, 1)
           for (int u = 0; u < 2; ++u) {
             const int r = cc * 32 + c + u;
             const bool vis = kp <= __float_as_int(rcb[384 + r]);
-            const float p = vis ? exp2f(fmaf(sv[c + u], a.scale_log2, rcb[coff + r])) : 0.f;
+            const float p = vis ? ex2_approx(fmaf(sv[c + u], a.scale_log2, rcb[coff + r])) : 0.f;
             p2[u] = p;
             d2[u] = vis ? p * (dv[c + u] - rcb[256 + r]) : 0.f;
           }
