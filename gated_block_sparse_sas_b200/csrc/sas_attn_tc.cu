@@ -283,8 +283,7 @@ __global__ void __launch_bounds__(tcf::kThreads, 1)
       uint32_t pk[kB / 2];
       if (__any_sync(0xffffffffu, has)) {
         float s[kB];
-        tmem_ld32(tmem + lane_addr + s_col, s);
-        tmem_ld32(tmem + lane_addr + s_col + 32, s + 32);
+        tmem_ld64(tmem + lane_addr + s_col, s);
         const int limit = (j == ct) ? (t - j * kB) : (kB - 1);   // last visible key column
         float smax = -INFINITY;                                   // max of the raw scores
         if (limit == kB - 1) {

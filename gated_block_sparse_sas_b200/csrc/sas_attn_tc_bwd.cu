@@ -351,10 +351,8 @@ __global__ void __launch_bounds__(tcb::kThreads, 1)
         uint32_t pk[kB / 2];
         if (__any_sync(0xffffffffu, hit)) {
           float s[kB], dp[kB];
-          tmem_ld32(tmem + lane_addr + 128 + bb * 128, s);
-          tmem_ld32(tmem + lane_addr + 128 + bb * 128 + 32, s + 32);
-          tmem_ld32(tmem + lane_addr + 128 + bb * 128 + 64, dp);
-          tmem_ld32(tmem + lane_addr + 128 + bb * 128 + 96, dp + 32);
+          tmem_ld64(tmem + lane_addr + 128 + bb * 128, s);
+          tmem_ld64(tmem + lane_addr + 128 + bb * 128 + 64, dp);
           const int limit = (j == ct) ? (t - j * kB) : (kB - 1);
           const float off = hit ? bias - lse2 : -INFINITY;   // P = 2^(s*scale + bias - lse)
 #pragma unroll

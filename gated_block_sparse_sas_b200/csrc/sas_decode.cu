@@ -8,8 +8,11 @@
 // (3) merge of the splits -> O. The attention only ever reads the selected blocks.
 #include <math.h>
 
+#include <type_traits>
+
 #include "sas_common.cuh"
 #include "sas_kernels.h"
+#include "sas_sm100.cuh"
 
 namespace sas {
 
@@ -84,16 +87,33 @@ __global__ void __launch_bounds__(kDecThreads) decode_gate_kernel(
     P[e] = (part == 2) ? x / (float)n : x;
   }
   __syncthreads();
-  // projections: 2 threads per output channel for each of q and k (H <= 128 -> <= 512 jobs)
-  for (int job = tid; job < 2 * H; job += kDecThreads) {
-    const bool isq = job < H;
-    const int i = isq ? job : job - H;
-    const T* w = isq ? wq + ((size_t)kv * H + i) * GD : wk + ((size_t)kv * H + i) * C;
+  // projections: one warp per output channel (q channels, then k channels), lanes across the
+  // input with 16-byte loads of the weight row, so every row is read coalesced
+  // Four channels per warp step, all their weight loads issued before any arithmetic, so a
+  // warp has several L2 round trips in flight instead of one per channel.
+  for (int job0 = warp * 4; job0 < 2 * H; job0 += kDecWarps * 4) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    const bool isq = job0 < H;   // H is a multiple of 4: a step never mixes q and k channels
     const float* x = isq ? qcat : P;
     const int n_in = isq ? GD : C;
-    float acc = 0.f;
-    for (int e = 0; e < n_in; ++e) acc = fmaf(to_f(w[e]), x[e], acc);
-    (isq ? xq : xk)[i] = acc;
+    for (int e0 = lane * 8; e0 < n_in; e0 += 256) {
+      float w8[4][8];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = (isq ? job0 : job0 - H) + u;
+        const T* w = isq ? wq + ((size_t)kv * H + i) * GD : wk + ((size_t)kv * H + i) * C;
+        load8<T>(w + e0, w8[u]);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 8; ++v) acc[u] = fmaf(w8[u][v], x[e0 + v], acc[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float r = warp_sum(acc[u]);
+      if (lane == 0) (isq ? xq : xk)[(isq ? job0 : job0 - H) + u] = r;
+    }
   }
   __syncthreads();
   if (warp == 0 || warp == 1) {
@@ -118,31 +138,38 @@ __global__ void __launch_bounds__(kDecThreads) decode_gate_kernel(
   }
   __syncthreads();
   const float sqrt_h = sqrtf((float)H);
-  // historical scores: 4 lanes per block, 8 blocks per warp pass
+  // historical scores: H/8 lanes per cached key row (16 bytes each, so a row is one
+  // coalesced segment), 32*8/H rows per warp instruction, 8 rows in flight per lane group
   {
-    const int sub = lane & 3, grp = lane >> 2;
-    constexpr int PER = H / 4;   // channels per lane
-    const __nv_bfloat16* base = gkc + ((size_t)b * Hkv + kv) * (size_t)NBmax * H;
-    for (int jb = warp * 8; jb < c; jb += 8 * kDecWarps) {   // warp-uniform trip count
-      const int j = jb + grp;
-      float acc = 0.f;
-      if (j < c) {
-        const __nv_bfloat16* kr = base + (size_t)j * H + sub * PER;
+    constexpr int LPR = H / 8, RPW = 32 / LPR, UNR = 8;
+    const int sub = lane % LPR, rsub = lane / LPR;
+    float qv[8];
 #pragma unroll
-        for (int e0 = 0; e0 < PER; e0 += 8) {
-          const uint4 uv = *reinterpret_cast<const uint4*>(kr + e0);
-          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&uv);
+    for (int u = 0; u < 8; ++u) qv[u] = xq[sub * 8 + u];
+    const __nv_bfloat16* base = gkc + ((size_t)b * Hkv + kv) * (size_t)NBmax * H + sub * 8;
+    for (int j0 = warp * RPW * UNR; j0 < c; j0 += kDecWarps * RPW * UNR) {   // warp-uniform
+      uint4 raw[UNR];
 #pragma unroll
-          for (int w2 = 0; w2 < 4; ++w2) {
-            const float2 f = __bfloat1622float2(h2[w2]);
-            acc = fmaf(xq[sub * PER + e0 + 2 * w2], f.x, acc);
-            acc = fmaf(xq[sub * PER + e0 + 2 * w2 + 1], f.y, acc);
-          }
-        }
+      for (int it = 0; it < UNR; ++it) {
+        const int j = j0 + it * RPW + rsub;
+        raw[it] = (j < c) ? __ldg(reinterpret_cast<const uint4*>(base + (size_t)j * H))
+                          : make_uint4(0u, 0u, 0u, 0u);
       }
-      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-      if (sub == 0 && j < c) s[j] = acc / sqrt_h;
+#pragma unroll
+      for (int it = 0; it < UNR; ++it) {
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw[it]);
+        float acc = 0.f;
+#pragma unroll
+        for (int w2 = 0; w2 < 4; ++w2) {
+          const float2 f = __bfloat1622float2(h2[w2]);
+          acc = fmaf(qv[2 * w2], f.x, acc);
+          acc = fmaf(qv[2 * w2 + 1], f.y, acc);
+        }
+#pragma unroll
+        for (int off = 1; off < LPR; off <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        const int j = j0 + it * RPW + rsub;
+        if (sub == 0 && j < c) s[j] = acc / sqrt_h;
+      }
     }
     if (warp == 0) {
       float dot = 0.f;
@@ -325,6 +352,240 @@ __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(
   }
 }
 
+// ---------------------------------------------------------------------------------------
+// (2') the same split-K attention for bf16, head_dim 128: each kept block's K and V rows
+// (contiguous, up to 16 KB each) are streamed into a 3-stage shared-memory ring by bulk
+// asynchronous copies issued by one thread, so many kilobytes per SM are in flight; all 256
+// threads then work from shared memory: scores (a warp per key, lanes across head_dim),
+// per-head online softmax (a warp per head), P.V (a thread per (head, 2 channels)).
+// ---------------------------------------------------------------------------------------
+constexpr int kAttStages = 3;
+constexpr int kAttRow = 128 * 2;                  // bytes of one bf16 K or V row (d = 128)
+constexpr int kAttBlk = 64 * kAttRow;             // one block of K (or V): 16 KB
+constexpr int kAttStage = 2 * kAttBlk;
+
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(sm100::smem_u32(bar))
+      : "memory");
+}
+
+template <int G>
+__global__ void __launch_bounds__(kDecThreads, 2) decode_attn_bulk_kernel(
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kc,
+    const __nv_bfloat16* __restrict__ vc, const int32_t* __restrict__ seqlens,
+    const int32_t* __restrict__ sel_idx, const float* __restrict__ sel_logg, int Hkv, int capacity,
+    int B, int K, int nsplit, float scale_log2, float* __restrict__ part_ml,
+    float* __restrict__ part_acc, int* __restrict__ err) {
+  using namespace sm100;
+  constexpr int D = 128;
+  constexpr int NP = (G * 64 + kDecThreads - 1) / kDecThreads;   // (head, 2-channel) pairs per thread
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
+                                           ~static_cast<uintptr_t>(127));
+  float* q_sm = reinterpret_cast<float*>(sm + kAttStages * kAttStage);   // [G][128]
+  float* s_sm = q_sm + G * D;                                            // [G][64]
+  float* st_sm = s_sm + G * 64;                                          // [3][8]: m, l, alpha
+  int* blk_j = reinterpret_cast<int*>(st_sm + 3 * 8);                    // [128] kept blocks
+  float* blk_b = reinterpret_cast<float*>(blk_j + 128);                  // their log-gates (log2)
+  uint64_t* full = reinterpret_cast<uint64_t*>(blk_b + 128);             // [kAttStages], 8-aligned
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(full + kAttStages);
+  int* nblk_s = reinterpret_cast<int*>(full + kAttStages) + 1;
+
+  const int kv = blockIdx.x, b = blockIdx.y, split = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int L = min(seqlens[b], capacity);
+  const int Hq = Hkv * G;
+  const int slots = K + 1;
+  const int per = (slots + nsplit - 1) / nsplit;
+  const int sl0 = split * per, sl1 = min(slots, sl0 + per);
+  const size_t srow = ((size_t)b * Hkv + kv) * (K + 1);
+  if (warp == 0) {   // this split's kept blocks, in slot order (at most 128 slots)
+    int n = 0;
+    for (int sl0w = sl0; sl0w < sl1; sl0w += 32) {
+      const int sl = sl0w + lane;
+      int j = -1;
+      float lg = 0.f;
+      if (sl < sl1) {
+        j = sel_idx[srow + sl];
+        lg = sel_logg[srow + sl];
+      }
+      const bool keep = j >= 0 && j * B < L;
+      const unsigned m = __ballot_sync(0xffffffffu, keep);
+      if (keep) {
+        const int pos = n + __popc(m & ((1u << lane) - 1u));
+        blk_j[pos] = j;
+        blk_b[pos] = lg * kLog2e;
+      }
+      n += __popc(m);
+    }
+    if (lane == 0) {
+      *nblk_s = n;
+      for (int s = 0; s < kAttStages; ++s) mbar_init(full + s, 1);
+      *abort_flag = 0;
+      fence_mbar_init();
+    }
+  }
+  for (int e = tid; e < G * D; e += kDecThreads)
+    q_sm[e] = __bfloat162float(q[((size_t)b * Hq + kv * G) * D + e]);
+  if (tid < G) {
+    st_sm[tid] = -INFINITY;
+    st_sm[8 + tid] = 0.f;
+  }
+  __syncthreads();
+  const int nblk = *nblk_s;
+  const __nv_bfloat16* kbase = kc + ((size_t)b * Hkv + kv) * (size_t)capacity * D;
+  const __nv_bfloat16* vbase = vc + ((size_t)b * Hkv + kv) * (size_t)capacity * D;
+  auto issue = [&](int n) {   // thread 0: copy block n's K and V rows into stage n % kAttStages
+    const int st = n % kAttStages;
+    const int i0 = blk_j[n] * B;
+    const int nk = min(B, L - i0);
+    const uint32_t bytes = (uint32_t)nk * kAttRow;
+    const uint32_t dst = smem_u32(sm + st * kAttStage);
+    mbar_arrive_expect_tx(full + st, 2 * bytes);
+    bulk_g2s(dst, kbase + (size_t)i0 * D, bytes, full + st);
+    bulk_g2s(dst + kAttBlk, vbase + (size_t)i0 * D, bytes, full + st);
+  };
+  int issued = 0;   // thread 0 only
+  if (tid == 0)
+    for (; issued < min(nblk, kAttStages); ++issued) issue(issued);
+
+  float acc[NP][2];
+#pragma unroll
+  for (int u = 0; u < NP; ++u) acc[u][0] = acc[u][1] = 0.f;
+  bool ok = true;
+  for (int n = 0; n < nblk; ++n) {
+    const int st = n % kAttStages;
+    const int i0 = blk_j[n] * B;
+    const int nk = min(B, L - i0);
+    const float bias = blk_b[n];
+    if (ok && !mbar_wait(full + st, (n / kAttStages) & 1, abort_flag)) {
+      *abort_flag = 1;
+      atomicCAS(err, 0, 41);
+      ok = false;
+    }
+    ok = __all_sync(0xffffffffu, ok);   // warp-uniform for the warp reductions below
+    const uint8_t* kst = sm + st * kAttStage;
+    const uint8_t* vst = kst + kAttBlk;
+    // scores: 8 lanes per key (16 channels each), 4 keys per warp step, 8 keys per warp
+    {
+      const int sub = lane & 7, kq = lane >> 3;
+#pragma unroll 1
+      for (int step = 0; step < 2; ++step) {
+        const int k = warp * 8 + step * 4 + kq;
+        float kf[16];
+        const bool live = ok && k < nk;
+        if (live) {
+          const uint4 a0 = *reinterpret_cast<const uint4*>(kst + k * kAttRow + sub * 32);
+          const uint4 a1 = *reinterpret_cast<const uint4*>(kst + k * kAttRow + sub * 32 + 16);
+          const __nv_bfloat162* h0 = reinterpret_cast<const __nv_bfloat162*>(&a0);
+          const __nv_bfloat162* h1 = reinterpret_cast<const __nv_bfloat162*>(&a1);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float2 f0 = __bfloat1622float2(h0[u]), f1 = __bfloat1622float2(h1[u]);
+            kf[2 * u] = f0.x; kf[2 * u + 1] = f0.y; kf[8 + 2 * u] = f1.x; kf[8 + 2 * u + 1] = f1.y;
+          }
+        } else {
+#pragma unroll
+          for (int u = 0; u < 16; ++u) kf[u] = 0.f;
+        }
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float* qh = q_sm + h * D + sub * 16;
+          float dot = 0.f;
+#pragma unroll
+          for (int u = 0; u < 16; u += 4) {
+            const float4 qq = *reinterpret_cast<const float4*>(qh + u);
+            dot = fmaf(qq.x, kf[u], dot);
+            dot = fmaf(qq.y, kf[u + 1], dot);
+            dot = fmaf(qq.z, kf[u + 2], dot);
+            dot = fmaf(qq.w, kf[u + 3], dot);
+          }
+          dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+          dot += __shfl_xor_sync(0xffffffffu, dot, 2);
+          dot += __shfl_xor_sync(0xffffffffu, dot, 4);
+          if (sub == 0) s_sm[h * 64 + k] = live ? fmaf(dot, scale_log2, bias) : -INFINITY;
+        }
+      }
+    }
+    __syncthreads();
+    // online softmax per head (warp h)
+    if (warp < G) {
+      const float s0v = s_sm[warp * 64 + lane], s1v = s_sm[warp * 64 + 32 + lane];
+      const float mx = warp_max(fmaxf(s0v, s1v));
+      const float m_old = st_sm[warp];
+      const float m_new = fmaxf(m_old, mx);
+      const float ref = (m_new == -INFINITY) ? 0.f : m_new;
+      const float p0 = exp2f(s0v - ref), p1 = exp2f(s1v - ref);
+      s_sm[warp * 64 + lane] = p0;
+      s_sm[warp * 64 + 32 + lane] = p1;
+      const float ps = warp_sum(p0 + p1);
+      if (lane == 0) {
+        const float alpha = (m_old == -INFINITY) ? 0.f : exp2f(m_old - ref);
+        st_sm[warp] = m_new;
+        st_sm[8 + warp] = st_sm[8 + warp] * alpha + ps;
+        st_sm[16 + warp] = alpha;
+      }
+    }
+    __syncthreads();
+    // P.V: thread owns (head, channel pair) o = tid + 256 u
+#pragma unroll
+    for (int u = 0; u < NP; ++u) {
+      const int o = tid + u * kDecThreads;
+      if (o < G * 64) {
+        const int h = o >> 6, d2 = (o & 63) * 2;
+        const float alpha = st_sm[16 + h];
+        float a0 = acc[u][0] * alpha, a1 = acc[u][1] * alpha;
+        const float* ph = s_sm + h * 64;
+        float b0 = 0.f, b1 = 0.f;   // second chain for instruction-level parallelism
+        int k = 0;
+        for (; k + 8 <= nk; k += 8) {
+#pragma unroll
+          for (int kk = 0; kk < 8; kk += 2) {
+            const float2 v0 = __bfloat1622float2(
+                *reinterpret_cast<const __nv_bfloat162*>(vst + (k + kk) * kAttRow + d2 * 2));
+            const float2 v1 = __bfloat1622float2(
+                *reinterpret_cast<const __nv_bfloat162*>(vst + (k + kk + 1) * kAttRow + d2 * 2));
+            a0 = fmaf(ph[k + kk], v0.x, a0);
+            a1 = fmaf(ph[k + kk], v0.y, a1);
+            b0 = fmaf(ph[k + kk + 1], v1.x, b0);
+            b1 = fmaf(ph[k + kk + 1], v1.y, b1);
+          }
+        }
+        for (; k < nk; ++k) {
+          const float2 v = __bfloat1622float2(
+              *reinterpret_cast<const __nv_bfloat162*>(vst + k * kAttRow + d2 * 2));
+          a0 = fmaf(ph[k], v.x, a0);
+          a1 = fmaf(ph[k], v.y, a1);
+        }
+        acc[u][0] = a0 + b0;
+        acc[u][1] = a1 + b1;
+      }
+    }
+    __syncthreads();   // stage and score buffer free again
+    if (tid == 0 && ok && issued < nblk) issue(issued++);
+  }
+  // no bulk copy may still be in flight at exit (normal path: every one was consumed)
+  if (tid == 0)
+    for (int m = max(0, issued - kAttStages); m < issued; ++m)
+      mbar_wait_drain(full + m % kAttStages, (m / kAttStages) & 1);
+  const size_t prow = (((size_t)b * Hkv + kv) * nsplit + split) * G;
+#pragma unroll
+  for (int u = 0; u < NP; ++u) {
+    const int o = tid + u * kDecThreads;
+    if (o < G * 64) {
+      const int h = o >> 6, d2 = (o & 63) * 2;
+      part_acc[(prow + h) * D + d2] = acc[u][0];
+      part_acc[(prow + h) * D + d2 + 1] = acc[u][1];
+    }
+  }
+  if (tid < G) {
+    part_ml[(prow + tid) * 2] = st_sm[tid];
+    part_ml[(prow + tid) * 2 + 1] = st_sm[8 + tid];
+  }
+}
+
 // (3) merge the splits (log2-domain maxima) and normalise.
 template <typename T, int D, int G>
 __global__ void decode_merge_kernel(const float* __restrict__ part_ml, const float* __restrict__ part_acc,
@@ -352,7 +613,7 @@ __global__ void decode_merge_kernel(const float* __restrict__ part_ml, const flo
 // ---------------------------------------------------------------------------------------
 int decode_nsplit(const sas_decode_problem& p) {
   const int pairs = p.batch * p.num_kv_heads;
-  int ns = (8 * 148 + pairs - 1) / pairs;
+  int ns = (4 * 148 + pairs - 1) / pairs;   // about 4 CTAs per SM, each a long stream
   if (ns < 1) ns = 1;
   if (ns > p.topk + 1) ns = p.topk + 1;
   return ns;
@@ -364,14 +625,34 @@ size_t decode_workspace_bytes(const sas_decode_problem& p) {
   const size_t ns = decode_nsplit(p);
   auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
   return al(pairs * (p.topk + 1) * 4) * 2 + al(pairs * ns * G * 2 * 4) +
-         al(pairs * ns * G * p.head_dim * 4);
+         al(pairs * ns * G * p.head_dim * 4) + 256;   // + error word
+}
+
+template <int G>
+static size_t decode_bulk_smem() {
+  return (size_t)kAttStages * kAttStage + (size_t)G * 128 * 4 + (size_t)G * 64 * 4 + 3 * 8 * 4 +
+         2 * 128 * 4 + kAttStages * 8 + 16 + 128;
 }
 
 template <typename T, int D, int G>
 static void decode_attn_launch(const sas_decode_problem& p, const void* q, const void* kc,
                                const void* vc, int32_t* sel_idx, float* sel_logg, float* part_ml,
-                               float* part_acc, void* o, int ns, cudaStream_t st) {
+                               float* part_acc, int* err, void* o, int ns, cudaStream_t st) {
   dim3 grid(p.num_kv_heads, p.batch, ns);
+  if constexpr (std::is_same<T, __nv_bfloat16>::value && D == 128) {
+    if (p.block <= 64) {   // bulk-copy streaming path
+      const size_t smem = decode_bulk_smem<G>();
+      cudaFuncSetAttribute(decode_attn_bulk_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem);
+      decode_attn_bulk_kernel<G><<<grid, kDecThreads, smem, st>>>(
+          (const __nv_bfloat16*)q, (const __nv_bfloat16*)kc, (const __nv_bfloat16*)vc, p.seqlens,
+          sel_idx, sel_logg, p.num_kv_heads, p.capacity, p.block, p.topk, ns,
+          kLog2e / sqrtf((float)D), part_ml, part_acc, err);
+      decode_merge_kernel<T, D, G><<<dim3(p.num_kv_heads, p.batch), 256, 0, st>>>(
+          part_ml, part_acc, p.num_kv_heads, ns, (T*)o);
+      return;
+    }
+  }
   decode_attn_kernel<T, D, G><<<grid, kDecThreads, 0, st>>>(
       (const T*)q, (const T*)kc, (const T*)vc, p.seqlens, sel_idx, sel_logg, p.num_kv_heads,
       p.capacity, p.block, p.topk, ns, kLog2e / sqrtf((float)D), part_ml, part_acc);
@@ -430,6 +711,8 @@ sas_status launch_decode(const sas_decode_problem& p, const void* q, const void*
   float* part_ml = (float*)w;
   w += al(pairs * ns * G * 2 * 4);
   float* part_acc = (float*)w;
+  w += al(pairs * ns * G * p.head_dim * 4);
+  int* err = (int*)w;
   if (p.dtype == SAS_BF16)
     decode_gate_launch<__nv_bfloat16>(p, q_nope, gkc, cur_pool, wq, qnorm_w, wk, knorm_w, sel_idx,
                                       sel_logg, idx_out, logg_out, st);
@@ -439,8 +722,8 @@ sas_status launch_decode(const sas_decode_problem& p, const void* q, const void*
   sas_status s = launch_status("decode gate", 1);
   if (s != SAS_OK) return s;
 #define SAS_DA(T, D, G)                                                                      \
-  decode_attn_launch<T, D, G>(p, q, k_cache, v_cache, sel_idx, sel_logg, part_ml, part_acc, o, \
-                              ns, st)
+  decode_attn_launch<T, D, G>(p, q, k_cache, v_cache, sel_idx, sel_logg, part_ml, part_acc, err, \
+                              o, ns, st)
 #define SAS_DA_G(T, D)                   \
   switch (G) {                           \
     case 1: SAS_DA(T, D, 1); break;      \
