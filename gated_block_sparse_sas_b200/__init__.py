@@ -209,6 +209,16 @@ def _workspace(fn, prob_ref, device):
     return torch.zeros(max(int(n.value), 256), dtype=torch.uint8, device=device)
 
 
+def attn_fwd_workspace(p: Problem):
+    """A zeroed workspace of the size sas_attn_fwd asks for (word 0: pipeline error code)."""
+    return _workspace(_lib.sas_attn_fwd_workspace_size, p.ref, p.device)
+
+
+def attn_bwd_workspace(p: Problem):
+    """A zeroed workspace of the size sas_attn_bwd asks for."""
+    return _workspace(_lib.sas_attn_bwd_workspace_size, p.ref, p.device)
+
+
 def sas_attn_fwd(p: Problem, q, k, v, idx, logg, o=None, lse=None, workspace=None, stream=None):
     if o is None:
         o = torch.empty((p.total_tokens, p.num_q_heads, p.head_dim), dtype=p.dtype, device=p.device)

@@ -172,7 +172,9 @@ sas_status sas_topk(const sas_problem* p, const float* scores, const float* lse,
 sas_status sas_attn_fwd_workspace_size(const sas_problem* p, size_t* bytes) {
   SAS_TRY(check_problem(p, false));
   SAS_CHECK_ARG(bytes != nullptr, "bytes is NULL");
-  *bytes = 256;   // word 0: pipeline error code of the tensor-core kernel (0 = none)
+  // word 0: pipeline error code of the tensor-core kernels (0 = none); the key-major path
+  // adds its accumulators, per-row references and inverted selection lists
+  *bytes = attn_fwd_km_supported(*p) ? attn_fwd_km_workspace_bytes(*p) : 256;
   return SAS_OK;
 }
 
@@ -188,11 +190,14 @@ sas_status sas_attn_fwd(const sas_problem* p, const void* q, const void* k, cons
   SAS_PTR(o);
   SAS_PTR(lse_attn);
   SAS_PTR(workspace);
-  if (workspace_bytes < 256) {
-    set_error("workspace too small: %zu < 256 bytes", workspace_bytes);
+  if (p->total_tokens == 0) return SAS_OK;
+  const size_t need = attn_fwd_km_supported(*p) ? attn_fwd_km_workspace_bytes(*p) : 256;
+  if (workspace_bytes < need) {
+    set_error("workspace too small: %zu < %zu bytes", workspace_bytes, need);
     return SAS_ERR_WORKSPACE;
   }
-  if (p->total_tokens == 0) return SAS_OK;
+  if (attn_fwd_km_supported(*p))
+    return launch_attn_fwd_km(*p, q, k, v, idx, logg, o, lse_attn, workspace, stream);
   if (attn_tc_supported(*p))
     return launch_attn_fwd_tc(*p, q, k, v, idx, logg, o, lse_attn, (int*)workspace, stream);
   return launch_attn_fwd_simt(*p, q, k, v, idx, logg, o, lse_attn, stream);

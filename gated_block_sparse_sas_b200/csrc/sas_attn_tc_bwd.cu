@@ -87,17 +87,6 @@ struct TcBwdArgs {
   float scale_log2, scale;
 };
 
-__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
-  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) &
-                                    ~static_cast<uintptr_t>(1023));
-}
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.wait_all;" ::: "memory");
-}
 
 // ---------------------------------------------------------------------------------------
 // pre-pass: bit t of pmask[b][kv][p] = token t of sequence b kept block 2p or 2p+1

@@ -44,6 +44,12 @@ sas_status launch_attn_fwd_tc(const sas_problem& p, const void* q, const void* k
                               const int32_t* idx, const float* logg, void* o, float* lse, int* err,
                               cudaStream_t st);
 
+bool attn_fwd_km_supported(const sas_problem& p);
+size_t attn_fwd_km_workspace_bytes(const sas_problem& p);
+sas_status launch_attn_fwd_km(const sas_problem& p, const void* q, const void* k, const void* v,
+                              const int32_t* idx, const float* logg, void* o, float* lse,
+                              void* workspace, cudaStream_t st);
+
 int decode_nsplit(const sas_decode_problem& p);
 size_t decode_workspace_bytes(const sas_decode_problem& p);
 sas_status launch_decode(const sas_decode_problem& p, const void* q, const void* q_nope,

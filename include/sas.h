@@ -160,7 +160,14 @@ sas_status sas_topk(const sas_problem* p, const float* scores, const float* lse,
  * O_t = softmax(z) V; lse_attn = natural-log logsumexp of z.
  * q dtype [T, Hq, d]; k, v dtype [T, Hkv, d] (rotated); idx/logg as from sas_topk
  * (any valid selection: ascending historical, current block, -1 padding);
- * o dtype [T, Hq, d]; lse_attn fp32 [T, Hq]. */
+ * o dtype [T, Hq, d]; lse_attn fp32 [T, Hq].
+ * Workspace: word 0 receives a pipeline error code (0 = none; checked by the caller after
+ * the stream completes). For bf16, d = 128, B = 64 the workspace also holds fp32 output
+ * accumulators [T, Hq, d + 1], per-row reference logits and the inverted selection lists
+ * (blocks -> kept tokens), about T*Hq*520 + T*Hkv*(K+1)*8 bytes. In that configuration the
+ * per-block partial sums are added with L2 reductions, so the low bits of o and lse_attn
+ * can change from run to run; a row whose largest logit exceeds the logit of its own key
+ * by more than ~97 nats sets error code 60 (its o is 0, lse_attn -inf). */
 sas_status sas_attn_fwd_workspace_size(const sas_problem* p, size_t* bytes);
 sas_status sas_attn_fwd(const sas_problem* p, const void* q, const void* k, const void* v,
                         const int32_t* idx, const float* logg, void* o, float* lse_attn,

@@ -43,7 +43,7 @@ def test_prefill_full_size_sampled(sas, name):
     dev = torch.device("cuda:0")
     g = si.prefill_inputs(shape, device=dev)
     prob = _problem(sas, shape, dev)
-    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    ws = sas.attn_fwd_workspace(prob)
     idx, logg = sas.prefill_selection(prob, g["q_nope"], g["k_nope"], g["wq"], g["qnorm_w"],
                                       g["wk"], g["knorm_w"])
     o, lse = sas.sas_attn_fwd(prob, g["q"], g["k"], g["v"], idx, logg, workspace=ws)

@@ -68,7 +68,7 @@ def test_gate_pipeline(sas, name):
 def test_attention_forward(sas, name):
     shape, inp, g, prob = _setup(sas, name, seed=200)
     idx, logg = si.random_selection(shape)
-    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    ws = sas.attn_fwd_workspace(prob)
     o, lse = sas.sas_attn_fwd(prob, g["q"], g["k"], g["v"], torch.from_numpy(idx).cuda(),
                               torch.from_numpy(logg).cuda(), workspace=ws)
     torch.cuda.synchronize()
@@ -78,6 +78,50 @@ def test_attention_forward(sas, name):
     fp32 = shape.dtype == "fp32"
     assert_out_close(o, O, fp32, "O")
     assert np.abs(to64(lse) - LSE).max() <= (1e-4 if fp32 else 2e-3)
+
+
+WINDOW_CASES = {
+    # lengths, Hq, Hkv, K: several 4096-token windows of the key-major forward, ragged tails,
+    # sequences shorter than a block, G = 4, 5, 8
+    "windows-G4": ([9000, 4100, 70], 8, 2, 7),
+    "windows-G5": ([4097, 5000, 1], 10, 2, 15),
+    "windows-G8": ([8200, 300], 16, 2, 31),
+}
+
+
+@pytest.mark.parametrize("name", list(WINDOW_CASES))
+def test_attention_forward_windows(sas, name):
+    """Forward over several token windows; every row of the GPU output is computed, the
+    oracle checks window edges, block edges, sequence ends and a random sample."""
+    lengths, Hq, Hkv, K = WINDOW_CASES[name]
+    shape = si.Shape(list(lengths), Hq, Hkv, 128, 64, K, 128, "bf16", seed=400)
+    inp = si.prefill_inputs(shape, with_dout=False)
+    dev = torch.device("cuda:0")
+    prob = sas.Problem.from_lengths(shape.lengths, dev, num_q_heads=Hq, num_kv_heads=Hkv,
+                                    head_dim=128, block=64, topk=K, gate_hidden=128,
+                                    dtype=torch.bfloat16)
+    idx, logg = si.random_selection(shape)
+    ws = sas.attn_fwd_workspace(prob)
+    o, lse = sas.sas_attn_fwd(prob, inp["q"].to(dev), inp["k"].to(dev), inp["v"].to(dev),
+                              torch.from_numpy(idx).to(dev), torch.from_numpy(logg).to(dev),
+                              workspace=ws)
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) == 0, "tensor-core pipeline reported an error"
+    o64, lse64 = to64(o), to64(lse)
+    assert np.isfinite(o64).all() and np.isfinite(lse64).all()
+    rng = np.random.default_rng(401)
+    rows = set()
+    for b, (s0, s1) in enumerate(zip(shape.cu_seqlens[:-1], shape.cu_seqlens[1:])):
+        L = int(s1 - s0)
+        for tl in (0, 1, 63, 64, 65, 4095, 4096, 4097, 8191, 8192, L - 2, L - 1):
+            if 0 <= tl < L:
+                rows.add(int(s0) + tl)
+    rows |= set(rng.choice(shape.total_tokens, 120, replace=False).tolist())
+    rows = np.array(sorted(rows))
+    O, LSE, _ = orc.attention_fwd(inp["q"], inp["k"], inp["v"], idx, logg, shape.cu_seqlens,
+                                  shape.block, rows=rows)
+    assert_out_close(o[torch.from_numpy(rows).to(dev)], O, False, "O")
+    assert np.abs(lse64[rows] - LSE).max() <= 2e-3
 
 
 @pytest.mark.parametrize("name", list(CASES))
