@@ -9,7 +9,7 @@
 //   S = Q K_j^T (M=128, N=64, K=128)
 //   P = 2^(S * log2e/sqrt(d) + log2e * log g_j - m_row)   (causal mask inside the current block)
 //   O_part = P V_j (M=128, N=128, K=64),  l_part = row sum of P (fp32, before rounding)
-// O_part and l_part are added into fp32 accumulators with L2 vector reductions. Splitting the
+// O_part and l_part are added into fp32 accumulators with L2 reductions. Splitting the
 // softmax sums over blocks this way is exact regrouping because each row uses ONE reference
 // m_row for all of its blocks (abstract: the gate enters the softmax in log form, so a
 // row's logits are z = q.k/sqrt(d) + log g whatever block they come from):
@@ -38,8 +38,9 @@
 //   warp 4      TMEM allocation; lane 0 issues the MMAs, S of tile n before PV of tile n-1.
 //   warps 8-11  softmax: TMEM lane r = tile row r; P as bf16 pairs over its S columns,
 //               l_part into a TMEM column once the epilogue has released tile n-2.
-//   warps 12-15 epilogue: O_part and l_part out of TMEM, through a row-major shared buffer,
-//               then one 512-byte red.global.add.v4.f32 per row and warp instruction.
+//   warps 12-15 epilogue: O_part and l_part out of TMEM; thread r writes row r to a shared
+//               buffer and hands it to the TMA unit as one 512-byte bulk fp32 reduction
+//               (cp.reduce.async.bulk .add.f32) into O_acc.
 // Every wait is bounded; a timeout records an error code in the workspace and all roles
 // wind down (copies drained, MMAs completed, TMEM released).
 #include <cuda.h>
@@ -540,6 +541,7 @@ __global__ void __launch_bounds__(kmf::kThreads, 1)
       if (!warp_wait(o_full + tb, (n >> 1) & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
       const uint32_t my_row = buf + (uint32_t)(lane * kEpiStride * 4);
+      bulk_wait_read0();   // the previous tile's reduction has read this row's buffer
 #pragma unroll 1
       for (int c0 = 0; c0 < kD; c0 += 32) {
         float v[32];
@@ -553,18 +555,15 @@ __global__ void __launch_bounds__(kmf::kThreads, 1)
       const float lsum = tmem_ld1(tmem + lane_addr + kColL + tb);
       tc_fence_before();
       mbar_arrive(o_empty + tb);   // TMEM buffer free for tile n+2
-      __syncwarp();
-#pragma unroll 4
-      for (int i = 0; i < 32; ++i) {   // row i of this warp: 32 lanes x 16 B = the whole row
-        const int drow = __shfl_sync(0xffffffffu, dst, i);
-        if (drow >= 0)
-          red_add_v4(a.oacc + (size_t)drow * kD + lane * 4,
-                     ld_shared_v4f(buf + (uint32_t)((i * kEpiStride + lane * 4) * 4)));
+      fence_async_smem();          // the row is read by the TMA unit (async proxy)
+      if (dst >= 0) {
+        bulk_reduce_add_f32(a.oacc + (size_t)dst * kD, my_row, kD * 4);
+        atomicAdd(a.lacc + dst, lsum);
       }
-      if (dst >= 0) atomicAdd(a.lacc + dst, lsum);
-      __syncwarp();
+      bulk_commit();
       mbar_arrive(rc_empty + rs);
     }
+    bulk_wait0();   // every reduction complete before the CTA exits
     if (!ok) tc_fail(a.err, 57, abort_flag);
   }
   tc_fence_before();
