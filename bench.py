@@ -195,38 +195,25 @@ def attended_pairs_gpu(idx: torch.Tensor, cu: torch.Tensor, block: int) -> int:
     return int(n.sum().item())
 
 
-def union_stats(idx: torch.Tensor, cu: torch.Tensor, lengths, Mq: int, Hkv: int, NBmax: int):
-    """Work the tensor-core kernels actually do on this selection.
+def km_stats(idx: torch.Tensor, cu: torch.Tensor, lengths, Mq: int, Hkv: int, NBmax: int):
+    """Work the key-major tensor-core kernels do on this selection.
 
-    U = sum over (tile of Mq tokens, kv head) of the number of distinct blocks its rows kept
-    (forward and query-major backward visit each once, 128 rows x 64 keys);
-    P = gathered 128-row tiles of the key-major backward: per (sequence, kv, block pair), the
-    tokens that kept a block of the pair, in tiles of Mq tokens (128 keys x 128 rows each).
+    Items are (kv head, sequence, 4096-token window, kept block); an item with c kept
+    (token, block) pairs runs ceil(c / Mq) gathered 128-row tiles. Returns (tiles, rows):
+    the tile count and the number of gathered (token, block) pairs (x G heads = MMA rows).
     """
     T = idx.shape[0]
     dev = idx.device
     cu64 = cu.long()
     tok = torch.arange(T, device=dev)
     seq = torch.searchsorted(cu64[1:], tok, right=True)
-    pos = tok - cu64[seq]
-    n_tiles = (max(lengths) + Mq - 1) // Mq
-    tile = seq * n_tiles + pos // Mq
+    w = (tok - cu64[seq]) // 4096
+    nW = (max(lengths) + 4095) // 4096
     j = idx.long()
     kvi = torch.arange(Hkv, device=dev)[None, :, None].expand_as(j)
-    nbp = NBmax + (NBmax & 1)
-    lin = (tile[:, None, None] * Hkv + kvi) * nbp + j.clamp(min=0)
-    mark = torch.zeros(len(lengths) * n_tiles * Hkv * nbp, dtype=torch.bool, device=dev)
-    mark[lin[j >= 0]] = True
-    m = mark.view(-1, nbp)
-    U = int(m.sum().item())
-    NP = nbp // 2
-    key = ((tok[:, None, None] * Hkv + kvi) * NP + (j.clamp(min=0) >> 1))[j >= 0]
-    key = torch.unique(key)
-    trow = key // (Hkv * NP)
-    grp = (seq[trow] * Hkv + (key // NP) % Hkv) * NP + key % NP
-    n_tok = torch.bincount(grp, minlength=len(lengths) * Hkv * NP)
-    P = int(((n_tok + Mq - 1) // Mq).sum().item())
-    return U, P
+    ent = ((kvi * len(lengths) + seq[:, None, None]) * nW + w[:, None, None]) * NBmax + j.clamp(min=0)
+    cnt = torch.bincount(ent[j >= 0], minlength=Hkv * len(lengths) * nW * NBmax)
+    return int(((cnt + Mq - 1) // Mq).sum().item()), int(cnt.sum().item())
 
 
 class Timer:
@@ -441,11 +428,12 @@ def main():
     fwd_flops = 4.0 * pairs * G * d
     bwd_flops = 2.5 * fwd_flops if backward else 0.0
     Mq = 25 if G == 5 else 128 // G
-    U, P = union_stats(out[2], prob.cu_seqlens, shape.lengths, Mq, shape.num_kv_heads,
-                       prob.max_blocks)
-    mma = 2.0 * 128 * 64 * d                           # one 128 x 64 x d product
-    comp_fwd = U * 2 * mma                             # QK^T + PV per visited block
-    comp_bwd = U * 3 * mma + P * 4 * (2.0 * 128 * 128 * d) if backward else 0.0
+    tiles, kept = km_stats(out[2], prob.cu_seqlens, shape.lengths, Mq, shape.num_kv_heads,
+                           prob.max_blocks)
+    mma = 2.0 * 128 * 64 * d                           # one 128-row x 64-key x d product
+    comp_fwd = tiles * 2 * mma                         # S = Q K^T, O = P V per gathered tile
+    comp_bwd = tiles * 5 * mma if backward else 0.0    # S, dP, dV^T, dK^T, dQ
+    red_bytes = kept * G * d * 4                       # fp32 partial rows reduced into L2
 
     timer = Timer()
     steps = []
@@ -494,12 +482,15 @@ def main():
                      "dense_causal_fraction": pairs / (shape.num_kv_heads * sum(
                          L * (L + 1) / 2 for L in shape.lengths))},
         "computed": {"fwd_tflop": comp_fwd / 1e12, "bwd_tflop": comp_bwd / 1e12,
-                     "union_blocks_per_tile": U / max(1, shape.num_kv_heads * sum(
-                         (L + Mq - 1) // Mq for L in shape.lengths)),
+                     "gathered_tiles": tiles,
                      "attended_over_computed": (fwd_flops + bwd_flops) / max(1.0, comp_fwd + comp_bwd),
                      "fwd_tflops": comp_fwd / (ops["sas_attn_fwd"] * 1e-3) / 1e12,
                      "bwd_tflops": (comp_bwd / (ops["sas_attn_bwd"] * 1e-3) / 1e12) if backward else None,
-                     "note": "tensor-core work of the tile-union kernels (rows x visited blocks)"},
+                     "l2_reduction_gb_per_pass": red_bytes / 1e9,
+                     "fwd_reduction_gbs": red_bytes / (ops["sas_attn_fwd"] * 1e-3) / 1e9,
+                     "note": "key-major kernels: gathered 128-row tiles per (kv, window, kept "
+                             "block); each kept (token, block) pair adds G fp32 rows of d "
+                             "values into L2 (O in the forward, dQ in the backward)"},
         "ops_ms": ops,
         "roofline": roof,
         "gpu_launches": launches,

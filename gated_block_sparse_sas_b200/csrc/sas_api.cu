@@ -87,12 +87,6 @@ static sas_status check_problem(const sas_problem* p, bool needs_rope) {
     SAS_CHECK_ARG(aligned16(ptr), "%s is not 16-byte aligned", #ptr);       \
   } while (0)
 
-#define SAS_TRY(expr)              \
-  do {                             \
-    sas_status s_ = (expr);        \
-    if (s_ != SAS_OK) return s_;   \
-  } while (0)
-
 }  // namespace sas
 
 using namespace sas;
@@ -206,6 +200,10 @@ sas_status sas_attn_fwd(const sas_problem* p, const void* q, const void* k, cons
 sas_status sas_attn_bwd_workspace_size(const sas_problem* p, size_t* bytes) {
   SAS_TRY(check_problem(p, false));
   SAS_CHECK_ARG(bytes != nullptr, "bytes is NULL");
+  if (attn_bwd_km_supported(*p)) {   // key-major path: accumulators and selection lists
+    *bytes = attn_bwd_km_workspace_bytes(*p);
+    return SAS_OK;
+  }
   // [256 B error word][D = rowsum(dO*O), fp32 T*Hq][per-tile union bitmasks (tensor-core path)]
   size_t n = 256 + ((((size_t)p->total_tokens * p->num_q_heads * sizeof(float)) + 255) & ~(size_t)255);
   if (attn_bwd_tc_supported(*p)) n += (attn_bwd_tc_tmask_bytes(*p) + 255) & ~(size_t)255;
@@ -241,6 +239,9 @@ sas_status sas_attn_bwd(const sas_problem* p, const void* q, const void* k, cons
     }
   }
   if (p->total_tokens == 0) return SAS_OK;
+  if (attn_bwd_km_supported(*p))
+    return launch_attn_bwd_km(*p, q, k, v, o, dout, lse_attn, idx, logg, dq, dk, dv, dlogg,
+                              workspace, stream);
   char* ws = (char*)workspace;
   int* err = (int*)ws;
   float* drow = (float*)(ws + 256);

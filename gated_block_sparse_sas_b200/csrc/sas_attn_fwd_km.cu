@@ -21,12 +21,8 @@
 // The finishing pass writes O = O_acc / l and LSE = (m_row + log2 l) ln 2. Summation order of
 // the reductions is not fixed, so results can differ in the last fp32 bits from run to run.
 //
-// Preparation (device only, no host synchronisation):
-//   row_ref  m_row per (token, query head)
-//   count    CTA per (window, sequence, kv head): shared-memory histogram of kept blocks
-//   scan     exclusive scan of the counts and the ascending list of non-empty items
-//   fill     CTA per (window, sequence, kv head): (token | slot << 24, log-gate) of every
-//            kept (token, block) pair, grouped by item (order inside an item arbitrary)
+// Preparation (device only, no host synchronisation): m_row per (token, query head), and
+// the inverted selection lists (sas_km.cuh).
 //
 // Main kernel: persistent, one CTA per SM; items are taken in ascending order from an atomic
 // counter, so the CTAs work on neighbouring windows and the accumulator rows they update stay
@@ -49,6 +45,7 @@
 
 #include "sas_common.cuh"
 #include "sas_kernels.h"
+#include "sas_km.cuh"
 #include "sas_sm100.cuh"
 
 namespace sas {
@@ -56,9 +53,6 @@ using namespace sm100;
 
 namespace kmf {
 constexpr int kD = 128, kB = 64, kM = 128;
-constexpr int kW = 4096;                 // tokens per window
-constexpr int kWB = kW / kB;             // blocks per window step (64)
-constexpr int kMaxBins = 2048;           // blocks a window can see (max_seqlen <= 131072)
 constexpr int kThreads = 512;
 constexpr float kRefShift = 32.f;        // m_row = own-key logit + 32 (log2 units)
 constexpr int kKVHalf = kB * 128;        // [64 keys][64 d] bf16, 128B rows: 8 KB
@@ -99,11 +93,6 @@ struct KmFwdArgs {
   float scale_log2;
 };
 
-// Entry index of (kv, sequence b, window w, block j < 64 (w+1)).
-__host__ __device__ __forceinline__ int km_entry(int kv, int b, int w, int j, int batch, int P) {
-  return (kv * batch + b) * P + kmf::kWB * (w * (w + 1) / 2) + j;
-}
-
 // ---------------------------------------------------------------------------------------
 // preparation
 // ---------------------------------------------------------------------------------------
@@ -141,101 +130,6 @@ __global__ void km_rowref_kernel(const __nv_bfloat16* __restrict__ q, const __nv
     const float2 q23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qr.y));
     const float dot = warp_sum(q01.x * k01.x + q01.y * k01.y + q23.x * k23.x + q23.y * k23.y);
     if (lane == 0) mref[row] = fmaf(dot, scale_log2, lg * kLog2e) + kmf::kRefShift;
-  }
-}
-
-// Histogram of the blocks kept by the tokens of window w of sequence b, kv head kv. Every
-// entry of the window (64 (w+1) blocks) is written, zeros included.
-__global__ void km_count_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ cu,
-                                int batch, int Hkv, int K, int P, int* __restrict__ cnt) {
-  __shared__ int hist[kmf::kMaxBins];
-  const int w = blockIdx.x, b = blockIdx.y, kv = blockIdx.z;
-  const int nbins = kmf::kWB * (w + 1);
-  for (int j = threadIdx.x; j < nbins; j += blockDim.x) hist[j] = 0;
-  __syncthreads();
-  const int s0 = cu[b], L = cu[b + 1] - s0;
-  const int t0 = w * kmf::kW, t1 = min(L, t0 + kmf::kW);
-  const int K1 = K + 1;
-  for (int e = threadIdx.x; e < (t1 - t0) * K1; e += blockDim.x) {   // empty when t0 >= L
-    const int tl = t0 + e / K1, s = e - (e / K1) * K1;
-    const int j = idx[((size_t)(s0 + tl) * Hkv + kv) * K1 + s];
-    if (j >= 0 && j < nbins) atomicAdd(&hist[j], 1);
-  }
-  __syncthreads();
-  const int base = km_entry(kv, b, w, 0, batch, P);
-  for (int j = threadIdx.x; j < nbins; j += blockDim.x) cnt[base + j] = hist[j];
-}
-
-// Exclusive scan of the E counts (one CTA of 1024 threads); ascending list of the non-empty
-// entries; ctl[0] = their number; the work counter is reset for the main kernel.
-__global__ void __launch_bounds__(1024) km_scan_kernel(const int* __restrict__ cnt, int E,
-                                                       int* __restrict__ off, int* __restrict__ items,
-                                                       int* __restrict__ ctl, int* __restrict__ next_item) {
-  __shared__ int ws_c[32], ws_n[32];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int per = (E + 1023) / 1024;
-  const int e0 = min(E, tid * per), e1 = min(E, e0 + per);
-  int sc = 0, sn = 0;
-  for (int e = e0; e < e1; ++e) {
-    const int c = cnt[e];
-    sc += c;
-    sn += c > 0;
-  }
-  int ic = sc, in = sn;   // inclusive warp scans
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int a = __shfl_up_sync(0xffffffffu, ic, o), bb = __shfl_up_sync(0xffffffffu, in, o);
-    if (lane >= o) { ic += a; in += bb; }
-  }
-  if (lane == 31) { ws_c[warp] = ic; ws_n[warp] = in; }
-  __syncthreads();
-  if (warp == 0) {
-    int vc = ws_c[lane], vn = ws_n[lane];
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int a = __shfl_up_sync(0xffffffffu, vc, o), bb = __shfl_up_sync(0xffffffffu, vn, o);
-      if (lane >= o) { vc += a; vn += bb; }
-    }
-    ws_c[lane] = vc;   // inclusive over warps
-    ws_n[lane] = vn;
-  }
-  __syncthreads();
-  int rc = ic - sc + (warp ? ws_c[warp - 1] : 0);
-  int rn = in - sn + (warp ? ws_n[warp - 1] : 0);
-  for (int e = e0; e < e1; ++e) {
-    const int c = cnt[e];
-    off[e] = rc;
-    rc += c;
-    if (c > 0) items[rn++] = e;
-  }
-  if (tid == 1023) {
-    ctl[0] = ws_n[31];
-    *next_item = 0;
-  }
-}
-
-// Place every kept (token, block) pair of window w at its item's next free position.
-__global__ void km_fill_kernel(const int32_t* __restrict__ idx, const float* __restrict__ logg,
-                               const int32_t* __restrict__ cu, int batch, int Hkv, int K, int P,
-                               const int* __restrict__ off, int2* __restrict__ list) {
-  __shared__ int cur[kmf::kMaxBins];
-  const int w = blockIdx.x, b = blockIdx.y, kv = blockIdx.z;
-  const int s0 = cu[b], L = cu[b + 1] - s0;
-  const int t0 = w * kmf::kW, t1 = min(L, t0 + kmf::kW);
-  if (t0 >= L) return;
-  const int nbins = kmf::kWB * (w + 1);
-  const int base = km_entry(kv, b, w, 0, batch, P);
-  for (int j = threadIdx.x; j < nbins; j += blockDim.x) cur[j] = off[base + j];
-  __syncthreads();
-  const int K1 = K + 1;
-  for (int e = threadIdx.x; e < (t1 - t0) * K1; e += blockDim.x) {
-    const int tl = t0 + e / K1, s = e - (e / K1) * K1;
-    const size_t gi = ((size_t)(s0 + tl) * Hkv + kv) * K1 + s;
-    const int j = idx[gi];
-    if (j >= 0 && j < nbins) {
-      const int pos = atomicAdd(&cur[j], 1);
-      list[pos] = make_int2((s0 + tl) | (s << 24), __float_as_int(logg[gi]));
-    }
   }
 }
 
@@ -342,11 +236,8 @@ __global__ void __launch_bounds__(kmf::kThreads, 1)
       if (stop) break;
       const int e = a.items[it];
       const int cnt = a.cnt[e], off = a.off[e];
-      const int kvb = e / a.P;
-      int rem = e - kvb * a.P, w = 0;
-      while (kWB * ((w + 1) * (w + 2) / 2) <= rem) ++w;
-      const int j = rem - kWB * (w * (w + 1) / 2);
-      const int kv = kvb / a.batch, b = kvb - kv * a.batch;
+      const km::Item itm = km::decode(e, a.batch, a.P);
+      const int kv = itm.kv, b = itm.b, j = itm.j;
       const int s0 = a.cu[b];
       const int kvs = item_seq & 1;
       if (r == 0 && ok) {   // this item's K/V block
@@ -579,48 +470,27 @@ __global__ void __launch_bounds__(kmf::kThreads, 1)
 // ---------------------------------------------------------------------------------------
 namespace {
 struct KmLayout {
-  size_t mref, oacc, lacc, cnt, off, items, ctl, list, total;
-  int nW, P, E;
+  size_t mref, oacc, lacc, lists, total;
 };
 
 size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 KmLayout km_layout(const sas_problem& p) {
   KmLayout L;
-  L.nW = (p.max_seqlen + kmf::kW - 1) / kmf::kW;
-  L.P = kmf::kWB * (L.nW * (L.nW + 1) / 2);
-  L.E = p.num_kv_heads * p.batch * L.P;
   const size_t rows = (size_t)p.total_tokens * p.num_q_heads;
   size_t o = 256;   // word 0: error code
   L.mref = o;  o += al256(rows * 4);
   L.oacc = o;  o += al256(rows * kmf::kD * 4);
   L.lacc = o;  o += al256(rows * 4);
-  L.cnt = o;   o += al256((size_t)L.E * 4);
-  L.off = o;   o += al256((size_t)L.E * 4);
-  L.items = o; o += al256((size_t)L.E * 4);
-  L.ctl = o;   o += 256;   // [0] items, [1] work counter
-  L.list = o;  o += al256((size_t)p.total_tokens * p.num_kv_heads * (p.topk + 1) * 8);
+  L.lists = o; o += km_lists_bytes(p);
   L.total = o;
   return L;
-}
-
-int sm_count() {
-  static int n = 0;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-      n = 148;
-  });
-  return n;
 }
 }  // namespace
 
 bool attn_fwd_km_supported(const sas_problem& p) {
   const int NBmax = (p.max_seqlen + p.block - 1) / p.block;
-  return attn_tc_supported(p) && p.max_seqlen <= kmf::kW * 32 && NBmax <= kmf::kMaxBins &&
-         p.total_tokens < (1 << 24) && p.topk + 1 <= 128;
+  return attn_tc_supported(p) && km_supported(p) && NBmax <= km::kMaxBins;
 }
 
 size_t attn_fwd_km_workspace_bytes(const sas_problem& p) { return km_layout(p).total; }
@@ -634,11 +504,7 @@ sas_status launch_attn_fwd_km(const sas_problem& p, const void* q, const void* k
   float* mref = reinterpret_cast<float*>(ws + L.mref);
   float* oacc = reinterpret_cast<float*>(ws + L.oacc);
   float* lacc = reinterpret_cast<float*>(ws + L.lacc);
-  int* cnt = reinterpret_cast<int*>(ws + L.cnt);
-  int* off = reinterpret_cast<int*>(ws + L.off);
-  int* items = reinterpret_cast<int*>(ws + L.items);
-  int* ctl = reinterpret_cast<int*>(ws + L.ctl);
-  int2* list = reinterpret_cast<int2*>(ws + L.list);
+  const KmLists lists = km_lists_carve(p, ws + L.lists);
   const int G = p.num_q_heads / p.num_kv_heads;
   const int Hkv = p.num_kv_heads;
   const int T = p.total_tokens;
@@ -651,7 +517,7 @@ sas_status launch_attn_fwd_km(const sas_problem& p, const void* q, const void* k
     return SAS_ERR_CUDA;
   }
   // O_acc and l_acc are adjacent: one clear
-  if (cudaMemsetAsync(oacc, 0, L.cnt - L.oacc, st) != cudaSuccess) {
+  if (cudaMemsetAsync(oacc, 0, L.lists - L.oacc, st) != cudaSuccess) {
     set_error("attn_fwd: clearing the accumulators failed");
     return SAS_ERR_CUDA;
   }
@@ -659,20 +525,17 @@ sas_status launch_attn_fwd_km(const sas_problem& p, const void* q, const void* k
   km_rowref_kernel<<<(wpr + 7) / 8, 256, 0, st>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
                                                   idx, logg, p.cu_seqlens, p.batch, T,
                                                   p.num_q_heads, Hkv, G, p.topk, scale_log2, mref);
-  const dim3 wgrid(L.nW, p.batch, Hkv);
-  km_count_kernel<<<wgrid, 512, 0, st>>>(idx, p.cu_seqlens, p.batch, Hkv, p.topk, L.P, cnt);
-  km_scan_kernel<<<1, 1024, 0, st>>>(cnt, L.E, off, items, ctl, ctl + 1);
-  km_fill_kernel<<<wgrid, 512, 0, st>>>(idx, logg, p.cu_seqlens, p.batch, Hkv, p.topk, L.P, off, list);
+  SAS_TRY(launch_km_lists(p, idx, logg, lists, st));
 
   KmFwdArgs a;
   a.cu = p.cu_seqlens;
   a.q = (const __nv_bfloat16*)q;
-  a.list = list;
-  a.cnt = cnt;
-  a.off = off;
-  a.items = items;
-  a.ctl = ctl;
-  a.next_item = ctl + 1;
+  a.list = lists.list;
+  a.cnt = lists.cnt;
+  a.off = lists.off;
+  a.items = lists.items;
+  a.ctl = lists.ctl;
+  a.next_item = lists.ctl + 1;
   a.mref = mref;
   a.oacc = oacc;
   a.lacc = lacc;
@@ -682,7 +545,7 @@ sas_status launch_attn_fwd_km(const sas_problem& p, const void* q, const void* k
   a.Hkv = Hkv;
   a.G = G;
   a.Mq = tc_rows_per_tile(G);
-  a.P = L.P;
+  a.P = lists.P;
   a.scale_log2 = scale_log2;
   static std::once_flag attr_once;
   std::call_once(attr_once, [] {
@@ -693,7 +556,7 @@ sas_status launch_attn_fwd_km(const sas_problem& p, const void* q, const void* k
   const int rows = T * p.num_q_heads;
   km_finalize_kernel<<<(rows + 7) / 8, 256, 0, st>>>(oacc, lacc, mref, rows,
                                                      (__nv_bfloat16*)o, lse, err);
-  return launch_status("attn_fwd (key-major tensor cores)", 6);
+  return launch_status("attn_fwd (key-major tensor cores)", 3);
 }
 
 }  // namespace sas

@@ -81,6 +81,13 @@ namespace sas {
 void set_error(const char* fmt, ...);
 sas_status launch_status(const char* what, int launches);
 void count_launches(int n);
+// Return the status of `expr` from the calling function unless it is SAS_OK.
+#define SAS_TRY(expr)              \
+  do {                             \
+    sas_status s_ = (expr);        \
+    if (s_ != SAS_OK) return s_;   \
+  } while (0)
+
 }  // namespace sas
 
 #define SAS_CHECK_ARG(cond, ...)                      \

@@ -5,6 +5,7 @@
 #include <stdint.h>
 
 #include <cuda.h>
+#include <vector_types.h>
 
 #include "sas.h"
 
@@ -44,11 +45,34 @@ sas_status launch_attn_fwd_tc(const sas_problem& p, const void* q, const void* k
                               const int32_t* idx, const float* logg, void* o, float* lse, int* err,
                               cudaStream_t st);
 
+// inverted selection lists of the key-major passes (sas_km.cuh)
+struct KmLists {
+  int* cnt;
+  int* off;
+  int* items;
+  int* ctl;      // [0] non-empty entries, [1] work counter
+  int2* list;
+  int nW, P, E;
+};
+bool km_supported(const sas_problem& p);
+size_t km_lists_bytes(const sas_problem& p);
+KmLists km_lists_carve(const sas_problem& p, uint8_t* base);
+sas_status launch_km_lists(const sas_problem& p, const int32_t* idx, const float* logg,
+                           const KmLists& L, cudaStream_t st);
+int sm_count();
+
 bool attn_fwd_km_supported(const sas_problem& p);
 size_t attn_fwd_km_workspace_bytes(const sas_problem& p);
 sas_status launch_attn_fwd_km(const sas_problem& p, const void* q, const void* k, const void* v,
                               const int32_t* idx, const float* logg, void* o, float* lse,
                               void* workspace, cudaStream_t st);
+
+bool attn_bwd_km_supported(const sas_problem& p);
+size_t attn_bwd_km_workspace_bytes(const sas_problem& p);
+sas_status launch_attn_bwd_km(const sas_problem& p, const void* q, const void* k, const void* v,
+                              const void* o, const void* dout, const float* lse,
+                              const int32_t* idx, const float* logg, void* dq, void* dk, void* dv,
+                              float* dlogg, void* workspace, cudaStream_t st);
 
 int decode_nsplit(const sas_decode_problem& p);
 size_t decode_workspace_bytes(const sas_decode_problem& p);

@@ -124,6 +124,59 @@ def test_attention_forward_windows(sas, name):
     assert np.abs(lse64[rows] - LSE).max() <= 2e-3
 
 
+@pytest.mark.parametrize("name", list(WINDOW_CASES))
+def test_attention_backward_windows(sas, name):
+    """Backward over several token windows: dQ/dlogg on window, block and sequence edges plus
+    random rows; dK/dV on first, middle and last (ragged) blocks of every sequence."""
+    lengths, Hq, Hkv, K = WINDOW_CASES[name]
+    shape = si.Shape(list(lengths), Hq, Hkv, 128, 64, K, 128, "bf16", seed=500)
+    inp = si.prefill_inputs(shape, with_dout=True)
+    dev = torch.device("cuda:0")
+    prob = sas.Problem.from_lengths(shape.lengths, dev, num_q_heads=Hq, num_kv_heads=Hkv,
+                                    head_dim=128, block=64, topk=K, gate_hidden=128,
+                                    dtype=torch.bfloat16)
+    g = {k: v.to(dev) for k, v in inp.items()}
+    idx, logg = si.random_selection(shape)
+    ti, tl = torch.from_numpy(idx).to(dev), torch.from_numpy(logg).to(dev)
+    o, lse = sas.sas_attn_fwd(prob, g["q"], g["k"], g["v"], ti, tl)
+    ws = sas.attn_bwd_workspace(prob)
+    dq, dk, dv, dl = sas.sas_attn_bwd(prob, g["q"], g["k"], g["v"], o, g["dout"], lse, ti, tl,
+                                      workspace=ws)
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) == 0, "tensor-core pipeline reported an error"
+    rng = np.random.default_rng(501)
+    rows = set()
+    cu = shape.cu_seqlens
+    for s0, s1 in zip(cu[:-1], cu[1:]):
+        L = int(s1 - s0)
+        for t in (0, 63, 64, 4095, 4096, 8191, 8192, L - 1):
+            if 0 <= t < L:
+                rows.add(int(s0) + t)
+    rows |= set(rng.choice(shape.total_tokens, 40, replace=False).tolist())
+    rows = np.array(sorted(rows))
+    dq_r, dl_r = orc.attention_bwd_rows(inp["q"], inp["k"], inp["v"], inp["dout"], idx, logg,
+                                        cu, shape.block, rows)
+    assert_grad_close(dq.cpu()[rows], dq_r, False, "dQ rows")
+    assert_grad_close(dl.cpu()[rows], dl_r, False, "dlogg rows")
+    assert (to64(dl)[idx < 0] == 0).all()
+    for b, (s0, s1) in enumerate(zip(cu[:-1], cu[1:])):
+        L = int(s1 - s0)
+        nb = (L + 63) // 64
+        for j, kv in sorted({(0, 0), (nb // 2, Hkv - 1), (nb - 1, 0)}):
+            lo, hi = j * 64, min((j + 1) * 64, L)
+            dk_r, dv_r = orc.attention_bwd_keys(inp["q"], inp["k"], inp["v"], inp["dout"], idx,
+                                                logg, cu, shape.block, b, kv, lo, hi)
+            gk = dk.cpu()[int(s0) + lo:int(s0) + hi, kv]
+            if np.linalg.norm(dk_r) < 1e-9:
+                # a one-token sequence: P = 1, so dS = dP - D = 0 and dK = 0 in exact
+                # arithmetic; only rounding noise of dP - D is left on the GPU
+                assert np.abs(to64(gk)).max() <= 1e-4, f"dK seq {b} block {j} not ~0"
+            else:
+                assert_grad_close(gk, dk_r, False, f"dK seq {b} block {j}")
+            assert_grad_close(dv.cpu()[int(s0) + lo:int(s0) + hi, kv], dv_r, False,
+                              f"dV seq {b} block {j}")
+
+
 @pytest.mark.parametrize("name", list(CASES))
 def test_attention_backward(sas, name):
     shape, inp, g, prob = _setup(sas, name, seed=300)
