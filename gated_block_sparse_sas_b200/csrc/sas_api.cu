@@ -192,8 +192,6 @@ sas_status sas_attn_fwd(const sas_problem* p, const void* q, const void* k, cons
   }
   if (attn_fwd_km_supported(*p))
     return launch_attn_fwd_km(*p, q, k, v, idx, logg, o, lse_attn, workspace, stream);
-  if (attn_tc_supported(*p))
-    return launch_attn_fwd_tc(*p, q, k, v, idx, logg, o, lse_attn, (int*)workspace, stream);
   return launch_attn_fwd_simt(*p, q, k, v, idx, logg, o, lse_attn, stream);
 }
 
@@ -204,10 +202,8 @@ sas_status sas_attn_bwd_workspace_size(const sas_problem* p, size_t* bytes) {
     *bytes = attn_bwd_km_workspace_bytes(*p);
     return SAS_OK;
   }
-  // [256 B error word][D = rowsum(dO*O), fp32 T*Hq][per-tile union bitmasks (tensor-core path)]
-  size_t n = 256 + ((((size_t)p->total_tokens * p->num_q_heads * sizeof(float)) + 255) & ~(size_t)255);
-  if (attn_bwd_tc_supported(*p)) n += (attn_bwd_tc_tmask_bytes(*p) + 255) & ~(size_t)255;
-  *bytes = n;
+  // [256 B error word][D = rowsum(dO*O), fp32 T*Hq] (CUDA-core path)
+  *bytes = 256 + ((((size_t)p->total_tokens * p->num_q_heads * sizeof(float)) + 255) & ~(size_t)255);
   return SAS_OK;
 }
 
@@ -242,16 +238,7 @@ sas_status sas_attn_bwd(const sas_problem* p, const void* q, const void* k, cons
   if (attn_bwd_km_supported(*p))
     return launch_attn_bwd_km(*p, q, k, v, o, dout, lse_attn, idx, logg, dq, dk, dv, dlogg,
                               workspace, stream);
-  char* ws = (char*)workspace;
-  int* err = (int*)ws;
-  float* drow = (float*)(ws + 256);
-  if (attn_bwd_tc_supported(*p)) {
-    uint32_t* tmask = (uint32_t*)(ws + 256 + ((((size_t)p->total_tokens * p->num_q_heads *
-                                                 sizeof(float)) + 255) & ~(size_t)255));
-    SAS_TRY(launch_rowdot(*p, o, dout, drow, stream));
-    return launch_attn_bwd_tc(*p, q, k, v, dout, lse_attn, drow, idx, logg, dq, dk, dv, dlogg,
-                              tmask, err, stream);
-  }
+  float* drow = (float*)((char*)workspace + 256);
   return launch_attn_bwd_simt(*p, q, k, v, o, dout, lse_attn, idx, logg, dq, dk, dv, dlogg, drow,
                               stream);
 }

@@ -24,9 +24,8 @@
 //               passes each item's K/V block to the loader.
 //   warp 5      K/V loader: lane 0 loads an item's K and V block by TMA into the single stage
 //               once the previous item's gradient MMAs have released it.
-//   warp 4      TMEM allocation; lane 0 issues the MMAs (S, dP of tile n before the gradient
-//               MMAs of tile n-1, except across an item boundary, where the K/V stage of the
-//               finished item must be released first).
+//   warp 4      TMEM allocation; lane 0 issues the MMAs, event-driven: S/dP of the next tile
+//               and the gradient MMAs of the oldest pending tile, each once its inputs are ready.
 //   warps 8-11  dS: TMEM lane r = row r: P and dS/sqrt(d) as bf16 into shared tiles (operands
 //               of the gradient MMAs); dlogg summed over the token's G rows.
 //   warps 12-15 epilogue: dQ of the tile from TMEM into the tile's own (now unused) Q/dO stage,
@@ -307,15 +306,12 @@ __global__ void __launch_bounds__(kmb::kThreads, 1)
       constexpr uint32_t kIdQ = idesc_bf16_f32(kM, kD, false, true);    // dQ
       const uint32_t k_addr = smem_u32(sm + OFF_K), v_addr = smem_u32(sm + OFF_V);
       const uint32_t p_addr = smem_u32(sm + OFF_P), ds_addr = smem_u32(sm + OFF_DS);
-      bool ok = true;
-      int item_seq = 0;
-      int pend = -1, pend_flags = 0, pend_item = 0;
-      auto grads = [&](int m, int flags, int item) -> bool {
-        if (!mbar_wait(ps_full, m & 1, abort_flag)) return false;
-        if (m >= 2 && !mbar_wait(dq_empty + (m & 1), ((m >> 1) - 1) & 1, abort_flag)) return false;
-        if ((flags & kFlagFirst) && item >= 1 && !mbar_wait(dkv_empty, (item - 1) & 1, abort_flag))
-          return false;
-        tc_fence_after();
+      // Event-driven issue: S/dP of the next tile and the gradient MMAs of the oldest
+      // pending tile are each issued as soon as their inputs are ready, so neither waits
+      // for the other's producer (the gather of tile n+1 does not hold up the gradients of
+      // tile n, and an item's last gradients release the K/V stage without waiting for the
+      // next item's block).
+      auto issue_grads = [&](int m, int flags) {
         const uint32_t q_addr = smem_u32(sm + OFF_QD + (m & 1) * kStage);
         const uint32_t do_addr = q_addr + kTile;
         const bool first = flags & kFlagFirst;
@@ -336,43 +332,68 @@ __global__ void __launch_bounds__(kmb::kThreads, 1)
         tc_commit(ps_empty);
         tc_commit(dq_full + (m & 1));
         if (flags & kFlagLast) tc_commit(kv_empty);
-        return true;
       };
-      int cur_item = 0;
-      for (int n = 0; ok; ++n) {
-        const int rs = n & 3, qs = n & 1;
-        if (!mbar_wait(rc_full + rs, (n >> 2) & 1, abort_flag)) { ok = false; break; }
-        const int flags = hdr[rs * 4];
-        if (flags & kFlagStop) break;
-        if (flags & kFlagFirst) {
-          // the previous item's last gradient MMAs release the single K/V stage that this
-          // item's block is loaded into: issue them before waiting for the load
-          if (pend >= 0 && !grads(pend, pend_flags, pend_item)) { ok = false; break; }
-          pend = -1;
-          if (!mbar_wait(kv_full, item_seq & 1, abort_flag)) { ok = false; break; }
-          cur_item = item_seq++;
-        }
-        if (!mbar_wait(qd_full + qs, (n >> 1) & 1, abort_flag)) { ok = false; break; }
-        if (n >= 1 && !mbar_wait(s_free, (n - 1) & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t q_addr = smem_u32(sm + OFF_QD + qs * kStage);
-        const uint32_t do_addr = q_addr + kTile;
+      bool ok = true, stop = false;
+      int n_s = 0, n_g = 0;          // next tile for S/dP, next tile for the gradients
+      int hflags = -1;               // header of tile n_s once read
+      int item_seq = 0, cur_item = 0;
+      int g_flags[4], g_item[4];     // tiles with S issued and gradients pending (n_g..n_s-1)
+      long long t_last = clock64();
+      while (true) {
+        bool progress = false;
+        if (!stop) {
+          const int rs = n_s & 3;
+          if (hflags < 0 && mbar_test(rc_full + rs, (n_s >> 2) & 1)) {
+            hflags = hdr[rs * 4];
+            if (hflags & kFlagStop) stop = true;
+          }
+          if (hflags >= 0 && !stop) {
+            bool ready = !(hflags & kFlagFirst) || mbar_test(kv_full, item_seq & 1);
+            ready = ready && mbar_test(qd_full + (n_s & 1), (n_s >> 1) & 1);
+            ready = ready && (n_s == 0 || mbar_test(s_free, (n_s - 1) & 1));
+            if (ready) {
+              if (hflags & kFlagFirst) cur_item = item_seq++;
+              tc_fence_after();
+              const uint32_t q_addr = smem_u32(sm + OFF_QD + (n_s & 1) * kStage);
+              const uint32_t do_addr = q_addr + kTile;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {   // S = Q K^T, dP = dO V^T (all K-major)
-          const uint32_t ro = (kk >> 2) * kHalf + (kk & 3) * 32;
-          const uint32_t ko = (kk >> 2) * kKVHalf + (kk & 3) * 32;
-          mma_bf16_ss(tmem + kColS, sdesc_sw128(q_addr + ro, 16, 1024),
-                      sdesc_sw128(k_addr + ko, 16, 1024), kIdS, kk > 0 ? 1u : 0u);
-          mma_bf16_ss(tmem + kColDP, sdesc_sw128(do_addr + ro, 16, 1024),
-                      sdesc_sw128(v_addr + ko, 16, 1024), kIdS, kk > 0 ? 1u : 0u);
+              for (int kk = 0; kk < 8; ++kk) {   // S = Q K^T, dP = dO V^T (all K-major)
+                const uint32_t ro = (kk >> 2) * kHalf + (kk & 3) * 32;
+                const uint32_t ko = (kk >> 2) * kKVHalf + (kk & 3) * 32;
+                mma_bf16_ss(tmem + kColS, sdesc_sw128(q_addr + ro, 16, 1024),
+                            sdesc_sw128(k_addr + ko, 16, 1024), kIdS, kk > 0 ? 1u : 0u);
+                mma_bf16_ss(tmem + kColDP, sdesc_sw128(do_addr + ro, 16, 1024),
+                            sdesc_sw128(v_addr + ko, 16, 1024), kIdS, kk > 0 ? 1u : 0u);
+              }
+              tc_commit(s_full);
+              g_flags[n_s & 3] = hflags;
+              g_item[n_s & 3] = cur_item;
+              ++n_s;
+              hflags = -1;
+              progress = true;
+            }
+          }
         }
-        tc_commit(s_full);
-        if (pend >= 0 && !grads(pend, pend_flags, pend_item)) { ok = false; break; }
-        pend = n;
-        pend_flags = flags;
-        pend_item = cur_item;
+        if (n_g < n_s) {
+          const int m = n_g, fl = g_flags[m & 3], it = g_item[m & 3];
+          bool ready = mbar_test(ps_full, m & 1);
+          ready = ready && (m < 2 || mbar_test(dq_empty + (m & 1), ((m >> 1) - 1) & 1));
+          ready = ready && (!(fl & kFlagFirst) || it < 1 || mbar_test(dkv_empty, (it - 1) & 1));
+          if (ready) {
+            tc_fence_after();
+            issue_grads(m, fl);
+            ++n_g;
+            progress = true;
+          }
+        }
+        if (stop && n_g == n_s) break;
+        if (progress) {
+          t_last = clock64();
+        } else if (*abort_flag || clock64() - t_last > kWaitCycles) {
+          ok = false;
+          break;
+        }
       }
-      if (ok && pend >= 0 && !grads(pend, pend_flags, pend_item)) ok = false;
       if (!ok) tc_fail(a.err, 75, abort_flag);
       tc_commit(final_bar);
       mbar_wait_drain(final_bar, 0);   // all MMAs done before the TMEM is released

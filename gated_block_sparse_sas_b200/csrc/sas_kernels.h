@@ -33,17 +33,8 @@ bool attn_tc_supported(const sas_problem& p);
 int tc_rows_per_tile(int G);
 bool make_tmap_bf16_3d(CUtensorMap* m, const void* base, uint64_t n0, uint64_t n1, uint64_t n2,
                        uint32_t b0, uint32_t b1, uint32_t b2);
-bool attn_bwd_tc_supported(const sas_problem& p);
-size_t attn_bwd_tc_tmask_bytes(const sas_problem& p);
-sas_status launch_attn_bwd_tc(const sas_problem& p, const void* q, const void* k, const void* v,
-                              const void* dout, const float* lse, const float* drow,
-                              const int32_t* idx, const float* logg, void* dq, void* dk, void* dv,
-                              float* dlogg, uint32_t* tmask, int* err, cudaStream_t st);
 sas_status launch_rowdot(const sas_problem& p, const void* o, const void* dout, float* drow,
                          cudaStream_t st);
-sas_status launch_attn_fwd_tc(const sas_problem& p, const void* q, const void* k, const void* v,
-                              const int32_t* idx, const float* logg, void* o, float* lse, int* err,
-                              cudaStream_t st);
 
 // inverted selection lists of the key-major passes (sas_km.cuh)
 struct KmLists {
