@@ -640,6 +640,12 @@ static void decode_attn_launch(const sas_decode_problem& p, const void* q, const
                                float* part_acc, int* err, void* o, int ns, cudaStream_t st) {
   dim3 grid(p.num_kv_heads, p.batch, ns);
   if constexpr (std::is_same<T, __nv_bfloat16>::value && D == 128) {
+    if (decode_attn_tc_supported(p)) {   // tensor-core path (sas_decode_tc.cu)
+      launch_decode_attn_tc(p, q, kc, vc, sel_idx, sel_logg, part_ml, part_acc, err, ns, st);
+      decode_merge_kernel<T, D, G><<<dim3(p.num_kv_heads, p.batch), 256, 0, st>>>(
+          part_ml, part_acc, p.num_kv_heads, ns, (T*)o);
+      return;
+    }
     if (p.block <= 64) {   // bulk-copy streaming path
       const size_t smem = decode_bulk_smem<G>();
       cudaFuncSetAttribute(decode_attn_bulk_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,

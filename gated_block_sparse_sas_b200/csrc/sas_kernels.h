@@ -65,6 +65,13 @@ sas_status launch_attn_bwd_km(const sas_problem& p, const void* q, const void* k
                               const int32_t* idx, const float* logg, void* dq, void* dk, void* dv,
                               float* dlogg, void* workspace, cudaStream_t st);
 
+bool tma_available();
+bool decode_attn_tc_supported(const sas_decode_problem& p);
+sas_status launch_decode_attn_tc(const sas_decode_problem& p, const void* q, const void* kc,
+                                 const void* vc, const int32_t* sel_idx, const float* sel_logg,
+                                 float* part_ml, float* part_acc, int* err, int ns,
+                                 cudaStream_t st);
+
 int decode_nsplit(const sas_decode_problem& p);
 size_t decode_workspace_bytes(const sas_decode_problem& p);
 sas_status launch_decode(const sas_decode_problem& p, const void* q, const void* q_nope,

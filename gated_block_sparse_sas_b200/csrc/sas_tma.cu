@@ -38,6 +38,8 @@ bool make_tmap_bf16_3d(CUtensorMap* m, const void* base, uint64_t n0, uint64_t n
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool tma_available() { return encode_fn() != nullptr; }
+
 // Tokens per 128-row tile: Mq tokens x G heads <= 128 (G = 5: 25 tokens, 125 rows).
 int tc_rows_per_tile(int G) { return G == 5 ? 25 : 128 / G; }
 
