@@ -62,7 +62,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_gate_kernel(
   float* xk = xq + H;                  // [H]
   float* s = xk + H;                   // [NBmax + 1]
   float* red = s + NBmax + 1;          // [kDecWarps]
-  int* cnt_red = reinterpret_cast<int*>(red + kDecWarps);  // [kDecWarps]
+  int* cnt_red = reinterpret_cast<int*>(red + kDecWarps);  // [2][kDecWarps]
 
   const int kv = blockIdx.x, b = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -79,6 +79,15 @@ __global__ void __launch_bounds__(kDecThreads) decode_gate_kernel(
     return;
   }
 
+  if (tid == 0 && c > 0) {   // start streaming this row's cached block keys into L2 now: the
+    // projections below take a while and the scores read these rows only afterwards
+    const char* src = reinterpret_cast<const char*>(gkc + ((size_t)b * Hkv + kv) * (size_t)NBmax * H);
+    const size_t bytes = (size_t)c * H * 2;   // a multiple of 16 (H >= 32)
+    for (size_t o = 0; o < bytes; o += 65536) {
+      const uint32_t n = (uint32_t)min((size_t)65536, bytes - o);
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src + o), "r"(n) : "memory");
+    }
+  }
   for (int e = tid; e < GD; e += kDecThreads)
     qcat[e] = to_f(q_nope[((size_t)b * Hq + (size_t)kv * G) * d + e]);
   for (int e = tid; e < C; e += kDecThreads) {
@@ -87,32 +96,76 @@ __global__ void __launch_bounds__(kDecThreads) decode_gate_kernel(
     P[e] = (part == 2) ? x / (float)n : x;
   }
   __syncthreads();
-  // projections: one warp per output channel (q channels, then k channels), lanes across the
-  // input with 16-byte loads of the weight row, so every row is read coalesced
-  // Four channels per warp step, all their weight loads issued before any arithmetic, so a
-  // warp has several L2 round trips in flight instead of one per channel.
-  for (int job0 = warp * 4; job0 < 2 * H; job0 += kDecWarps * 4) {
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    const bool isq = job0 < H;   // H is a multiple of 4: a step never mixes q and k channels
-    const float* x = isq ? qcat : P;
-    const int n_in = isq ? GD : C;
-    for (int e0 = lane * 8; e0 < n_in; e0 += 256) {
-      float w8[4][8];
+  // projections: warp-coalesced weight rows (lanes across the input, 16-byte loads), eight
+  // output channels per warp step with all their loads issued before any arithmetic
+  if constexpr (!std::is_same<T, __nv_bfloat16>::value) {   // fp32 weights: one row per step
+    for (int job = warp; job < 2 * H; job += kDecWarps) {
+      const bool isq = job < H;
+      const int i = isq ? job : job - H;
+      const T* w = isq ? wq + ((size_t)kv * H + i) * GD : wk + ((size_t)kv * H + i) * C;
+      const float* x = isq ? qcat : P;
+      const int n_in = isq ? GD : C;
+      float acc = 0.f;
+      for (int e0 = lane * 8; e0 < n_in; e0 += 256) {
+        float w8[8];
+        load8<T>(w + e0, w8);
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int i = (isq ? job0 : job0 - H) + u;
-        const T* w = isq ? wq + ((size_t)kv * H + i) * GD : wk + ((size_t)kv * H + i) * C;
-        load8<T>(w + e0, w8[u]);
+        for (int u = 0; u < 8; ++u) acc = fmaf(w8[u], x[e0 + u], acc);
+      }
+      acc = warp_sum(acc);
+      if (lane == 0) (isq ? xq : xk)[i] = acc;
+    }
+  } else {
+    constexpr int R = 8;
+    for (int job0 = warp * R; job0 < 2 * H; job0 += kDecWarps * R) {
+      const bool isq = job0 < H;   // H is a multiple of 8: a step never mixes q and k rows
+      const int i0 = isq ? job0 : job0 - H;
+      const T* w = isq ? wq + ((size_t)kv * H + i0) * GD : wk + ((size_t)kv * H + i0) * C;
+      const int n_in = isq ? GD : C;
+      const float* x = isq ? qcat : P;
+      const int nv = n_in / 8;   // 16-byte vectors per row
+      float acc[R];
+#pragma unroll
+      for (int u = 0; u < R; ++u) acc[u] = 0.f;
+      for (int v0 = 0; v0 < nv; v0 += 64) {   // two vectors per lane per row in flight
+        uint4 raw[R][2];
+#pragma unroll
+        for (int u = 0; u < R; ++u)
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int v = v0 + h2 * 32 + lane;
+            raw[u][h2] = v < nv ? __ldg(reinterpret_cast<const uint4*>(w + (size_t)u * n_in) + v)
+                                : make_uint4(0u, 0u, 0u, 0u);
+          }
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int v = v0 + h2 * 32 + lane;
+          if (v < nv) {
+            const float4 xa = *reinterpret_cast<const float4*>(x + v * 8);
+            const float4 xb = *reinterpret_cast<const float4*>(x + v * 8 + 4);
+#pragma unroll
+            for (int u = 0; u < R; ++u) {
+              float f[8];
+              const __nv_bfloat162* hh = reinterpret_cast<const __nv_bfloat162*>(&raw[u][h2]);
+#pragma unroll
+              for (int q2 = 0; q2 < 4; ++q2) {
+                const float2 ff = __bfloat1622float2(hh[q2]);
+                f[2 * q2] = ff.x;
+                f[2 * q2 + 1] = ff.y;
+              }
+              acc[u] = fmaf(f[0], xa.x, acc[u]); acc[u] = fmaf(f[1], xa.y, acc[u]);
+              acc[u] = fmaf(f[2], xa.z, acc[u]); acc[u] = fmaf(f[3], xa.w, acc[u]);
+              acc[u] = fmaf(f[4], xb.x, acc[u]); acc[u] = fmaf(f[5], xb.y, acc[u]);
+              acc[u] = fmaf(f[6], xb.z, acc[u]); acc[u] = fmaf(f[7], xb.w, acc[u]);
+            }
+          }
+        }
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-#pragma unroll
-        for (int v = 0; v < 8; ++v) acc[u] = fmaf(w8[u][v], x[e0 + v], acc[u]);
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const float r = warp_sum(acc[u]);
-      if (lane == 0) (isq ? xq : xk)[(isq ? job0 : job0 - H) + u] = r;
+      for (int u = 0; u < R; ++u) {
+        const float r = warp_sum(acc[u]);
+        if (lane == 0) (isq ? xq : xk)[i0 + u] = r;
+      }
     }
   }
   __syncthreads();
@@ -206,18 +259,20 @@ __global__ void __launch_bounds__(kDecThreads) decode_gate_kernel(
     key[r] = (j < c) ? order_key(s[j]) : 0u;
   }
   uint32_t thr = 0;
+  __syncthreads();   // s[] complete before the keys are read below; cnt_red free
 #pragma unroll 1
-  for (int bit = 31; bit >= 0; --bit) {
+  for (int bit = 31; bit >= 0; --bit) {   // counters double-buffered: one barrier per bit
     const uint32_t cand = thr | (1u << bit);
     int cn = 0;
 #pragma unroll
     for (int r = 0; r < NPT; ++r) cn += key[r] >= cand;
     cn = __reduce_add_sync(0xffffffffu, cn);
-    __syncthreads();
-    if (lane == 0) cnt_red[warp] = cn;
+    int* cb = cnt_red + (bit & 1) * kDecWarps;
+    if (lane == 0) cb[warp] = cn;
     __syncthreads();
     int tot = 0;
-    for (int w = 0; w < kDecWarps; ++w) tot += cnt_red[w];
+#pragma unroll
+    for (int w = 0; w < kDecWarps; ++w) tot += cb[w];
     if (tot >= K) thr = cand;
   }
   int gt = 0;
@@ -674,7 +729,7 @@ static void decode_gate_launch(const sas_decode_problem& p, const void* q_nope, 
   const int NBmax = (p.capacity + p.block - 1) / p.block;
   const int G = p.num_q_heads / p.num_kv_heads;
   const size_t smem = (size_t)(G * p.head_dim + 3 * p.head_dim + 2 * p.gate_hidden + NBmax + 1 +
-                               2 * kDecWarps) * sizeof(float);
+                               3 * kDecWarps) * sizeof(float);
   dim3 grid(p.num_kv_heads, p.batch);
 #define SAS_DG(H, NPT)                                                                           \
   {                                                                                              \
