@@ -12,7 +12,7 @@
 //   dV_j^T += dO^T P,  dK_j^T += Q^T dS / sqrt(d)     (M=128 d, N=64 keys, K=128 rows)
 //   dQ_rows = dS K_j / sqrt(d)                         (M=128 rows, N=128 d, K=64 keys)
 // dV^T and dK^T stay in TMEM over the item and are added to fp32 dK/dV accumulators at its
-// end; dQ of every tile is added to an fp32 accumulator with a TMA bulk reduction per row;
+// end; dQ of every tile is added to an fp32 accumulator with L2 vector reductions;
 // a last pass rounds the three accumulators to bf16. dlogg needs no reduction: each kept
 // (token, block) pair lives in exactly one tile. Summation order of the reductions is not
 // fixed, so gradients can differ in the last fp32 bits from run to run.
@@ -28,9 +28,10 @@
 //               and the gradient MMAs of the oldest pending tile, each once its inputs are ready.
 //   warps 8-11  dS: TMEM lane r = row r: P and dS/sqrt(d) as bf16 into shared tiles (operands
 //               of the gradient MMAs); dlogg summed over the token's G rows.
-//   warps 12-15 epilogue: dQ of the tile from TMEM into the tile's own (now unused) Q/dO stage,
-//               one 512-byte bulk fp32 reduction per row; at an item's end dK/dV from TMEM
-//               (lane = d, column = key) into the accumulators with coalesced reductions.
+//   warps 12-15 epilogue: dQ of the tile from TMEM, 32 columns at a time through a per-warp
+//               transpose buffer, into dQ_acc with coalesced red.global.add.v4.f32 (so a Q/dO
+//               stage is free as soon as the tile's gradient MMAs are done); at an item's end
+//               dK/dV from TMEM (lane = d, column = key) into the accumulators.
 // Every wait is bounded; a timeout records an error code in the workspace and all roles
 // wind down (copies drained, MMAs completed, TMEM released).
 #include <cuda.h>
@@ -50,8 +51,8 @@ constexpr int kD = 128, kB = 64, kM = 128;
 constexpr int kThreads = 512;
 constexpr int kHalf = kM * 128;              // [128 rows][64 d] bf16: 16 KB
 constexpr int kTile = 2 * kHalf;             // [128 rows][128 d] as two d halves: 32 KB
-constexpr int kStgStride = 132;              // floats per dQ staging row (528 B)
-constexpr int kStage = 2 * kTile + 3072;     // Q tile, dO tile; later the dQ staging (67584 B)
+constexpr int kStage = 2 * kTile;            // Q tile, dO tile
+constexpr int kEpiStride = 36;               // floats per row of a warp's dQ transpose buffer
 constexpr int kKVHalf = kB * 128;            // [64 keys][64 d]: 8 KB
 constexpr int OFF_QD = 0;                    // 2 stages
 constexpr int OFF_K = OFF_QD + 2 * kStage;   // [64 keys][128 d] as two halves
@@ -60,7 +61,8 @@ constexpr int OFF_P = OFF_V + 2 * kKVHalf;   // [128 rows][64 keys] bf16, 128B-s
 constexpr int OFF_DS = OFF_P + kM * 128;
 constexpr int kRcArrays = 5;                 // c1, D, limit, dst, dlogg index
 constexpr int OFF_RC = OFF_DS + kM * 128;    // [4 slots][5][128]
-constexpr int OFF_HDR = OFF_RC + 4 * kRcArrays * kM * 4;  // [4 slots][4]
+constexpr int OFF_EPI = OFF_RC + 4 * kRcArrays * kM * 4;  // [4 warps][32 rows][36] fp32
+constexpr int OFF_HDR = OFF_EPI + 4 * 32 * kEpiStride * 4; // [4 slots][4]
 constexpr int OFF_DESC = OFF_HDR + 4 * 4 * 4;             // [2 slots][2] item K/V rows, kv
 constexpr int OFF_BAR = OFF_DESC + 2 * 2 * 4;
 constexpr int kNumBars = 28;
@@ -132,7 +134,7 @@ __global__ void __launch_bounds__(kmb::kThreads, 1)
     mbar_init(kv_empty, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(qd_full + i, 128);
-      mbar_init(qd_empty + i, 128);
+      mbar_init(qd_empty + i, 1);
       mbar_init(dq_full + i, 1);
       mbar_init(dq_empty + i, 128);
     }
@@ -330,6 +332,7 @@ __global__ void __launch_bounds__(kmb::kThreads, 1)
           mma_bf16_ss(tmem + kColDQ + (m & 1) * kD, sdesc_sw128(ds_addr + kk * 32, 16, 1024),
                       sdesc_sw128(k_addr + kk * 2048, kKVHalf, 1024), kIdQ, kk > 0 ? 1u : 0u);
         tc_commit(ps_empty);
+        tc_commit(qd_empty + (m & 1));   // the tile's Q/dO stage is read by no later MMA
         tc_commit(dq_full + (m & 1));
         if (flags & kFlagLast) tc_commit(kv_empty);
       };
@@ -472,25 +475,34 @@ __global__ void __launch_bounds__(kmb::kThreads, 1)
       const int dst = rci[rc_slot(rs, 3) + r];
       if (!warp_wait(dq_full + qs, (n >> 1) & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      // the tile's Q/dO stage is no longer read by any MMA: it becomes the dQ staging
-      const uint32_t my_row = smem_u32(sm + OFF_QD + qs * kStage) + (uint32_t)(r * kStgStride * 4);
+      // dQ rows: 32 columns at a time through the warp's transpose buffer, then one
+      // red.global.add.v4.f32 per 4 rows x 128 bytes (8 lanes per row segment)
+      const uint32_t buf = smem_u32(sm + OFF_EPI) + (uint32_t)(ew * 32 * kEpiStride * 4);
+      const uint32_t my_row = buf + (uint32_t)(lane * kEpiStride * 4);
 #pragma unroll 1
       for (int c0 = 0; c0 < kD; c0 += 32) {
         float v[32];
         tmem_ld32(tmem + lane_addr + kColDQ + qs * kD + c0, v);
+        if (c0 == kD - 32) {
+          tc_fence_before();
+          mbar_arrive(dq_empty + qs);   // TMEM dQ buffer free for tile n+2
+        }
 #pragma unroll
         for (int i = 0; i < 8; ++i)
-          st_shared_v4(my_row + (uint32_t)((c0 + 4 * i) * 4), __float_as_uint(v[4 * i]),
+          st_shared_v4(my_row + (uint32_t)(4 * i * 4), __float_as_uint(v[4 * i]),
                        __float_as_uint(v[4 * i + 1]), __float_as_uint(v[4 * i + 2]),
                        __float_as_uint(v[4 * i + 3]));
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int row = i * 4 + (lane >> 3), seg = lane & 7;
+          const int drow = __shfl_sync(0xffffffffu, dst, row);
+          if (drow >= 0)
+            red_add_v4(a.dq_acc + (size_t)drow * kD + c0 + seg * 4,
+                       ld_shared_v4f(buf + (uint32_t)((row * kEpiStride + seg * 4) * 4)));
+        }
+        __syncwarp();
       }
-      tc_fence_before();
-      mbar_arrive(dq_empty + qs);   // TMEM dQ buffer free for tile n+2
-      fence_async_smem();
-      if (dst >= 0) bulk_reduce_add_f32(a.dq_acc + (size_t)dst * kD, my_row, kD * 4);
-      bulk_commit();
-      bulk_wait_read0();
-      mbar_arrive(qd_empty + qs);   // the stage may take tile n+2's rows
       if (flags & kFlagLast) {      // the item's dK^T, dV^T are complete (same commit as dQ)
         const int key0 = hdr[rs * 4 + 1], nkeys = hdr[rs * 4 + 2], kv = hdr[rs * 4 + 3];
         // thread r = TMEM lane r = channel d = r; column c = key c of the block
@@ -516,7 +528,6 @@ __global__ void __launch_bounds__(kmb::kThreads, 1)
       }
       mbar_arrive(rc_empty + rs);
     }
-    bulk_wait0();
     if (!ok) tc_fail(a.err, 77, abort_flag);
   }
   tc_fence_before();
