@@ -4,8 +4,9 @@
 // kernel and leave the selection in the workspace.
 //
 // CTA = (kv head, sequence, split of the kept-block slots). Kept blocks are taken in pairs
-// (128 keys): both blocks' K and V rows arrive by TMA (3-D boxes of 64 keys x 64 channels,
-// 128B swizzle) in a 2-stage ring, and per pair
+// (128 keys): both blocks' K rows, then their V rows, arrive by TMA (3-D boxes of 64 keys x 64
+// channels, 128B swizzle) into a ring of three 32 KB slots (K of pair n, V of pair n, K of pair
+// n+1, ...; two CTAs fit on an SM), and per pair
 //   S^T = K Q^T        (M = 128 keys, N = 16: the G query heads padded with zero rows, K = d)
 //   P   = 2^(S^T log2e/sqrt(d) + log2e log g_block - m_h)   (0 past the sequence end)
 //   O^T += V^T P        (M = 128 channels, N = 16, K = 128 keys), accumulated in TMEM.
@@ -34,18 +35,17 @@ constexpr int kD = 128, kB = 64;
 constexpr int kThreads = 256;
 constexpr int kHalfBlk = kB * 128;          // one block, one 64-channel half: [64 keys][128 B] = 8 KB
 constexpr int kHalfPair = 2 * kHalfBlk;     // both blocks of a pair, one half: [128 keys][128 B]
-constexpr int kKV = 2 * kHalfPair;          // K (or V) of a pair: 32 KB
-constexpr int kStage = 2 * kKV;             // K then V: 64 KB
-constexpr int kStages = 2;
+constexpr int kKV = 2 * kHalfPair;          // K (or V) of a pair: 32 KB = one ring slot
+constexpr int kSlots = 3;
 constexpr int kN = 16;                      // padded head count (MMA N)
 constexpr int OFF_STAGE = 0;
-constexpr int OFF_Q = kStages * kStage;     // [16 heads][128 d] K-major: 2 halves x 2 KB
+constexpr int OFF_Q = kSlots * kKV;         // [16 heads][128 d] K-major: 2 halves x 2 KB
 constexpr int OFF_P = OFF_Q + 2 * kN * 128; // 2 buffers x P^T [16 heads][128 keys]: 2 halves x 2 KB
 constexpr int OFF_BLK = OFF_P + 2 * 2 * kN * 128;   // [128] kept block ids, [128] log-gates (log2)
 constexpr int OFF_RED = OFF_BLK + 2 * 128 * 4;      // [4 warps][16] row-sum partials
 constexpr int OFF_MREF = OFF_RED + 4 * kN * 4;      // [16]
 constexpr int OFF_BAR = OFF_MREF + kN * 4;
-constexpr int kNumBars = 2 * kStages + 2 + 2 + 2 + 1;   // full, empty, s_full, p_full, p_empty, final
+constexpr int kNumBars = 2 * kSlots + 2 + 2 + 2 + 1;   // full, empty, s_full, p_full, p_empty, final
 constexpr int OFF_MISC = OFF_BAR + kNumBars * 8;
 constexpr int kSmemBytes = OFF_MISC + 64 + 1024;
 constexpr uint32_t kTmemCols = 64;          // S0 0..15, S1 16..31, O^T 32..47
@@ -65,7 +65,7 @@ struct DecTcArgs {
   float scale_log2;
 };
 
-__global__ void __launch_bounds__(dtc::kThreads, 1)
+__global__ void __launch_bounds__(dtc::kThreads, 2)
     decode_attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                           const DecTcArgs a) {
   using namespace dtc;
@@ -82,9 +82,9 @@ __global__ void __launch_bounds__(dtc::kThreads, 1)
   const size_t srow = ((size_t)b * a.Hkv + kv) * K1;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
-  uint64_t* full = bars;                 // [2]
-  uint64_t* empty = bars + kStages;      // [2]
-  uint64_t* s_full = bars + 2 * kStages; // [2]
+  uint64_t* full = bars;                 // [3] ring slots
+  uint64_t* empty = bars + kSlots;       // [3]
+  uint64_t* s_full = bars + 2 * kSlots;  // [2]
   uint64_t* p_full = s_full + 2;         // [2]
   uint64_t* p_empty = p_full + 2;        // [2]
   uint64_t* final_bar = p_empty + 2;
@@ -118,7 +118,7 @@ __global__ void __launch_bounds__(dtc::kThreads, 1)
     }
     if (lane == 0) {
       *nblk_s = n;
-      for (int i = 0; i < kStages; ++i) {
+      for (int i = 0; i < kSlots; ++i) {
         mbar_init(full + i, 1);
         mbar_init(empty + i, 1);
       }
@@ -192,28 +192,28 @@ __global__ void __launch_bounds__(dtc::kThreads, 1)
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
       const int z = b * a.Hkv + kv;
-      int issued = 0;
-      for (int n = 0; n < npairs; ++n) {
-        const int st = n & 1;
-        if (n >= kStages && !mbar_wait(empty + st, ((n >> 1) - 1) & 1, abort_flag)) {
+      int issued = 0;   // ring loads issued: load i = K (i even) or V (i odd) of pair i / 2
+      for (int i = 0; i < 2 * npairs; ++i) {
+        const int slot = i % kSlots;
+        if (i >= kSlots && !mbar_wait(empty + slot, ((i / kSlots) - 1) & 1, abort_flag)) {
           tc_fail(a.err, 81, abort_flag);
           break;
         }
-        uint8_t* stg = sm + OFF_STAGE + st * kStage;
+        const int n = i >> 1;
+        const CUtensorMap* map = (i & 1) ? &tmV : &tmK;
+        uint8_t* dst = sm + OFF_STAGE + slot * kKV;
         const int ja = blk_j[2 * n];
         const int jb = (2 * n + 1 < nblk) ? blk_j[2 * n + 1] : ja;   // odd count: masked copy
-        mbar_arrive_expect_tx(full + st, kStage);
+        mbar_arrive_expect_tx(full + slot, kKV);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          tma_load_3d(stg + h * kHalfPair, &tmK, full + st, 64 * h, ja * kB, z);
-          tma_load_3d(stg + h * kHalfPair + kHalfBlk, &tmK, full + st, 64 * h, jb * kB, z);
-          tma_load_3d(stg + kKV + h * kHalfPair, &tmV, full + st, 64 * h, ja * kB, z);
-          tma_load_3d(stg + kKV + h * kHalfPair + kHalfBlk, &tmV, full + st, 64 * h, jb * kB, z);
+          tma_load_3d(dst + h * kHalfPair, map, full + slot, 64 * h, ja * kB, z);
+          tma_load_3d(dst + h * kHalfPair + kHalfBlk, map, full + slot, 64 * h, jb * kB, z);
         }
-        issued = n + 1;
+        issued = i + 1;
       }
-      for (int n = max(0, issued - kStages); n < issued; ++n)   // none in flight at exit
-        mbar_wait_drain(full + (n & 1), (n >> 1) & 1);
+      for (int i = max(0, issued - kSlots); i < issued; ++i)   // none in flight at exit
+        mbar_wait_drain(full + i % kSlots, (i / kSlots) & 1);
     }
   } else if (warp == 1) {
     // ---------------- MMA issue ----------------
@@ -223,24 +223,26 @@ __global__ void __launch_bounds__(dtc::kThreads, 1)
       const uint32_t q_addr = smem_u32(sm + OFF_Q);
       bool ok = true;
       auto pv = [&](int m) -> bool {
+        const int vi = 2 * m + 1, vslot = vi % kSlots;
+        if (!mbar_wait(full + vslot, (vi / kSlots) & 1, abort_flag)) return false;
         if (!mbar_wait(p_full + (m & 1), (m >> 1) & 1, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t v_addr = smem_u32(sm + OFF_STAGE + (m & 1) * kStage + kKV);
+        const uint32_t v_addr = smem_u32(sm + OFF_STAGE + vslot * kKV);
         const uint32_t p_addr = smem_u32(sm + OFF_P + (m & 1) * 2 * kN * 128);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)   // 16 keys per step; A = V (MN-major), B = P^T (K-major)
           mma_bf16_ss(tmem + kColO, sdesc_sw128(v_addr + kk * 2048, kHalfPair, 1024),
                       sdesc_sw128(p_addr + (kk >> 2) * (kN * 128) + (kk & 3) * 32, 16, 1024),
                       kIdO, (m > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(empty + (m & 1));
+        tc_commit(empty + vslot);
         tc_commit(p_empty + (m & 1));
         return true;
       };
       for (int n = 0; n < npairs; ++n) {
-        const int st = n & 1;
-        if (!mbar_wait(full + st, (n >> 1) & 1, abort_flag)) { ok = false; break; }
+        const int st = n & 1, ki = 2 * n, kslot = ki % kSlots;
+        if (!mbar_wait(full + kslot, (ki / kSlots) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t k_addr = smem_u32(sm + OFF_STAGE + st * kStage);
+        const uint32_t k_addr = smem_u32(sm + OFF_STAGE + kslot * kKV);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)   // 16 channels per step
           mma_bf16_ss(tmem + kColS + st * kN,
@@ -248,6 +250,7 @@ __global__ void __launch_bounds__(dtc::kThreads, 1)
                       sdesc_sw128(q_addr + (kk >> 2) * (kN * 128) + (kk & 3) * 32, 16, 1024),
                       kIdS, kk > 0 ? 1u : 0u);
         tc_commit(s_full + st);
+        tc_commit(empty + kslot);   // K of pair n is read by no later MMA
         if (n >= 1 && !pv(n - 1)) { ok = false; break; }
       }
       if (ok && npairs >= 1 && !pv(npairs - 1)) ok = false;
@@ -292,12 +295,13 @@ __global__ void __launch_bounds__(dtc::kThreads, 1)
           *reinterpret_cast<__nv_bfloat16*>(pb + h * 128 + ((((kk >> 3) ^ (h & 7)) << 4) | ((kk & 7) << 1))) =
               __float2bfloat16_rn(p[h]);
       // keys past the sequence end (or of a missing block): V row := 0 once the copy has landed
-      if (__any_sync(0xffffffffu, !valid) && !warp_wait(full + st, (n >> 1) & 1, abort_flag)) {
+      const int vi = 2 * n + 1, vslot = vi % kSlots;
+      if (__any_sync(0xffffffffu, !valid) && !warp_wait(full + vslot, (vi / kSlots) & 1, abort_flag)) {
         ok = false;
         break;
       }
       if (!valid) {
-        uint8_t* vrow = sm + OFF_STAGE + st * kStage + kKV + (r >> 6) * kHalfBlk + (r & 63) * 128;
+        uint8_t* vrow = sm + OFF_STAGE + vslot * kKV + (r >> 6) * kHalfBlk + (r & 63) * 128;
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2)
 #pragma unroll
