@@ -245,7 +245,7 @@ def train_step(sas, prob, g, backward: bool, timer: Timer | None = None):
                                                         gate_keys=g["_gk"]))
     scores, lse = run("sas_gate_scores", lambda: sas.sas_gate_scores(
         prob, g["q_nope"], g["k_nope"], gk, g["wq"], g["qnorm_w"], g["wk"], g["knorm_w"],
-        scores=g["_scores"], lse=g["_glse"]))
+        scores=g["_scores"], lse=g["_glse"], workspace=g["_wsg"]))
     idx, logg = run("sas_topk", lambda: sas.sas_topk(prob, scores, lse, idx=g["_idx"],
                                                      logg=g["_logg"]))
     o, alse = run("sas_attn_fwd", lambda: sas.sas_attn_fwd(prob, g["q"], g["k"], g["v"], idx, logg,
@@ -275,6 +275,8 @@ def alloc_outputs(sas, prob, g, backward):
     g["_alse"] = torch.empty((T, Hq), dtype=torch.float32, device=dev)
     lib = sas.lib_handle()
     n = ctypes.c_size_t(0)
+    lib.sas_gate_scores_workspace_size(prob.ref, ctypes.byref(n))
+    g["_wsg"] = torch.empty(max(256, n.value), dtype=torch.uint8, device=dev)
     lib.sas_attn_fwd_workspace_size(prob.ref, ctypes.byref(n))
     g["_wsf"] = torch.empty(max(256, n.value), dtype=torch.uint8, device=dev)
     if backward:

@@ -50,7 +50,8 @@ _SIGS = {
     "sas_rope_tables": ([_i32, _i32, ctypes.c_double, _vp, _vp], ctypes.c_int),
     "sas_pool_keys": ([_P, _vp, _vp, _vp], ctypes.c_int),
     "sas_gate_keys": ([_P, _vp, _vp, _vp, _vp, _vp], ctypes.c_int),
-    "sas_gate_scores": ([_P] + [_vp] * 10, ctypes.c_int),
+    "sas_gate_scores_workspace_size": ([_P, ctypes.POINTER(_sz)], ctypes.c_int),
+    "sas_gate_scores": ([_P] + [_vp] * 9 + [_vp, _sz, _vp], ctypes.c_int),
     "sas_topk": ([_P, _vp, _vp, _vp, _vp, _vp], ctypes.c_int),
     "sas_attn_fwd_workspace_size": ([_P, ctypes.POINTER(_sz)], ctypes.c_int),
     "sas_attn_fwd": ([_P] + [_vp] * 8 + [_sz, _vp], ctypes.c_int),
@@ -178,16 +179,22 @@ def sas_gate_keys(p: Problem, pooled, wk, knorm_w, gate_keys=None, stream=None):
     return gate_keys
 
 
+def gate_scores_workspace(p: Problem):
+    """A workspace of the size sas_gate_scores asks for."""
+    return _workspace(_lib.sas_gate_scores_workspace_size, p.ref, p.device)
+
+
 def sas_gate_scores(p: Problem, q_nope, k_nope, gate_keys, wq, qnorm_w, wk, knorm_w,
-                    scores=None, lse=None, stream=None):
+                    scores=None, lse=None, workspace=None, stream=None):
     if scores is None:
         scores = torch.empty((p.total_tokens, p.num_kv_heads, p.max_blocks), dtype=torch.float32,
                              device=p.device)
     if lse is None:
         lse = torch.empty((p.total_tokens, p.num_kv_heads), dtype=torch.float32, device=p.device)
+    ws = workspace if workspace is not None else gate_scores_workspace(p)
     _check(_lib.sas_gate_scores(p.ref, _ptr(q_nope), _ptr(k_nope), _ptr(gate_keys), _ptr(wq),
                                 _ptr(qnorm_w), _ptr(wk), _ptr(knorm_w), _ptr(scores), _ptr(lse),
-                                _stream(stream)), "sas_gate_scores")
+                                _ptr(ws), ws.numel(), _stream(stream)), "sas_gate_scores")
     return scores, lse
 
 

@@ -133,10 +133,17 @@ sas_status sas_gate_keys(const sas_problem* p, const float* pooled, const void* 
   return launch_gate_keys(*p, pooled, wk, knorm_w, gate_keys, stream);
 }
 
+sas_status sas_gate_scores_workspace_size(const sas_problem* p, size_t* bytes) {
+  SAS_TRY(check_problem(p, true));
+  SAS_CHECK_ARG(bytes != nullptr, "bytes is NULL");
+  *bytes = gate_scores_workspace_bytes(*p);
+  return SAS_OK;
+}
+
 sas_status sas_gate_scores(const sas_problem* p, const void* q_nope, const void* k_nope,
                            const float* gate_keys, const void* wq, const float* qnorm_w,
                            const void* wk, const float* knorm_w, float* scores, float* lse,
-                           cudaStream_t stream) {
+                           void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   SAS_TRY(check_problem(p, true));
   SAS_PTR(q_nope);
   SAS_PTR(k_nope);
@@ -148,8 +155,14 @@ sas_status sas_gate_scores(const sas_problem* p, const void* q_nope, const void*
   SAS_PTR(scores);
   SAS_PTR(lse);
   if (p->total_tokens == 0) return SAS_OK;
+  SAS_PTR(workspace);
+  const size_t need = gate_scores_workspace_bytes(*p);
+  if (workspace_bytes < need) {
+    set_error("workspace too small: %zu < %zu bytes", workspace_bytes, need);
+    return SAS_ERR_WORKSPACE;
+  }
   return launch_gate_scores(*p, q_nope, k_nope, gate_keys, wq, qnorm_w, wk, knorm_w, scores, lse,
-                            stream);
+                            workspace, stream);
 }
 
 sas_status sas_topk(const sas_problem* p, const float* scores, const float* lse, int32_t* idx,

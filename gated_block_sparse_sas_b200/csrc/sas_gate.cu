@@ -8,6 +8,8 @@
 // bit for bit except at near-ties, so no reduced-precision tensor-core math here.
 #include <math.h>
 
+#include <mutex>
+
 #include "sas_common.cuh"
 #include "sas_kernels.h"
 
@@ -182,7 +184,7 @@ constexpr int kGsThreads = 256;
 constexpr int kKC = 32;         // reduction chunk of the query projection
 constexpr int kAP = kTQ + 4;    // padded row of transposed A tiles
 
-template <int H>
+template <int H, bool PROJ = false>
 struct GsSmem {
   // floats
   static constexpr int QT = H * kAP;                  // q~ transposed [H][kAP]
@@ -194,20 +196,23 @@ struct GsSmem {
   static constexpr int R1 = (P1 > X ? P1 : X);
   static constexpr int R2a = KT + P2;
   static constexpr int R2 = (R2a > X + KT ? R2a : X + KT);
-  static constexpr int RMAX0 = (R1 > R2 ? R1 : R2);
+  static constexpr int RMAX0 = PROJ ? X : (R1 > R2 ? R1 : R2);   // PROJ: only row staging
   static constexpr int RMAX = (RMAX0 > P3 ? RMAX0 : P3);
   static constexpr int TOTAL = QT + RMAX + kTQ;       // + s_cur[64]
 };
 
-template <typename T, int H>
+// PROJ: the two projections come precomputed (tensor-core GEMMs, sas_gate_tc.cu) as
+// qproj / kproj [T, Hkv, H] fp32, so phases 1 and 2 only load, normalise and rotate them.
+template <typename T, int H, bool PROJ>
 __global__ void __launch_bounds__(kGsThreads) gate_scores_kernel(
     const T* __restrict__ q_nope, const T* __restrict__ k_nope, const float* __restrict__ gkeys,
     const T* __restrict__ wq, const float* __restrict__ qnorm_w, const T* __restrict__ wk,
     const float* __restrict__ knorm_w, const int32_t* __restrict__ cu,
     const float* __restrict__ rc, const float* __restrict__ rs, int Hq, int Hkv, int d, int B,
-    int NBmax, float eps, float* __restrict__ scores, float* __restrict__ lse) {
+    int NBmax, float eps, const float* __restrict__ qproj, const float* __restrict__ kproj,
+    float* __restrict__ scores, float* __restrict__ lse) {
   extern __shared__ float smem[];
-  using S = GsSmem<H>;
+  using S = GsSmem<H, PROJ>;
   constexpr int NO = H / 16;   // outputs per thread in the 64 x H GEMMs
   float* Qt = smem;            // [H][kAP]
   float* R = smem + S::QT;     // phase-dependent region
@@ -223,7 +228,22 @@ __global__ void __launch_bounds__(kGsThreads) gate_scores_kernel(
   const int warp = tid >> 5, lane = tid & 31;
 
   // ---------------- phase 1: query projection ----------------
-  {
+  if constexpr (PROJ) {
+    float* X = R;  // [64][H+1]
+    for (int e = tid; e < kTQ * H; e += kGsThreads) {
+      const int t = e / H, c = e - t * H;
+      X[t * (H + 1) + c] = (t < nt) ? qproj[((size_t)(s0 + t0 + t) * Hkv + kv) * H + c] : 0.f;
+    }
+    __syncthreads();
+    for (int t = warp; t < kTQ; t += kGsThreads / 32) {
+      if (t < nt) {
+        norm_rope_row<H>(X + t * (H + 1), qnorm_w, eps, rc, rs, t0 + t, X + t * (H + 1), lane);
+      }
+      __syncwarp();
+      for (int e = lane; e < H; e += 32) Qt[e * kAP + t] = (t < nt) ? X[t * (H + 1) + e] : 0.f;
+    }
+    __syncthreads();
+  } else {
     float acc[4][NO];
 #pragma unroll
     for (int a = 0; a < 4; ++a)
@@ -283,7 +303,26 @@ __global__ void __launch_bounds__(kGsThreads) gate_scores_kernel(
   }
 
   // ---------------- phase 2: current-block keys ----------------
-  {
+  if constexpr (PROJ) {
+    float* X = R;  // [64][H+1]
+    for (int e = tid; e < kTQ * H; e += kGsThreads) {
+      const int t = e / H, c = e - t * H;
+      X[t * (H + 1) + c] = (t < nt) ? kproj[((size_t)(s0 + t0 + t) * Hkv + kv) * H + c] : 0.f;
+    }
+    __syncthreads();
+    for (int t = warp; t < kTQ; t += kGsThreads / 32) {
+      if (t < nt) {
+        const int cb = ((t0 + t) / B) * B;
+        norm_rope_row<H>(X + t * (H + 1), knorm_w, eps, rc, rs, cb, X + t * (H + 1), lane);
+        __syncwarp();
+        float dot = 0.f;
+        for (int e = lane; e < H; e += 32) dot += Qt[e * kAP + t] * X[t * (H + 1) + e];
+        dot = warp_sum(dot);
+        if (lane == 0) scur[t] = dot / sqrtf((float)H);
+      }
+    }
+    __syncthreads();
+  } else {
     float* KT = R;                       // [64][d+1] token keys of this kv head (fp32)
     float* As = R + S::KT;               // [64 pooled channels][kAP]
     float* Bs = As + 64 * kAP;           // [64][H+4]
@@ -436,18 +475,33 @@ template <typename T>
 static sas_status gate_scores_dispatch(const sas_problem& p, const void* q_nope, const void* k_nope,
                                        const float* gkeys, const void* wq, const float* qnorm_w,
                                        const void* wk, const float* knorm_w, float* scores,
-                                       float* lse, cudaStream_t st) {
+                                       float* lse, void* workspace, cudaStream_t st) {
   const int NBmax = (p.max_seqlen + p.block - 1) / p.block;
   dim3 grid((p.max_seqlen + kTQ - 1) / kTQ, p.batch, p.num_kv_heads);
+  if (gate_tc_supported(p)) {   // projections on the tensor cores, then norms, rotary, scores
+    float *qproj = nullptr, *kproj = nullptr;
+    SAS_TRY(launch_gate_proj_tc(p, q_nope, k_nope, wq, wk, workspace, &qproj, &kproj, st));
+    const size_t smem = (size_t)GsSmem<128, true>::TOTAL * sizeof(float);
+    static std::once_flag once;
+    std::call_once(once, [smem] {
+      cudaFuncSetAttribute(gate_scores_kernel<T, 128, true>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    });
+    gate_scores_kernel<T, 128, true><<<grid, kGsThreads, smem, st>>>(
+        (const T*)q_nope, (const T*)k_nope, gkeys, (const T*)wq, qnorm_w, (const T*)wk, knorm_w,
+        p.cu_seqlens, p.gate_rope_cos, p.gate_rope_sin, p.num_q_heads, p.num_kv_heads,
+        p.head_dim, p.block, NBmax, p.rms_eps, qproj, kproj, scores, lse);
+    return launch_status("gate_scores (tensor-core projections)", 4);
+  }
 #define SAS_GS(H)                                                                             \
   {                                                                                           \
     const size_t smem = (size_t)GsSmem<H>::TOTAL * sizeof(float);                             \
-    cudaFuncSetAttribute(gate_scores_kernel<T, H>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                         (int)smem);                                                          \
-    gate_scores_kernel<T, H><<<grid, kGsThreads, smem, st>>>(                                 \
+    cudaFuncSetAttribute(gate_scores_kernel<T, H, false>,                                     \
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);              \
+    gate_scores_kernel<T, H, false><<<grid, kGsThreads, smem, st>>>(                          \
         (const T*)q_nope, (const T*)k_nope, gkeys, (const T*)wq, qnorm_w, (const T*)wk,        \
         knorm_w, p.cu_seqlens, p.gate_rope_cos, p.gate_rope_sin, p.num_q_heads,               \
-        p.num_kv_heads, p.head_dim, p.block, NBmax, p.rms_eps, scores, lse);                   \
+        p.num_kv_heads, p.head_dim, p.block, NBmax, p.rms_eps, nullptr, nullptr, scores, lse); \
   }
   switch (p.gate_hidden) {
     case 32: SAS_GS(32); break;
@@ -458,15 +512,19 @@ static sas_status gate_scores_dispatch(const sas_problem& p, const void* q_nope,
   return launch_status("gate_scores", 1);
 }
 
+size_t gate_scores_workspace_bytes(const sas_problem& p) {
+  return gate_tc_supported(p) ? gate_tc_workspace_bytes(p) : 256;
+}
+
 sas_status launch_gate_scores(const sas_problem& p, const void* q_nope, const void* k_nope,
                               const float* gkeys, const void* wq, const float* qnorm_w,
                               const void* wk, const float* knorm_w, float* scores, float* lse,
-                              cudaStream_t st) {
+                              void* workspace, cudaStream_t st) {
   if (p.dtype == SAS_BF16)
     return gate_scores_dispatch<__nv_bfloat16>(p, q_nope, k_nope, gkeys, wq, qnorm_w, wk, knorm_w,
-                                               scores, lse, st);
+                                               scores, lse, workspace, st);
   return gate_scores_dispatch<float>(p, q_nope, k_nope, gkeys, wq, qnorm_w, wk, knorm_w, scores,
-                                     lse, st);
+                                     lse, workspace, st);
 }
 
 // ---------------------------------------------------------------------------------------

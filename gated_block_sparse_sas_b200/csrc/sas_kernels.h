@@ -14,10 +14,11 @@ namespace sas {
 sas_status launch_pool_keys(const sas_problem& p, const void* k_nope, float* pooled, cudaStream_t st);
 sas_status launch_gate_keys(const sas_problem& p, const float* pooled, const void* wk,
                             const float* knorm_w, float* gkeys, cudaStream_t st);
+size_t gate_scores_workspace_bytes(const sas_problem& p);
 sas_status launch_gate_scores(const sas_problem& p, const void* q_nope, const void* k_nope,
                               const float* gkeys, const void* wq, const float* qnorm_w,
                               const void* wk, const float* knorm_w, float* scores, float* lse,
-                              cudaStream_t st);
+                              void* workspace, cudaStream_t st);
 sas_status launch_topk(const sas_problem& p, const float* scores, const float* lse, int32_t* idx,
                        float* logg, cudaStream_t st);
 
@@ -66,6 +67,13 @@ sas_status launch_attn_bwd_km(const sas_problem& p, const void* q, const void* k
                               float* dlogg, void* workspace, cudaStream_t st);
 
 bool tma_available();
+bool make_tmap_bf16_2d(CUtensorMap* m, const void* base, uint64_t n0, uint64_t n1,
+                       uint64_t row_bytes, uint32_t b0, uint32_t b1);
+bool gate_tc_supported(const sas_problem& p);
+size_t gate_tc_workspace_bytes(const sas_problem& p);
+sas_status launch_gate_proj_tc(const sas_problem& p, const void* q_nope, const void* k_nope,
+                               const void* wq, const void* wk, void* workspace, float** qproj,
+                               float** kproj, cudaStream_t st);
 bool decode_attn_tc_supported(const sas_decode_problem& p);
 sas_status launch_decode_attn_tc(const sas_decode_problem& p, const void* q, const void* kc,
                                  const void* vc, const int32_t* sel_idx, const float* sel_logg,

@@ -140,11 +140,16 @@ sas_status sas_gate_keys(const sas_problem* p, const float* pooled, const void* 
  * k_nope, wk, knorm_w); s = -inf for j > c_t. lse[t, kv] = logsumexp_{j<=c_t} s.
  * q_nope dtype [T, Hq, d]; k_nope dtype [T, Hkv, d]; gate_keys fp32 [batch, NBmax,
  * Hkv, h]; wq dtype [Hkv, h, G*d]; wk dtype [Hkv, h, 3d]; qnorm_w, knorm_w fp32 [h];
- * scores fp32 [T, Hkv, NBmax]; lse fp32 [T, Hkv]. */
+ * scores fp32 [T, Hkv, NBmax]; lse fp32 [T, Hkv].
+ * Workspace (size from sas_gate_scores_workspace_size): for bf16, d = 128, h = 128 the two
+ * projections run as tensor-core GEMMs and the workspace holds their inputs and outputs
+ * (per token and kv head: the current block's prefix max, min and mean as exact bf16 parts,
+ * 1280 B, and the two projections, 1024 B); otherwise 256 B suffice. */
+sas_status sas_gate_scores_workspace_size(const sas_problem* p, size_t* bytes);
 sas_status sas_gate_scores(const sas_problem* p, const void* q_nope, const void* k_nope,
                            const float* gate_keys, const void* wq, const float* qnorm_w,
                            const void* wk, const float* knorm_w, float* scores, float* lse,
-                           cudaStream_t stream);
+                           void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /* A4 -- Top-K selection (README (b); model card: Training Top-K 31 historical blocks).
  * Per (t, kv): the min(K, c_t) historical blocks with the highest score (ties to

@@ -115,3 +115,17 @@ def test_empty_problem_is_a_no_op(sas):
     ptrs = [0x10000 + 0x100 * i for i in range(8)]
     assert lib.sas_attn_fwd(ctypes.byref(p), *ptrs[:7], 0x90000, 256, None) == 0
     assert lib.sas_topk(ctypes.byref(p), *ptrs[:4], None) == 0
+
+
+def test_binding_argument_counts_match_the_header(sas):
+    """Every ctypes signature of the binding takes as many arguments as include/sas.h
+    declares (a mismatch would pass a wrong stream or size without any error)."""
+    import re
+    src = open(os.path.join(ROOT, "include", "sas.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    decls = dict(re.findall(r"\b(sas_\w+)\s*\(([^)]*)\)\s*;", src))
+    assert decls, "no declarations parsed"
+    for name, (args, _res) in sas._SIGS.items():
+        params = decls[name].strip()
+        n = 0 if params in ("", "void") else params.count(",") + 1
+        assert n == len(args), f"{name}: header {n} parameters, binding {len(args)}"
