@@ -533,28 +533,11 @@ sas_status launch_gate_scores(const sas_problem& p, const void* q_nope, const vo
 // row is emitted in ascending block order with ballots: every key above the threshold,
 // plus the lowest-index ties at the threshold until K are kept.
 // ---------------------------------------------------------------------------------------
+// One row with c > K historical candidates held as NPL keys per lane (c <= 32 NPL).
 template <int NPL>
-__global__ void topk_kernel(const float* __restrict__ scores, const float* __restrict__ lse,
-                            const int32_t* __restrict__ cu, int batch, int T, int Hkv, int NBmax,
-                            int B, int K, int32_t* __restrict__ idx, float* __restrict__ logg) {
-  const int row = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= T * Hkv) return;
-  const int tg = row / Hkv;
-  const int b = seq_of(cu, batch, tg);
-  const int t = tg - cu[b];
-  const int c = t / B;
-  const float* srow = scores + (size_t)row * NBmax;
-  const float l = lse[row];
-  int32_t* irow = idx + (size_t)row * (K + 1);
-  float* grow = logg + (size_t)row * (K + 1);
-  if (c <= K) {
-    for (int s = lane; s <= K; s += 32) {
-      if (s <= c) { irow[s] = s; grow[s] = srow[s] - l; }
-      else { irow[s] = -1; grow[s] = 0.f; }
-    }
-    return;
-  }
+__device__ __forceinline__ void topk_row(const float* __restrict__ srow, float l, int c, int K,
+                                         int lane, int32_t* __restrict__ irow,
+                                         float* __restrict__ grow) {
   uint32_t key[NPL];
 #pragma unroll
   for (int r = 0; r < NPL; ++r) {
@@ -594,6 +577,39 @@ __global__ void topk_kernel(const float* __restrict__ scores, const float* __res
     out += __popc(selm);
     eq_seen += __popc(eqm);
   }
+}
+
+// The key count per lane follows the row's own candidate count c_t (warp-uniform), so the
+// work of a row scales with its visible blocks, not with the longest sequence. MAXNPL bounds
+// the instantiated sizes (and so the registers) by the problem's NBmax.
+template <int MAXNPL>
+__global__ void topk_kernel(const float* __restrict__ scores, const float* __restrict__ lse,
+                            const int32_t* __restrict__ cu, int batch, int T, int Hkv, int NBmax,
+                            int B, int K, int32_t* __restrict__ idx, float* __restrict__ logg) {
+  const int row = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= T * Hkv) return;
+  const int tg = row / Hkv;
+  const int b = seq_of(cu, batch, tg);
+  const int t = tg - cu[b];
+  const int c = t / B;
+  const float* srow = scores + (size_t)row * NBmax;
+  const float l = lse[row];
+  int32_t* irow = idx + (size_t)row * (K + 1);
+  float* grow = logg + (size_t)row * (K + 1);
+  if (c <= K) {
+    for (int s = lane; s <= K; s += 32) {
+      if (s <= c) { irow[s] = s; grow[s] = srow[s] - l; }
+      else { irow[s] = -1; grow[s] = 0.f; }
+    }
+    return;
+  }
+  if (MAXNPL <= 2 || c <= 64) topk_row<2>(srow, l, c, K, lane, irow, grow);
+  else if (MAXNPL <= 4 || c <= 128) topk_row<(MAXNPL < 4 ? MAXNPL : 4)>(srow, l, c, K, lane, irow, grow);
+  else if (MAXNPL <= 8 || c <= 256) topk_row<(MAXNPL < 8 ? MAXNPL : 8)>(srow, l, c, K, lane, irow, grow);
+  else if (MAXNPL <= 16 || c <= 512) topk_row<(MAXNPL < 16 ? MAXNPL : 16)>(srow, l, c, K, lane, irow, grow);
+  else if (MAXNPL <= 32 || c <= 1024) topk_row<(MAXNPL < 32 ? MAXNPL : 32)>(srow, l, c, K, lane, irow, grow);
+  else topk_row<MAXNPL>(srow, l, c, K, lane, irow, grow);
   if (lane == 0) {
     irow[K] = c;
     grow[K] = srow[c] - l;
@@ -611,6 +627,7 @@ sas_status launch_topk(const sas_problem& p, const float* scores, const float* l
                                            p.num_kv_heads, NBmax, p.block, p.topk, idx, logg)
   if (NBmax <= 64) SAS_TK(2);
   else if (NBmax <= 256) SAS_TK(8);
+  else if (NBmax <= 512) SAS_TK(16);
   else if (NBmax <= 1024) SAS_TK(32);
   else SAS_TK(64);
 #undef SAS_TK
