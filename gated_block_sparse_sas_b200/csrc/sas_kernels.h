@@ -42,6 +42,7 @@ struct KmLists {
   int* cnt;
   int* off;
   int* items;
+  int* cnt_q;    // per entry and window quarter
   int* ctl;      // [0] non-empty entries, [1] work counter
   int2* list;
   int nW, P, E;

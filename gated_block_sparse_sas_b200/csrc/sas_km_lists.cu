@@ -1,9 +1,11 @@
 // Construction of the inverted selection lists of the key-major attention passes (layout in
-// sas_km.cuh). Three launches, no global atomics and no host synchronisation:
-//   count  CTA per (window, sequence, kv head): shared-memory histogram of the kept blocks
-//   scan   one CTA: exclusive scan of the counts, ascending list of non-empty entries
-//   fill   CTA per (window, sequence, kv head): every kept (token, block) pair placed at its
-//          entry's next free position (order inside an entry arbitrary)
+// sas_km.cuh). Three launches and a clear, no host synchronisation:
+//   count  CTA per (window quarter, sequence, kv head): shared-memory histogram of the kept
+//          blocks of 1024 tokens; per-quarter counts, entry totals by global atomics
+//   scan   one CTA: exclusive scan of the entry totals, ascending list of non-empty entries
+//   fill   CTA per (window quarter, sequence, kv head): every kept (token, block) pair placed
+//          at its entry's offset + the counts of the window's earlier quarters + a shared
+//          atomic cursor (order inside an entry arbitrary)
 #include <mutex>
 
 #include "sas_common.cuh"
@@ -12,17 +14,22 @@
 
 namespace sas {
 
-// Histogram of the blocks kept by the tokens of window w of sequence b, kv head kv. Every
-// entry of the window (64 (w+1) blocks) is written, zeros included.
+constexpr int kQuarters = 4;   // CTAs per window
+constexpr int kQTok = km::kW / kQuarters;
+
+// Histogram of the blocks kept by the tokens of quarter q of window w of sequence b, kv head
+// kv: cnt_q[e][q] for every entry of the window (zeros included), cnt[e] += (cleared before).
 __global__ void km_count_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ cu,
-                                int batch, int Hkv, int K, int P, int* __restrict__ cnt) {
+                                int batch, int Hkv, int K, int P, int* __restrict__ cnt,
+                                int* __restrict__ cnt_q) {
   __shared__ int hist[km::kMaxBins];
-  const int w = blockIdx.x, b = blockIdx.y, kv = blockIdx.z;
+  const int w = blockIdx.x / kQuarters, qt = blockIdx.x - w * kQuarters;
+  const int b = blockIdx.y, kv = blockIdx.z;
   const int nbins = km::kWB * (w + 1);
   for (int j = threadIdx.x; j < nbins; j += blockDim.x) hist[j] = 0;
   __syncthreads();
   const int s0 = cu[b], L = cu[b + 1] - s0;
-  const int t0 = w * km::kW, t1 = min(L, t0 + km::kW);
+  const int t0 = w * km::kW + qt * kQTok, t1 = min(L, t0 + kQTok);
   const int K1 = K + 1;
   for (int e = threadIdx.x; e < (t1 - t0) * K1; e += blockDim.x) {   // empty when t0 >= L
     const int tl = t0 + e / K1, s = e - (e / K1) * K1;
@@ -31,7 +38,11 @@ __global__ void km_count_kernel(const int32_t* __restrict__ idx, const int32_t* 
   }
   __syncthreads();
   const int base = km::entry(kv, b, w, 0, batch, P);
-  for (int j = threadIdx.x; j < nbins; j += blockDim.x) cnt[base + j] = hist[j];
+  for (int j = threadIdx.x; j < nbins; j += blockDim.x) {
+    const int h = hist[j];
+    cnt_q[(size_t)(base + j) * kQuarters + qt] = h;
+    if (h) atomicAdd(cnt + base + j, h);
+  }
 }
 
 // Exclusive scan of the E counts (one CTA of 1024 threads); ascending list of the non-empty
@@ -82,18 +93,25 @@ __global__ void __launch_bounds__(1024) km_scan_kernel(const int* __restrict__ c
   }
 }
 
-// Place every kept (token, block) pair of window w at its entry's next free position.
+// Place every kept (token, block) pair of quarter q of window w at its entry's next free
+// position: entry offset + the earlier quarters' counts + a shared atomic cursor.
 __global__ void km_fill_kernel(const int32_t* __restrict__ idx, const float* __restrict__ logg,
                                const int32_t* __restrict__ cu, int batch, int Hkv, int K, int P,
-                               const int* __restrict__ off, int2* __restrict__ list) {
+                               const int* __restrict__ off, const int* __restrict__ cnt_q,
+                               int2* __restrict__ list) {
   __shared__ int cur[km::kMaxBins];
-  const int w = blockIdx.x, b = blockIdx.y, kv = blockIdx.z;
+  const int w = blockIdx.x / kQuarters, qt = blockIdx.x - w * kQuarters;
+  const int b = blockIdx.y, kv = blockIdx.z;
   const int s0 = cu[b], L = cu[b + 1] - s0;
-  const int t0 = w * km::kW, t1 = min(L, t0 + km::kW);
+  const int t0 = w * km::kW + qt * kQTok, t1 = min(L, t0 + kQTok);
   if (t0 >= L) return;
   const int nbins = km::kWB * (w + 1);
   const int base = km::entry(kv, b, w, 0, batch, P);
-  for (int j = threadIdx.x; j < nbins; j += blockDim.x) cur[j] = off[base + j];
+  for (int j = threadIdx.x; j < nbins; j += blockDim.x) {
+    int o = off[base + j];
+    for (int q = 0; q < qt; ++q) o += cnt_q[(size_t)(base + j) * kQuarters + q];
+    cur[j] = o;
+  }
   __syncthreads();
   const int K1 = K + 1;
   for (int e = threadIdx.x; e < (t1 - t0) * K1; e += blockDim.x) {
@@ -125,7 +143,7 @@ bool km_supported(const sas_problem& p) {
 size_t km_lists_bytes(const sas_problem& p) {
   int nW, P, E;
   km_dims(p, &nW, &P, &E);
-  return 3 * al256((size_t)E * 4) + 256 +
+  return 3 * al256((size_t)E * 4) + al256((size_t)E * kQuarters * 4) + 256 +
          al256((size_t)p.total_tokens * p.num_kv_heads * (p.topk + 1) * 8);
 }
 
@@ -136,6 +154,7 @@ KmLists km_lists_carve(const sas_problem& p, uint8_t* base) {
   L.cnt = reinterpret_cast<int*>(base + o);   o += al256((size_t)L.E * 4);
   L.off = reinterpret_cast<int*>(base + o);   o += al256((size_t)L.E * 4);
   L.items = reinterpret_cast<int*>(base + o); o += al256((size_t)L.E * 4);
+  L.cnt_q = reinterpret_cast<int*>(base + o); o += al256((size_t)L.E * kQuarters * 4);
   L.ctl = reinterpret_cast<int*>(base + o);   o += 256;
   L.list = reinterpret_cast<int2*>(base + o);
   return L;
@@ -143,12 +162,16 @@ KmLists km_lists_carve(const sas_problem& p, uint8_t* base) {
 
 sas_status launch_km_lists(const sas_problem& p, const int32_t* idx, const float* logg,
                            const KmLists& L, cudaStream_t st) {
-  const dim3 wgrid(L.nW, p.batch, p.num_kv_heads);
+  const dim3 wgrid(L.nW * kQuarters, p.batch, p.num_kv_heads);
+  if (cudaMemsetAsync(L.cnt, 0, (size_t)L.E * 4, st) != cudaSuccess) {
+    set_error("key-major lists: clearing the counts failed");
+    return SAS_ERR_CUDA;
+  }
   km_count_kernel<<<wgrid, 512, 0, st>>>(idx, p.cu_seqlens, p.batch, p.num_kv_heads, p.topk, L.P,
-                                         L.cnt);
+                                         L.cnt, L.cnt_q);
   km_scan_kernel<<<1, 1024, 0, st>>>(L.cnt, L.E, L.off, L.items, L.ctl);
   km_fill_kernel<<<wgrid, 512, 0, st>>>(idx, logg, p.cu_seqlens, p.batch, p.num_kv_heads, p.topk,
-                                        L.P, L.off, L.list);
+                                        L.P, L.off, L.cnt_q, L.list);
   return launch_status("key-major selection lists", 3);
 }
 
