@@ -28,10 +28,13 @@
 //               and the gradient MMAs of the oldest pending tile, each once its inputs are ready.
 //   warps 8-11  dS: TMEM lane r = row r: P and dS/sqrt(d) as bf16 into shared tiles (operands
 //               of the gradient MMAs); dlogg summed over the token's G rows.
-//   warps 12-15 epilogue: dQ of the tile from TMEM, 32 columns at a time through a per-warp
-//               transpose buffer, into dQ_acc with coalesced red.global.add.v4.f32 (so a Q/dO
-//               stage is free as soon as the tile's gradient MMAs are done); at an item's end
-//               dK/dV from TMEM (lane = d, column = key) into the accumulators.
+//   warps 12-15 epilogue: dQ of the tile from TMEM, 32 columns at a time, into a dense per-warp
+//               buffer [32 rows][32 columns] (each lane's 16-byte pieces rotated by lane so the
+//               stores hit distinct banks), then one TMA tensor reduction (cp.reduce.async.bulk
+//               .tensor .add, fp32) per token: the G rows of a token are its G adjacent query
+//               heads in dQ_acc (a Q/dO stage is free as soon as the tile's gradient MMAs are
+//               done); at an item's end dK/dV from TMEM (lane = d, column = key) into the
+//               accumulators.
 // Every wait is bounded; a timeout records an error code in the workspace and all roles
 // wind down (copies drained, MMAs completed, TMEM released).
 #include <cuda.h>
@@ -52,7 +55,7 @@ constexpr int kThreads = 512;
 constexpr int kHalf = kM * 128;              // [128 rows][64 d] bf16: 16 KB
 constexpr int kTile = 2 * kHalf;             // [128 rows][128 d] as two d halves: 32 KB
 constexpr int kStage = 2 * kTile;            // Q tile, dO tile
-constexpr int kEpiStride = 36;               // floats per row of a warp's dQ transpose buffer
+constexpr int kEpiBytes = 32 * 32 * 4;       // a warp's dQ buffer: [32 rows][32 fp32 columns]
 constexpr int kKVHalf = kB * 128;            // [64 keys][64 d]: 8 KB
 constexpr int OFF_QD = 0;                    // 2 stages
 constexpr int OFF_K = OFF_QD + 2 * kStage;   // [64 keys][128 d] as two halves
@@ -61,8 +64,8 @@ constexpr int OFF_P = OFF_V + 2 * kKVHalf;   // [128 rows][64 keys] bf16, 128B-s
 constexpr int OFF_DS = OFF_P + kM * 128;
 constexpr int kRcArrays = 5;                 // c1, D, limit, dst, dlogg index
 constexpr int OFF_RC = OFF_DS + kM * 128;    // [4 slots][5][128]
-constexpr int OFF_EPI = OFF_RC + 4 * kRcArrays * kM * 4;  // [4 warps][32 rows][36] fp32
-constexpr int OFF_HDR = OFF_EPI + 4 * 32 * kEpiStride * 4; // [4 slots][4]
+constexpr int OFF_EPI = OFF_RC + 4 * kRcArrays * kM * 4;  // [4 warps][32 rows][32] fp32
+constexpr int OFF_HDR = OFF_EPI + 4 * kEpiBytes;           // [4 slots][4]
 constexpr int OFF_DESC = OFF_HDR + 4 * 4 * 4;             // [2 slots][2] item K/V rows, kv
 constexpr int OFF_BAR = OFF_DESC + 2 * 2 * 4;
 constexpr int kNumBars = 28;
@@ -97,7 +100,7 @@ struct KmBwdArgs {
 
 __global__ void __launch_bounds__(kmb::kThreads, 1)
     attn_bwd_km_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                       const KmBwdArgs a) {
+                       const __grid_constant__ CUtensorMap tmDQ, const KmBwdArgs a) {
   using namespace kmb;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
@@ -466,6 +469,13 @@ __global__ void __launch_bounds__(kmb::kThreads, 1)
     // ------------------------------ epilogue ------------------------------
     const int r = tid - 384, ew = warp - 12;
     const uint32_t lane_addr = (uint32_t)(ew * 32) << 16;
+    // one reduction box per token (its G rows) when G divides 32, so no token straddles two
+    // warps; otherwise one box per row
+    const int Gb = (32 % G) == 0 ? G : 1;
+    const bool issuer = (lane % Gb) == 0;
+    const int rot = lane & 7;
+    const uint32_t my_row = smem_u32(sm + OFF_EPI) + (uint32_t)(ew * kEpiBytes + lane * 128);
+    if (lane == 0) prefetch_tmap(&tmDQ);
     bool ok = true;
     for (int n = 0;; ++n) {
       const int rs = n & 3, qs = n & 1;
@@ -475,10 +485,7 @@ __global__ void __launch_bounds__(kmb::kThreads, 1)
       const int dst = rci[rc_slot(rs, 3) + r];
       if (!warp_wait(dq_full + qs, (n >> 1) & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      // dQ rows: 32 columns at a time through the warp's transpose buffer, then one
-      // red.global.add.v4.f32 per 4 rows x 128 bytes (8 lanes per row segment)
-      const uint32_t buf = smem_u32(sm + OFF_EPI) + (uint32_t)(ew * 32 * kEpiStride * 4);
-      const uint32_t my_row = buf + (uint32_t)(lane * kEpiStride * 4);
+      const int tok = dst >= 0 ? dst / a.Hq : 0, head = dst - tok * a.Hq;
 #pragma unroll 1
       for (int c0 = 0; c0 < kD; c0 += 32) {
         float v[32];
@@ -487,21 +494,34 @@ __global__ void __launch_bounds__(kmb::kThreads, 1)
           tc_fence_before();
           mbar_arrive(dq_empty + qs);   // TMEM dQ buffer free for tile n+2
         }
+        // piece k of the store sequence is column group (k + rot) & 7 of this lane's row
+        float4 w[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) w[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+#pragma unroll
+        for (int b = 1; b < 8; b <<= 1) {
+          const bool on = (rot & b) != 0;
+          float4 t[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) t[i] = w[(i + b) & 7];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            w[i].x = on ? t[i].x : w[i].x;
+            w[i].y = on ? t[i].y : w[i].y;
+            w[i].z = on ? t[i].z : w[i].z;
+            w[i].w = on ? t[i].w : w[i].w;
+          }
+        }
+        bulk_wait_read0();   // the previous chunk's reductions have read the buffer
+        __syncwarp();
 #pragma unroll
         for (int i = 0; i < 8; ++i)
-          st_shared_v4(my_row + (uint32_t)(4 * i * 4), __float_as_uint(v[4 * i]),
-                       __float_as_uint(v[4 * i + 1]), __float_as_uint(v[4 * i + 2]),
-                       __float_as_uint(v[4 * i + 3]));
+          st_shared_v4(my_row + (uint32_t)(((i + rot) & 7) << 4), __float_as_uint(w[i].x),
+                       __float_as_uint(w[i].y), __float_as_uint(w[i].z), __float_as_uint(w[i].w));
+        fence_async_smem();   // the rows are read by the TMA unit (async proxy)
         __syncwarp();
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int row = i * 4 + (lane >> 3), seg = lane & 7;
-          const int drow = __shfl_sync(0xffffffffu, dst, row);
-          if (drow >= 0)
-            red_add_v4(a.dq_acc + (size_t)drow * kD + c0 + seg * 4,
-                       ld_shared_v4f(buf + (uint32_t)((row * kEpiStride + seg * 4) * 4)));
-        }
-        __syncwarp();
+        if (issuer && dst >= 0) tma_reduce_add_3d(&tmDQ, my_row, c0, head, tok);
+        bulk_commit();
       }
       if (flags & kFlagLast) {      // the item's dK^T, dV^T are complete (same commit as dQ)
         const int key0 = hdr[rs * 4 + 1], nkeys = hdr[rs * 4 + 2], kv = hdr[rs * 4 + 3];
@@ -528,6 +548,7 @@ __global__ void __launch_bounds__(kmb::kThreads, 1)
       }
       mbar_arrive(rc_empty + rs);
     }
+    bulk_wait0();   // every reduction complete before the CTA exits
     if (!ok) tc_fail(a.err, 77, abort_flag);
   }
   tc_fence_before();
@@ -593,9 +614,11 @@ sas_status launch_attn_bwd_km(const sas_problem& p, const void* q, const void* k
   const int Hkv = p.num_kv_heads;
   const int T = p.total_tokens;
 
-  CUtensorMap tk, tv;
+  CUtensorMap tk, tv, tdq;
+  const uint32_t box_rows = (32 % G) == 0 ? (uint32_t)G : 1u;   // the epilogue's box per token
   if (!make_tmap_bf16_3d(&tk, k, 128, Hkv, T, 64, 1, 64) ||
-      !make_tmap_bf16_3d(&tv, v, 128, Hkv, T, 64, 1, 64)) {
+      !make_tmap_bf16_3d(&tv, v, 128, Hkv, T, 64, 1, 64) ||
+      !make_tmap_f32_3d(&tdq, dq_acc, 128, p.num_q_heads, T, 32, box_rows, 1)) {
     set_error("attn_bwd: TMA descriptor creation failed");
     return SAS_ERR_CUDA;
   }
@@ -638,7 +661,7 @@ sas_status launch_attn_bwd_km(const sas_problem& p, const void* q, const void* k
     cudaFuncSetAttribute(attn_bwd_km_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          kmb::kSmemBytes);
   });
-  attn_bwd_km_kernel<<<sm_count(), kmb::kThreads, kmb::kSmemBytes, st>>>(tk, tv, a);
+  attn_bwd_km_kernel<<<sm_count(), kmb::kThreads, kmb::kSmemBytes, st>>>(tk, tv, tdq, a);
   const size_t nq4 = (size_t)T * p.num_q_heads * kmb::kD / 4;
   const size_t nk4 = (size_t)T * Hkv * kmb::kD / 4;
   km_bwd_finalize_kernel<<<4 * sm_count(), 256, 0, st>>>((const float4*)dq_acc, nq4, (uint2*)dq);

@@ -34,6 +34,8 @@ bool attn_tc_supported(const sas_problem& p);
 int tc_rows_per_tile(int G);
 bool make_tmap_bf16_3d(CUtensorMap* m, const void* base, uint64_t n0, uint64_t n1, uint64_t n2,
                        uint32_t b0, uint32_t b1, uint32_t b2);
+bool make_tmap_f32_3d(CUtensorMap* m, const void* base, uint64_t n0, uint64_t n1, uint64_t n2,
+                      uint32_t b0, uint32_t b1, uint32_t b2);
 sas_status launch_rowdot(const sas_problem& p, const void* o, const void* dout, float* drow,
                          cudaStream_t st);
 

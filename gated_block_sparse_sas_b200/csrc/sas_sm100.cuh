@@ -335,6 +335,16 @@ __device__ __forceinline__ void bulk_reduce_add_f32(void* dst, uint32_t src, uin
                : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// global tensor box at (c0, c1, c2) += shared box (the map's element type; no swizzle: the
+// shared box is dense), by the TMA unit, tracked by the issuing thread's bulk groups
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, uint32_t src, int c0,
+                                                  int c1, int c2) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group"
+      " [%0, {%2, %3, %4}], [%1];" ::"l"(reinterpret_cast<uint64_t>(map)),
+      "r"(src), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
 // this thread's committed bulk operations have finished reading their shared sources
 __device__ __forceinline__ void bulk_wait_read0() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");

@@ -53,6 +53,21 @@ bool make_tmap_bf16_2d(CUtensorMap* m, const void* base, uint64_t n0, uint64_t n
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D fp32 map over [n2][n1][n0] (n0 contiguous) with a (b0, b1, b2) box, no swizzle (the
+// shared box is dense: b0 * 4 bytes per row).
+bool make_tmap_f32_3d(CUtensorMap* m, const void* base, uint64_t n0, uint64_t n1, uint64_t n2,
+                      uint32_t b0, uint32_t b1, uint32_t b2) {
+  PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {n0, n1, n2};
+  cuuint64_t strides[2] = {n0 * 4, n0 * n1 * 4};
+  cuuint32_t box[3] = {b0, b1, b2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool tma_available() { return encode_fn() != nullptr; }
 
 // Tokens per 128-row tile: Mq tokens x G heads <= 128 (G = 5: 25 tokens, 125 rows).
