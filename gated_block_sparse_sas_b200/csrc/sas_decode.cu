@@ -63,6 +63,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_gate_kernel(
   float* s = xk + H;                   // [NBmax + 1]
   float* red = s + NBmax + 1;          // [kDecWarps]
   int* cnt_red = reinterpret_cast<int*>(red + kDecWarps);  // [2][kDecWarps]
+  int* misc = cnt_red + 2 * kDecWarps;                      // [4]
+  int* hist = misc + 4;                                     // [256] radix histogram
 
   const int kv = blockIdx.x, b = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -251,69 +253,116 @@ __global__ void __launch_bounds__(kDecThreads) decode_gate_kernel(
     }
     return;
   }
-  // exact K-th largest of s[0..c-1] by a bitwise search over order-preserving keys
+  // exact K-th largest of s[0..c-1] over order-preserving keys, by a radix select: four
+  // rounds of an 8-bit digit histogram; `need` is the wanted rank among the keys that share the
+  // digits chosen so far (padding keys are 0, below every real key, and c > K)
   uint32_t key[NPT];
 #pragma unroll
   for (int r = 0; r < NPT; ++r) {
     const int j = tid + r * kDecThreads;
     key[r] = (j < c) ? order_key(s[j]) : 0u;
   }
-  uint32_t thr = 0;
-  __syncthreads();   // s[] complete before the keys are read below; cnt_red free
+  uint32_t thr = 0, pmask = 0;
+  int need = K;
 #pragma unroll 1
-  for (int bit = 31; bit >= 0; --bit) {   // counters double-buffered: one barrier per bit
-    const uint32_t cand = thr | (1u << bit);
-    int cn = 0;
-#pragma unroll
-    for (int r = 0; r < NPT; ++r) cn += key[r] >= cand;
-    cn = __reduce_add_sync(0xffffffffu, cn);
-    int* cb = cnt_red + (bit & 1) * kDecWarps;
-    if (lane == 0) cb[warp] = cn;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = tid; i < 256; i += kDecThreads) hist[i] = 0;
     __syncthreads();
-    int tot = 0;
 #pragma unroll
-    for (int w = 0; w < kDecWarps; ++w) tot += cb[w];
-    if (tot >= K) thr = cand;
-  }
-  int gt = 0;
+    for (int r = 0; r < NPT; ++r) {   // one shared atomic per distinct digit in the warp
+      const bool in = (key[r] & pmask) == thr;
+      const int bin = in ? (int)((key[r] >> shift) & 255u) : 256;
+      const unsigned peers = __match_any_sync(0xffffffffu, bin);
+      if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+    }
+    __syncthreads();
+    if (warp == 0) {   // lane owns digits 8 lane .. 8 lane + 7; find the digit where the
+                       // count of keys with a larger-or-equal digit first reaches `need`
+      int hv[8], loc = 0;
 #pragma unroll
-  for (int r = 0; r < NPT; ++r) gt += key[r] > thr;
-  gt = __reduce_add_sync(0xffffffffu, gt);
-  __syncthreads();
-  if (lane == 0) cnt_red[warp] = gt;
-  __syncthreads();
-  int gtot = 0;
-  for (int w = 0; w < kDecWarps; ++w) gtot += cnt_red[w];
-  const int need_eq = K - gtot;
-  if (warp == 0) {   // ordered emission by one warp
-    const unsigned below = (1u << lane) - 1u;
-    int out = 0, eq_seen = 0;
-    for (int j0 = 0; j0 < c; j0 += 32) {
-      const int j = j0 + lane;
-      const uint32_t kk = (j < c) ? order_key(s[j]) : 0u;
-      const bool is_gt = kk > thr, is_eq = kk == thr;
-      const unsigned eqm = __ballot_sync(0xffffffffu, is_eq);
-      const int eq_rank = eq_seen + __popc(eqm & below);
-      const bool sel = is_gt || (is_eq && eq_rank < need_eq);
-      const unsigned selm = __ballot_sync(0xffffffffu, sel);
-      if (sel) {
-        const int pos = out + __popc(selm & below);
-        const float lg = s[j] - lse;
-        sel_idx[orow + pos] = j;
-        sel_logg[orow + pos] = lg;
-        if (idx_out) idx_out[orow + pos] = j;
-        if (logg_out) logg_out[orow + pos] = lg;
+      for (int k = 0; k < 8; ++k) {
+        hv[k] = hist[8 * lane + k];
+        loc += hv[k];
       }
-      out += __popc(selm);
-      eq_seen += __popc(eqm);
+      int incl = loc;   // keys in this lane's digits and all larger ones
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_down_sync(0xffffffffu, incl, o);
+        if (lane + o < 32) incl += v;
+      }
+      int acc = incl - loc, found = -1, rest = 0;
+#pragma unroll
+      for (int k = 7; k >= 0; --k) {
+        if (found < 0 && acc < need && acc + hv[k] >= need) {
+          found = 8 * lane + k;
+          rest = need - acc;
+        }
+        acc += hv[k];
+      }
+      const unsigned who = __ballot_sync(0xffffffffu, found >= 0);   // exactly one lane
+      const int src = who ? __ffs(who) - 1 : 0;
+      const int dsel = __shfl_sync(0xffffffffu, found, src);
+      const int nrest = __shfl_sync(0xffffffffu, rest, src);
+      if (lane == 0) {
+        misc[1] = dsel;
+        misc[2] = nrest;
+      }
     }
-    if (lane == 0) {
-      const float lg = s[c] - lse;
-      sel_idx[orow + K] = c;
-      sel_logg[orow + K] = lg;
-      if (idx_out) idx_out[orow + K] = c;
-      if (logg_out) logg_out[orow + K] = lg;
+    __syncthreads();
+    thr |= (uint32_t)misc[1] << shift;
+    pmask |= 255u << shift;
+    need = misc[2];
+  }
+  const int need_eq = need;   // keys equal to thr to take, lowest block indices first
+  // ordered emission: warp w takes a contiguous range of blocks; a first pass counts its keys
+  // above and equal to thr, a second writes its selected blocks at their global positions
+  const int per = (c + kDecWarps - 1) / kDecWarps;
+  const int wj0 = min(c, warp * per), wj1 = min(c, wj0 + per);
+  const unsigned below = (1u << lane) - 1u;
+  int n_gt = 0, n_eq = 0;
+  for (int j0 = wj0; j0 < wj1; j0 += 32) {
+    const int j = j0 + lane;
+    const uint32_t kk = j < wj1 ? order_key(s[j]) : 0u;
+    n_gt += __popc(__ballot_sync(0xffffffffu, j < wj1 && kk > thr));
+    n_eq += __popc(__ballot_sync(0xffffffffu, j < wj1 && kk == thr));
+  }
+  if (lane == 0) {
+    cnt_red[warp] = n_gt;
+    cnt_red[kDecWarps + warp] = n_eq;
+  }
+  __syncthreads();
+  int gt_before = 0, eq_seen = 0;
+  for (int w = 0; w < warp; ++w) {
+    gt_before += cnt_red[w];
+    eq_seen += cnt_red[kDecWarps + w];
+  }
+  int out = gt_before + min(eq_seen, need_eq);
+  for (int j0 = wj0; j0 < wj1; j0 += 32) {
+    const int j = j0 + lane;
+    const bool valid = j < wj1;
+    const uint32_t kk = valid ? order_key(s[j]) : 0u;
+    const bool is_gt = valid && kk > thr, is_eq = valid && kk == thr;
+    const unsigned eqm = __ballot_sync(0xffffffffu, is_eq);
+    const int eq_rank = eq_seen + __popc(eqm & below);
+    const bool sel = is_gt || (is_eq && eq_rank < need_eq);
+    const unsigned selm = __ballot_sync(0xffffffffu, sel);
+    if (sel) {
+      const int pos = out + __popc(selm & below);
+      const float lg = s[j] - lse;
+      sel_idx[orow + pos] = j;
+      sel_logg[orow + pos] = lg;
+      if (idx_out) idx_out[orow + pos] = j;
+      if (logg_out) logg_out[orow + pos] = lg;
     }
+    out += __popc(selm);
+    eq_seen += __popc(eqm);
+  }
+  if (tid == 0) {
+    const float lg = s[c] - lse;
+    sel_idx[orow + K] = c;
+    sel_logg[orow + K] = lg;
+    if (idx_out) idx_out[orow + K] = c;
+    if (logg_out) logg_out[orow + K] = lg;
   }
 }
 
@@ -729,7 +778,7 @@ static void decode_gate_launch(const sas_decode_problem& p, const void* q_nope, 
   const int NBmax = (p.capacity + p.block - 1) / p.block;
   const int G = p.num_q_heads / p.num_kv_heads;
   const size_t smem = (size_t)(G * p.head_dim + 3 * p.head_dim + 2 * p.gate_hidden + NBmax + 1 +
-                               3 * kDecWarps) * sizeof(float);
+                               3 * kDecWarps + 4 + 256) * sizeof(float);
   dim3 grid(p.num_kv_heads, p.batch);
 #define SAS_DG(H, NPT)                                                                           \
   {                                                                                              \
