@@ -39,7 +39,8 @@ class SasDecodeProblem(ctypes.Structure):
     _fields_ = [("batch", _i32), ("capacity", _i32), ("num_q_heads", _i32),
                 ("num_kv_heads", _i32), ("head_dim", _i32), ("block", _i32), ("topk", _i32),
                 ("gate_hidden", _i32), ("rms_eps", _f32), ("dtype", ctypes.c_int),
-                ("seqlens", _vp), ("gate_rope_cos", _vp), ("gate_rope_sin", _vp)]
+                ("seqlens", _vp), ("gate_rope_cos", _vp), ("gate_rope_sin", _vp),
+                ("ungated", _i32)]
 
 
 _P = ctypes.POINTER(SasProblem)
@@ -275,6 +276,7 @@ class DecodeProblem:
     gate_rope_base: float = 1e6
     rope_cos: torch.Tensor | None = None
     rope_sin: torch.Tensor | None = None
+    gated: bool = True              # False: hard selection, no log-gate in the attention logits
 
     def __post_init__(self):
         if self.rope_cos is None:
@@ -285,7 +287,8 @@ class DecodeProblem:
         self._c = SasDecodeProblem(len(self.seqlens), self.capacity, self.num_q_heads,
                                    self.num_kv_heads, self.head_dim, self.block, self.topk,
                                    self.gate_hidden, self.rms_eps, _dtype_code(self.dtype),
-                                   _ptr(self.seqlens), _ptr(self.rope_cos), _ptr(self.rope_sin))
+                                   _ptr(self.seqlens), _ptr(self.rope_cos), _ptr(self.rope_sin),
+                                   0 if self.gated else 1)
 
     @property
     def batch(self) -> int:

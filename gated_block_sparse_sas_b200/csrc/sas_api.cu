@@ -290,6 +290,7 @@ static sas_status check_decode(const sas_decode_problem* p) {
   SAS_CHECK_ARG(p->seqlens != nullptr, "seqlens is NULL");
   SAS_CHECK_ARG(p->gate_rope_cos != nullptr && p->gate_rope_sin != nullptr,
                 "gate rotary tables are NULL");
+  SAS_CHECK_ARG(p->ungated == 0 || p->ungated == 1, "ungated must be 0 or 1 (got %d)", p->ungated);
   return SAS_OK;
 }
 

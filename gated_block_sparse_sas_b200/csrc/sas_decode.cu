@@ -52,8 +52,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_gate_kernel(
     const float* __restrict__ cur_pool, const T* __restrict__ wq, const float* __restrict__ qnorm_w,
     const T* __restrict__ wk, const float* __restrict__ knorm_w, const int32_t* __restrict__ seqlens,
     const float* __restrict__ rc, const float* __restrict__ rs, int Hq, int Hkv, int d, int B, int K,
-    int NBmax, int capacity, float eps, int32_t* __restrict__ sel_idx, float* __restrict__ sel_logg,
-    int32_t* __restrict__ idx_out, float* __restrict__ logg_out) {
+    int NBmax, int capacity, float eps, int ungated, int32_t* __restrict__ sel_idx,
+    float* __restrict__ sel_logg, int32_t* __restrict__ idx_out, float* __restrict__ logg_out) {
   extern __shared__ float smem[];
   const int G = Hq / Hkv, GD = G * d, C = 3 * d;
   float* qcat = smem;                  // [GD]
@@ -247,7 +247,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_gate_kernel(
       const int jj = sl <= c ? sl : -1;
       const float lg = sl <= c ? s[sl] - lse : 0.f;
       sel_idx[orow + sl] = jj;
-      sel_logg[orow + sl] = lg;
+      sel_logg[orow + sl] = ungated ? 0.f : lg;   // the attention's bias
       if (idx_out) idx_out[orow + sl] = jj;
       if (logg_out) logg_out[orow + sl] = lg;
     }
@@ -350,7 +350,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_gate_kernel(
       const int pos = out + __popc(selm & below);
       const float lg = s[j] - lse;
       sel_idx[orow + pos] = j;
-      sel_logg[orow + pos] = lg;
+      sel_logg[orow + pos] = ungated ? 0.f : lg;
       if (idx_out) idx_out[orow + pos] = j;
       if (logg_out) logg_out[orow + pos] = lg;
     }
@@ -360,7 +360,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_gate_kernel(
   if (tid == 0) {
     const float lg = s[c] - lse;
     sel_idx[orow + K] = c;
-    sel_logg[orow + K] = lg;
+    sel_logg[orow + K] = ungated ? 0.f : lg;
     if (idx_out) idx_out[orow + K] = c;
     if (logg_out) logg_out[orow + K] = lg;
   }
@@ -787,8 +787,8 @@ static void decode_gate_launch(const sas_decode_problem& p, const void* q_nope, 
     decode_gate_kernel<T, H, NPT><<<grid, kDecThreads, smem, st>>>(                              \
         (const T*)q_nope, (const __nv_bfloat16*)gkc, cur_pool, (const T*)wq, qnorm_w, (const T*)wk, \
         knorm_w, p.seqlens, p.gate_rope_cos, p.gate_rope_sin, p.num_q_heads, p.num_kv_heads,      \
-        p.head_dim, p.block, p.topk, NBmax, p.capacity, p.rms_eps, sel_idx, sel_logg, idx_out,   \
-        logg_out);                                                                               \
+        p.head_dim, p.block, p.topk, NBmax, p.capacity, p.rms_eps, p.ungated, sel_idx, sel_logg, \
+        idx_out, logg_out);                                                                      \
   }
 #define SAS_DG_H(NPT)                              \
   switch (p.gate_hidden) {                         \

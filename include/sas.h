@@ -101,6 +101,13 @@ typedef struct sas_decode_problem {
   const int32_t* seqlens;      /* device [batch]: L_b in 1..capacity, newest token at L_b-1 */
   const float* gate_rope_cos;  /* device [capacity, h/2]                           */
   const float* gate_rope_sin;
+  /* 0 (default): the kept blocks' log-gates are added to the attention logits, as in the
+   * prefill operator. 1: hard selection only -- the gate still picks the blocks (and
+   * idx_out / logg_out still report them with their log-gates), but the attention is a plain
+   * softmax over the kept keys, as a serving backend that uses the gate for selection alone
+   * would compute it (Hugging Face card "tencent/Simple-Attention-Sparsification", SGLang
+   * seer_attn backend section). */
+  int32_t ungated;
 } sas_decode_problem;
 
 /* Reason for the last non-OK status returned on this thread ("" if none). */

@@ -434,13 +434,16 @@ def prefill_selection(q_nope, k_nope, wq, qnorm_w, wk, knorm_w, cu_seqlens, bloc
 # ------------------------------------------------------------------------------------------
 
 def decode(q, q_nope, k_cache, v_cache, lengths, gate_key_cache, cur_pool, wq, qnorm_w, wk, knorm_w,
-           block: int, K: int, eps: float, base: float, rows=None):
+           block: int, K: int, eps: float, base: float, rows=None, gated: bool = True):
     """One decode step for (some) sequences.
 
     Sequence b has L_b tokens cached, the newest at position L_b-1 with c = (L_b-1)//B.
     Gate: q~ at position L_b-1; historical keys k~_j (j < c) read from the cache; the current
     block key from the running pool state (max, min, sum/n), n = L_b - c*B, at position c*B.
     Then the same softmax gates, Top-K and gated attention as the prefill row L_b-1.
+    gated=False keeps the selection but drops the log-gate from the attention logits (hard
+    selection, as a serving backend that uses the gate only to pick blocks computes it;
+    Hugging Face card "tencent/Simple-Attention-Sparsification", SGLang seer_attn section).
     Returns O [n, Hq, d], idx [n, Hkv, K+1], logg [n, Hkv, K+1], margin [n, Hkv].
     """
     q, qn = as64(q), as64(q_nope)
@@ -477,7 +480,7 @@ def decode(q, q_nope, k_cache, v_cache, lengths, gate_key_cache, cur_pool, wq, q
             margin[r, kv] = mg
             bias = np.full(L, NEG_INF)
             for j, lg in zip(ids, s[ids] - lse):
-                bias[j * block: min((j + 1) * block, L)] = lg
+                bias[j * block: min((j + 1) * block, L)] = lg if gated else 0.0
             kk, vv = kcache[kv, :L], vcache[kv, :L]
             for g in range(G):
                 hq = kv * G + g

@@ -30,3 +30,37 @@ def test_decode_equals_prefill_last_row(L):
     np.testing.assert_array_equal(idx[0], sel["idx"][L - 1])
     np.testing.assert_allclose(logg[0], sel["logg"][L - 1], rtol=1e-11, atol=1e-12)
     np.testing.assert_allclose(Od[0], O[L - 1], rtol=1e-11, atol=1e-12)
+
+
+def test_ungated_decode_is_softmax_over_kept_keys():
+    """Hard selection (gated=False): same blocks, and O is a plain softmax attention over the
+    kept keys -- checked against torch's scaled_dot_product_attention with a boolean mask
+    built from the oracle's own selection (a library routine, independent of the oracle's
+    softmax); the gated result differs whenever the kept log-gates differ."""
+    import torch
+
+    shp = si.DecodeShape([200, 37, 129], 256, 4, 2, 16, 16, 3, 16, seed=31, dtype="fp32")
+    inp = si.decode_inputs(shp)
+    args = (inp["q"], inp["q_nope"], inp["k_cache"], inp["v_cache"], shp.lengths,
+            inp["gate_key_cache"], inp["cur_pool"], inp["wq"], inp["qnorm_w"], inp["wk"],
+            inp["knorm_w"], shp.block, shp.topk, 1e-6, 1e6)
+    Og, idx_g, logg_g, _ = orc.decode(*args)
+    Ou, idx_u, logg_u, _ = orc.decode(*args, gated=False)
+    np.testing.assert_array_equal(idx_u, idx_g)
+    np.testing.assert_array_equal(logg_u, logg_g)
+    G = shp.num_q_heads // shp.num_kv_heads
+    for b, L in enumerate(shp.lengths):
+        for kv in range(shp.num_kv_heads):
+            keep = np.zeros(L, dtype=bool)
+            for j in idx_u[b, kv]:
+                if j >= 0:
+                    keep[j * shp.block: min((j + 1) * shp.block, L)] = True
+            kk = torch.from_numpy(orc.as64(inp["k_cache"][b, kv, :L]))
+            vv = torch.from_numpy(orc.as64(inp["v_cache"][b, kv, :L]))
+            for g in range(G):
+                hq = kv * G + g
+                qq = torch.from_numpy(orc.as64(inp["q"][b, hq]))[None, None, None]
+                ref = torch.nn.functional.scaled_dot_product_attention(
+                    qq, kk[None, None], vv[None, None], attn_mask=torch.from_numpy(keep)[None, None, None])
+                np.testing.assert_allclose(Ou[b, hq], ref[0, 0, 0].numpy(), rtol=1e-10, atol=1e-12)
+    assert np.abs(Ou - Og).max() > 1e-6

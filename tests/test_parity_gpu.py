@@ -226,24 +226,30 @@ DEC_CASES = {
     "bf16-d128-B64": ([1, 64, 65, 700, 2048, 1500], 2048, 8, 2, 128, 64, 7, 128),
     "bf16-d128-B64-G4-K31": ([4000, 129, 2500], 4096, 16, 4, 128, 64, 31, 128),
     "bf16-d64-B16": ([30, 17, 300], 512, 4, 2, 64, 16, 5, 32),
+    # the card's other decode budgets: 1,024 tokens (K 15) and 4,096 tokens (K 63)
+    "bf16-budget1024-K15": ([3000, 1100, 70, 2048], 4096, 32, 8, 128, 64, 15, 128),
+    "bf16-budget4096-K63": ([6000, 4200, 130, 5000], 8192, 16, 4, 128, 64, 63, 128),
 }
 
 
-@pytest.mark.parametrize("name", list(DEC_CASES))
-def test_decode(sas, name):
+@pytest.mark.parametrize("name,gated", [(n, True) for n in DEC_CASES] +
+                         [("bf16-d128-B64-G4-K31", False), ("bf16-d64-B16", False)])
+def test_decode(sas, name, gated):
     lengths, cap, Hq, Hkv, d, B, K, h = DEC_CASES[name]
     shp = si.DecodeShape(list(lengths), cap, Hq, Hkv, d, B, K, h, seed=400)
     inp = si.decode_inputs(shp)
     g = {k: v.cuda() for k, v in inp.items()}
     prob = sas.DecodeProblem(seqlens=g["lengths"], capacity=cap, num_q_heads=Hq, num_kv_heads=Hkv,
-                             head_dim=d, block=B, topk=K, gate_hidden=h, dtype=torch.bfloat16)
+                             head_dim=d, block=B, topk=K, gate_hidden=h, dtype=torch.bfloat16,
+                             gated=gated)
     o, idx, logg = sas.sas_decode(prob, g["q"], g["q_nope"], g["k_cache"], g["v_cache"],
                                   g["gate_key_cache"], g["cur_pool"], g["wq"], g["qnorm_w"], g["wk"],
                                   g["knorm_w"], want_selection=True)
     torch.cuda.synchronize()
     O, ridx, rlogg, margin = orc.decode(inp["q"], inp["q_nope"], inp["k_cache"], inp["v_cache"],
                                         lengths, inp["gate_key_cache"], inp["cur_pool"], inp["wq"],
-                                        inp["qnorm_w"], inp["wk"], inp["knorm_w"], B, K, 1e-6, 1e6)
+                                        inp["qnorm_w"], inp["wk"], inp["knorm_w"], B, K, 1e-6, 1e6,
+                                        gated=gated)
     compare_selection(idx.cpu().numpy(), logg, ridx, rlogg, margin)
     same = (idx.cpu().numpy() == ridx).all(axis=-1).all(axis=-1)
     assert_out_close(o[torch.from_numpy(same)], O[same], False, "O")
