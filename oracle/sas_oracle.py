@@ -46,6 +46,8 @@ Where the pages leave a step open, the reading used here is stated at that step:
       selection held fixed (Top-K is piecewise constant).
   R11 decode is the same operator evaluated for the newest token; cached gate keys
       are inputs as given.
+  R13 router backward: gradients of the gate parameters through the kept blocks'
+      log-gates with the selection fixed (see gate_backward).
 
 Parity pins live in tests/test_oracle_*.py. The gate's composition (R3-R5, R7) has
 no worked example on the pages: its parts are pinned by properties (rotary relative
@@ -427,6 +429,97 @@ def prefill_selection(q_nope, k_nope, wq, qnorm_w, wk, knorm_w, cu_seqlens, bloc
     idx, logg, margin = topk(s, lse, pos, block, K)
     return dict(idx=idx, logg=logg, margin=margin, scores=s, lse=lse, rows=rows, pooled=pooled,
                 gate_keys=gk)
+
+
+# ------------------------------------------------------------------------------------------
+# Router backward  [README (b): the loss reaches the selector; ABSTRACT: end-to-end
+# optimisation of the context ranking]  (R13)
+# ------------------------------------------------------------------------------------------
+#
+# R13 the gate parameters (Wq, Wk and the two RMSNorm weights) get the gradient of the
+#     loss through the log-gates of the kept blocks, with the selection held fixed:
+#     dL/ds[t, j] = sum over the slots holding j of dlogg - softmax_j(s[t, :c_t+1]) * sum of
+#     all dlogg of the row, then back through s = q~.k~/sqrt(h), the rotary, the RMSNorm and
+#     the projections (historical block keys from the pooled blocks, the current block's key
+#     from its visible prefix).
+
+def rms_norm_backward(x: np.ndarray, w: np.ndarray, eps: float, dy: np.ndarray):
+    """Gradients of y = x / r * w, r = sqrt(mean(x^2) + eps), over the last axis.
+
+    Returns (dx, dw) with dw summed over the leading axes."""
+    H = x.shape[-1]
+    r = np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+    u = x / r
+    dw = (dy * u).reshape(-1, H).sum(axis=0)
+    du = dy * w
+    dx = du / r - x * np.sum(du * x, axis=-1, keepdims=True) / (H * r ** 3)
+    return dx, dw
+
+
+def gate_backward(q_nope, k_nope, wq, qnorm_w, wk, knorm_w, idx, dlogg, cu_seqlens, block: int,
+                  eps: float, base: float):
+    """Router parameter gradients (R13) for the full problem.
+
+    idx, dlogg [T, Hkv, K+1] (the forward's selection and the loss gradient of its
+    log-gates). Returns dict(dwq [Hkv, h, G*d], dqnorm_w [h], dwk [Hkv, h, 3d], dknorm_w [h]).
+    """
+    q, k = as64(q_nope), as64(k_nope)
+    wq_, wk_, qw, kw = as64(wq), as64(wk), as64(qnorm_w), as64(knorm_w)
+    idx = np.asarray(idx)
+    dl = as64(dlogg)
+    T, Hq, d = q.shape
+    Hkv, h = wq_.shape[0], wq_.shape[1]
+    G = Hq // Hkv
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    seqs = seq_ranges(cu)
+    dwq = np.zeros_like(wq_)
+    dwk = np.zeros_like(wk_)
+    dqw = np.zeros(h)
+    dkw = np.zeros(h)
+    sq = np.sqrt(h)
+    for s0, s1 in seqs:
+        L = s1 - s0
+        nb = (L + block - 1) // block
+        # historical block keys of this sequence: pre-norm projections and final keys
+        P = np.stack([pool_tokens(k[s0 + j * block: s0 + min(L, (j + 1) * block)])
+                      for j in range(nb)])                                      # [nb, Hkv, 3d]
+        xk = np.einsum("khc,jkc->jkh", wk_, P)                                  # [nb, Hkv, h]
+        kt = rope_rotate(rms_norm(xk, kw, eps), (np.arange(nb) * block)[:, None], base)
+        dkt = np.zeros_like(kt)                                                 # dL/dk~_j
+        for t in range(L):
+            tg = s0 + t
+            c = t // block
+            a = q[tg].reshape(Hkv, G * d)
+            xq = np.einsum("khc,kc->kh", wq_, a)                                # [Hkv, h]
+            qt = rope_rotate(rms_norm(xq, qw, eps), float(t), base)
+            Pc = pool_tokens(k[s0 + c * block: tg + 1])                         # prefix (R7)
+            xc = np.einsum("khc,kc->kh", wk_, Pc)
+            kc = rope_rotate(rms_norm(xc, kw, eps), float(c * block), base)
+            keys = np.concatenate([kt[:c], kc[None]], axis=0)                   # [c+1, Hkv, h]
+            sc = np.einsum("kh,jkh->kj", qt, keys) / sq                         # [Hkv, c+1]
+            p = np.exp(sc - sc.max(axis=1, keepdims=True))
+            p /= p.sum(axis=1, keepdims=True)
+            ds = -p * dl[tg].sum(axis=1, keepdims=True)                         # LSE term
+            for kv in range(Hkv):
+                for sl in range(idx.shape[2]):
+                    j = int(idx[tg, kv, sl])
+                    if j >= 0:
+                        ds[kv, j] += dl[tg, kv, sl]
+            dqt = np.einsum("kj,jkh->kh", ds, keys) / sq
+            dkeys = np.einsum("kj,kh->jkh", ds, qt) / sq
+            dkt[:c] += dkeys[:c]
+            # current block key: rotary back (rotation by -angle), RMSNorm, Kproj
+            dxc, dw_ = rms_norm_backward(xc, kw, eps, rope_rotate(dkeys[c], -float(c * block), base))
+            dkw += dw_
+            dwk += np.einsum("kh,kc->khc", dxc, Pc)
+            dxq, dw_ = rms_norm_backward(xq, qw, eps, rope_rotate(dqt, -float(t), base))
+            dqw += dw_
+            dwq += np.einsum("kh,kc->khc", dxq, a)
+        dxk, dw_ = rms_norm_backward(xk, kw, eps,
+                                     rope_rotate(dkt, -(np.arange(nb) * block)[:, None].astype(F64), base))
+        dkw += dw_
+        dwk += np.einsum("jkh,jkc->khc", dxk, P)
+    return dict(dwq=dwq, dqnorm_w=dqw, dwk=dwk, dknorm_w=dkw)
 
 
 # ------------------------------------------------------------------------------------------
