@@ -288,6 +288,36 @@ def alloc_outputs(sas, prob, g, backward):
         g["_wsb"] = torch.empty(max(256, n.value), dtype=torch.uint8, device=dev)
 
 
+def bench_router_bwd(sas, prob, g, flush, steps):
+    """The router backward (gate parameter gradients from the step's own dlogg), timed on its
+    own after the step: it is not part of the timed step."""
+    import ctypes
+    n = ctypes.c_size_t(0)
+    if sas.lib_handle().sas_gate_bwd_workspace_size(prob.ref, ctypes.byref(n)) != 0:
+        return {"unsupported": sas.lib_handle().sas_last_error().decode()}
+    ws = torch.empty(max(256, n.value), dtype=torch.uint8, device=prob.device)
+    args = (prob, g["q_nope"], g["k_nope"], g["_pooled"], g["wq"], g["qnorm_w"], g["wk"],
+            g["knorm_w"], g["_idx"], g["_dlogg"])
+    for _ in range(2):
+        sas.sas_gate_bwd(*args, workspace=ws)
+    times = []
+    for _ in range(steps):
+        flush.zero_()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        sas.sas_gate_bwd(*args, workspace=ws)
+        e.record()
+        times.append((s, e))
+    torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in times) / len(times)
+    T, Hkv, h, d = prob.total_tokens, prob.num_kv_heads, prob.gate_hidden, prob.head_dim
+    G = prob.num_q_heads // Hkv
+    outer = 2.0 * T * Hkv * h * (G * d + 3 * d) + 2.0 * prob.batch * prob.max_blocks * Hkv * h * 3 * d
+    return {"ms": ms, "outer_product_gflop": outer / 1e9, "achieved_tflops": outer / (ms * 1e-3) / 1e12,
+            "note": "dWq, dWk, norm-weight gradients from the step's dlogg; fp32 CUDA-core outer "
+                    "products; timed separately, not part of the step"}
+
+
 # ------------------------------------------------------------------------------------------
 # oracle sample (CPU baseline and the reference arm)
 # ------------------------------------------------------------------------------------------
@@ -500,6 +530,8 @@ def main():
     cs = clk.summary()
     if cs:
         line["clocks"] = cs
+    if backward:
+        line["router_bwd"] = bench_router_bwd(sas, prob, g, flush, max(3, a.steps))
 
     if not a.no_decode:
         try:

@@ -54,6 +54,8 @@ _SIGS = {
     "sas_gate_scores_workspace_size": ([_P, ctypes.POINTER(_sz)], ctypes.c_int),
     "sas_gate_scores": ([_P] + [_vp] * 9 + [_vp, _sz, _vp], ctypes.c_int),
     "sas_topk": ([_P, _vp, _vp, _vp, _vp, _vp], ctypes.c_int),
+    "sas_gate_bwd_workspace_size": ([_P, ctypes.POINTER(_sz)], ctypes.c_int),
+    "sas_gate_bwd": ([_P] + [_vp] * 13 + [_vp, _sz, _vp], ctypes.c_int),
     "sas_attn_fwd_workspace_size": ([_P, ctypes.POINTER(_sz)], ctypes.c_int),
     "sas_attn_fwd": ([_P] + [_vp] * 8 + [_sz, _vp], ctypes.c_int),
     "sas_attn_bwd_workspace_size": ([_P, ctypes.POINTER(_sz)], ctypes.c_int),
@@ -197,6 +199,27 @@ def sas_gate_scores(p: Problem, q_nope, k_nope, gate_keys, wq, qnorm_w, wk, knor
                                 _ptr(qnorm_w), _ptr(wk), _ptr(knorm_w), _ptr(scores), _ptr(lse),
                                 _ptr(ws), ws.numel(), _stream(stream)), "sas_gate_scores")
     return scores, lse
+
+
+def gate_bwd_workspace(p: Problem):
+    """A workspace of the size sas_gate_bwd asks for."""
+    return _workspace(_lib.sas_gate_bwd_workspace_size, p.ref, p.device)
+
+
+def sas_gate_bwd(p: Problem, q_nope, k_nope, pooled, wq, qnorm_w, wk, knorm_w, idx, dlogg,
+                 workspace=None, stream=None):
+    """Router backward: (dwq, dqnorm_w, dwk, dknorm_w), fp32, through the kept log-gates."""
+    G, h, d, Hkv = p.num_q_heads // p.num_kv_heads, p.gate_hidden, p.head_dim, p.num_kv_heads
+    dwq = torch.empty((Hkv, h, G * d), dtype=torch.float32, device=p.device)
+    dwk = torch.empty((Hkv, h, 3 * d), dtype=torch.float32, device=p.device)
+    dqn = torch.empty((h,), dtype=torch.float32, device=p.device)
+    dkn = torch.empty((h,), dtype=torch.float32, device=p.device)
+    ws = workspace if workspace is not None else gate_bwd_workspace(p)
+    _check(_lib.sas_gate_bwd(p.ref, _ptr(q_nope), _ptr(k_nope), _ptr(pooled), _ptr(wq),
+                             _ptr(qnorm_w), _ptr(wk), _ptr(knorm_w), _ptr(idx), _ptr(dlogg),
+                             _ptr(dwq), _ptr(dqn), _ptr(dwk), _ptr(dkn), _ptr(ws), ws.numel(),
+                             _stream(stream)), "sas_gate_bwd")
+    return dwq, dqn, dwk, dkn
 
 
 def sas_topk(p: Problem, scores, lse, idx=None, logg=None, stream=None):

@@ -165,6 +165,61 @@ sas_status sas_gate_scores(const sas_problem* p, const void* q_nope, const void*
                             workspace, stream);
 }
 
+sas_status sas_gate_bwd_workspace_size(const sas_problem* p, size_t* bytes) {
+  SAS_TRY(check_problem(p, true));
+  SAS_CHECK_ARG(bytes != nullptr, "bytes is NULL");
+  if (!gate_bwd_supported(*p)) {
+    set_error("gate_bwd: supported for bf16, head_dim 128, gate_hidden 128, block <= 128");
+    return SAS_ERR_UNSUPPORTED;
+  }
+  *bytes = gate_bwd_workspace_bytes(*p);
+  return SAS_OK;
+}
+
+sas_status sas_gate_bwd(const sas_problem* p, const void* q_nope, const void* k_nope,
+                        const float* pooled, const void* wq, const float* qnorm_w, const void* wk,
+                        const float* knorm_w, const int32_t* idx, const float* dlogg, float* dwq,
+                        float* dqnorm_w, float* dwk, float* dknorm_w, void* workspace,
+                        size_t workspace_bytes, cudaStream_t stream) {
+  SAS_TRY(check_problem(p, true));
+  SAS_PTR(q_nope);
+  SAS_PTR(k_nope);
+  SAS_PTR(pooled);
+  SAS_PTR(wq);
+  SAS_PTR(qnorm_w);
+  SAS_PTR(wk);
+  SAS_PTR(knorm_w);
+  SAS_PTR(idx);
+  SAS_PTR(dlogg);
+  SAS_PTR(dwq);
+  SAS_PTR(dqnorm_w);
+  SAS_PTR(dwk);
+  SAS_PTR(dknorm_w);
+  if (!gate_bwd_supported(*p)) {
+    set_error("gate_bwd: supported for bf16, head_dim 128, gate_hidden 128, block <= 128");
+    return SAS_ERR_UNSUPPORTED;
+  }
+  if (p->total_tokens == 0) {   // no rows: every gradient is zero
+    const int G = p->num_q_heads / p->num_kv_heads, h = p->gate_hidden, d = p->head_dim;
+    if (cudaMemsetAsync(dwq, 0, (size_t)p->num_kv_heads * h * G * d * 4, stream) != cudaSuccess ||
+        cudaMemsetAsync(dwk, 0, (size_t)p->num_kv_heads * h * 3 * d * 4, stream) != cudaSuccess ||
+        cudaMemsetAsync(dqnorm_w, 0, (size_t)h * 4, stream) != cudaSuccess ||
+        cudaMemsetAsync(dknorm_w, 0, (size_t)h * 4, stream) != cudaSuccess) {
+      set_error("gate_bwd: clearing the outputs failed");
+      return SAS_ERR_CUDA;
+    }
+    return SAS_OK;
+  }
+  SAS_PTR(workspace);
+  const size_t need = gate_bwd_workspace_bytes(*p);
+  if (workspace_bytes < need) {
+    set_error("workspace too small: %zu < %zu bytes", workspace_bytes, need);
+    return SAS_ERR_WORKSPACE;
+  }
+  return launch_gate_bwd(*p, q_nope, k_nope, pooled, wq, qnorm_w, wk, knorm_w, idx, dlogg, dwq,
+                         dqnorm_w, dwk, dknorm_w, workspace, stream);
+}
+
 sas_status sas_topk(const sas_problem* p, const float* scores, const float* lse, int32_t* idx,
                     float* logg, cudaStream_t stream) {
   SAS_TRY(check_problem(p, false));

@@ -1,0 +1,447 @@
+// Router backward: gradients of the gate parameters (Wq, Wk and the two RMSNorm weights)
+// through the log-gates of the kept blocks, with the selection held fixed. The project
+// README (intro item (b)) and the paper abstract make the selector trainable end to end
+// from the language-model loss; this is that gradient for one layer's gate.
+//
+// Forward being differentiated (per token t, kv head; h = 128):
+//   xq_t = Wq . concat_g q_nope[t, kv*G+g],  q~_t = rope_t(RMSNorm(xq_t) * qnorm_w)
+//   xk_j = Wk . P_j (pooled block j),        k~_j = rope_{jB}(RMSNorm(xk_j) * knorm_w)
+//   xc_t = Wk . P_cur(t) (block c_t's prefix up to t), k~c_t = rope_{c_t B}(...)
+//   s[t, j] = q~_t . k~_j / sqrt(h),  log g = s - logsumexp over visible blocks
+// Given dlogg[t, kv, slot]: dL/ds[t, j] = dlogg on the kept slots. The logsumexp term
+// (- softmax_j * sum of the row's dlogg) is zero: the attention is unchanged when every
+// log-gate of a row moves by one constant, so the row sums of the dlogg it returns are zero.
+//
+// Passes (fp32 throughout; h = 128, bf16 inputs):
+//   0. xq, xc for every (t, kv): the tensor-core projections of the forward gate.
+//   1. block keys: xk_j and k~_j per (sequence, block, kv), one warp per row.
+//   2. rows: per (t, kv) one warp: q~, k~c; dq~ = sum_slots ds k~_j; dk~_j += ds q~ (L2
+//      reductions into a per-block buffer); dk~c = ds_c q~; both back through the rotary and
+//      the RMSNorm -> dxq, dxc and the norm-weight gradients.
+//   3. block keys backward: dk~_j -> dxk_j and the knorm_w gradient.
+//   4. weight gradients as sums of outer products over rows, register-tiled 64 x 64 tiles:
+//      dWq += dxq (x) q_nope group, dWk += dxk (x) P_j + dxc (x) P_cur(t) (the prefix pools
+//      rebuilt per block by a running max / min / sum).
+#include "sas_common.cuh"
+#include "sas_kernels.h"
+
+namespace sas {
+
+namespace gbw {
+constexpr int H = 128;           // gate hidden of the supported configuration
+constexpr int kRowThreads = 256;
+constexpr int kTile = 64;        // outer-product tile (rows of W x columns of W)
+constexpr int kKs = 16;          // rows per step of the outer-product kernel
+}  // namespace gbw
+
+// One row of h = 128 values per warp: lane holds e = lane + 32 u (u = 0..3); the rotary
+// pairs (e, e + 64) are (u = 0, 2) and (u = 1, 3) of the same lane.
+__device__ __forceinline__ void gbw_norm_rope_fwd(const float x[4], const float* __restrict__ w,
+                                                  const float* __restrict__ rc,
+                                                  const float* __restrict__ rs, int pos, float eps,
+                                                  int lane, float out[4], float u[4], float& r) {
+  float ss = x[0] * x[0] + x[1] * x[1] + x[2] * x[2] + x[3] * x[3];
+  ss = warp_sum(ss);
+  r = sqrtf(ss / (float)gbw::H + eps);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) u[k] = x[k] / r;
+#pragma unroll
+  for (int p = 0; p < 2; ++p) {
+    const int e = lane + 32 * p;
+    const float a = u[p] * w[e], b = u[p + 2] * w[e + 64];
+    const float c = rc[(size_t)pos * 64 + e], s = rs[(size_t)pos * 64 + e];
+    out[p] = a * c - b * s;
+    out[p + 2] = b * c + a * s;
+  }
+}
+
+// Backward of gbw_norm_rope_fwd: dout = dL/d(rotated output) -> dx; dw += dL/dw.
+__device__ __forceinline__ void gbw_norm_rope_bwd(const float x[4], const float u[4], float r,
+                                                  const float* __restrict__ w,
+                                                  const float* __restrict__ rc,
+                                                  const float* __restrict__ rs, int pos, int lane,
+                                                  const float dout[4], float dx[4], float dw[4]) {
+  float dy[4];
+#pragma unroll
+  for (int p = 0; p < 2; ++p) {   // the rotation's transpose: rotation by -angle
+    const int e = lane + 32 * p;
+    const float c = rc[(size_t)pos * 64 + e], s = rs[(size_t)pos * 64 + e];
+    dy[p] = dout[p] * c + dout[p + 2] * s;
+    dy[p + 2] = dout[p + 2] * c - dout[p] * s;
+  }
+  float du[4], dot = 0.f;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float wk = w[lane + 32 * k];
+    dw[k] += dy[k] * u[k];
+    du[k] = dy[k] * wk;
+    dot += du[k] * x[k];
+  }
+  dot = warp_sum(dot);
+  const float r3 = r * r * r * (float)gbw::H;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) dx[k] = du[k] / r - x[k] * dot / r3;
+}
+
+// Sum the CTA's per-lane norm-weight gradients (4 per lane and warp) into dw[128].
+__device__ __forceinline__ void gbw_cta_add_dw(const float acc[4], float* red, float* __restrict__ dw) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nw = blockDim.x >> 5;
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < 4; ++k) red[warp * gbw::H + lane + 32 * k] = acc[k];
+  __syncthreads();
+  for (int e = threadIdx.x; e < gbw::H; e += blockDim.x) {
+    float s = 0.f;
+    for (int w = 0; w < nw; ++w) s += red[w * gbw::H + e];
+    atomicAdd(dw + e, s);
+  }
+}
+
+// (1) block keys: xk = Wk . P_j and k~_j, one warp per (sequence, block, kv); zeros past a
+// sequence's end.
+__global__ void __launch_bounds__(gbw::kRowThreads) gbw_block_fwd_kernel(
+    const float* __restrict__ pooled, const __nv_bfloat16* __restrict__ wk,
+    const float* __restrict__ knorm_w, const int32_t* __restrict__ cu, const float* __restrict__ rc,
+    const float* __restrict__ rs, int batch, int NBmax, int Hkv, int d, int B, float eps,
+    float* __restrict__ xk_out, float* __restrict__ kt_out) {
+  const int lane = threadIdx.x & 31;
+  const int C = 3 * d;   // <= 384: 12 inputs per lane
+  const size_t nrows = (size_t)batch * NBmax * Hkv;
+  for (size_t row = (blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5; row < nrows;
+       row += (gridDim.x * (size_t)blockDim.x) >> 5) {
+    const int kv = (int)(row % Hkv);
+    const size_t bj = row / Hkv;
+    const int b = (int)(bj / NBmax), j = (int)(bj % NBmax);
+    const int L = cu[b + 1] - cu[b];
+    float* xo = xk_out + row * gbw::H;
+    float* ko = kt_out + row * gbw::H;
+    if (j * B >= L) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) xo[lane + 32 * k] = ko[lane + 32 * k] = 0.f;
+      continue;
+    }
+    float pv[12];
+    const float* P = pooled + row * C;
+#pragma unroll
+    for (int m = 0; m < 12; ++m) pv[m] = (lane + 32 * m < C) ? P[lane + 32 * m] : 0.f;
+    const __nv_bfloat16* W = wk + (size_t)kv * gbw::H * C;
+    float x[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      x[u] = 0.f;
+#pragma unroll 1
+      for (int ii = 0; ii < 32; ++ii) {
+        const __nv_bfloat16* wr = W + (size_t)(32 * u + ii) * C;
+        float part = 0.f;
+#pragma unroll
+        for (int m = 0; m < 12; ++m)
+          if (lane + 32 * m < C) part = fmaf(__bfloat162float(wr[lane + 32 * m]), pv[m], part);
+        part = warp_sum(part);
+        if (lane == ii) x[u] = part;
+      }
+    }
+    float out[4], uu[4], r;
+    gbw_norm_rope_fwd(x, knorm_w, rc, rs, j * B, eps, lane, out, uu, r);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      xo[lane + 32 * k] = x[k];
+      ko[lane + 32 * k] = out[k];
+    }
+  }
+}
+
+// (2) rows: one warp per (token, kv head).
+__global__ void __launch_bounds__(gbw::kRowThreads) gbw_row_kernel(
+    const float* __restrict__ xq_all, const float* __restrict__ xc_all,
+    const float* __restrict__ kt_hist, const int32_t* __restrict__ idx,
+    const float* __restrict__ dlogg, const float* __restrict__ qnorm_w,
+    const float* __restrict__ knorm_w, const int32_t* __restrict__ cu, const float* __restrict__ rc,
+    const float* __restrict__ rs, int batch, int T, int NBmax, int Hkv, int B, int K1, float eps,
+    float* __restrict__ dkt_hist, float* __restrict__ dxq_out, float* __restrict__ dxc_out,
+    float* __restrict__ dqnorm_w, float* __restrict__ dknorm_w) {
+  __shared__ float red[(gbw::kRowThreads / 32) * gbw::H];
+  const int lane = threadIdx.x & 31;
+  const float inv_sqrt_h = 1.f / sqrtf((float)gbw::H);
+  float dwq[4] = {0.f, 0.f, 0.f, 0.f}, dwk[4] = {0.f, 0.f, 0.f, 0.f};
+  const size_t nrows = (size_t)T * Hkv;
+  for (size_t row = (blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5; row < nrows;
+       row += (gridDim.x * (size_t)blockDim.x) >> 5) {
+    const int tg = (int)(row / Hkv), kv = (int)(row % Hkv);
+    const int b = seq_of(cu, batch, tg);
+    const int t = tg - cu[b], c = t / B;
+    float xq[4], xc[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      xq[k] = xq_all[row * gbw::H + lane + 32 * k];
+      xc[k] = xc_all[row * gbw::H + lane + 32 * k];
+    }
+    float qt[4], uq[4], rq, kc[4], uc[4], rcn;
+    gbw_norm_rope_fwd(xq, qnorm_w, rc, rs, t, eps, lane, qt, uq, rq);
+    gbw_norm_rope_fwd(xc, knorm_w, rc, rs, c * B, eps, lane, kc, uc, rcn);
+    float dqt[4] = {0.f, 0.f, 0.f, 0.f}, dkc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int sl = 0; sl < K1; ++sl) {   // warp-uniform: every lane reads the same slot
+      const int j = idx[row * K1 + sl];
+      if (j < 0) continue;
+      const float ds = dlogg[row * K1 + sl] * inv_sqrt_h;
+      if (j == c) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          dqt[k] = fmaf(ds, kc[k], dqt[k]);
+          dkc[k] = fmaf(ds, qt[k], dkc[k]);
+        }
+      } else {
+        const size_t kr = (((size_t)b * NBmax + j) * Hkv + kv) * gbw::H;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          dqt[k] = fmaf(ds, kt_hist[kr + lane + 32 * k], dqt[k]);
+          atomicAdd(dkt_hist + kr + lane + 32 * k, ds * qt[k]);
+        }
+      }
+    }
+    float dx[4];
+    gbw_norm_rope_bwd(xq, uq, rq, qnorm_w, rc, rs, t, lane, dqt, dx, dwq);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) dxq_out[row * gbw::H + lane + 32 * k] = dx[k];
+    gbw_norm_rope_bwd(xc, uc, rcn, knorm_w, rc, rs, c * B, lane, dkc, dx, dwk);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) dxc_out[row * gbw::H + lane + 32 * k] = dx[k];
+  }
+  gbw_cta_add_dw(dwq, red, dqnorm_w);
+  gbw_cta_add_dw(dwk, red, dknorm_w);
+}
+
+// (3) block keys backward: dk~_j -> dxk_j, knorm_w gradient.
+__global__ void __launch_bounds__(gbw::kRowThreads) gbw_block_bwd_kernel(
+    const float* __restrict__ xk_hist, const float* __restrict__ dkt_hist,
+    const float* __restrict__ knorm_w, const int32_t* __restrict__ cu, const float* __restrict__ rc,
+    const float* __restrict__ rs, int batch, int NBmax, int Hkv, int B, float eps,
+    float* __restrict__ dxk_out, float* __restrict__ dknorm_w) {
+  __shared__ float red[(gbw::kRowThreads / 32) * gbw::H];
+  const int lane = threadIdx.x & 31;
+  float dwk[4] = {0.f, 0.f, 0.f, 0.f};
+  const size_t nrows = (size_t)batch * NBmax * Hkv;
+  for (size_t row = (blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5; row < nrows;
+       row += (gridDim.x * (size_t)blockDim.x) >> 5) {
+    const size_t bj = row / Hkv;
+    const int b = (int)(bj / NBmax), j = (int)(bj % NBmax);
+    float* xo = dxk_out + row * gbw::H;
+    if (j * B >= cu[b + 1] - cu[b]) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) xo[lane + 32 * k] = 0.f;
+      continue;
+    }
+    float x[4], g[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      x[k] = xk_hist[row * gbw::H + lane + 32 * k];
+      g[k] = dkt_hist[row * gbw::H + lane + 32 * k];
+    }
+    float out[4], u[4], r, dx[4];
+    gbw_norm_rope_fwd(x, knorm_w, rc, rs, j * B, eps, lane, out, u, r);
+    gbw_norm_rope_bwd(x, u, r, knorm_w, rc, rs, j * B, lane, g, dx, dwk);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) xo[lane + 32 * k] = dx[k];
+  }
+  gbw_cta_add_dw(dwk, red, dknorm_w);
+}
+
+// (4) dW[kv][i][c] += sum over rows of X[row][kv][i] * Y[row][kv][c], a 64 x 64 tile of dW per
+// CTA (64 threads, 8 x 8 outputs each), rows split over gridDim.z / Hkv chunks, the partial
+// tile added with fp32 atomics.
+//   MODE 0: rows = tokens, X = dxq, Y = q_nope[t, kv*G .. kv*G+G-1, :] (C = G d)
+//   MODE 1: rows = (sequence, block), X = dxk, Y = pooled (C = 3d)
+//   MODE 2: rows = tokens taken block by block, X = dxc, Y = the block's prefix pool up to
+//           the token (running max | min | sum / count, C = 3d)
+template <int MODE>
+__global__ void __launch_bounds__(64) gbw_outer_kernel(
+    const float* __restrict__ X, const __nv_bfloat16* __restrict__ q_nope,
+    const float* __restrict__ pooled, const __nv_bfloat16* __restrict__ k_nope,
+    const int32_t* __restrict__ cu, int batch, int T, int Hq, int Hkv, int d, int B, int NBmax,
+    int C, int nsplit, float* __restrict__ dW) {
+  __shared__ float Xs[gbw::kKs][gbw::kTile];
+  __shared__ float Ys[gbw::kKs][gbw::kTile];
+  const int tid = threadIdx.x, ty = tid >> 3, tx = tid & 7;
+  const int c0 = blockIdx.x * gbw::kTile, i0 = blockIdx.y * gbw::kTile;
+  const int kv = blockIdx.z % Hkv, split = blockIdx.z / Hkv;
+  const int G = Hq / Hkv;
+  float acc[8][8];
+#pragma unroll
+  for (int a = 0; a < 8; ++a)
+#pragma unroll
+    for (int bb = 0; bb < 8; ++bb) acc[a][bb] = 0.f;
+
+  auto fma_step = [&](int nk) {
+    __syncthreads();
+    for (int k = 0; k < nk; ++k) {
+      float xv[8], yv[8];
+#pragma unroll
+      for (int a = 0; a < 8; ++a) xv[a] = Xs[k][ty + 8 * a];
+#pragma unroll
+      for (int bb = 0; bb < 8; ++bb) yv[bb] = Ys[k][tx + 8 * bb];
+#pragma unroll
+      for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int bb = 0; bb < 8; ++bb) acc[a][bb] = fmaf(xv[a], yv[bb], acc[a][bb]);
+    }
+    __syncthreads();
+  };
+
+  if constexpr (MODE == 0 || MODE == 1) {
+    const int nrows = MODE == 0 ? T : batch * NBmax;
+    const int per = (nrows + nsplit - 1) / nsplit;
+    const int r0 = split * per, r1 = min(nrows, r0 + per);
+    for (int rb = r0; rb < r1; rb += gbw::kKs) {
+      const int nk = min(gbw::kKs, r1 - rb);
+      for (int e = tid; e < gbw::kKs * gbw::kTile; e += 64) {
+        const int k = e / gbw::kTile, col = e % gbw::kTile;
+        const int r = rb + k;
+        float xv = 0.f, yv = 0.f;
+        if (k < nk) {
+          xv = X[((size_t)r * Hkv + kv) * gbw::H + i0 + col];
+          if constexpr (MODE == 0)
+            yv = __bfloat162float(q_nope[((size_t)r * Hq + (size_t)kv * G) * d + c0 + col]);
+          else
+            yv = pooled[((size_t)r * Hkv + kv) * C + c0 + col];
+        }
+        Xs[k][col] = xv;
+        Ys[k][col] = yv;
+      }
+      fma_step(nk);
+    }
+  } else {
+    const int nblk = batch * NBmax;
+    const int per = (nblk + nsplit - 1) / nsplit;
+    const int q0 = split * per, q1 = min(nblk, q0 + per);
+    // column owned by this thread in the prefix scan: c0 + tid -> (part, channel)
+    const int col = c0 + tid, part = col / d, ch = col - part * d;
+    for (int bj = q0; bj < q1; ++bj) {
+      const int b = bj / NBmax, j = bj % NBmax;
+      const int s0 = cu[b], L = cu[b + 1] - s0;
+      if (j * B >= L) continue;   // uniform over the CTA
+      const int n = min(B, L - j * B);
+      float run = 0.f;
+      for (int rb = 0; rb < n; rb += gbw::kKs) {
+        const int nk = min(gbw::kKs, n - rb);
+        float kvv[gbw::kKs];
+#pragma unroll
+        for (int k = 0; k < gbw::kKs; ++k)
+          kvv[k] = k < nk ? __bfloat162float(
+                                k_nope[((size_t)(s0 + j * B + rb + k) * Hkv + kv) * d + ch])
+                          : 0.f;
+#pragma unroll
+        for (int k = 0; k < gbw::kKs; ++k) {
+          if (k < nk) {
+            const int cnt = rb + k + 1;
+            const float v = kvv[k];
+            if (cnt == 1) run = v;
+            else if (part == 0) run = fmaxf(run, v);
+            else if (part == 1) run = fminf(run, v);
+            else run += v;
+            Ys[k][tid] = part == 2 ? run / (float)cnt : run;
+          } else {
+            Ys[k][tid] = 0.f;
+          }
+        }
+        for (int e = tid; e < gbw::kKs * gbw::kTile; e += 64) {
+          const int k = e / gbw::kTile, cc = e % gbw::kTile;
+          Xs[k][cc] = k < nk ? X[((size_t)(s0 + j * B + rb + k) * Hkv + kv) * gbw::H + i0 + cc] : 0.f;
+        }
+        fma_step(nk);
+      }
+    }
+  }
+#pragma unroll
+  for (int a = 0; a < 8; ++a)
+#pragma unroll
+    for (int bb = 0; bb < 8; ++bb)
+      atomicAdd(dW + ((size_t)kv * gbw::H + i0 + ty + 8 * a) * C + c0 + tx + 8 * bb, acc[a][bb]);
+}
+
+// ---------------------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------------------
+namespace {
+struct GbwLayout {
+  size_t tc, xk, kt, dkt, dxk, dxq, dxc, total;
+};
+size_t al256w(size_t x) { return (x + 255) & ~(size_t)255; }
+GbwLayout gbw_layout(const sas_problem& p) {
+  GbwLayout L;
+  const int NBmax = (p.max_seqlen + p.block - 1) / p.block;
+  const size_t brow = (size_t)p.batch * NBmax * p.num_kv_heads * gbw::H * 4;
+  const size_t trow = (size_t)p.total_tokens * p.num_kv_heads * gbw::H * 4;
+  size_t o = 0;
+  L.tc = o;  o += al256w(gate_tc_workspace_bytes(p));
+  L.xk = o;  o += al256w(brow);
+  L.kt = o;  o += al256w(brow);
+  L.dkt = o; o += al256w(brow);
+  L.dxk = o; o += al256w(brow);
+  L.dxq = o; o += al256w(trow);
+  L.dxc = o; o += al256w(trow);
+  L.total = o;
+  return L;
+}
+}  // namespace
+
+bool gate_bwd_supported(const sas_problem& p) {
+  return gate_tc_supported(p) && p.gate_hidden == gbw::H && p.head_dim == 128;
+}
+
+size_t gate_bwd_workspace_bytes(const sas_problem& p) { return gbw_layout(p).total; }
+
+sas_status launch_gate_bwd(const sas_problem& p, const void* q_nope, const void* k_nope,
+                           const float* pooled, const void* wq, const float* qnorm_w,
+                           const void* wk, const float* knorm_w, const int32_t* idx,
+                           const float* dlogg, float* dwq, float* dqnorm_w, float* dwk,
+                           float* dknorm_w, void* workspace, cudaStream_t st) {
+  const GbwLayout L = gbw_layout(p);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int Hkv = p.num_kv_heads, Hq = p.num_q_heads, G = Hq / Hkv, d = p.head_dim;
+  const int T = p.total_tokens, B = p.block;
+  const int NBmax = (p.max_seqlen + B - 1) / B;
+  float* xk = reinterpret_cast<float*>(ws + L.xk);
+  float* kt = reinterpret_cast<float*>(ws + L.kt);
+  float* dkt = reinterpret_cast<float*>(ws + L.dkt);
+  float* dxk = reinterpret_cast<float*>(ws + L.dxk);
+  float* dxq = reinterpret_cast<float*>(ws + L.dxq);
+  float* dxc = reinterpret_cast<float*>(ws + L.dxc);
+  const size_t brow = (size_t)p.batch * NBmax * Hkv * gbw::H * 4;
+  if (cudaMemsetAsync(dwq, 0, (size_t)Hkv * gbw::H * G * d * 4, st) != cudaSuccess ||
+      cudaMemsetAsync(dwk, 0, (size_t)Hkv * gbw::H * 3 * d * 4, st) != cudaSuccess ||
+      cudaMemsetAsync(dqnorm_w, 0, gbw::H * 4, st) != cudaSuccess ||
+      cudaMemsetAsync(dknorm_w, 0, gbw::H * 4, st) != cudaSuccess ||
+      cudaMemsetAsync(dkt, 0, brow, st) != cudaSuccess) {
+    set_error("gate_bwd: clearing the outputs failed");
+    return SAS_ERR_CUDA;
+  }
+  float *xq_all = nullptr, *xc_all = nullptr;
+  SAS_TRY(launch_gate_proj_tc(p, q_nope, k_nope, wq, wk, ws + L.tc, &xq_all, &xc_all, st));
+  const int nsm = sm_count();
+  const __nv_bfloat16* qn = static_cast<const __nv_bfloat16*>(q_nope);
+  const __nv_bfloat16* kn = static_cast<const __nv_bfloat16*>(k_nope);
+  gbw_block_fwd_kernel<<<2 * nsm, gbw::kRowThreads, 0, st>>>(
+      pooled, static_cast<const __nv_bfloat16*>(wk), knorm_w, p.cu_seqlens, p.gate_rope_cos,
+      p.gate_rope_sin, p.batch, NBmax, Hkv, d, B, p.rms_eps, xk, kt);
+  gbw_row_kernel<<<4 * nsm, gbw::kRowThreads, 0, st>>>(
+      xq_all, xc_all, kt, idx, dlogg, qnorm_w, knorm_w, p.cu_seqlens, p.gate_rope_cos,
+      p.gate_rope_sin, p.batch, T, NBmax, Hkv, B, p.topk + 1, p.rms_eps, dkt, dxq, dxc, dqnorm_w,
+      dknorm_w);
+  gbw_block_bwd_kernel<<<2 * nsm, gbw::kRowThreads, 0, st>>>(
+      xk, dkt, knorm_w, p.cu_seqlens, p.gate_rope_cos, p.gate_rope_sin, p.batch, NBmax, Hkv, B,
+      p.rms_eps, dxk, dknorm_w);
+  // outer products: enough row splits that the grid covers every SM a few times
+  const int CQ = G * d, CK = 3 * d;
+  const int tq = (CQ / gbw::kTile) * (gbw::H / gbw::kTile) * Hkv;
+  const int tk = (CK / gbw::kTile) * (gbw::H / gbw::kTile) * Hkv;
+  const int sq = max(1, min(64, 4 * nsm / tq)), sk = max(1, min(64, 4 * nsm / tk));
+  gbw_outer_kernel<0><<<dim3(CQ / gbw::kTile, gbw::H / gbw::kTile, Hkv * sq), 64, 0, st>>>(
+      dxq, qn, pooled, kn, p.cu_seqlens, p.batch, T, Hq, Hkv, d, B, NBmax, CQ, sq, dwq);
+  gbw_outer_kernel<1><<<dim3(CK / gbw::kTile, gbw::H / gbw::kTile, Hkv * sk), 64, 0, st>>>(
+      dxk, qn, pooled, kn, p.cu_seqlens, p.batch, T, Hq, Hkv, d, B, NBmax, CK, sk, dwk);
+  gbw_outer_kernel<2><<<dim3(CK / gbw::kTile, gbw::H / gbw::kTile, Hkv * sk), 64, 0, st>>>(
+      dxc, qn, pooled, kn, p.cu_seqlens, p.batch, T, Hq, Hkv, d, B, NBmax, CK, sk, dwk);
+  return launch_status("gate backward", 9);   // + the prefix pass and two projection GEMMs
+}
+
+}  // namespace sas

@@ -21,6 +21,13 @@ sas_status launch_gate_scores(const sas_problem& p, const void* q_nope, const vo
                               void* workspace, cudaStream_t st);
 sas_status launch_topk(const sas_problem& p, const float* scores, const float* lse, int32_t* idx,
                        float* logg, cudaStream_t st);
+bool gate_bwd_supported(const sas_problem& p);
+size_t gate_bwd_workspace_bytes(const sas_problem& p);
+sas_status launch_gate_bwd(const sas_problem& p, const void* q_nope, const void* k_nope,
+                           const float* pooled, const void* wq, const float* qnorm_w,
+                           const void* wk, const float* knorm_w, const int32_t* idx,
+                           const float* dlogg, float* dwq, float* dqnorm_w, float* dwk,
+                           float* dknorm_w, void* workspace, cudaStream_t st);
 
 sas_status launch_attn_fwd_simt(const sas_problem& p, const void* q, const void* k, const void* v,
                                 const int32_t* idx, const float* logg, void* o, float* lse,

@@ -158,6 +158,28 @@ sas_status sas_gate_scores(const sas_problem* p, const void* q_nope, const void*
                            const void* wk, const float* knorm_w, float* scores, float* lse,
                            void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* Router backward (README intro item (b): the loss reaches the selector; paper abstract:
+ * end-to-end optimisation of the context ranking) -- gradients of one layer's gate
+ * parameters through the log-gates of the kept blocks, the selection held fixed:
+ * dL/ds[t, kv, idx[t, kv, slot]] = dlogg[t, kv, slot], then back through
+ * s = q~.k~/sqrt(h), the gate rotary, the RMSNorm and the two projections (the historical
+ * block keys from `pooled`, the current block's key from its visible prefix of k_nope).
+ * The softmax term of the gate (- softmax_j * the row sum of dlogg) is left out: it is zero
+ * for the dlogg returned by sas_attn_bwd, whose row sums vanish because the attention does
+ * not change when all log-gates of a row move by one constant.
+ * Inputs as sas_gate_scores, plus pooled fp32 [batch, NBmax, Hkv, 3d] (sas_pool_keys),
+ * idx int32 / dlogg fp32 [T, Hkv, K+1]. Outputs (overwritten, fp32): dwq [Hkv, h, G*d],
+ * dqnorm_w [h], dwk [Hkv, h, 3d], dknorm_w [h]; sums of floating-point atomics, so their low
+ * bits can change from run to run. Supported: bf16, head_dim 128, gate_hidden 128,
+ * block <= 128 (SAS_ERR_UNSUPPORTED otherwise). Workspace (sas_gate_bwd_workspace_size):
+ * word 0 receives the pipeline error code of the tensor-core projections (0 = none). */
+sas_status sas_gate_bwd_workspace_size(const sas_problem* p, size_t* bytes);
+sas_status sas_gate_bwd(const sas_problem* p, const void* q_nope, const void* k_nope,
+                        const float* pooled, const void* wq, const float* qnorm_w, const void* wk,
+                        const float* knorm_w, const int32_t* idx, const float* dlogg, float* dwq,
+                        float* dqnorm_w, float* dwk, float* dknorm_w, void* workspace,
+                        size_t workspace_bytes, cudaStream_t stream);
+
 /* A4 -- Top-K selection (README (b); model card: Training Top-K 31 historical blocks).
  * Per (t, kv): the min(K, c_t) historical blocks with the highest score (ties to
  * the lower index), ascending, then the current block c_t, then -1 padding.

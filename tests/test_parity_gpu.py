@@ -7,7 +7,7 @@ import torch
 
 import sas_inputs as si
 from oracle import sas_oracle as orc
-from parity_utils import (assert_grad_close, assert_out_close, compare_selection, to64,
+from parity_utils import (assert_grad_close, assert_out_close, compare_selection, rel_l2, to64,
                           GATE_ABS)
 
 pytestmark = pytest.mark.gpu
@@ -286,3 +286,44 @@ def test_decode_equals_prefill_row(sas):
     assert torch.equal(di[0], idx[L - 1])
     assert (dl[0] - logg[L - 1]).abs().max().item() <= GATE_ABS
     assert (od[0].float() - o[L - 1].float()).abs().max().item() <= 2e-2
+
+
+GATE_BWD_CASES = {
+    # lengths, Hq, Hkv, d, B, K, h (bf16; the router backward's supported shape)
+    "bf16-G4-K7-ragged": ([700, 300, 64, 1], 16, 4, 128, 64, 7, 128),
+    "bf16-G8-K3": ([1100, 129], 16, 2, 128, 64, 3, 128),
+}
+
+
+@pytest.mark.parametrize("name", list(GATE_BWD_CASES))
+def test_gate_backward(sas, name):
+    """Router backward vs the oracle (both fed the GPU's selection): dWq, dWk and the two
+    RMSNorm weight gradients, fp32, relative L2 <= 2e-3. dlogg is random with zero row sums
+    over the kept slots, as the attention backward's own dlogg has."""
+    lengths, Hq, Hkv, d, B, K, h = GATE_BWD_CASES[name]
+    shape = si.Shape(list(lengths), Hq, Hkv, d, B, K, h, "bf16", seed=501)
+    inp = si.prefill_inputs(shape)
+    dev = torch.device("cuda:0")
+    g = {k: v.to(dev) for k, v in inp.items() if isinstance(v, torch.Tensor)}
+    prob = sas.Problem.from_lengths(shape.lengths, dev, num_q_heads=Hq, num_kv_heads=Hkv,
+                                    head_dim=d, block=B, topk=K, gate_hidden=h,
+                                    dtype=torch.bfloat16)
+    idx, _ = sas.prefill_selection(prob, g["q_nope"], g["k_nope"], g["wq"], g["qnorm_w"], g["wk"],
+                                   g["knorm_w"])
+    pooled = sas.sas_pool_keys(prob, g["k_nope"])
+    idx_np = idx.cpu().numpy()
+    valid = idx_np >= 0
+    rng = np.random.default_rng(3)
+    dl = rng.standard_normal(idx_np.shape) * valid
+    dl -= valid * (dl.sum(axis=2, keepdims=True) / np.maximum(valid.sum(axis=2, keepdims=True), 1))
+    dlogg = torch.from_numpy(dl.astype(np.float32)).to(dev)
+    dwq, dqn, dwk, dkn = sas.sas_gate_bwd(prob, g["q_nope"], g["k_nope"], pooled, g["wq"],
+                                          g["qnorm_w"], g["wk"], g["knorm_w"], idx, dlogg)
+    torch.cuda.synchronize()
+    ref = orc.gate_backward(inp["q_nope"], inp["k_nope"], inp["wq"], inp["qnorm_w"], inp["wk"],
+                            inp["knorm_w"], idx_np, dlogg.cpu().numpy().astype(np.float64),
+                            np.asarray(shape.cu_seqlens), B, 1e-6, 1e6)
+    for gpu, key in ((dwq, "dwq"), (dqn, "dqnorm_w"), (dwk, "dwk"), (dkn, "dknorm_w")):
+        e = rel_l2(gpu, ref[key])
+        assert np.isfinite(to64(gpu)).all(), key
+        assert e <= 2e-3, f"{key}: rel-L2 {e:.3e}"
