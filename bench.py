@@ -530,8 +530,6 @@ def main():
     cs = clk.summary()
     if cs:
         line["clocks"] = cs
-    if backward:
-        line["router_bwd"] = bench_router_bwd(sas, prob, g, flush, max(3, a.steps))
 
     if not a.no_decode:
         try:
@@ -542,6 +540,9 @@ def main():
 
     if not a.no_e2e:
         line["e2e"] = e2e(sas, prob, g, backward, work, dev, a, ws)
+
+    if backward:   # after the step, decode and e2e legs, so it cannot perturb them
+        line["router_bwd"] = bench_router_bwd(sas, prob, g, flush, max(3, a.steps))
 
     if rank == 0 and ws == 1 and not a.no_cpu_baseline:
         cpu = cpu_inputs_from(g)

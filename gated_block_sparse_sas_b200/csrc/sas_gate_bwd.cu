@@ -24,8 +24,10 @@
 //      rebuilt per block by a running max / min / sum).
 #include "sas_common.cuh"
 #include "sas_kernels.h"
+#include "sas_sm100.cuh"
 
 namespace sas {
+using sm100::red_add_v4;
 
 namespace gbw {
 constexpr int H = 128;           // gate hidden of the supported configuration
@@ -83,13 +85,65 @@ __device__ __forceinline__ void gbw_norm_rope_bwd(const float x[4], const float 
   for (int k = 0; k < 4; ++k) dx[k] = du[k] / r - x[k] * dot / r3;
 }
 
+// The same two steps with lane holding 4 consecutive values e = 4 lane + k (so a row moves
+// as one 16-byte vector per lane); the rotary partner of e (e +- 64) sits in lane ^ 16.
+__device__ __forceinline__ void gbw_norm_rope_fwd_v(const float x[4], const float* __restrict__ w,
+                                                    const float* __restrict__ rc,
+                                                    const float* __restrict__ rs, int pos,
+                                                    float eps, int lane, float out[4], float u[4],
+                                                    float& r) {
+  float ss = x[0] * x[0] + x[1] * x[1] + x[2] * x[2] + x[3] * x[3];
+  ss = warp_sum(ss);
+  r = sqrtf(ss / (float)gbw::H + eps);
+  const bool lo = lane < 16;
+  const int e0 = 4 * lane, t0 = lo ? e0 : e0 - 64;   // rotary table index of e0
+  float y[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    u[k] = x[k] / r;
+    y[k] = u[k] * w[e0 + k];
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float yp = __shfl_xor_sync(0xffffffffu, y[k], 16);
+    const float c = rc[(size_t)pos * 64 + t0 + k], s = rs[(size_t)pos * 64 + t0 + k];
+    out[k] = lo ? y[k] * c - yp * s : y[k] * c + yp * s;
+  }
+}
+
+__device__ __forceinline__ void gbw_norm_rope_bwd_v(const float x[4], const float u[4], float r,
+                                                    const float* __restrict__ w,
+                                                    const float* __restrict__ rc,
+                                                    const float* __restrict__ rs, int pos,
+                                                    int lane, const float dout[4], float dx[4],
+                                                    float dw[4]) {
+  const bool lo = lane < 16;
+  const int e0 = 4 * lane, t0 = lo ? e0 : e0 - 64;
+  float du[4], dot = 0.f;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {   // the rotation's transpose: rotation by -angle
+    const float dp = __shfl_xor_sync(0xffffffffu, dout[k], 16);
+    const float c = rc[(size_t)pos * 64 + t0 + k], s = rs[(size_t)pos * 64 + t0 + k];
+    const float dy = lo ? dout[k] * c + dp * s : dout[k] * c - dp * s;
+    dw[k] += dy * u[k];
+    du[k] = dy * w[e0 + k];
+    dot += du[k] * x[k];
+  }
+  dot = warp_sum(dot);
+  const float r3 = r * r * r * (float)gbw::H;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) dx[k] = du[k] / r - x[k] * dot / r3;
+}
+
 // Sum the CTA's per-lane norm-weight gradients (4 per lane and warp) into dw[128].
-__device__ __forceinline__ void gbw_cta_add_dw(const float acc[4], float* red, float* __restrict__ dw) {
+__device__ __forceinline__ void gbw_cta_add_dw(const float acc[4], float* red, float* __restrict__ dw,
+                                               bool vec_layout) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nw = blockDim.x >> 5;
   __syncthreads();
 #pragma unroll
-  for (int k = 0; k < 4; ++k) red[warp * gbw::H + lane + 32 * k] = acc[k];
+  for (int k = 0; k < 4; ++k)
+    red[warp * gbw::H + (vec_layout ? 4 * lane + k : lane + 32 * k)] = acc[k];
   __syncthreads();
   for (int e = threadIdx.x; e < gbw::H; e += blockDim.x) {
     float s = 0.f;
@@ -170,45 +224,65 @@ __global__ void __launch_bounds__(gbw::kRowThreads) gbw_row_kernel(
     const int tg = (int)(row / Hkv), kv = (int)(row % Hkv);
     const int b = seq_of(cu, batch, tg);
     const int t = tg - cu[b], c = t / B;
-    float xq[4], xc[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      xq[k] = xq_all[row * gbw::H + lane + 32 * k];
-      xc[k] = xc_all[row * gbw::H + lane + 32 * k];
-    }
+    // lane holds e = 4 lane .. 4 lane + 3 of every row (16-byte vectors)
+    const float4 xq4 = reinterpret_cast<const float4*>(xq_all + row * gbw::H)[lane];
+    const float4 xc4 = reinterpret_cast<const float4*>(xc_all + row * gbw::H)[lane];
+    const float xq[4] = {xq4.x, xq4.y, xq4.z, xq4.w}, xc[4] = {xc4.x, xc4.y, xc4.z, xc4.w};
     float qt[4], uq[4], rq, kc[4], uc[4], rcn;
-    gbw_norm_rope_fwd(xq, qnorm_w, rc, rs, t, eps, lane, qt, uq, rq);
-    gbw_norm_rope_fwd(xc, knorm_w, rc, rs, c * B, eps, lane, kc, uc, rcn);
+    gbw_norm_rope_fwd_v(xq, qnorm_w, rc, rs, t, eps, lane, qt, uq, rq);
+    gbw_norm_rope_fwd_v(xc, knorm_w, rc, rs, c * B, eps, lane, kc, uc, rcn);
     float dqt[4] = {0.f, 0.f, 0.f, 0.f}, dkc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int sl = 0; sl < K1; ++sl) {   // warp-uniform: every lane reads the same slot
-      const int j = idx[row * K1 + sl];
-      if (j < 0) continue;
-      const float ds = dlogg[row * K1 + sl] * inv_sqrt_h;
-      if (j == c) {
+    // slots 32 at a time: lane l reads slot base + l once; the kept keys of 4 slots are
+    // loaded together before their arithmetic
+    const size_t krow = (size_t)b * NBmax;
+    for (int base = 0; base < K1; base += 32) {
+      const int my = base + lane;
+      const int jl = my < K1 ? idx[row * K1 + my] : -1;
+      const float dsl = my < K1 ? dlogg[row * K1 + my] * inv_sqrt_h : 0.f;
+      const int ns = min(32, K1 - base);
+      for (int s0 = 0; s0 < ns; s0 += 4) {
+        int jj[4];
+        float dd[4];
+        float4 kj[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          dqt[k] = fmaf(ds, kc[k], dqt[k]);
-          dkc[k] = fmaf(ds, qt[k], dkc[k]);
+        for (int u = 0; u < 4; ++u) {
+          jj[u] = __shfl_sync(0xffffffffu, jl, (s0 + u) & 31);
+          dd[u] = __shfl_sync(0xffffffffu, dsl, (s0 + u) & 31);
+          if (s0 + u >= ns) jj[u] = -1;
+          kj[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (jj[u] >= 0 && jj[u] != c)
+            kj[u] = reinterpret_cast<const float4*>(
+                kt_hist + ((krow + jj[u]) * Hkv + kv) * gbw::H)[lane];
         }
-      } else {
-        const size_t kr = (((size_t)b * NBmax + j) * Hkv + kv) * gbw::H;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          dqt[k] = fmaf(ds, kt_hist[kr + lane + 32 * k], dqt[k]);
-          atomicAdd(dkt_hist + kr + lane + 32 * k, ds * qt[k]);
+        for (int u = 0; u < 4; ++u) {   // warp-uniform branches: every lane holds slot u
+          if (jj[u] < 0) continue;
+          const float ds = dd[u];
+          if (jj[u] == c) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              dqt[k] = fmaf(ds, kc[k], dqt[k]);
+              dkc[k] = fmaf(ds, qt[k], dkc[k]);
+            }
+          } else {
+            dqt[0] = fmaf(ds, kj[u].x, dqt[0]);
+            dqt[1] = fmaf(ds, kj[u].y, dqt[1]);
+            dqt[2] = fmaf(ds, kj[u].z, dqt[2]);
+            dqt[3] = fmaf(ds, kj[u].w, dqt[3]);
+            red_add_v4(dkt_hist + ((krow + jj[u]) * Hkv + kv) * gbw::H + 4 * lane,
+                       make_float4(ds * qt[0], ds * qt[1], ds * qt[2], ds * qt[3]));
+          }
         }
       }
     }
     float dx[4];
-    gbw_norm_rope_bwd(xq, uq, rq, qnorm_w, rc, rs, t, lane, dqt, dx, dwq);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) dxq_out[row * gbw::H + lane + 32 * k] = dx[k];
-    gbw_norm_rope_bwd(xc, uc, rcn, knorm_w, rc, rs, c * B, lane, dkc, dx, dwk);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) dxc_out[row * gbw::H + lane + 32 * k] = dx[k];
+    gbw_norm_rope_bwd_v(xq, uq, rq, qnorm_w, rc, rs, t, lane, dqt, dx, dwq);
+    reinterpret_cast<float4*>(dxq_out + row * gbw::H)[lane] = make_float4(dx[0], dx[1], dx[2], dx[3]);
+    gbw_norm_rope_bwd_v(xc, uc, rcn, knorm_w, rc, rs, c * B, lane, dkc, dx, dwk);
+    reinterpret_cast<float4*>(dxc_out + row * gbw::H)[lane] = make_float4(dx[0], dx[1], dx[2], dx[3]);
   }
-  gbw_cta_add_dw(dwq, red, dqnorm_w);
-  gbw_cta_add_dw(dwk, red, dknorm_w);
+  gbw_cta_add_dw(dwq, red, dqnorm_w, true);
+  gbw_cta_add_dw(dwk, red, dknorm_w, true);
 }
 
 // (3) block keys backward: dk~_j -> dxk_j, knorm_w gradient.
@@ -243,7 +317,7 @@ __global__ void __launch_bounds__(gbw::kRowThreads) gbw_block_bwd_kernel(
 #pragma unroll
     for (int k = 0; k < 4; ++k) xo[lane + 32 * k] = dx[k];
   }
-  gbw_cta_add_dw(dwk, red, dknorm_w);
+  gbw_cta_add_dw(dwk, red, dknorm_w, false);
 }
 
 // (4) dW[kv][i][c] += sum over rows of X[row][kv][i] * Y[row][kv][c], a 64 x 64 tile of dW per
@@ -291,22 +365,35 @@ __global__ void __launch_bounds__(64) gbw_outer_kernel(
     const int nrows = MODE == 0 ? T : batch * NBmax;
     const int per = (nrows + nsplit - 1) / nsplit;
     const int r0 = split * per, r1 = min(nrows, r0 + per);
+    // the next step's 16 x 64 tiles are loaded into registers while this step computes
+    constexpr int kPer = gbw::kKs * gbw::kTile / 64;   // elements of each tile per thread
+    float xr[kPer], yr[kPer];
+    auto load = [&](int rb) {
+#pragma unroll
+      for (int q = 0; q < kPer; ++q) {
+        const int e = tid + 64 * q, k = e / gbw::kTile, col = e % gbw::kTile;
+        const int r = rb + k;
+        xr[q] = 0.f;
+        yr[q] = 0.f;
+        if (r < r1) {
+          xr[q] = X[((size_t)r * Hkv + kv) * gbw::H + i0 + col];
+          if constexpr (MODE == 0)
+            yr[q] = __bfloat162float(q_nope[((size_t)r * Hq + (size_t)kv * G) * d + c0 + col]);
+          else
+            yr[q] = pooled[((size_t)r * Hkv + kv) * C + c0 + col];
+        }
+      }
+    };
+    if (r0 < r1) load(r0);
     for (int rb = r0; rb < r1; rb += gbw::kKs) {
       const int nk = min(gbw::kKs, r1 - rb);
-      for (int e = tid; e < gbw::kKs * gbw::kTile; e += 64) {
-        const int k = e / gbw::kTile, col = e % gbw::kTile;
-        const int r = rb + k;
-        float xv = 0.f, yv = 0.f;
-        if (k < nk) {
-          xv = X[((size_t)r * Hkv + kv) * gbw::H + i0 + col];
-          if constexpr (MODE == 0)
-            yv = __bfloat162float(q_nope[((size_t)r * Hq + (size_t)kv * G) * d + c0 + col]);
-          else
-            yv = pooled[((size_t)r * Hkv + kv) * C + c0 + col];
-        }
-        Xs[k][col] = xv;
-        Ys[k][col] = yv;
+#pragma unroll
+      for (int q = 0; q < kPer; ++q) {
+        const int e = tid + 64 * q;
+        Xs[e / gbw::kTile][e % gbw::kTile] = xr[q];
+        Ys[e / gbw::kTile][e % gbw::kTile] = yr[q];
       }
+      if (rb + gbw::kKs < r1) load(rb + gbw::kKs);
       fma_step(nk);
     }
   } else {
@@ -434,7 +521,7 @@ sas_status launch_gate_bwd(const sas_problem& p, const void* q_nope, const void*
   const int CQ = G * d, CK = 3 * d;
   const int tq = (CQ / gbw::kTile) * (gbw::H / gbw::kTile) * Hkv;
   const int tk = (CK / gbw::kTile) * (gbw::H / gbw::kTile) * Hkv;
-  const int sq = max(1, min(64, 4 * nsm / tq)), sk = max(1, min(64, 4 * nsm / tk));
+  const int sq = max(1, min(64, 16 * nsm / tq)), sk = max(1, min(64, 16 * nsm / tk));
   gbw_outer_kernel<0><<<dim3(CQ / gbw::kTile, gbw::H / gbw::kTile, Hkv * sq), 64, 0, st>>>(
       dxq, qn, pooled, kn, p.cu_seqlens, p.batch, T, Hq, Hkv, d, B, NBmax, CQ, sq, dwq);
   gbw_outer_kernel<1><<<dim3(CK / gbw::kTile, gbw::H / gbw::kTile, Hkv * sk), 64, 0, st>>>(
