@@ -292,6 +292,7 @@ GATE_BWD_CASES = {
     # lengths, Hq, Hkv, d, B, K, h (bf16; the router backward's supported shape)
     "bf16-G4-K7-ragged": ([700, 300, 64, 1], 16, 4, 128, 64, 7, 128),
     "bf16-G8-K3": ([1100, 129], 16, 2, 128, 64, 3, 128),
+    "bf16-G5-K15-long": ([5000, 300], 10, 2, 128, 64, 15, 128),
 }
 
 
