@@ -129,3 +129,29 @@ def test_binding_argument_counts_match_the_header(sas):
         params = decls[name].strip()
         n = 0 if params in ("", "void") else params.count(",") + 1
         assert n == len(args), f"{name}: header {n} parameters, binding {len(args)}"
+
+
+def test_gate_bwd_argument_checks(sas):
+    """Router backward: NULL outputs and unsupported shapes are rejected before any launch."""
+    lib = sas.lib_handle()
+    p = _prob(sas)
+    ptrs = [0x10000 + 0x100 * i for i in range(13)]
+    ptrs[12] = 0   # dknorm_w
+    st = lib.sas_gate_bwd(ctypes.byref(p), *ptrs, 0x90000, 1 << 30, None)
+    assert st == sas.SAS_ERR_INVALID_ARG and "NULL" in lib.sas_last_error().decode()
+    n = ctypes.c_size_t(0)
+    p32 = _prob(sas, dtype=sas.SAS_FP32)
+    assert lib.sas_gate_bwd_workspace_size(ctypes.byref(p32), ctypes.byref(n)) == sas.SAS_ERR_UNSUPPORTED
+    assert "gate_bwd" in lib.sas_last_error().decode()
+
+
+def test_decode_ungated_flag_is_checked(sas):
+    lib = sas.lib_handle()
+    n = ctypes.c_size_t(0)
+    d = sas.SasDecodeProblem(batch=4, capacity=4096, num_q_heads=32, num_kv_heads=8, head_dim=128,
+                             block=64, topk=31, gate_hidden=128, rms_eps=1e-6, dtype=sas.SAS_BF16,
+                             seqlens=0x1000, gate_rope_cos=0x2000, gate_rope_sin=0x3000, ungated=1)
+    assert lib.sas_decode_workspace_size(ctypes.byref(d), ctypes.byref(n)) == 0
+    d.ungated = 2
+    assert lib.sas_decode_workspace_size(ctypes.byref(d), ctypes.byref(n)) == sas.SAS_ERR_INVALID_ARG
+    assert "ungated" in lib.sas_last_error().decode()
