@@ -7,9 +7,10 @@ import sas_inputs as si
 from oracle import sas_oracle as orc
 
 
-@pytest.mark.parametrize("L", [1, 16, 17, 63, 100, 128])
-def test_decode_equals_prefill_last_row(L):
-    B, K, h = 16, 3, 16
+@pytest.mark.parametrize("L,K", [(1, 3), (16, 3), (17, 3), (63, 3), (100, 3), (128, 3),
+                                 (300, 15), (290, 7)])
+def test_decode_equals_prefill_last_row(L, K):
+    B, h = 16, 16
     shape = si.Shape([L], 4, 2, 8, B, K, h, "fp32", seed=20 + L)
     inp = si.prefill_inputs(shape)
     sel = orc.prefill_selection(inp["q_nope"], inp["k_nope"], inp["wq"], inp["qnorm_w"], inp["wk"],
