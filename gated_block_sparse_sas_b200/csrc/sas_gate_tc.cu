@@ -214,7 +214,7 @@ sas_status launch_gate_proj_tc(const sas_problem& p, const void* q_nope, const v
       !make_tmap_bf16_2d(&tAk, ak, (uint64_t)Hkv * gtc::kKCols, T, (uint64_t)Hkv * gtc::kKCols * 2,
                          64, 128) ||
       !make_tmap_bf16_2d(&tBk, wk, 384, (uint64_t)Hkv * 128, 384 * 2, 64, 128)) {
-    set_error("gate_scores: TMA descriptor creation failed");
+    set_error("gate projections: TMA descriptor creation failed");
     return SAS_ERR_CUDA;
   }
   static std::once_flag attr_once;
