@@ -63,6 +63,7 @@ _SIGS = {
     "sas_decode_workspace_size": ([_DP, ctypes.POINTER(_sz)], ctypes.c_int),
     "sas_decode": ([_DP] + [_vp] * 14 + [_sz, _vp], ctypes.c_int),
     "sas_decode_noalloc": ([_DP] + [_vp] * 13 + [_vp], ctypes.c_int),
+    "sas_decode_noalloc_error_word": ([ctypes.POINTER(_vp)], ctypes.c_int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -79,6 +80,64 @@ class SasError(RuntimeError):
 def _check(status: int, where: str):
     if status != SAS_OK:
         raise SasError(status, where)
+
+
+# Device-side error codes written to word 0 of a workspace (include/sas.h, "Device-side errors").
+ERROR_CODES = {
+    41: "decode attention: a bounded wait gave up",
+    51: "attn_fwd: a bounded wait gave up", 52: "attn_fwd: a bounded wait gave up",
+    53: "attn_fwd: a bounded wait gave up", 54: "attn_fwd: a bounded wait gave up",
+    55: "attn_fwd: a bounded wait gave up", 56: "attn_fwd: a bounded wait gave up",
+    57: "attn_fwd: a bounded wait gave up",
+    60: "attn_fwd: a row's largest logit exceeds its own key's by more than ~97 nats",
+    61: "decode: a row's largest logit exceeds its own key's by more than ~97 nats",
+    71: "attn_bwd: a bounded wait gave up", 72: "attn_bwd: a bounded wait gave up",
+    73: "attn_bwd: a bounded wait gave up", 74: "attn_bwd: a bounded wait gave up",
+    75: "attn_bwd: a bounded wait gave up", 76: "attn_bwd: a bounded wait gave up",
+    77: "attn_bwd: a bounded wait gave up", 78: "attn_bwd: a bounded wait gave up",
+    79: "attn_bwd: a bounded wait gave up",
+    81: "decode attention: a bounded wait gave up", 82: "decode attention: a bounded wait gave up",
+    83: "decode attention: a bounded wait gave up",
+    91: "gate projections: a bounded wait gave up", 92: "gate projections: a bounded wait gave up",
+    93: "gate projections: a bounded wait gave up",
+}
+
+
+class SasDeviceError(RuntimeError):
+    """A kernel reported a device-side failure through a workspace's error word."""
+
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: device error code {code}: "
+                         f"{ERROR_CODES.get(code, 'unknown code')}")
+
+
+def error_code(workspace) -> int:
+    """Word 0 of a workspace after its call: 0, or the device-side error code. Reading it
+    waits for the work queued so far on the workspace's device."""
+    return int(workspace[:4].view(torch.int32).item())
+
+
+def check_workspace(workspace, where: str = "sas"):
+    """Raise SasDeviceError if the call that used `workspace` reported a device-side error."""
+    code = error_code(workspace)
+    if code != 0:
+        raise SasDeviceError(code, where)
+
+
+def decode_noalloc_error_code() -> int:
+    """Error word of the last sas_decode_noalloc call on the current device (0 = none). The
+    read is ordered after the work queued on the current stream."""
+    addr = _vp()
+    _check(_lib.sas_decode_noalloc_error_word(ctypes.byref(addr)), "sas_decode_noalloc_error_word")
+    out = np.zeros(1, dtype=np.int32)
+    torch.cuda.current_stream().synchronize()
+    cudart = ctypes.CDLL("libcudart.so.12")          # the runtime torch has already loaded
+    cudart.cudaMemcpy.argtypes = [_vp, _vp, _sz, ctypes.c_int]
+    err = cudart.cudaMemcpy(out.ctypes.data, addr.value, 4, 2)   # 2 = device to host
+    if err != 0:
+        raise RuntimeError(f"reading the no-alloc error word failed: cudaError {err}")
+    return int(out[0])
 
 
 def _ptr(t):
@@ -250,7 +309,10 @@ def attn_bwd_workspace(p: Problem):
     return _workspace(_lib.sas_attn_bwd_workspace_size, p.ref, p.device)
 
 
-def sas_attn_fwd(p: Problem, q, k, v, idx, logg, o=None, lse=None, workspace=None, stream=None):
+def sas_attn_fwd(p: Problem, q, k, v, idx, logg, o=None, lse=None, workspace=None, stream=None,
+                 check: bool = False):
+    """Gated sparse attention forward. check=True waits for the call and raises
+    SasDeviceError if its workspace error word is set."""
     if o is None:
         o = torch.empty((p.total_tokens, p.num_q_heads, p.head_dim), dtype=p.dtype, device=p.device)
     if lse is None:
@@ -258,11 +320,14 @@ def sas_attn_fwd(p: Problem, q, k, v, idx, logg, o=None, lse=None, workspace=Non
     ws = workspace if workspace is not None else _workspace(_lib.sas_attn_fwd_workspace_size, p.ref, p.device)
     _check(_lib.sas_attn_fwd(p.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(logg), _ptr(o),
                              _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)), "sas_attn_fwd")
+    if check:
+        check_workspace(ws, "sas_attn_fwd")
     return o, lse
 
 
 def sas_attn_bwd(p: Problem, q, k, v, o, dout, lse, idx, logg, dq=None, dk=None, dv=None,
-                 dlogg=None, workspace=None, stream=None):
+                 dlogg=None, workspace=None, stream=None, check: bool = False):
+    """Backward of the gated sparse attention; check=True as in sas_attn_fwd."""
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
@@ -273,6 +338,8 @@ def sas_attn_bwd(p: Problem, q, k, v, o, dout, lse, idx, logg, dq=None, dk=None,
     _check(_lib.sas_attn_bwd(p.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
                              _ptr(idx), _ptr(logg), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dlogg),
                              _ptr(ws), ws.numel(), _stream(stream)), "sas_attn_bwd")
+    if check:
+        check_workspace(ws, "sas_attn_bwd")
     return dq, dk, dv, dlogg
 
 
@@ -328,7 +395,9 @@ class DecodeProblem:
 
 def sas_decode(p: DecodeProblem, q, q_nope, k_cache, v_cache, gate_key_cache, cur_pool, wq,
                qnorm_w, wk, knorm_w, o=None, idx_out=None, logg_out=None, workspace=None,
-               stream=None, want_selection: bool = False):
+               stream=None, want_selection: bool = False, check: bool = False):
+    """One sparse decode step; check=True waits for the call and raises SasDeviceError if
+    its workspace error word is set."""
     if o is None:
         o = torch.empty((p.batch, p.num_q_heads, p.head_dim), dtype=p.dtype, device=p.device)
     if want_selection and idx_out is None:
@@ -341,6 +410,8 @@ def sas_decode(p: DecodeProblem, q, q_nope, k_cache, v_cache, gate_key_cache, cu
                            _ptr(gate_key_cache), _ptr(cur_pool), _ptr(wq), _ptr(qnorm_w), _ptr(wk),
                            _ptr(knorm_w), _ptr(o), _ptr(idx_out), _ptr(logg_out), _ptr(ws),
                            ws.numel(), _stream(stream)), "sas_decode")
+    if check:
+        check_workspace(ws, "sas_decode")
     return (o, idx_out, logg_out) if want_selection else o
 
 

@@ -81,6 +81,16 @@ static sas_status check_problem(const sas_problem* p, bool needs_rope) {
   return SAS_OK;
 }
 
+// Word 0 of a workspace is the call's pipeline error code: cleared (stream-ordered) before the
+// call's kernels, so after the stream completes it holds this call's code and no earlier one.
+static sas_status clear_error_word(void* workspace, cudaStream_t stream) {
+  if (cudaMemsetAsync(workspace, 0, sizeof(int32_t), stream) != cudaSuccess) {
+    set_error("clearing the workspace error word failed");
+    return SAS_ERR_CUDA;
+  }
+  return SAS_OK;
+}
+
 #define SAS_PTR(ptr)                                                        \
   do {                                                                      \
     SAS_CHECK_ARG((ptr) != nullptr, "%s is NULL", #ptr);                    \
@@ -161,6 +171,7 @@ sas_status sas_gate_scores(const sas_problem* p, const void* q_nope, const void*
     set_error("workspace too small: %zu < %zu bytes", workspace_bytes, need);
     return SAS_ERR_WORKSPACE;
   }
+  SAS_TRY(clear_error_word(workspace, stream));
   return launch_gate_scores(*p, q_nope, k_nope, gate_keys, wq, qnorm_w, wk, knorm_w, scores, lse,
                             workspace, stream);
 }
@@ -216,6 +227,7 @@ sas_status sas_gate_bwd(const sas_problem* p, const void* q_nope, const void* k_
     set_error("workspace too small: %zu < %zu bytes", workspace_bytes, need);
     return SAS_ERR_WORKSPACE;
   }
+  SAS_TRY(clear_error_word(workspace, stream));
   return launch_gate_bwd(*p, q_nope, k_nope, pooled, wq, qnorm_w, wk, knorm_w, idx, dlogg, dwq,
                          dqnorm_w, dwk, dknorm_w, workspace, stream);
 }
@@ -258,6 +270,7 @@ sas_status sas_attn_fwd(const sas_problem* p, const void* q, const void* k, cons
     set_error("workspace too small: %zu < %zu bytes", workspace_bytes, need);
     return SAS_ERR_WORKSPACE;
   }
+  SAS_TRY(clear_error_word(workspace, stream));
   if (attn_fwd_km_supported(*p))
     return launch_attn_fwd_km(*p, q, k, v, idx, logg, o, lse_attn, workspace, stream);
   return launch_attn_fwd_simt(*p, q, k, v, idx, logg, o, lse_attn, stream);
@@ -303,6 +316,7 @@ sas_status sas_attn_bwd(const sas_problem* p, const void* q, const void* k, cons
     }
   }
   if (p->total_tokens == 0) return SAS_OK;
+  SAS_TRY(clear_error_word(workspace, stream));
   if (attn_bwd_km_supported(*p))
     return launch_attn_bwd_km(*p, q, k, v, o, dout, lse_attn, idx, logg, dq, dk, dv, dlogg,
                               workspace, stream);

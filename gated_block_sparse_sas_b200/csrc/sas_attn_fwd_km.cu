@@ -145,9 +145,11 @@ __global__ void km_finalize_kernel(const float* __restrict__ oacc, const float* 
   const bool good = l > 0.f && isfinite(l);
   const float inv = good ? 1.f / l : 0.f;
   const float4 x = reinterpret_cast<const float4*>(oacc + (size_t)row * kmf::kD)[lane];
-  uint2 pk;
-  pk.x = pack_bf16x2(x.x * inv, x.y * inv);
-  pk.y = pack_bf16x2(x.z * inv, x.w * inv);
+  uint2 pk = make_uint2(0u, 0u);   // a row outside the reference's range (error 60) is 0
+  if (good) {
+    pk.x = pack_bf16x2(x.x * inv, x.y * inv);
+    pk.y = pack_bf16x2(x.z * inv, x.w * inv);
+  }
   reinterpret_cast<uint2*>(o + (size_t)row * kmf::kD)[lane] = pk;
   if (lane == 0) {
     lse[row] = good ? (mref[row] + log2f(l)) * kLn2 : -INFINITY;

@@ -710,7 +710,9 @@ __global__ void decode_merge_kernel(const float* __restrict__ part_ml, const flo
       ls += part_ml[pr * 2 + 1] * f;
       as += part_acc[pr * D + ch] * f;
     }
-    o[((size_t)b * Hq + kv * G + g) * D + ch] = from_f<T>(ls > 0.f ? as / ls : 0.f);
+    // a head outside the fixed reference's range (error 61: ls overflowed) is written as 0
+    o[((size_t)b * Hq + kv * G + g) * D + ch] =
+        from_f<T>(ls > 0.f && isfinite(ls) ? as / ls : 0.f);
   }
 }
 
@@ -728,8 +730,8 @@ size_t decode_workspace_bytes(const sas_decode_problem& p) {
   const size_t pairs = (size_t)p.batch * p.num_kv_heads;
   const size_t ns = decode_nsplit(p);
   auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
-  return al(pairs * (p.topk + 1) * 4) * 2 + al(pairs * ns * G * 2 * 4) +
-         al(pairs * ns * G * p.head_dim * 4) + 256;   // + error word
+  return 256 /* error word */ + al(pairs * (p.topk + 1) * 4) * 2 + al(pairs * ns * G * 2 * 4) +
+         al(pairs * ns * G * p.head_dim * 4);
 }
 
 template <int G>
@@ -814,6 +816,13 @@ sas_status launch_decode(const sas_decode_problem& p, const void* q, const void*
   const int ns = decode_nsplit(p);
   auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
   char* w = (char*)ws;
+  // word 0: this call's error code (0 = none), cleared first so it never reports an earlier call
+  int* err = (int*)w;
+  if (cudaMemsetAsync(err, 0, sizeof(int), st) != cudaSuccess) {
+    set_error("decode: clearing the error word failed");
+    return SAS_ERR_CUDA;
+  }
+  w += 256;
   int32_t* sel_idx = (int32_t*)w;
   w += al(pairs * (p.topk + 1) * 4);
   float* sel_logg = (float*)w;
@@ -822,7 +831,6 @@ sas_status launch_decode(const sas_decode_problem& p, const void* q, const void*
   w += al(pairs * ns * G * 2 * 4);
   float* part_acc = (float*)w;
   w += al(pairs * ns * G * p.head_dim * 4);
-  int* err = (int*)w;
   if (p.dtype == SAS_BF16)
     decode_gate_launch<__nv_bfloat16>(p, q_nope, gkc, cur_pool, wq, qnorm_w, wk, knorm_w, sel_idx,
                                       sel_logg, idx_out, logg_out, st);

@@ -13,8 +13,15 @@
 // sas_decode_workspace_size reports) exceeds that is rejected with SAS_ERR_UNSUPPORTED.
 // All calls on a device share the one array: calls whose kernels overlap on the GPU (two
 // streams, or two threads) race on it, so serialise them. The array keeps whatever the
-// previous call left; the decode kernels write every scratch element they later read, so
-// nothing has to start at zero.
+// previous call left; the decode kernels write every scratch element they later read, and
+// the one word that must start at zero -- the error word, the array's first int32 -- is
+// cleared by each call on its stream (cudaMemsetAsync, which allocates nothing).
+// sas_decode_noalloc_error_word hands out that word's device address so the caller can read
+// the status of its last call.
+//
+// The address of the array is looked up once per device ordinal and cached. The stream must
+// belong to the current device, and a cudaDeviceReset of that device (which would reload the
+// module at a new address) is not supported while the library stays loaded.
 #include <mutex>
 
 #include "sas_common.cuh"
@@ -80,4 +87,16 @@ extern "C" sas_status sas_decode_noalloc(const sas_decode_problem* p, const void
   if (s2 != SAS_OK) return s2;
   return sas_decode(p, q, q_nope, k_cache, v_cache, gate_key_cache, cur_pool, wq, qnorm_w, wk,
                     knorm_w, o, idx_out, logg_out, scratch, sas::kNoAllocScratchBytes, stream);
+}
+
+extern "C" sas_status sas_decode_noalloc_error_word(const int32_t** word) {
+  if (word == nullptr) {
+    sas::set_error("sas_decode_noalloc_error_word: word is NULL");
+    return SAS_ERR_INVALID_ARG;
+  }
+  void* scratch = nullptr;
+  const sas_status st = sas::scratch_on_current_device(&scratch);
+  if (st != SAS_OK) return st;
+  *word = static_cast<const int32_t*>(scratch);   // word 0 of the scratch: the error code
+  return SAS_OK;
 }

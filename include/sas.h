@@ -42,6 +42,16 @@
  *     and return a negative status; sas_last_error() (thread-local) then holds
  *     the reason. A failed launch returns SAS_ERR_CUDA. Nothing is launched
  *     after the first error of a call.
+ *   - Device-side errors: every entry point that takes a workspace uses its first
+ *     int32 (word 0) as the call's error word. The call clears it on `stream`
+ *     before its kernels run, and a kernel that meets a device-side failure
+ *     writes a nonzero code there; read it once the stream has completed
+ *     (0 = none). Codes: 41, 81-83 decode waits that gave up (bounded mbarrier
+ *     waits, about one second); 51-57 forward, 71-79 backward, 91-93 gate
+ *     projection waits that gave up; 60 forward / 61 decode: a row whose largest
+ *     logit exceeds its own key's logit by more than ~97 nats (outside the fixed
+ *     per-row reference's fp32 range; that row's output is 0 and its lse -inf).
+ *     The outputs of a call with a nonzero code are not valid.
  *   - Supported: d in {64, 128}; B in {16, 32, 64}; 1 <= K <= 127;
  *     h in {32, 64, 128}; G in {1, 2, 4, 5, 8}; NBmax <= 2048 (prefill) or
  *     ceil(capacity / B) <= 4096 (decode). Anything else returns
@@ -172,7 +182,7 @@ sas_status sas_gate_scores(const sas_problem* p, const void* q_nope, const void*
  * dqnorm_w [h], dwk [Hkv, h, 3d], dknorm_w [h]; sums of floating-point atomics, so their low
  * bits can change from run to run. Supported: bf16, head_dim 128, gate_hidden 128,
  * block <= 128 (SAS_ERR_UNSUPPORTED otherwise). Workspace (sas_gate_bwd_workspace_size):
- * word 0 receives the pipeline error code of the tensor-core projections (0 = none). */
+ * word 0 is the call's error word (the tensor-core projections' codes 91-93; 0 = none). */
 sas_status sas_gate_bwd_workspace_size(const sas_problem* p, size_t* bytes);
 sas_status sas_gate_bwd(const sas_problem* p, const void* q_nope, const void* k_nope,
                         const float* pooled, const void* wq, const float* qnorm_w, const void* wk,
@@ -195,8 +205,8 @@ sas_status sas_topk(const sas_problem* p, const float* scores, const float* lse,
  * q dtype [T, Hq, d]; k, v dtype [T, Hkv, d] (rotated); idx/logg as from sas_topk
  * (any valid selection: ascending historical, current block, -1 padding);
  * o dtype [T, Hq, d]; lse_attn fp32 [T, Hq].
- * Workspace: word 0 receives a pipeline error code (0 = none; checked by the caller after
- * the stream completes). For bf16, d = 128, B = 64 the workspace also holds fp32 output
+ * Workspace: word 0 is the call's error word (cleared by the call; 0 = none; read by the
+ * caller after the stream completes). For bf16, d = 128, B = 64 the workspace also holds fp32 output
  * accumulators [T, Hq, d + 1], per-row reference logits and the inverted selection lists
  * (blocks -> kept tokens), about T*Hq*520 + T*Hkv*(K+1)*8 bytes. In that configuration the
  * per-block partial sums are added with L2 reductions, so the low bits of o and lse_attn
@@ -229,7 +239,9 @@ sas_status sas_attn_bwd(const sas_problem* p, const void* q, const void* k, cons
  * k_cache, v_cache dtype [batch, Hkv, capacity, d]; gate_key_cache bf16
  * [batch, Hkv, NBmax, h] (entries j < c read); cur_pool fp32 [batch, Hkv, 3, d]
  * (max, min, sum over tokens c*B..L_b-1); wq, wk, qnorm_w, knorm_w as A3;
- * o dtype [batch, Hq, d]; idx_out int32 / logg_out fp32 [batch, Hkv, K+1] may be NULL. */
+ * o dtype [batch, Hq, d]; idx_out int32 / logg_out fp32 [batch, Hkv, K+1] may be NULL.
+ * Workspace (sas_decode_workspace_size): word 0 is the call's error word (cleared by the
+ * call; 41 / 81-83 a bounded wait gave up, 61 a row outside the fixed reference's range). */
 sas_status sas_decode_workspace_size(const sas_decode_problem* p, size_t* bytes);
 sas_status sas_decode(const sas_decode_problem* p, const void* q, const void* q_nope,
                       const void* k_cache, const void* v_cache, const void* gate_key_cache,
@@ -246,15 +258,28 @@ sas_status sas_decode(const sas_decode_problem* p, const void* q, const void* q_
  * array inside the library, held on every GPU that loads the library until the process
  * exits. Problems needing more scratch than that (sas_decode_workspace_size) return
  * SAS_ERR_UNSUPPORTED. The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress); make that first call before any stream capture. Calls whose
- * kernels overlap on the GPU share the one array and race: serialise them. Nothing in the
- * scratch needs to start at zero. Allocates nothing (no cudaMalloc/cudaFree). */
+ * (cudaGetSymbolAddress); make that first call before any stream capture. The stream must
+ * belong to the current device; a cudaDeviceReset while the library stays loaded is not
+ * supported (the cached address would be stale). Calls whose kernels overlap on the GPU
+ * share the one array and race: serialise them. The only scratch word that must start at
+ * zero, the error word (word 0, as sas_decode's workspace word 0), is cleared by each call
+ * on its stream; sas_decode_noalloc_error_word gives its address. Allocates nothing (no
+ * cudaMalloc/cudaFree). */
 sas_status sas_decode_noalloc(const sas_decode_problem* p, const void* q, const void* q_nope,
                               const void* k_cache, const void* v_cache,
                               const void* gate_key_cache, const float* cur_pool,
                               const void* wq, const float* qnorm_w, const void* wk,
                               const float* knorm_w, void* o, int32_t* idx_out,
                               float* logg_out, cudaStream_t stream);
+
+/* Device address of sas_decode_noalloc's error word on the current device (no counterpart
+ * in the SAS pages). The word is the first int32 of the built-in scratch: each
+ * sas_decode_noalloc call clears it on its stream and its kernels write a nonzero code on a
+ * device-side failure (the codes of sas_decode's workspace word 0). Read it after the call
+ * with a stream-ordered copy on the same stream, e.g. cudaMemcpyAsync into a host int32 and
+ * a stream synchronise. Like the decode call, the first use on a device looks the address
+ * up. Allocates nothing. */
+sas_status sas_decode_noalloc_error_word(const int32_t** word);
 
 #ifdef __cplusplus
 }

@@ -49,11 +49,14 @@ Where the pages leave a step open, the reading used here is stated at that step:
   R13 router backward: gradients of the gate parameters through the kept blocks'
       log-gates with the selection fixed (see gate_backward).
 
-Parity pins live in tests/test_oracle_*.py. The gate's composition (R3-R5, R7) has
-no worked example on the pages: its parts are pinned by properties (rotary relative
-position, RMSNorm scale invariance, prefix/full-block pooling agreement, the
-parameter-count arithmetic) but the exact composition and the 1/sqrt(h) scale are
-readings -- parity unpinned for those.
+Parity pins live in tests/test_oracle_*.py and tests/test_gate_second_impl.py. The
+gate's composition (R1-R7) has no worked example on the pages; besides the properties of
+its parts (rotary relative position, RMSNorm scale invariance, prefix/full-block pooling
+agreement, the parameter-count arithmetic) it is pinned by a second, independently
+structured implementation of the same readings (torch fp64, explicit per-head and
+per-block loops, complex-exponential rotary) on several sequences with non-unit norm
+weights. The readings themselves (concatenation order, norm before rotary, the 1/sqrt(h)
+scale, the prefix-pooled current key) remain readings of the pages.
 """
 from __future__ import annotations
 
@@ -527,7 +530,8 @@ def gate_backward(q_nope, k_nope, wq, qnorm_w, wk, knorm_w, idx, dlogg, cu_seqle
 # ------------------------------------------------------------------------------------------
 
 def decode(q, q_nope, k_cache, v_cache, lengths, gate_key_cache, cur_pool, wq, qnorm_w, wk, knorm_w,
-           block: int, K: int, eps: float, base: float, rows=None, gated: bool = True):
+           block: int, K: int, eps: float, base: float, rows=None, gated: bool = True,
+           selection=None):
     """One decode step for (some) sequences.
 
     Sequence b has L_b tokens cached, the newest at position L_b-1 with c = (L_b-1)//B.
@@ -537,6 +541,9 @@ def decode(q, q_nope, k_cache, v_cache, lengths, gate_key_cache, cur_pool, wq, q
     gated=False keeps the selection but drops the log-gate from the attention logits (hard
     selection, as a serving backend that uses the gate only to pick blocks computes it;
     Hugging Face card "tencent/Simple-Attention-Sparsification", SGLang seer_attn section).
+    `selection` = (idx, logg) [n, Hkv, K+1] replaces the gate's own Top-K in the attention:
+    at a near-tie two selections are both correct, and the attention is then evaluated on
+    the one given (the gate's own selection is still returned).
     Returns O [n, Hq, d], idx [n, Hkv, K+1], logg [n, Hkv, K+1], margin [n, Hkv].
     """
     q, qn = as64(q), as64(q_nope)
@@ -571,8 +578,14 @@ def decode(q, q_nope, k_cache, v_cache, lengths, gate_key_cache, cur_pool, wq, q
             idx[r, kv, : len(ids)] = ids
             logg[r, kv, : len(ids)] = s[ids] - lse
             margin[r, kv] = mg
+            if selection is None:
+                use_ids, use_lg = ids, s[ids] - lse
+            else:
+                keep = np.asarray(selection[0][r, kv]) >= 0
+                use_ids = np.asarray(selection[0][r, kv])[keep]
+                use_lg = as64(selection[1][r, kv])[keep]
             bias = np.full(L, NEG_INF)
-            for j, lg in zip(ids, s[ids] - lse):
+            for j, lg in zip(use_ids, use_lg):
                 bias[j * block: min((j + 1) * block, L)] = lg if gated else 0.0
             kk, vv = kcache[kv, :L], vcache[kv, :L]
             for g in range(G):

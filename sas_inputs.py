@@ -240,12 +240,19 @@ def workload(name: str) -> Shape:
     raise KeyError(name)
 
 
+def norm_weight(seed: int, name: str, h: int, device) -> torch.Tensor:
+    """A learnable RMSNorm weight as a trained gate would hold it: 1 + 0.25 z, z ~ N(0,1),
+    fp32 (one rounding). Not all ones, so the weight's place in the gate is exercised."""
+    z = draw(seed, name, (h,), device=device)
+    return z * torch.tensor(np.float32(0.25), device=z.device) + 1.0
+
+
 def prefill_inputs(shape: Shape, device="cpu", *, with_dout: bool = False) -> dict:
     """Pre-rotary and rotated Q/K, V, gate weights (and dO) for a packed prefill problem.
 
-    Values: N(0,1) for Q/K/V/dO; gate weights N(0,1)/sqrt(fan_in); norm weights 1.
-    Everything is rounded once to the problem dtype (gate weights included); norm
-    weights stay fp32.
+    Values: N(0,1) for Q/K/V/dO; gate weights N(0,1)/sqrt(fan_in); RMSNorm weights
+    1 + 0.25 N(0,1). Everything is rounded once to the problem dtype (gate weights
+    included); norm weights stay fp32.
     """
     T, Hq, Hkv, d, h, G = (shape.total_tokens, shape.num_q_heads, shape.num_kv_heads,
                           shape.head_dim, shape.gate_hidden, shape.group)
@@ -259,8 +266,8 @@ def prefill_inputs(shape: Shape, device="cpu", *, with_dout: bool = False) -> di
         "v": draw(s, "v", (T, Hkv, d), dtype=dt, device=device),
         "wq": draw(s, "wq", (Hkv, h, G * d), dtype=dt, device=device, scale=1.0 / math.sqrt(G * d)),
         "wk": draw(s, "wk", (Hkv, h, 3 * d), dtype=dt, device=device, scale=1.0 / math.sqrt(3 * d)),
-        "qnorm_w": torch.ones(h, dtype=torch.float32, device=device),
-        "knorm_w": torch.ones(h, dtype=torch.float32, device=device),
+        "qnorm_w": norm_weight(s, "qnorm_w", h, device),
+        "knorm_w": norm_weight(s, "knorm_w", h, device),
         "cu_seqlens": torch.from_numpy(shape.cu_seqlens).to(device),
     }
     # the attention reads rotated Q/K; rotate the already-rounded pre-rotary values
@@ -399,6 +406,6 @@ def decode_inputs(shape: DecodeShape, device="cpu", *, batch_rows=None) -> dict:
         "cur_pool": cur_pool,
         "wq": draw(s, "wq", (Hkv, h, G * d), dtype=dt, device=device, scale=1.0 / math.sqrt(G * d)),
         "wk": draw(s, "wk", (Hkv, h, 3 * d), dtype=dt, device=device, scale=1.0 / math.sqrt(3 * d)),
-        "qnorm_w": torch.ones(h, dtype=torch.float32, device=device),
-        "knorm_w": torch.ones(h, dtype=torch.float32, device=device),
+        "qnorm_w": norm_weight(s, "qnorm_w", h, device),
+        "knorm_w": norm_weight(s, "knorm_w", h, device),
     }

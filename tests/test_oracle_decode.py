@@ -65,3 +65,38 @@ def test_ungated_decode_is_softmax_over_kept_keys():
                     qq, kk[None, None], vv[None, None], attn_mask=torch.from_numpy(keep)[None, None, None])
                 np.testing.assert_allclose(Ou[b, hq], ref[0, 0, 0].numpy(), rtol=1e-10, atol=1e-12)
     assert np.abs(Ou - Og).max() > 1e-6
+
+
+def test_decode_on_a_given_selection_equals_prefill_row_on_it():
+    """decode(selection=...) evaluates the newest token's attention on the selection given
+    (a near-tie's other correct answer): it equals the prefill row's attention on that same
+    selection, and on the gate's own selection it changes nothing."""
+    L, B, K, h = 150, 16, 3, 16
+    shape = si.Shape([L], 4, 2, 8, B, K, h, "fp32", seed=77)
+    inp = si.prefill_inputs(shape)
+    sel = orc.prefill_selection(inp["q_nope"], inp["k_nope"], inp["wq"], inp["qnorm_w"], inp["wk"],
+                                inp["knorm_w"], shape.cu_seqlens, B, K, 1e-6, 1e6)
+    k = orc.as64(inp["k_nope"])
+    c = (L - 1) // B
+    cur = k[c * B: L]
+    pool = np.stack([cur.max(0), cur.min(0), cur.sum(0)], axis=1)[None]
+    gkc = sel["gate_keys"].transpose(0, 2, 1, 3)
+    kc = orc.as64(inp["k"]).transpose(1, 0, 2)[None]
+    vc = orc.as64(inp["v"]).transpose(1, 0, 2)[None]
+    args = (orc.as64(inp["q"])[L - 1:L], orc.as64(inp["q_nope"])[L - 1:L], kc, vc, [L], gkc, pool,
+            inp["wq"], inp["qnorm_w"], inp["wk"], inp["knorm_w"], B, K, 1e-6, 1e6)
+    O0, idx0, logg0, _ = orc.decode(*args)
+    O1, _, _, _ = orc.decode(*args, selection=(idx0, logg0))
+    np.testing.assert_array_equal(O1, O0)
+    # another valid selection: historical blocks 0, 2, 5 with arbitrary log-gates
+    other = np.array([[[0, 2, 5, c]] * 2], dtype=np.int32)
+    lg = np.array([[[-0.5, -1.5, -2.0, -0.7], [-3.0, -0.1, -0.2, -1.0]]])
+    O2, idx2, _, _ = orc.decode(*args, selection=(other, lg))
+    np.testing.assert_array_equal(idx2, idx0)          # the gate's own selection is still returned
+    full_idx = np.full((L, 2, K + 1), -1, np.int32)
+    full_lg = np.zeros((L, 2, K + 1))
+    full_idx[L - 1], full_lg[L - 1] = other[0], lg[0]
+    O, _, _ = orc.attention_fwd(inp["q"], inp["k"], inp["v"], full_idx, full_lg, shape.cu_seqlens, B,
+                                rows=np.array([L - 1]))
+    np.testing.assert_allclose(O2, O, rtol=1e-11, atol=1e-12)
+    assert np.abs(O2 - O0).max() > 1e-6

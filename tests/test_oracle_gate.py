@@ -81,7 +81,8 @@ def test_prefix_key_at_block_end_equals_block_key():
     k = orc.as64(inp["k_nope"])
     for j in (0, 3, 11):
         t = 16 * j + 15
-        kc = orc.current_block_key(k, t, 16, orc.as64(inp["wk"]), np.ones(16), 1e-6, 1e6)
+        kc = orc.current_block_key(k, t, 16, orc.as64(inp["wk"]), orc.as64(inp["knorm_w"]), 1e-6,
+                                    1e6)
         np.testing.assert_allclose(kc, gk[0, j], rtol=1e-12, atol=1e-13)
 
 

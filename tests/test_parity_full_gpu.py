@@ -90,6 +90,40 @@ def test_train_full_size_backward_sampled(sas):
         assert_grad_close(dv.cpu()[j * 64:(j + 1) * 64, kv], dv_r, False, f"dV block {j}")
 
 
+def test_varlen_full_size_backward_sampled(sas):
+    """The 14B varlen workload (4 packed sequences, G 5, K 63) forward + backward at full size
+    on the gate's own selection, as bench.py runs it: dQ/dlogg rows and dK/dV of late blocks
+    (few query rows reach them, so the oracle stays small) against the oracle."""
+    shape = si.workload("qwen3-14b-varlen-4seq")
+    dev = torch.device("cuda:0")
+    g = si.prefill_inputs(shape, device=dev, with_dout=True)
+    prob = _problem(sas, shape, dev)
+    idx, logg = sas.prefill_selection(prob, g["q_nope"], g["k_nope"], g["wq"], g["qnorm_w"],
+                                      g["wk"], g["knorm_w"])
+    wsf, wsb = sas.attn_fwd_workspace(prob), sas.attn_bwd_workspace(prob)
+    o, lse = sas.sas_attn_fwd(prob, g["q"], g["k"], g["v"], idx, logg, workspace=wsf)
+    dq, dk, dv, dl = sas.sas_attn_bwd(prob, g["q"], g["k"], g["v"], o, g["dout"], lse, idx, logg,
+                                      workspace=wsb)
+    torch.cuda.synchronize()
+    assert sas.error_code(wsf) == 0 and sas.error_code(wsb) == 0
+    cpu = {k: v.cpu() for k, v in g.items()}
+    ig, lg = idx.cpu().numpy(), logg.cpu().numpy()
+    rows = _rows(shape, 12, 13)
+    dq_r, dl_r = orc.attention_bwd_rows(cpu["q"], cpu["k"], cpu["v"], cpu["dout"], ig, lg,
+                                        shape.cu_seqlens, shape.block, rows)
+    assert_grad_close(dq.cpu()[rows], dq_r, False, "dQ rows")
+    assert_grad_close(dl.cpu()[rows], dl_r, False, "dlogg rows")
+    b = int(np.argmin(shape.lengths))
+    L, s0 = shape.lengths[b], int(shape.cu_seqlens[b])
+    nb = (L + 63) // 64
+    for j, kv in ((nb - 4, 0), (nb - 1, 7)):
+        lo, hi = j * 64, min((j + 1) * 64, L)
+        dk_r, dv_r = orc.attention_bwd_keys(cpu["q"], cpu["k"], cpu["v"], cpu["dout"], ig, lg,
+                                            shape.cu_seqlens, shape.block, b, kv, lo, hi)
+        assert_grad_close(dk.cpu()[s0 + lo:s0 + hi, kv], dk_r, False, f"dK block {j}")
+        assert_grad_close(dv.cpu()[s0 + lo:s0 + hi, kv], dv_r, False, f"dV block {j}")
+
+
 def test_decode_full_size_sampled(sas):
     shp = si.decode_workload("qwen3-8b-decode-b64")
     dev = torch.device("cuda:0")
@@ -102,7 +136,10 @@ def test_decode_full_size_sampled(sas):
                                   g["gate_key_cache"], g["cur_pool"], g["wq"], g["qnorm_w"],
                                   g["wk"], g["knorm_w"], want_selection=True)
     torch.cuda.synchronize()
-    for b in (0, 17, 63):
+    L = np.array(shp.lengths)
+    pick = sorted({0, 17, 63, int(L.argmin()), int(L.argmax())} |
+                  set(np.random.default_rng(14).choice(64, 8, replace=False).tolist()))
+    for b in pick:
         sl = slice(b, b + 1)
         O, ridx, rlogg, margin = orc.decode(
             g["q"][sl].cpu(), g["q_nope"][sl].cpu(), g["k_cache"][sl].cpu(), g["v_cache"][sl].cpu(),
@@ -112,3 +149,11 @@ def test_decode_full_size_sampled(sas):
         compare_selection(idx[sl].cpu().numpy(), logg[sl].cpu(), ridx, rlogg, margin)
         if (idx[sl].cpu().numpy() == ridx).all():
             assert_out_close(o[sl].cpu(), O, False, f"O seq {b}")
+        else:   # a near-tie: the oracle's attention on the GPU's own selection
+            Og, _, _, _ = orc.decode(
+                g["q"][sl].cpu(), g["q_nope"][sl].cpu(), g["k_cache"][sl].cpu(),
+                g["v_cache"][sl].cpu(), [shp.lengths[b]], g["gate_key_cache"][sl].cpu(),
+                g["cur_pool"][sl].cpu(), g["wq"].cpu(), g["qnorm_w"].cpu(), g["wk"].cpu(),
+                g["knorm_w"].cpu(), shp.block, shp.topk, shp.rms_eps, shp.gate_rope_base,
+                selection=(idx[sl].cpu().numpy(), logg[sl].cpu().numpy()))
+            assert_out_close(o[sl].cpu(), Og, False, f"O seq {b} (GPU selection)")
