@@ -2,9 +2,12 @@
 """Benchmark of the SAS gated block-sparse attention hot path on B200.
 
 One step = one pass of the whole prefill/training path over the workload's inputs
-(already resident in HBM): key pooling -> gate keys -> gate scores -> Top-K -> gated
-attention forward -> gated attention backward. A decode step of the batch-64 decode
-workload is measured beside it and reported in the same line.
+(already resident in HBM): key pooling -> gate keys -> gate scores + Top-K (one fused pass)
+-> gated attention forward -> gated attention backward. The headline workload is the largest
+single-GPU configuration, the Qwen3-14B-shaped varlen training step (4 packed sequences of
+8k..64k tokens, 40 query / 8 KV heads, Top-K 63). The Qwen3-4B 32k training step, the 32k
+forward-only prefill and the batch-64 decode step are measured beside it and reported under
+their own keys in the same line.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl sas|reference]
 
@@ -34,7 +37,9 @@ import torch  # noqa: E402
 import sas_inputs as si  # noqa: E402
 
 METRIC = "gated sparse attn TFLOP/s (attended, fwd/bwd) + decode tok/s; % of B200 roofline"
-TRAIN_WORKLOAD = "qwen3-4b-train-32k"
+HEADLINE_WORKLOAD = "qwen3-14b-varlen-4seq"      # the largest single-GPU configuration
+EXTRA_WORKLOADS = ("qwen3-4b-train-32k", "qwen3-4b-prefill-32k")
+EXTRA_KEYS = {"qwen3-4b-train-32k": "train_32k", "qwen3-4b-prefill-32k": "prefill_32k"}
 DECODE_WORKLOAD = "qwen3-8b-decode-b64"
 L2_FLUSH_BYTES = 256 << 20
 
@@ -45,7 +50,9 @@ def parse():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="sas", choices=["sas", "reference"])
-    ap.add_argument("--workload", default=TRAIN_WORKLOAD)
+    ap.add_argument("--workload", default=HEADLINE_WORKLOAD)
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the other prefill/training workloads (profiling)")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-train", action="store_true", help="decode step only (profiling)")
     ap.add_argument("--decode-workload", default=DECODE_WORKLOAD)
@@ -165,12 +172,13 @@ def source_sha(files) -> str:
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(op: str):
-    """dram bytes per launch of `op` from the committed ncu summary, if its sources match."""
+def ncu_traffic(op: str, workload: str):
+    """DRAM bytes per launch of `op` on `workload` from the committed ncu summary, if the
+    kernel sources it was taken with are unchanged (None otherwise)."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(p):
         return None
-    d = json.load(open(p)).get(op)
+    d = json.load(open(p)).get(f"{op}@{workload}")
     if not d:
         return None
     try:
@@ -243,11 +251,9 @@ def train_step(sas, prob, g, backward: bool, timer: Timer | None = None):
     pooled = run("sas_pool_keys", lambda: sas.sas_pool_keys(prob, g["k_nope"], pooled=g["_pooled"]))
     gk = run("sas_gate_keys", lambda: sas.sas_gate_keys(prob, pooled, g["wk"], g["knorm_w"],
                                                         gate_keys=g["_gk"]))
-    scores, lse = run("sas_gate_scores", lambda: sas.sas_gate_scores(
+    idx, logg = run("sas_gate_select", lambda: sas.sas_gate_select(
         prob, g["q_nope"], g["k_nope"], gk, g["wq"], g["qnorm_w"], g["wk"], g["knorm_w"],
-        scores=g["_scores"], lse=g["_glse"], workspace=g["_wsg"]))
-    idx, logg = run("sas_topk", lambda: sas.sas_topk(prob, scores, lse, idx=g["_idx"],
-                                                     logg=g["_logg"]))
+        idx=g["_idx"], logg=g["_logg"], workspace=g["_wsg"]))
     o, alse = run("sas_attn_fwd", lambda: sas.sas_attn_fwd(prob, g["q"], g["k"], g["v"], idx, logg,
                                                            o=g["_o"], lse=g["_alse"],
                                                            workspace=g["_wsf"]))
@@ -267,15 +273,13 @@ def alloc_outputs(sas, prob, g, backward):
                                prob.head_dim, prob.topk, prob.max_blocks, prob.gate_hidden)
     g["_pooled"] = torch.empty((prob.batch, NB, Hkv, 3 * d), dtype=torch.float32, device=dev)
     g["_gk"] = torch.empty((prob.batch, NB, Hkv, h), dtype=torch.float32, device=dev)
-    g["_scores"] = torch.empty((T, Hkv, NB), dtype=torch.float32, device=dev)
-    g["_glse"] = torch.empty((T, Hkv), dtype=torch.float32, device=dev)
     g["_idx"] = torch.empty((T, Hkv, K + 1), dtype=torch.int32, device=dev)
     g["_logg"] = torch.empty((T, Hkv, K + 1), dtype=torch.float32, device=dev)
     g["_o"] = torch.empty((T, Hq, d), dtype=prob.dtype, device=dev)
     g["_alse"] = torch.empty((T, Hq), dtype=torch.float32, device=dev)
     lib = sas.lib_handle()
     n = ctypes.c_size_t(0)
-    lib.sas_gate_scores_workspace_size(prob.ref, ctypes.byref(n))
+    lib.sas_gate_select_workspace_size(prob.ref, ctypes.byref(n))
     g["_wsg"] = torch.empty(max(256, n.value), dtype=torch.uint8, device=dev)
     lib.sas_attn_fwd_workspace_size(prob.ref, ctypes.byref(n))
     g["_wsf"] = torch.empty(max(256, n.value), dtype=torch.uint8, device=dev)
@@ -384,6 +388,7 @@ def bench_decode(sas, dev, steps, warmup, flush, hbm_peak, name=DECODE_WORKLOAD)
     for _ in range(warmup):
         step()
     torch.cuda.synchronize()
+    sas.check_workspace(ws, "sas_decode")
     ts = []
     for _ in range(steps):
         flush.zero_()
@@ -416,10 +421,135 @@ def bench_decode(sas, dev, steps, warmup, flush, hbm_peak, name=DECODE_WORKLOAD)
                                       "context_min": int(L.min()), "context_max": int(L.max()),
                                       "budget_tokens": (shp.topk + 1) * B},
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": gbs / hbm_peak, "traffic": ncu_traffic("sas_decode"),
+                     "frac": gbs / hbm_peak, "traffic": ncu_traffic("sas_decode", name),
                      "algorithmic_bytes": total, "selected_kv_bytes": kv_bytes,
                      "gate_key_bytes": gk_bytes, "peak_source": "measured copy, of measured"},
         "selected_kv_gbs": kv_bytes / (ms * 1e-3) / 1e9,
+    }
+
+
+# ------------------------------------------------------------------------------------------
+# one prefill / training workload: resident inputs, timed steps, per-op events
+# ------------------------------------------------------------------------------------------
+
+def setup_workload(sas, name, dev):
+    shape = si.workload(name)
+    backward = "train" in name or "varlen" in name
+    g = si.prefill_inputs(shape, device=dev, with_dout=backward)
+    prob = sas.Problem.from_lengths(shape.lengths, dev, num_q_heads=shape.num_q_heads,
+                                    num_kv_heads=shape.num_kv_heads, head_dim=shape.head_dim,
+                                    block=shape.block, topk=shape.topk,
+                                    gate_hidden=shape.gate_hidden, dtype=shape.torch_dtype)
+    alloc_outputs(sas, prob, g, backward)
+    return shape, backward, g, prob
+
+
+def check_error_words(sas, g, backward):
+    """The device-side error words of the step's last calls (0 = none); raises otherwise."""
+    sas.check_workspace(g["_wsg"], "sas_gate_select")
+    sas.check_workspace(g["_wsf"], "sas_attn_fwd")
+    if backward:
+        sas.check_workspace(g["_wsb"], "sas_attn_bwd")
+
+
+def time_workload(sas, name, shape, backward, g, prob, steps, warmup, flush, ws, dev, clk=None):
+    """Warm up, check the error words, then time `steps` whole steps (L2 flushed between
+    steps) with CUDA events around the step and around each op."""
+    for _ in range(max(3, warmup)):
+        out = train_step(sas, prob, g, backward)
+    torch.cuda.synchronize()
+    check_error_words(sas, g, backward)
+    pairs = attended_pairs_gpu(out[2], prob.cu_seqlens, shape.block)
+    G, d = shape.group, shape.head_dim
+    fwd_flops = 4.0 * pairs * G * d
+    bwd_flops = 2.5 * fwd_flops if backward else 0.0
+    Mq = 25 if G == 5 else 128 // G
+    tiles, kept = km_stats(out[2], prob.cu_seqlens, shape.lengths, Mq, shape.num_kv_heads,
+                           prob.max_blocks)
+    timer = Timer()
+    evs = []
+    barrier(ws)
+    torch.cuda.synchronize()
+    n0 = sas.kernel_launches()
+    ctx = clk if clk is not None else _Null()
+    with ctx:
+        for _ in range(steps):
+            flush.zero_()
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record()
+            train_step(sas, prob, g, backward, timer)
+            e.record()
+            evs.append((s, e))
+        torch.cuda.synchronize()
+    barrier(ws)
+    launches = sas.kernel_launches() - n0
+    check_error_words(sas, g, backward)
+    ms = sum(x.elapsed_time(y) for x, y in evs) / len(evs)
+    ms = max_over_ranks(ms, ws, dev)
+    return dict(ms=ms, ops=timer.mean_ms(), pairs=pairs, fwd_flops=fwd_flops, bwd_flops=bwd_flops,
+                tiles=tiles, kept=kept, launches=launches)
+
+
+class _Null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        return False
+
+
+def choose_tc_peak(clocks, burst, sustained, src):
+    """The bf16 denominator for the clocks seen during the timed region: the burst figure
+    when the SM clock held its maximum, the sustained (power-capped) figure otherwise."""
+    if clocks and clocks.get("sm_max_mhz") and clocks["sm_mhz"] >= 0.95 * clocks["sm_max_mhz"]:
+        return burst, (f"bf16 dense burst (SM clock at its maximum, median "
+                       f"{clocks['sm_mhz']:.0f} MHz, during the timed region), of {src}")
+    return sustained, f"bf16 dense sustained (power-capped clocks), of {src}"
+
+
+def summarise(name, shape, backward, r, peak, peak_note, ws):
+    """The workload's numbers: attended TFLOP/s, per-op times, roofline of the dominant
+    attention pass, the key-major kernels' computed work and L2 reduction traffic."""
+    ops = r["ops"]
+    G, d = shape.group, shape.head_dim
+    work = r["fwd_flops"] + r["bwd_flops"]
+    mma = 2.0 * 128 * 64 * d                           # one 128-row x 64-key x d product
+    comp_fwd = r["tiles"] * 2 * mma                    # S = Q K^T, O = P V per gathered tile
+    comp_bwd = r["tiles"] * 5 * mma if backward else 0.0   # S, dP, dV^T, dK^T, dQ
+    red_bytes = r["kept"] * G * d * 4                  # fp32 partial rows reduced into L2
+    dom = max(("sas_attn_fwd", "sas_attn_bwd") if backward else ("sas_attn_fwd",),
+              key=lambda k: ops[k])
+    dflops = r["fwd_flops"] if dom == "sas_attn_fwd" else r["bwd_flops"]
+    ach = dflops / (ops[dom] * 1e-3) / 1e12
+    return {
+        "value": work * ws / (r["ms"] * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": r["ms"],
+        "config": {"workload": name, "batch": shape.batch, "seq_len": shape.max_seqlen,
+                   "seq_lens": list(shape.lengths), "total_tokens": shape.total_tokens,
+                   "num_q_heads": shape.num_q_heads, "num_kv_heads": shape.num_kv_heads,
+                   "head_dim": d, "block": shape.block, "topk": shape.topk,
+                   "gate_hidden": shape.gate_hidden, "passes": "fwd+bwd" if backward else "fwd",
+                   "parallelism": f"replicas x{ws}", "l2": "flushed (256 MiB write) between steps"},
+        "attended": {"pairs_per_kv_head_total": r["pairs"], "fwd_tflop": r["fwd_flops"] / 1e12,
+                     "bwd_tflop": r["bwd_flops"] / 1e12,
+                     "dense_causal_fraction": r["pairs"] / (shape.num_kv_heads * sum(
+                         L * (L + 1) / 2 for L in shape.lengths))},
+        "computed": {"fwd_tflop": comp_fwd / 1e12, "bwd_tflop": comp_bwd / 1e12,
+                     "gathered_tiles": r["tiles"],
+                     "attended_over_computed": work / max(1.0, comp_fwd + comp_bwd),
+                     "fwd_tflops": comp_fwd / (ops["sas_attn_fwd"] * 1e-3) / 1e12,
+                     "bwd_tflops": (comp_bwd / (ops["sas_attn_bwd"] * 1e-3) / 1e12) if backward else None,
+                     "l2_reduction_gb_per_pass": red_bytes / 1e9,
+                     "fwd_l2_reduction_gbs": red_bytes / (ops["sas_attn_fwd"] * 1e-3) / 1e9,
+                     "bwd_l2_reduction_gbs": (red_bytes / (ops["sas_attn_bwd"] * 1e-3) / 1e9)
+                     if backward else None,
+                     "note": "key-major kernels: gathered 128-row tiles per (kv, window, kept "
+                             "block); each kept (token, block) pair adds G fp32 rows of d "
+                             "values into L2 (O in the forward, dQ in the backward)"},
+        "ops_ms": ops,
+        "roofline": {"bound": "tensor", "kernel": dom, "achieved": ach, "peak": peak,
+                     "unit": "TFLOP/s", "frac": ach / peak, "traffic": ncu_traffic(dom, name),
+                     "peak_source": peak_note, "algorithmic_flops_per_launch": dflops},
+        "gpu_launches": r["launches"],
     }
 
 
@@ -435,101 +565,57 @@ def main():
     import gated_block_sparse_sas_b200 as sas
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    hbm_peak, tc_peak, tc_sust, peak_src = measured_peaks()
+    hbm_peak, tc_burst, tc_sust, peak_src = measured_peaks()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     if a.no_train:
-        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
         print(json.dumps(bench_decode(sas, dev, max(1, a.steps), max(3, a.warmup), flush, hbm_peak,
                                       a.decode_workload)), flush=True)
         return
 
-    shape = si.workload(a.workload)
-    backward = "train" in a.workload or "varlen" in a.workload
-    g = si.prefill_inputs(shape, device=dev, with_dout=backward)
-    prob = sas.Problem.from_lengths(shape.lengths, dev, num_q_heads=shape.num_q_heads,
-                                    num_kv_heads=shape.num_kv_heads, head_dim=shape.head_dim,
-                                    block=shape.block, topk=shape.topk,
-                                    gate_hidden=shape.gate_hidden, dtype=shape.torch_dtype)
-    alloc_outputs(sas, prob, g, backward)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-
-    for _ in range(max(3, a.warmup)):
-        out = train_step(sas, prob, g, backward)
-    torch.cuda.synchronize()
-    pairs = attended_pairs_gpu(out[2], prob.cu_seqlens, shape.block)
-    G, d = shape.group, shape.head_dim
-    fwd_flops = 4.0 * pairs * G * d
-    bwd_flops = 2.5 * fwd_flops if backward else 0.0
-    Mq = 25 if G == 5 else 128 // G
-    tiles, kept = km_stats(out[2], prob.cu_seqlens, shape.lengths, Mq, shape.num_kv_heads,
-                           prob.max_blocks)
-    mma = 2.0 * 128 * 64 * d                           # one 128-row x 64-key x d product
-    comp_fwd = tiles * 2 * mma                         # S = Q K^T, O = P V per gathered tile
-    comp_bwd = tiles * 5 * mma if backward else 0.0    # S, dP, dV^T, dK^T, dQ
-    red_bytes = kept * G * d * 4                       # fp32 partial rows reduced into L2
-
-    timer = Timer()
-    steps = []
-    barrier(ws)
-    torch.cuda.synchronize()
-    n0 = sas.kernel_launches()
-    with ClockSampler(dev.index) as clk:
-        for _ in range(a.steps):
-            flush.zero_()
-            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            s.record()
-            train_step(sas, prob, g, backward, timer)
-            e.record()
-            steps.append((s, e))
-        torch.cuda.synchronize()
-    barrier(ws)
-    launches = sas.kernel_launches() - n0
-    ms = sum(x.elapsed_time(y) for x, y in steps) / len(steps)
-    ms = max_over_ranks(ms, ws, dev)
-    ops = timer.mean_ms()
-    work = fwd_flops + bwd_flops
-    value = work * ws / (ms * 1e-3) / 1e12
-
-    # dominant kernel roofline (tensor-bound attention; peak: sustained, timed inside a long step)
-    dom = max(("sas_attn_fwd", "sas_attn_bwd") if backward else ("sas_attn_fwd",),
-              key=lambda k: ops[k])
-    dflops = fwd_flops if dom == "sas_attn_fwd" else bwd_flops
-    ach = dflops / (ops[dom] * 1e-3) / 1e12
-    roof = {"bound": "tensor", "kernel": dom, "achieved": ach, "peak": tc_sust, "unit": "TFLOP/s",
-            "frac": ach / tc_sust, "traffic": ncu_traffic(dom),
-            "peak_source": f"bf16 dense sustained, of {peak_src}",
-            "algorithmic_flops_per_launch": dflops}
-
-    line = {
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws, "steps": a.steps,
-        "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16" if shape.dtype == "bf16" else "f32",
-        "data": "synthetic (seeded counter-based generator, approx. N(0,1))",
-        "config": {"workload": a.workload, "batch": shape.batch, "seq_len": shape.max_seqlen,
-                   "num_q_heads": shape.num_q_heads, "num_kv_heads": shape.num_kv_heads,
-                   "head_dim": d, "block": shape.block, "topk": shape.topk,
-                   "gate_hidden": shape.gate_hidden, "passes": "fwd+bwd" if backward else "fwd",
-                   "parallelism": f"replicas x{ws}", "l2": "flushed (256 MiB write) between steps"},
-        "attended": {"pairs_per_kv_head_total": pairs, "fwd_tflop": fwd_flops / 1e12,
-                     "bwd_tflop": bwd_flops / 1e12,
-                     "dense_causal_fraction": pairs / (shape.num_kv_heads * sum(
-                         L * (L + 1) / 2 for L in shape.lengths))},
-        "computed": {"fwd_tflop": comp_fwd / 1e12, "bwd_tflop": comp_bwd / 1e12,
-                     "gathered_tiles": tiles,
-                     "attended_over_computed": (fwd_flops + bwd_flops) / max(1.0, comp_fwd + comp_bwd),
-                     "fwd_tflops": comp_fwd / (ops["sas_attn_fwd"] * 1e-3) / 1e12,
-                     "bwd_tflops": (comp_bwd / (ops["sas_attn_bwd"] * 1e-3) / 1e12) if backward else None,
-                     "l2_reduction_gb_per_pass": red_bytes / 1e9,
-                     "fwd_reduction_gbs": red_bytes / (ops["sas_attn_fwd"] * 1e-3) / 1e9,
-                     "note": "key-major kernels: gathered 128-row tiles per (kv, window, kept "
-                             "block); each kept (token, block) pair adds G fp32 rows of d "
-                             "values into L2 (O in the forward, dQ in the backward)"},
-        "ops_ms": ops,
-        "roofline": roof,
-        "gpu_launches": launches,
-    }
+    # ---- the headline workload ------------------------------------------------------------
+    shape, backward, g, prob = setup_workload(sas, a.workload, dev)
+    clk = ClockSampler(dev.index)
+    r = time_workload(sas, a.workload, shape, backward, g, prob, a.steps, a.warmup, flush, ws, dev,
+                      clk)
     cs = clk.summary()
+    peak, peak_note = choose_tc_peak(cs, tc_burst, tc_sust, peak_src)
+    head = summarise(a.workload, shape, backward, r, peak, peak_note, ws)
+    line = {
+        "metric": METRIC, "value": head["value"], "unit": "TFLOP/s", "n_gpus": ws,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": head["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if shape.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded counter-based generator, approx. N(0,1))",
+        "config": head["config"], "attended": head["attended"], "computed": head["computed"],
+        "ops_ms": head["ops_ms"], "roofline": head["roofline"], "gpu_launches": head["gpu_launches"],
+    }
     if cs:
         line["clocks"] = cs
+    if not a.no_e2e:
+        line["e2e"] = e2e(sas, prob, g, backward, r["fwd_flops"] + r["bwd_flops"], dev, a, ws)
+    if backward:   # after the timed step and e2e legs, so it cannot perturb them
+        line["router_bwd"] = bench_router_bwd(sas, prob, g, flush, max(3, a.steps))
+    if rank == 0 and ws == 1 and not a.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(g, shape, backward, a)
+    del g, prob
+    torch.cuda.empty_cache()
+
+    # ---- the other prefill / training workloads, each its own key -------------------------
+    if not a.no_extra:
+        for name in EXTRA_WORKLOADS:
+            if name == a.workload:
+                continue
+            shp, bwd, ge, pe = setup_workload(sas, name, dev)
+            ce = ClockSampler(dev.index)
+            re_ = time_workload(sas, name, shp, bwd, ge, pe, a.steps, a.warmup, flush, ws, dev, ce)
+            cse = ce.summary()
+            pk, pn = choose_tc_peak(cse, tc_burst, tc_sust, peak_src)
+            ex = summarise(name, shp, bwd, re_, pk, pn, ws)
+            if cse:
+                ex["clocks"] = cse
+            line[EXTRA_KEYS[name]] = ex
+            del ge, pe
+            torch.cuda.empty_cache()
 
     if not a.no_decode:
         try:
@@ -538,29 +624,35 @@ def main():
         except torch.OutOfMemoryError as ex:   # pragma: no cover
             line["decode"] = {"error": f"out of memory: {ex}"[:200]}
 
-    if not a.no_e2e:
-        line["e2e"] = e2e(sas, prob, g, backward, work, dev, a, ws)
-
-    if backward:   # after the step, decode and e2e legs, so it cannot perturb them
-        line["router_bwd"] = bench_router_bwd(sas, prob, g, flush, max(3, a.steps))
-
-    if rank == 0 and ws == 1 and not a.no_cpu_baseline:
-        cpu = cpu_inputs_from(g)
-        rows = sample_rows(shape, a.cpu_rows, 7)
-        threads = torch.get_num_threads()
-        t0 = time.perf_counter()
-        fl = oracle_sample(cpu, shape, rows, backward)
-        dt = time.perf_counter() - t0
-        line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads,
-                                "kind": "oracle", "seconds": dt,
-                                "sample": f"{len(rows)} random query rows of {a.workload} "
-                                          "(gate, Top-K, attention fwd" +
-                                          (" + dQ/dlogg rows" if backward else "") +
-                                          ") at full sequence length, fp64 numpy"}
+    line["extra_keys"] = [k for k in line if k in ("train_32k", "prefill_32k", "decode",
+                                                   "router_bwd", "computed", "attended", "ops_ms")]
     if rank == 0:
         print(json.dumps(line), flush=True)
     if ws > 1:
         torch.distributed.destroy_process_group()
+
+
+def cpu_baseline(g, shape, backward, a):
+    """The oracle, as it stands, on sampled query rows of the workload's shortest sequence at
+    its full length (rows of different sequences are independent), timed on the host cores."""
+    b = int(np.argmin(shape.lengths))
+    s0, L = int(shape.cu_seqlens[b]), shape.lengths[b]
+    one = si.sequence_shape(shape, b)
+    keys = ("q_nope", "k_nope", "q", "k", "v", "dout", "wq", "wk", "qnorm_w", "knorm_w")
+    tok = ("q_nope", "k_nope", "q", "k", "v", "dout")
+    cpu = {k: (g[k][s0:s0 + L] if k in tok else g[k]).float().cpu().numpy().astype(np.float64)
+           for k in keys if k in g}
+    rows = sample_rows(one, a.cpu_rows, 7)
+    threads = torch.get_num_threads()
+    t0 = time.perf_counter()
+    fl = oracle_sample(cpu, one, rows, backward)
+    dt = time.perf_counter() - t0
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "seconds": dt,
+            "sample": f"{len(rows)} random query rows of sequence {b} ({L} tokens) of "
+                      f"{a.workload} (gate, Top-K, attention fwd" +
+                      (" + dQ/dlogg rows" if backward else "") +
+                      ") at full sequence length, fp64 numpy"}
 
 
 def e2e(sas, prob, g, backward, work, dev, a, ws):
@@ -621,21 +713,25 @@ def e2e(sas, prob, g, backward, work, dev, a, ws):
 
 
 def reference_arm(a, ws, rank):
-    """The oracle, as it stands, on the machine's host cores (rank 0 only)."""
+    """The oracle, as it stands, on the machine's host cores (rank 0 only). Each step is a
+    bounded sample: random query rows of the workload's shortest sequence at full length
+    (rows of different sequences are independent), drawn with the same generator."""
     if rank != 0:
         return
     shape = si.workload(a.workload)
     backward = "train" in a.workload or "varlen" in a.workload
-    inp = si.prefill_inputs(shape, device="cpu", with_dout=backward)
+    b = int(np.argmin(shape.lengths))
+    one = si.sequence_shape(shape, b)
+    inp = si.prefill_inputs(shape, device="cpu", with_dout=backward, sequence=b)
     cpu = {k: v.float().numpy().astype(np.float64) for k, v in inp.items() if k != "cu_seqlens"}
     for i in range(a.warmup):
-        oracle_sample(cpu, shape, sample_rows(shape, 1, 100 + i), backward)
+        oracle_sample(cpu, one, sample_rows(one, 1, 100 + i), backward)
     t = []
     fl = 0.0
     for i in range(a.steps):
-        rows = sample_rows(shape, 8, 1000 + i)
+        rows = sample_rows(one, 8, 1000 + i)
         t0 = time.perf_counter()
-        fl += oracle_sample(cpu, shape, rows, backward)
+        fl += oracle_sample(cpu, one, rows, backward)
         t.append(time.perf_counter() - t0)
     tot = sum(t)
     val = fl / tot / 1e12
@@ -647,8 +743,11 @@ def reference_arm(a, ws, rank):
             "config": {"workload": a.workload, "batch": shape.batch, "seq_len": shape.max_seqlen,
                        "passes": "fwd+bwd" if backward else "fwd", "parallelism": "cpu oracle"},
             "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-                             "sample": f"8 random query rows per step of {a.workload} (gate, "
-                                       "Top-K, attention fwd + dQ/dlogg rows), fp64 numpy"},
+                             "sample": f"8 random query rows per step of sequence {b} "
+                                       f"({shape.lengths[b]} tokens) of {a.workload} (gate, "
+                                       "Top-K, attention fwd" +
+                                       (" + dQ/dlogg rows" if backward else "") +
+                                       ") at full sequence length, fp64 numpy"},
             "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)

@@ -54,6 +54,8 @@ _SIGS = {
     "sas_gate_scores_workspace_size": ([_P, ctypes.POINTER(_sz)], ctypes.c_int),
     "sas_gate_scores": ([_P] + [_vp] * 9 + [_vp, _sz, _vp], ctypes.c_int),
     "sas_topk": ([_P, _vp, _vp, _vp, _vp, _vp], ctypes.c_int),
+    "sas_gate_select_workspace_size": ([_P, ctypes.POINTER(_sz)], ctypes.c_int),
+    "sas_gate_select": ([_P] + [_vp] * 10 + [_vp, _sz, _vp], ctypes.c_int),
     "sas_gate_bwd_workspace_size": ([_P, ctypes.POINTER(_sz)], ctypes.c_int),
     "sas_gate_bwd": ([_P] + [_vp] * 13 + [_vp, _sz, _vp], ctypes.c_int),
     "sas_attn_fwd_workspace_size": ([_P, ctypes.POINTER(_sz)], ctypes.c_int),
@@ -62,6 +64,7 @@ _SIGS = {
     "sas_attn_bwd": ([_P] + [_vp] * 13 + [_sz, _vp], ctypes.c_int),
     "sas_decode_workspace_size": ([_DP, ctypes.POINTER(_sz)], ctypes.c_int),
     "sas_decode": ([_DP] + [_vp] * 14 + [_sz, _vp], ctypes.c_int),
+    "sas_decode_paged": ([_DP, _vp, _i32] + [_vp] * 14 + [_sz, _vp], ctypes.c_int),
     "sas_decode_noalloc": ([_DP] + [_vp] * 13 + [_vp], ctypes.c_int),
     "sas_decode_noalloc_error_word": ([ctypes.POINTER(_vp)], ctypes.c_int),
 }
@@ -91,6 +94,7 @@ ERROR_CODES = {
     57: "attn_fwd: a bounded wait gave up",
     60: "attn_fwd: a row's largest logit exceeds its own key's by more than ~97 nats",
     61: "decode: a row's largest logit exceeds its own key's by more than ~97 nats",
+    62: "paged decode: a page id out of range",
     71: "attn_bwd: a bounded wait gave up", 72: "attn_bwd: a bounded wait gave up",
     73: "attn_bwd: a bounded wait gave up", 74: "attn_bwd: a bounded wait gave up",
     75: "attn_bwd: a bounded wait gave up", 76: "attn_bwd: a bounded wait gave up",
@@ -343,10 +347,37 @@ def sas_attn_bwd(p: Problem, q, k, v, o, dout, lse, idx, logg, dq=None, dk=None,
     return dq, dk, dv, dlogg
 
 
-def prefill_selection(p: Problem, q_nope, k_nope, wq, qnorm_w, wk, knorm_w, stream=None):
-    """A1..A4 in order: pool -> gate keys -> scores -> Top-K. Returns (idx, logg)."""
+def gate_select_workspace(p: Problem):
+    """A workspace of the size sas_gate_select asks for."""
+    return _workspace(_lib.sas_gate_select_workspace_size, p.ref, p.device)
+
+
+def sas_gate_select(p: Problem, q_nope, k_nope, gate_keys, wq, qnorm_w, wk, knorm_w, idx=None,
+                    logg=None, lse=None, workspace=None, stream=None, want_lse: bool = False):
+    """Gate scores + Top-K in one pass (scores never written for the fused shapes).
+    Returns (idx, logg), or (idx, logg, lse) with want_lse."""
+    shape = (p.total_tokens, p.num_kv_heads, p.topk + 1)
+    if idx is None:
+        idx = torch.empty(shape, dtype=torch.int32, device=p.device)
+    if logg is None:
+        logg = torch.empty(shape, dtype=torch.float32, device=p.device)
+    if want_lse and lse is None:
+        lse = torch.empty((p.total_tokens, p.num_kv_heads), dtype=torch.float32, device=p.device)
+    ws = workspace if workspace is not None else gate_select_workspace(p)
+    _check(_lib.sas_gate_select(p.ref, _ptr(q_nope), _ptr(k_nope), _ptr(gate_keys), _ptr(wq),
+                                _ptr(qnorm_w), _ptr(wk), _ptr(knorm_w), _ptr(idx), _ptr(logg),
+                                _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)), "sas_gate_select")
+    return (idx, logg, lse) if want_lse else (idx, logg)
+
+
+def prefill_selection(p: Problem, q_nope, k_nope, wq, qnorm_w, wk, knorm_w, stream=None,
+                      fused: bool = True):
+    """A1..A4 in order: pool -> gate keys -> scores + Top-K (one fused pass, or the separate
+    score and Top-K calls with fused=False). Returns (idx, logg)."""
     pooled = sas_pool_keys(p, k_nope, stream=stream)
     gk = sas_gate_keys(p, pooled, wk, knorm_w, stream=stream)
+    if fused:
+        return sas_gate_select(p, q_nope, k_nope, gk, wq, qnorm_w, wk, knorm_w, stream=stream)
     scores, lse = sas_gate_scores(p, q_nope, k_nope, gk, wq, qnorm_w, wk, knorm_w, stream=stream)
     return sas_topk(p, scores, lse, stream=stream)
 
@@ -412,6 +443,30 @@ def sas_decode(p: DecodeProblem, q, q_nope, k_cache, v_cache, gate_key_cache, cu
                            ws.numel(), _stream(stream)), "sas_decode")
     if check:
         check_workspace(ws, "sas_decode")
+    return (o, idx_out, logg_out) if want_selection else o
+
+
+def sas_decode_paged(p: DecodeProblem, page_table, num_pages: int, q, q_nope, k_pages, v_pages,
+                     gate_key_pages, cur_pool, wq, qnorm_w, wk, knorm_w, o=None, idx_out=None,
+                     logg_out=None, workspace=None, stream=None, want_selection: bool = False,
+                     check: bool = False):
+    """One sparse decode step over paged caches: page_table int32 [batch, ceil(capacity/B)],
+    k_pages / v_pages [num_pages, Hkv, B, d], gate_key_pages bf16 [num_pages, Hkv, h]."""
+    if o is None:
+        o = torch.empty((p.batch, p.num_q_heads, p.head_dim), dtype=p.dtype, device=p.device)
+    if want_selection and idx_out is None:
+        idx_out = torch.empty((p.batch, p.num_kv_heads, p.topk + 1), dtype=torch.int32,
+                              device=p.device)
+        logg_out = torch.empty((p.batch, p.num_kv_heads, p.topk + 1), dtype=torch.float32,
+                               device=p.device)
+    ws = workspace if workspace is not None else _workspace(_lib.sas_decode_workspace_size, p.ref, p.device)
+    _check(_lib.sas_decode_paged(p.ref, _ptr(page_table), int(num_pages), _ptr(q), _ptr(q_nope),
+                                 _ptr(k_pages), _ptr(v_pages), _ptr(gate_key_pages), _ptr(cur_pool),
+                                 _ptr(wq), _ptr(qnorm_w), _ptr(wk), _ptr(knorm_w), _ptr(o),
+                                 _ptr(idx_out), _ptr(logg_out), _ptr(ws), ws.numel(),
+                                 _stream(stream)), "sas_decode_paged")
+    if check:
+        check_workspace(ws, "sas_decode_paged")
     return (o, idx_out, logg_out) if want_selection else o
 
 

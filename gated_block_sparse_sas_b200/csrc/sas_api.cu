@@ -176,6 +176,41 @@ sas_status sas_gate_scores(const sas_problem* p, const void* q_nope, const void*
                             workspace, stream);
 }
 
+sas_status sas_gate_select_workspace_size(const sas_problem* p, size_t* bytes) {
+  SAS_TRY(check_problem(p, true));
+  SAS_CHECK_ARG(bytes != nullptr, "bytes is NULL");
+  *bytes = gate_select_workspace_bytes(*p);
+  return SAS_OK;
+}
+
+sas_status sas_gate_select(const sas_problem* p, const void* q_nope, const void* k_nope,
+                           const float* gate_keys, const void* wq, const float* qnorm_w,
+                           const void* wk, const float* knorm_w, int32_t* idx, float* logg,
+                           float* lse, void* workspace, size_t workspace_bytes,
+                           cudaStream_t stream) {
+  SAS_TRY(check_problem(p, true));
+  SAS_PTR(q_nope);
+  SAS_PTR(k_nope);
+  SAS_PTR(gate_keys);
+  SAS_PTR(wq);
+  SAS_PTR(qnorm_w);
+  SAS_PTR(wk);
+  SAS_PTR(knorm_w);
+  SAS_PTR(idx);
+  SAS_PTR(logg);
+  if (lse != nullptr) SAS_CHECK_ARG(aligned16(lse), "lse is not 16-byte aligned");
+  if (p->total_tokens == 0) return SAS_OK;
+  SAS_PTR(workspace);
+  const size_t need = gate_select_workspace_bytes(*p);
+  if (workspace_bytes < need) {
+    set_error("workspace too small: %zu < %zu bytes", workspace_bytes, need);
+    return SAS_ERR_WORKSPACE;
+  }
+  SAS_TRY(clear_error_word(workspace, stream));
+  return launch_gate_select(*p, q_nope, k_nope, gate_keys, wq, qnorm_w, wk, knorm_w, idx, logg,
+                            lse, workspace, stream);
+}
+
 sas_status sas_gate_bwd_workspace_size(const sas_problem* p, size_t* bytes) {
   SAS_TRY(check_problem(p, true));
   SAS_CHECK_ARG(bytes != nullptr, "bytes is NULL");
@@ -397,7 +432,47 @@ sas_status sas_decode(const sas_decode_problem* p, const void* q, const void* q_
     return SAS_ERR_WORKSPACE;
   }
   return launch_decode(*p, q, q_nope, k_cache, v_cache, gate_key_cache, cur_pool, wq, qnorm_w, wk,
-                       knorm_w, o, idx_out, logg_out, workspace, stream);
+                       knorm_w, o, idx_out, logg_out, workspace, DecodePaging{}, stream);
+}
+
+sas_status sas_decode_paged(const sas_decode_problem* p, const int32_t* page_table,
+                            int32_t num_pages, const void* q, const void* q_nope,
+                            const void* k_pages, const void* v_pages, const void* gate_key_pages,
+                            const float* cur_pool, const void* wq, const float* qnorm_w,
+                            const void* wk, const float* knorm_w, void* o, int32_t* idx_out,
+                            float* logg_out, void* workspace, size_t workspace_bytes,
+                            cudaStream_t stream) {
+  SAS_TRY(check_decode(p));
+  if (!decode_attn_tc_supported(*p)) {
+    set_error("decode_paged: supported for bf16, head_dim 128, block 64 (one block per page)");
+    return SAS_ERR_UNSUPPORTED;
+  }
+  SAS_CHECK_ARG(num_pages >= 1, "num_pages must be >= 1 (got %d)", num_pages);
+  SAS_PTR(page_table);
+  SAS_PTR(q);
+  SAS_PTR(q_nope);
+  SAS_PTR(k_pages);
+  SAS_PTR(v_pages);
+  SAS_PTR(gate_key_pages);
+  SAS_PTR(cur_pool);
+  SAS_PTR(wq);
+  SAS_PTR(qnorm_w);
+  SAS_PTR(wk);
+  SAS_PTR(knorm_w);
+  SAS_PTR(o);
+  SAS_PTR(workspace);
+  if (idx_out) SAS_CHECK_ARG(aligned16(idx_out), "idx_out is not 16-byte aligned");
+  if (logg_out) SAS_CHECK_ARG(aligned16(logg_out), "logg_out is not 16-byte aligned");
+  const size_t need = decode_workspace_bytes(*p);
+  if (workspace_bytes < need) {
+    set_error("workspace too small: %zu < %zu bytes", workspace_bytes, need);
+    return SAS_ERR_WORKSPACE;
+  }
+  DecodePaging pg;
+  pg.pt = page_table;
+  pg.num_pages = num_pages;
+  return launch_decode(*p, q, q_nope, k_pages, v_pages, gate_key_pages, cur_pool, wq, qnorm_w, wk,
+                       knorm_w, o, idx_out, logg_out, workspace, pg, stream);
 }
 
 }  // extern "C"

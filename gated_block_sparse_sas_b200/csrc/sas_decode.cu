@@ -53,7 +53,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_gate_kernel(
     const T* __restrict__ wk, const float* __restrict__ knorm_w, const int32_t* __restrict__ seqlens,
     const float* __restrict__ rc, const float* __restrict__ rs, int Hq, int Hkv, int d, int B, int K,
     int NBmax, int capacity, float eps, int ungated, int32_t* __restrict__ sel_idx,
-    float* __restrict__ sel_logg, int32_t* __restrict__ idx_out, float* __restrict__ logg_out) {
+    float* __restrict__ sel_logg, int32_t* __restrict__ idx_out, float* __restrict__ logg_out,
+    const int32_t* __restrict__ pt, int num_pages, int* __restrict__ err) {
   extern __shared__ float smem[];
   const int G = Hq / Hkv, GD = G * d, C = 3 * d;
   float* qcat = smem;                  // [GD]
@@ -65,13 +66,27 @@ __global__ void __launch_bounds__(kDecThreads) decode_gate_kernel(
   int* cnt_red = reinterpret_cast<int*>(red + kDecWarps);  // [2][kDecWarps]
   int* misc = cnt_red + 2 * kDecWarps;                      // [4]
   int* hist = misc + 4;                                     // [256] radix histogram
+  int* pages = hist + 256;                                  // [NBmax] paged caches: page of block j
 
   const int kv = blockIdx.x, b = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int L = seqlens[b];
   const int t = L - 1, c = t / B, n = L - c * B;
   const size_t orow = ((size_t)b * Hkv + kv) * (K + 1);
-  if (L < 1 || L > capacity) {   // invalid length: empty selection, the merge writes 0
+  bool empty = L < 1 || L > capacity;   // invalid length: empty selection, the merge writes 0
+  if (!empty && pt != nullptr) {   // paged caches: the pages of blocks 0..c, range-checked
+    int bad = 0;
+    for (int j = tid; j <= c; j += kDecThreads) {
+      const int pg = pt[(size_t)b * NBmax + j];
+      bad |= (pg < 0 || pg >= num_pages) ? 1 : 0;
+      pages[j] = pg;
+    }
+    if (__syncthreads_or(bad)) {   // a page id out of range: report it, read nothing
+      if (tid == 0) atomicCAS(err, 0, 62);
+      empty = true;
+    }
+  }
+  if (empty) {
     for (int sl = tid; sl <= K; sl += kDecThreads) {
       sel_idx[orow + sl] = -1;
       sel_logg[orow + sl] = 0.f;
@@ -81,7 +96,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_gate_kernel(
     return;
   }
 
-  if (tid == 0 && c > 0) {   // start streaming this row's cached block keys into L2 now: the
+  if (tid == 0 && c > 0 && pt == nullptr) {   // start streaming this row's cached block keys into L2 now: the
     // projections below take a while and the scores read these rows only afterwards
     const char* src = reinterpret_cast<const char*>(gkc + ((size_t)b * Hkv + kv) * (size_t)NBmax * H);
     const size_t bytes = (size_t)c * H * 2;   // a multiple of 16 (H >= 32)
@@ -207,8 +222,10 @@ __global__ void __launch_bounds__(kDecThreads) decode_gate_kernel(
 #pragma unroll
       for (int it = 0; it < UNR; ++it) {
         const int j = j0 + it * RPW + rsub;
-        raw[it] = (j < c) ? __ldg(reinterpret_cast<const uint4*>(base + (size_t)j * H))
-                          : make_uint4(0u, 0u, 0u, 0u);
+        const __nv_bfloat16* row =
+            pt != nullptr ? gkc + ((size_t)pages[j < c ? j : 0] * Hkv + kv) * H + sub * 8
+                          : base + (size_t)j * H;
+        raw[it] = (j < c) ? __ldg(reinterpret_cast<const uint4*>(row)) : make_uint4(0u, 0u, 0u, 0u);
       }
 #pragma unroll
       for (int it = 0; it < UNR; ++it) {
@@ -743,11 +760,12 @@ static size_t decode_bulk_smem() {
 template <typename T, int D, int G>
 static void decode_attn_launch(const sas_decode_problem& p, const void* q, const void* kc,
                                const void* vc, int32_t* sel_idx, float* sel_logg, float* part_ml,
-                               float* part_acc, int* err, void* o, int ns, cudaStream_t st) {
+                               float* part_acc, int* err, void* o, int ns,
+                               const DecodePaging& pg, cudaStream_t st) {
   dim3 grid(p.num_kv_heads, p.batch, ns);
   if constexpr (std::is_same<T, __nv_bfloat16>::value && D == 128) {
     if (decode_attn_tc_supported(p)) {   // tensor-core path (sas_decode_tc.cu)
-      launch_decode_attn_tc(p, q, kc, vc, sel_idx, sel_logg, part_ml, part_acc, err, ns, st);
+      launch_decode_attn_tc(p, q, kc, vc, sel_idx, sel_logg, part_ml, part_acc, err, ns, pg, st);
       decode_merge_kernel<T, D, G><<<dim3(p.num_kv_heads, p.batch), 256, 0, st>>>(
           part_ml, part_acc, p.num_kv_heads, ns, (T*)o);
       return;
@@ -776,11 +794,12 @@ template <typename T>
 static void decode_gate_launch(const sas_decode_problem& p, const void* q_nope, const void* gkc,
                                const float* cur_pool, const void* wq, const float* qnorm_w,
                                const void* wk, const float* knorm_w, int32_t* sel_idx,
-                               float* sel_logg, int32_t* idx_out, float* logg_out, cudaStream_t st) {
+                               float* sel_logg, int32_t* idx_out, float* logg_out,
+                               const DecodePaging& pg, int* err, cudaStream_t st) {
   const int NBmax = (p.capacity + p.block - 1) / p.block;
   const int G = p.num_q_heads / p.num_kv_heads;
   const size_t smem = (size_t)(G * p.head_dim + 3 * p.head_dim + 2 * p.gate_hidden + NBmax + 1 +
-                               3 * kDecWarps + 4 + 256) * sizeof(float);
+                               3 * kDecWarps + 4 + 256 + NBmax) * sizeof(float);
   dim3 grid(p.num_kv_heads, p.batch);
 #define SAS_DG(H, NPT)                                                                           \
   {                                                                                              \
@@ -790,7 +809,7 @@ static void decode_gate_launch(const sas_decode_problem& p, const void* q_nope, 
         (const T*)q_nope, (const __nv_bfloat16*)gkc, cur_pool, (const T*)wq, qnorm_w, (const T*)wk, \
         knorm_w, p.seqlens, p.gate_rope_cos, p.gate_rope_sin, p.num_q_heads, p.num_kv_heads,      \
         p.head_dim, p.block, p.topk, NBmax, p.capacity, p.rms_eps, p.ungated, sel_idx, sel_logg, \
-        idx_out, logg_out);                                                                      \
+        idx_out, logg_out, pg.pt, pg.num_pages, err);                                           \
   }
 #define SAS_DG_H(NPT)                              \
   switch (p.gate_hidden) {                         \
@@ -810,7 +829,7 @@ sas_status launch_decode(const sas_decode_problem& p, const void* q, const void*
                          const void* k_cache, const void* v_cache, const void* gkc,
                          const float* cur_pool, const void* wq, const float* qnorm_w,
                          const void* wk, const float* knorm_w, void* o, int32_t* idx_out,
-                         float* logg_out, void* ws, cudaStream_t st) {
+                         float* logg_out, void* ws, const DecodePaging& pg, cudaStream_t st) {
   const int G = p.num_q_heads / p.num_kv_heads;
   const size_t pairs = (size_t)p.batch * p.num_kv_heads;
   const int ns = decode_nsplit(p);
@@ -833,15 +852,15 @@ sas_status launch_decode(const sas_decode_problem& p, const void* q, const void*
   w += al(pairs * ns * G * p.head_dim * 4);
   if (p.dtype == SAS_BF16)
     decode_gate_launch<__nv_bfloat16>(p, q_nope, gkc, cur_pool, wq, qnorm_w, wk, knorm_w, sel_idx,
-                                      sel_logg, idx_out, logg_out, st);
+                                      sel_logg, idx_out, logg_out, pg, err, st);
   else
     decode_gate_launch<float>(p, q_nope, gkc, cur_pool, wq, qnorm_w, wk, knorm_w, sel_idx, sel_logg,
-                              idx_out, logg_out, st);
+                              idx_out, logg_out, pg, err, st);
   sas_status s = launch_status("decode gate", 1);
   if (s != SAS_OK) return s;
 #define SAS_DA(T, D, G)                                                                      \
   decode_attn_launch<T, D, G>(p, q, k_cache, v_cache, sel_idx, sel_logg, part_ml, part_acc, err, \
-                              o, ns, st)
+                              o, ns, pg, st)
 #define SAS_DA_G(T, D)                   \
   switch (G) {                           \
     case 1: SAS_DA(T, D, 1); break;      \

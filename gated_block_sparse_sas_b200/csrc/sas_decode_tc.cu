@@ -63,6 +63,8 @@ struct DecTcArgs {
   int* err;
   int Hkv, G, capacity, K, nsplit;
   float scale_log2;
+  const int32_t* pt;            // paged caches: page of block j of sequence b ([batch][NBmax]); or null
+  int nbmax, num_pages;
 };
 
 __global__ void __launch_bounds__(dtc::kThreads, 2)
@@ -75,7 +77,13 @@ __global__ void __launch_bounds__(dtc::kThreads, 2)
   const int kv = blockIdx.x, b = blockIdx.y, split = blockIdx.z;
   const int G = a.G, Hq = a.Hkv * G, K1 = a.K + 1;
   const int Lraw = a.seqlens[b];
-  const bool seq_ok = Lraw >= 1 && Lraw <= a.capacity;
+  bool len_ok = Lraw >= 1 && Lraw <= a.capacity;
+  int own_page = 0;   // paged caches: the page of the newest token's block, range-checked
+  if (len_ok && a.pt != nullptr) {
+    own_page = a.pt[(size_t)b * a.nbmax + (Lraw - 1) / kB];
+    len_ok = own_page >= 0 && own_page < a.num_pages;
+  }
+  const bool seq_ok = len_ok;
   const int L = seq_ok ? Lraw : 0;
   const int per = (K1 + a.nsplit - 1) / a.nsplit;
   const int sl0 = split * per, sl1 = min(K1, sl0 + per);
@@ -165,8 +173,10 @@ __global__ void __launch_bounds__(dtc::kThreads, 2)
     for (int h = w4; h < G; h += 4) {
       float dot = 0.f;
       if (seq_ok) {
-        const uint2 kr = *reinterpret_cast<const uint2*>(
-            a.kc + (((size_t)b * a.Hkv + kv) * a.capacity + (L - 1)) * kD + lane * 4);
+        const size_t own = a.pt != nullptr
+                               ? ((size_t)own_page * a.Hkv + kv) * kB + (L - 1) % kB
+                               : ((size_t)b * a.Hkv + kv) * a.capacity + (L - 1);
+        const uint2 kr = *reinterpret_cast<const uint2*>(a.kc + own * kD + lane * 4);
         const uint2 qr = *reinterpret_cast<const uint2*>(a.q + ((size_t)b * Hq + kv * G + h) * kD + lane * 4);
         const float2 k01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&kr.x));
         const float2 k23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&kr.y));
@@ -204,11 +214,20 @@ __global__ void __launch_bounds__(dtc::kThreads, 2)
         uint8_t* dst = sm + OFF_STAGE + slot * kKV;
         const int ja = blk_j[2 * n];
         const int jb = (2 * n + 1 < nblk) ? blk_j[2 * n + 1] : ja;   // odd count: masked copy
+        // block j's 64 keys: rows j*64.. of (b, kv) in the contiguous cache, or all 64 rows of
+        // (page of j, kv) in the paged one (pages range-checked by the gate; a TMA box outside
+        // the tensor is filled, never read)
+        int ya = ja * kB, yb = jb * kB, za = z, zb = z;
+        if (a.pt != nullptr) {
+          ya = yb = 0;
+          za = a.pt[(size_t)b * a.nbmax + ja] * a.Hkv + kv;
+          zb = a.pt[(size_t)b * a.nbmax + jb] * a.Hkv + kv;
+        }
         mbar_arrive_expect_tx(full + slot, kKV);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          tma_load_3d(dst + h * kHalfPair, map, full + slot, 64 * h, ja * kB, z);
-          tma_load_3d(dst + h * kHalfPair + kHalfBlk, map, full + slot, 64 * h, jb * kB, z);
+          tma_load_3d(dst + h * kHalfPair, map, full + slot, 64 * h, ya, za);
+          tma_load_3d(dst + h * kHalfPair + kHalfBlk, map, full + slot, 64 * h, yb, zb);
         }
         issued = i + 1;
       }
@@ -353,11 +372,14 @@ bool decode_attn_tc_supported(const sas_decode_problem& p) {
 sas_status launch_decode_attn_tc(const sas_decode_problem& p, const void* q, const void* kc,
                                  const void* vc, const int32_t* sel_idx, const float* sel_logg,
                                  float* part_ml, float* part_acc, int* err, int ns,
-                                 cudaStream_t st) {
+                                 const DecodePaging& pg, cudaStream_t st) {
   CUtensorMap tk, tv;
-  const uint64_t rows = (uint64_t)p.batch * p.num_kv_heads;
-  if (!make_tmap_bf16_3d(&tk, kc, 128, p.capacity, rows, 64, 64, 1) ||
-      !make_tmap_bf16_3d(&tv, vc, 128, p.capacity, rows, 64, 64, 1)) {
+  // contiguous: [batch*Hkv][capacity][128]; paged: [num_pages*Hkv][64][128]
+  const uint64_t rows = pg.pt != nullptr ? (uint64_t)pg.num_pages * p.num_kv_heads
+                                         : (uint64_t)p.batch * p.num_kv_heads;
+  const uint64_t keys = pg.pt != nullptr ? (uint64_t)dtc::kB : (uint64_t)p.capacity;
+  if (!make_tmap_bf16_3d(&tk, kc, 128, keys, rows, 64, 64, 1) ||
+      !make_tmap_bf16_3d(&tv, vc, 128, keys, rows, 64, 64, 1)) {
     set_error("decode: TMA descriptor creation failed");
     return SAS_ERR_CUDA;
   }
@@ -376,6 +398,9 @@ sas_status launch_decode_attn_tc(const sas_decode_problem& p, const void* q, con
   a.K = p.topk;
   a.nsplit = ns;
   a.scale_log2 = kLog2e / sqrtf(128.f);
+  a.pt = pg.pt;
+  a.nbmax = (p.capacity + p.block - 1) / p.block;
+  a.num_pages = pg.num_pages;
   static std::once_flag attr_once;
   std::call_once(attr_once, [] {
     cudaFuncSetAttribute(decode_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "sas_common.cuh"
+#include "sas_gate.cuh"
 #include "sas_kernels.h"
 
 namespace sas {
@@ -61,28 +62,6 @@ sas_status launch_pool_keys(const sas_problem& p, const void* k_nope, float* poo
     pool_keys_kernel<<<grid, 256, 0, st>>>((const float*)k_nope, p.cu_seqlens, p.num_kv_heads,
                                            p.head_dim, p.block, NBmax, pooled);
   return launch_status("pool_keys", 1);
-}
-
-// ---------------------------------------------------------------------------------------
-// Shared epilogue: RMSNorm over h (x / sqrt(mean x^2 + eps) * w), then rotate-half rotary
-// at position pos using the fp32 tables (built in double on the host). One warp per row.
-// ---------------------------------------------------------------------------------------
-template <int H>
-__device__ __forceinline__ void norm_rope_row(const float* x, const float* __restrict__ w, float eps,
-                                              const float* __restrict__ rc, const float* __restrict__ rs,
-                                              int pos, float* dst, int lane) {
-  float ss = 0.f;
-  for (int e = lane; e < H; e += 32) ss += x[e] * x[e];
-  ss = warp_sum(ss);
-  const float rn = sqrtf(ss / (float)H + eps);
-  const float* c = rc + (size_t)pos * (H / 2);
-  const float* s = rs + (size_t)pos * (H / 2);
-  for (int e = lane; e < H / 2; e += 32) {
-    const float a = x[e] / rn * w[e];
-    const float b = x[e + H / 2] / rn * w[e + H / 2];
-    dst[e] = a * c[e] - b * s[e];
-    dst[e + H / 2] = b * c[e] + a * s[e];
-  }
 }
 
 // ---------------------------------------------------------------------------------------
@@ -533,52 +512,6 @@ sas_status launch_gate_scores(const sas_problem& p, const void* q_nope, const vo
 // row is emitted in ascending block order with ballots: every key above the threshold,
 // plus the lowest-index ties at the threshold until K are kept.
 // ---------------------------------------------------------------------------------------
-// One row with c > K historical candidates held as NPL keys per lane (c <= 32 NPL).
-template <int NPL>
-__device__ __forceinline__ void topk_row(const float* __restrict__ srow, float l, int c, int K,
-                                         int lane, int32_t* __restrict__ irow,
-                                         float* __restrict__ grow) {
-  uint32_t key[NPL];
-#pragma unroll
-  for (int r = 0; r < NPL; ++r) {
-    const int j = r * 32 + lane;
-    key[r] = (j < c) ? order_key(srow[j]) : 0u;
-  }
-  uint32_t thr = 0;
-#pragma unroll 1
-  for (int bit = 31; bit >= 0; --bit) {
-    const uint32_t cand = thr | (1u << bit);
-    int cnt = 0;
-#pragma unroll
-    for (int r = 0; r < NPL; ++r) cnt += (key[r] >= cand) ? 1 : 0;
-    cnt = __reduce_add_sync(0xffffffffu, cnt);
-    if (cnt >= K) thr = cand;
-  }
-  int gt = 0;
-#pragma unroll
-  for (int r = 0; r < NPL; ++r) gt += (key[r] > thr) ? 1 : 0;
-  gt = __reduce_add_sync(0xffffffffu, gt);
-  const int need_eq = K - gt;
-  const unsigned below = (1u << lane) - 1u;
-  int out = 0, eq_seen = 0;
-#pragma unroll
-  for (int r = 0; r < NPL; ++r) {
-    const bool is_gt = key[r] > thr, is_eq = key[r] == thr;
-    const unsigned eqm = __ballot_sync(0xffffffffu, is_eq);
-    const int eq_rank = eq_seen + __popc(eqm & below);
-    const bool sel = is_gt || (is_eq && eq_rank < need_eq);
-    const unsigned selm = __ballot_sync(0xffffffffu, sel);
-    if (sel) {
-      const int pos = out + __popc(selm & below);
-      const int j = r * 32 + lane;
-      irow[pos] = j;
-      grow[pos] = srow[j] - l;
-    }
-    out += __popc(selm);
-    eq_seen += __popc(eqm);
-  }
-}
-
 // The key count per lane follows the row's own candidate count c_t (warp-uniform), so the
 // work of a row scales with its visible blocks, not with the longest sequence. MAXNPL bounds
 // the instantiated sizes (and so the registers) by the problem's NBmax.

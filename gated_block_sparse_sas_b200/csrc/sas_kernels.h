@@ -19,6 +19,12 @@ sas_status launch_gate_scores(const sas_problem& p, const void* q_nope, const vo
                               const float* gkeys, const void* wq, const float* qnorm_w,
                               const void* wk, const float* knorm_w, float* scores, float* lse,
                               void* workspace, cudaStream_t st);
+bool gate_select_fused(const sas_problem& p);
+size_t gate_select_workspace_bytes(const sas_problem& p);
+sas_status launch_gate_select(const sas_problem& p, const void* q_nope, const void* k_nope,
+                              const float* gkeys, const void* wq, const float* qnorm_w,
+                              const void* wk, const float* knorm_w, int32_t* idx, float* logg,
+                              float* lse, void* workspace, cudaStream_t st);
 sas_status launch_topk(const sas_problem& p, const float* scores, const float* lse, int32_t* idx,
                        float* logg, cudaStream_t st);
 bool gate_bwd_supported(const sas_problem& p);
@@ -84,11 +90,18 @@ size_t gate_tc_workspace_bytes(const sas_problem& p);
 sas_status launch_gate_proj_tc(const sas_problem& p, const void* q_nope, const void* k_nope,
                                const void* wq, const void* wk, void* workspace, float** qproj,
                                float** kproj, cudaStream_t st);
+// Paged decode caches: pt = page table [batch, ceil(capacity / B)] (page of block j of
+// sequence b), pages of [Hkv, B, d] keys / values and [Hkv, h] gate keys; pt == nullptr for
+// the contiguous [batch, Hkv, capacity, d] layout.
+struct DecodePaging {
+  const int32_t* pt = nullptr;
+  int num_pages = 0;
+};
 bool decode_attn_tc_supported(const sas_decode_problem& p);
 sas_status launch_decode_attn_tc(const sas_decode_problem& p, const void* q, const void* kc,
                                  const void* vc, const int32_t* sel_idx, const float* sel_logg,
                                  float* part_ml, float* part_acc, int* err, int ns,
-                                 cudaStream_t st);
+                                 const DecodePaging& pg, cudaStream_t st);
 
 int decode_nsplit(const sas_decode_problem& p);
 size_t decode_workspace_bytes(const sas_decode_problem& p);
@@ -96,6 +109,6 @@ sas_status launch_decode(const sas_decode_problem& p, const void* q, const void*
                          const void* k_cache, const void* v_cache, const void* gkc,
                          const float* cur_pool, const void* wq, const float* qnorm_w,
                          const void* wk, const float* knorm_w, void* o, int32_t* idx_out,
-                         float* logg_out, void* ws, cudaStream_t st);
+                         float* logg_out, void* ws, const DecodePaging& pg, cudaStream_t st);
 
 }  // namespace sas

@@ -50,7 +50,8 @@
  *     waits, about one second); 51-57 forward, 71-79 backward, 91-93 gate
  *     projection waits that gave up; 60 forward / 61 decode: a row whose largest
  *     logit exceeds its own key's logit by more than ~97 nats (outside the fixed
- *     per-row reference's fp32 range; that row's output is 0 and its lse -inf).
+ *     per-row reference's fp32 range; that row's output is 0 and its lse -inf);
+ *     62 paged decode: a page id out of range.
  *     The outputs of a call with a nonzero code are not valid.
  *   - Supported: d in {64, 128}; B in {16, 32, 64}; 1 <= K <= 127;
  *     h in {32, 64, 128}; G in {1, 2, 4, 5, 8}; NBmax <= 2048 (prefill) or
@@ -168,6 +169,24 @@ sas_status sas_gate_scores(const sas_problem* p, const void* q_nope, const void*
                            const void* wk, const float* knorm_w, float* scores, float* lse,
                            void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* A3 + A4 fused -- gate scores and Top-K selection in one pass (paper abstract: Top-K keeps
+ * the computation sparse; model card: Qproj, Q/K normalisation, gate RoPE, Top-K).
+ * Same inputs as sas_gate_scores, same results as sas_gate_scores followed by sas_topk:
+ * idx int32 / logg fp32 [T, Hkv, K+1] (ids ascending, current block last, -1 padding),
+ * and, if lse is not NULL, the gate logsumexp fp32 [T, Hkv]. For bf16, d = 128, h = 128
+ * and NBmax <= 1024 the scores live only in shared memory (one kernel holds a tile's score
+ * rows, selects and writes the kept ids); the scores are bit-identical to sas_gate_scores',
+ * so the ids are too, and the log-gates agree to fp32 rounding (the logsumexp is summed in
+ * another order). Other shapes run the two unfused kernels through the workspace, which
+ * then also holds the scores. Workspace (sas_gate_select_workspace_size): word 0 is the
+ * call's error word (codes 91-93). */
+sas_status sas_gate_select_workspace_size(const sas_problem* p, size_t* bytes);
+sas_status sas_gate_select(const sas_problem* p, const void* q_nope, const void* k_nope,
+                           const float* gate_keys, const void* wq, const float* qnorm_w,
+                           const void* wk, const float* knorm_w, int32_t* idx, float* logg,
+                           float* lse, void* workspace, size_t workspace_bytes,
+                           cudaStream_t stream);
+
 /* Router backward (README intro item (b): the loss reaches the selector; paper abstract:
  * end-to-end optimisation of the context ranking) -- gradients of one layer's gate
  * parameters through the log-gates of the kept blocks, the selection held fixed:
@@ -249,6 +268,26 @@ sas_status sas_decode(const sas_decode_problem* p, const void* q, const void* q_
                       const void* wk, const float* knorm_w, void* o, int32_t* idx_out,
                       float* logg_out, void* workspace, size_t workspace_bytes,
                       cudaStream_t stream);
+
+/* A7 over paged caches -- the decode step of sas_decode with the KV cache in fixed-size pages
+ * (one KV block per page), as a paged serving backend holds it (README "Acknowledgements":
+ * the SGLang block-sparse fork; model card, SGLang seer_attn launch section). Same operator,
+ * same results as sas_decode on the same cached values (bit-identical: the same kernels read
+ * the same numbers in the same order). Layout: page_table int32 [batch, ceil(capacity / B)],
+ * entry (b, j) = the page holding block j of sequence b (entries j <= (L_b - 1) / B are read);
+ * k_pages, v_pages dtype [num_pages, Hkv, B, d]; gate_key_pages bf16 [num_pages, Hkv, h] (the
+ * cached gate key of the page's block, read for complete blocks). Other arguments and the
+ * workspace (sas_decode_workspace_size) as sas_decode. A page id outside [0, num_pages) sets
+ * error code 62 in workspace word 0; that sequence's output is 0 and nothing is read through
+ * the bad entry. Supported: bf16, head_dim 128, B = 64 (the tensor-core decode);
+ * SAS_ERR_UNSUPPORTED otherwise. */
+sas_status sas_decode_paged(const sas_decode_problem* p, const int32_t* page_table,
+                            int32_t num_pages, const void* q, const void* q_nope,
+                            const void* k_pages, const void* v_pages, const void* gate_key_pages,
+                            const float* cur_pool, const void* wq, const float* qnorm_w,
+                            const void* wk, const float* knorm_w, void* o, int32_t* idx_out,
+                            float* logg_out, void* workspace, size_t workspace_bytes,
+                            cudaStream_t stream);
 
 /* Allocation-free variant of sas_decode (no counterpart in the SAS pages; a library
  * convenience). For callers that cannot allocate device memory around a decode step --

@@ -247,36 +247,49 @@ def norm_weight(seed: int, name: str, h: int, device) -> torch.Tensor:
     return z * torch.tensor(np.float32(0.25), device=z.device) + 1.0
 
 
-def prefill_inputs(shape: Shape, device="cpu", *, with_dout: bool = False) -> dict:
+def prefill_inputs(shape: Shape, device="cpu", *, with_dout: bool = False,
+                   sequence: int | None = None) -> dict:
     """Pre-rotary and rotated Q/K, V, gate weights (and dO) for a packed prefill problem.
 
     Values: N(0,1) for Q/K/V/dO; gate weights N(0,1)/sqrt(fan_in); RMSNorm weights
     1 + 0.25 N(0,1). Everything is rounded once to the problem dtype (gate weights
     included); norm weights stay fp32.
+    `sequence` = b draws only sequence b's tokens (the same values as in the packed draw)
+    and returns them as a one-sequence problem (see `sequence_shape`).
     """
-    T, Hq, Hkv, d, h, G = (shape.total_tokens, shape.num_q_heads, shape.num_kv_heads,
-                          shape.head_dim, shape.gate_hidden, shape.group)
+    Hq, Hkv, d, h, G = (shape.num_q_heads, shape.num_kv_heads, shape.head_dim,
+                        shape.gate_hidden, shape.group)
     dt, s = shape.torch_dtype, shape.seed
-    pos = shape.positions()
-    q_nope = draw(s, "q_nope", (T, Hq, d), device=device)
-    k_nope = draw(s, "k_nope", (T, Hkv, d), device=device)
+    if sequence is None:
+        T, t0, pos, cu = shape.total_tokens, 0, shape.positions(), shape.cu_seqlens
+    else:
+        T, t0 = shape.lengths[sequence], int(shape.cu_seqlens[sequence])
+        pos = np.arange(T, dtype=np.int64)
+        cu = np.array([0, T], dtype=np.int32)
+    q_nope = draw(s, "q_nope", (T, Hq, d), device=device, offset=t0 * Hq * d)
+    k_nope = draw(s, "k_nope", (T, Hkv, d), device=device, offset=t0 * Hkv * d)
     out = {
         "q_nope": q_nope.to(dt),
         "k_nope": k_nope.to(dt),
-        "v": draw(s, "v", (T, Hkv, d), dtype=dt, device=device),
+        "v": draw(s, "v", (T, Hkv, d), dtype=dt, device=device, offset=t0 * Hkv * d),
         "wq": draw(s, "wq", (Hkv, h, G * d), dtype=dt, device=device, scale=1.0 / math.sqrt(G * d)),
         "wk": draw(s, "wk", (Hkv, h, 3 * d), dtype=dt, device=device, scale=1.0 / math.sqrt(3 * d)),
         "qnorm_w": norm_weight(s, "qnorm_w", h, device),
         "knorm_w": norm_weight(s, "knorm_w", h, device),
-        "cu_seqlens": torch.from_numpy(shape.cu_seqlens).to(device),
+        "cu_seqlens": torch.from_numpy(cu).to(device),
     }
     # the attention reads rotated Q/K; rotate the already-rounded pre-rotary values
     out["q"] = backbone_rotate(out["q_nope"].float(), pos, dt, shape.attn_rope_base)
     out["k"] = backbone_rotate(out["k_nope"].float(), pos, dt, shape.attn_rope_base)
     del q_nope, k_nope
     if with_dout:
-        out["dout"] = draw(s, "dout", (T, Hq, d), dtype=dt, device=device)
+        out["dout"] = draw(s, "dout", (T, Hq, d), dtype=dt, device=device, offset=t0 * Hq * d)
     return out
+
+
+def sequence_shape(shape: Shape, b: int) -> Shape:
+    """Sequence b of a packed problem as a one-sequence problem (prefill_inputs(sequence=b))."""
+    return dataclasses.replace(shape, lengths=[shape.lengths[b]])
 
 
 def random_selection(shape: Shape, seed: int | None = None):

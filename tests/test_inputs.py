@@ -51,3 +51,15 @@ def test_random_selection_structure():
             assert len(set(row[:k])) == k and all(0 <= j < c for j in row[:k])
             assert list(row[:k]) == sorted(row[:k])
     assert (logg[idx >= 0] <= -1).all() and (logg[idx < 0] == 0).all()
+
+
+def test_sequence_draw_matches_packed_draw():
+    shp = si.Shape([40, 70, 33], 4, 2, 8, 16, 2, 8, "bf16", seed=6)
+    full = si.prefill_inputs(shp, with_dout=True)
+    one = si.prefill_inputs(shp, with_dout=True, sequence=1)
+    for k in ("q_nope", "k_nope", "q", "k", "v", "dout"):
+        assert torch.equal(full[k][40:110], one[k]), k
+    for k in ("wq", "wk", "qnorm_w", "knorm_w"):
+        assert torch.equal(full[k], one[k]), k
+    assert one["cu_seqlens"].tolist() == [0, 70]
+    assert si.sequence_shape(shp, 1).lengths == [70]

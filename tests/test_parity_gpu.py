@@ -337,3 +337,117 @@ def test_gate_backward(sas, name):
         e = rel_l2(gpu, ref[key])
         assert np.isfinite(to64(gpu)).all(), key
         assert e <= 2e-3, f"{key}: rel-L2 {e:.3e}"
+
+
+SELECT_CASES = {
+    # fused path, 64-token tiles (NBmax <= 512), ragged sequences, G 4 and 5
+    "bf16-d128-B64-ragged": ([300, 64, 1, 130], 8, 2, 128, 64, 3, 128, "bf16"),
+    "bf16-d128-B64-G5": ([513, 77, 4100], 10, 2, 128, 64, 31, 128, "bf16"),
+    # fused path, 32-token tiles (512 < NBmax <= 1024), K 63 as the 14B varlen workload
+    "bf16-G5-K63-40k": ([40000, 333], 10, 2, 128, 64, 63, 128, "bf16"),
+    # shapes outside the fused kernel: the unfused kernels through the workspace
+    "bf16-d64-B32": ([257, 33], 8, 4, 64, 32, 5, 64, "bf16"),
+    "fp32-d64-B16-tiny-shape": ([1024], 2, 1, 64, 16, 4, 32, "fp32"),
+}
+
+
+@pytest.mark.parametrize("name", list(SELECT_CASES))
+def test_gate_select_fused(sas, name):
+    """sas_gate_select (scores + Top-K in one pass, scores kept on chip) against the unfused
+    sas_gate_scores + sas_topk on the GPU (ids bit-identical, log-gates and logsumexp to fp32
+    rounding) and against the oracle on window/block/sequence edges and random rows."""
+    lengths, Hq, Hkv, d, B, K, h, dt = SELECT_CASES[name]
+    shape = si.Shape(list(lengths), Hq, Hkv, d, B, K, h, dt, seed=700)
+    inp = si.prefill_inputs(shape)
+    dev = torch.device("cuda:0")
+    g = {k: v.to(dev) for k, v in inp.items()}
+    prob = sas.Problem.from_lengths(shape.lengths, dev, num_q_heads=Hq, num_kv_heads=Hkv,
+                                    head_dim=d, block=B, topk=K, gate_hidden=h,
+                                    dtype=shape.torch_dtype)
+    pooled = sas.sas_pool_keys(prob, g["k_nope"])
+    gk = sas.sas_gate_keys(prob, pooled, g["wk"], g["knorm_w"])
+    ws = sas.gate_select_workspace(prob)
+    idx, logg, lse = sas.sas_gate_select(prob, g["q_nope"], g["k_nope"], gk, g["wq"], g["qnorm_w"],
+                                         g["wk"], g["knorm_w"], workspace=ws, want_lse=True)
+    scores, lse_u = sas.sas_gate_scores(prob, g["q_nope"], g["k_nope"], gk, g["wq"], g["qnorm_w"],
+                                        g["wk"], g["knorm_w"])
+    idx_u, logg_u = sas.sas_topk(prob, scores, lse_u)
+    torch.cuda.synchronize()
+    assert sas.error_code(ws) == 0
+    assert torch.equal(idx, idx_u), "fused and unfused selections differ"
+    assert (logg - logg_u).abs().max().item() <= 2e-6
+    assert (lse - lse_u).abs().max().item() <= 2e-6
+    rng = np.random.default_rng(701)
+    rows = set()
+    for s0, s1 in zip(shape.cu_seqlens[:-1], shape.cu_seqlens[1:]):
+        L = int(s1 - s0)
+        for t in (0, 63, 64, 2047, 4095, 4096, 32767, 32768, L - 1):
+            if 0 <= t < L:
+                rows.add(int(s0) + t)
+    rows |= set(rng.choice(shape.total_tokens, 60, replace=False).tolist())
+    rows = np.array(sorted(rows))
+    ref = orc.prefill_selection(inp["q_nope"], inp["k_nope"], inp["wq"], inp["qnorm_w"], inp["wk"],
+                                inp["knorm_w"], shape.cu_seqlens, B, K, 1e-6, 1e6, rows)
+    compare_selection(idx.cpu().numpy()[rows], logg.cpu().numpy()[rows], ref["idx"], ref["logg"],
+                      ref["margin"])
+    assert np.abs(to64(lse)[rows] - ref["lse"]).max() <= GATE_ABS
+
+
+def _paged_from_contiguous(inp, shp, seed, spare=17):
+    """Scatter contiguous decode caches into shuffled pages of one block each (plus unused
+    pages full of large values that must never be read)."""
+    NB = shp.capacity // shp.block
+    nb = shp.batch
+    n_pages = nb * NB + spare
+    perm = np.random.default_rng(seed).permutation(n_pages)
+    pt = perm[:nb * NB].reshape(nb, NB).astype(np.int32)
+    Hkv, d, h, B = shp.num_kv_heads, shp.head_dim, shp.gate_hidden, shp.block
+    kp = torch.full((n_pages, Hkv, B, d), 300.0, dtype=inp["k_cache"].dtype)
+    vp = torch.full((n_pages, Hkv, B, d), -300.0, dtype=inp["v_cache"].dtype)
+    gp = torch.full((n_pages, Hkv, h), 300.0, dtype=torch.bfloat16)
+    for b in range(nb):
+        for j in range(NB):
+            kp[pt[b, j]] = inp["k_cache"][b, :, j * B:(j + 1) * B]
+            vp[pt[b, j]] = inp["v_cache"][b, :, j * B:(j + 1) * B]
+            gp[pt[b, j]] = inp["gate_key_cache"][b, :, j]
+    return torch.from_numpy(pt), n_pages, kp, vp, gp
+
+
+PAGED_CASES = {
+    "budget2048-K31": ([3000, 65, 1, 1777, 4096], 4096, 16, 4, 128, 64, 31, 128),
+    "budget4096-K63-G5": ([6000, 4200, 130, 64], 8192, 20, 4, 128, 64, 63, 128),
+}
+
+
+@pytest.mark.parametrize("name", list(PAGED_CASES))
+def test_decode_paged_equals_contiguous(sas, name):
+    """sas_decode_paged over shuffled one-block pages gives exactly sas_decode's results on the
+    same cached values (same kernels, same numbers, same order), and a page id out of range
+    is reported (code 62) with that sequence's output 0 and the others unchanged."""
+    lengths, cap, Hq, Hkv, d, B, K, h = PAGED_CASES[name]
+    shp = si.DecodeShape(list(lengths), cap, Hq, Hkv, d, B, K, h, seed=410)
+    inp = si.decode_inputs(shp)
+    g = {k: v.cuda() for k, v in inp.items()}
+    prob = sas.DecodeProblem(seqlens=g["lengths"], capacity=cap, num_q_heads=Hq, num_kv_heads=Hkv,
+                             head_dim=d, block=B, topk=K, gate_hidden=h, dtype=torch.bfloat16)
+    common = (g["cur_pool"], g["wq"], g["qnorm_w"], g["wk"], g["knorm_w"])
+    o_c, i_c, l_c = sas.sas_decode(prob, g["q"], g["q_nope"], g["k_cache"], g["v_cache"],
+                                   g["gate_key_cache"], *common, want_selection=True, check=True)
+    pt, n_pages, kp, vp, gp = _paged_from_contiguous(inp, shp, 411)
+    pt, kp, vp, gp = pt.cuda(), kp.cuda(), vp.cuda(), gp.cuda()
+    o_p, i_p, l_p = sas.sas_decode_paged(prob, pt, n_pages, g["q"], g["q_nope"], kp, vp, gp, *common,
+                                         want_selection=True, check=True)
+    torch.cuda.synchronize()
+    assert torch.equal(i_p, i_c)
+    assert torch.equal(l_p, l_c)
+    assert torch.equal(o_p, o_c)
+    # a bad page id in sequence 0's history
+    bad = pt.clone()
+    bad[0, 3] = n_pages + 5
+    ws = sas._workspace(sas.lib_handle().sas_decode_workspace_size, prob.ref, prob.device)
+    o_b = sas.sas_decode_paged(prob, bad, n_pages, g["q"], g["q_nope"], kp, vp, gp, *common,
+                               workspace=ws)
+    torch.cuda.synchronize()
+    assert sas.error_code(ws) == 62
+    assert torch.count_nonzero(o_b[0]).item() == 0
+    assert torch.equal(o_b[1:], o_c[1:])
