@@ -24,7 +24,12 @@ Where the pages leave a step open, the reading used here is stated at that step:
 
   R1  selection is per query token; one gate per (token, KV head), shared by the G
       query heads of that KV group; Qproj reads the G pre-rotary query heads
-      concatenated (G*d -> h).
+      concatenated (G*d -> h). Variant (one gate per query head): Qproj reads each
+      query head alone (d -> h, Wq [Hq, h, d]), the head's query is scored against its
+      KV head's block keys, and every query head keeps its own blocks. The number of
+      gate ("selection") heads Hs is read off Wq's first axis (Hs = Hkv or Hq) and off
+      idx's second axis; query head hq uses selection head hq // (Hq/Hs) and KV head
+      hq // (Hq/Hkv).
   R2  the gate reads pre-rotary Q and K and applies its own rotary embedding
       (rotate-half over h, base 1e6) at position t (query) and jB (block start).
   R3  pooled block key = concat[max, min, mean] over the block's tokens (3d);
@@ -147,9 +152,9 @@ def gate_keys(pooled, wk, knorm_w, block: int, eps: float, base: float, lengths=
 
 
 def gate_query(q_nope_rows: np.ndarray, wq: np.ndarray, qnorm_w, eps: float, pos, base: float):
-    """q~ = rope(RMSNorm(Wq . concat_g Q_nope[t, kv*G+g]), pos = t)  (R1, R2, R4).
+    """q~ = rope(RMSNorm(Wq . concat_g Q_nope[t, s*Gs+g]), pos = t)  (R1, R2, R4).
 
-    q_nope_rows [n, Hq, d] -> [n, Hkv, h].
+    q_nope_rows [n, Hq, d], wq [Hs, h, Gs*d] -> [n, Hs, h] (Hs gate heads of Gs query heads).
     """
     n, Hq, d = q_nope_rows.shape
     Hkv = wq.shape[0]
@@ -167,11 +172,11 @@ def current_block_key(k_nope_seq: np.ndarray, t: int, block: int, wk, knorm_w, e
 
 def gate_scores(q_nope, k_nope, gkeys, wq, qnorm_w, wk, knorm_w, cu_seqlens, block, eps, base,
                 rows=None):
-    """A3: scores s[t, kv, j] = q~_t . k~_j / sqrt(h) over visible blocks j <= c_t, and lse[t, kv].
+    """A3: scores s[t, s, j] = q~_t,s . k~_j / sqrt(h) over visible blocks j <= c_t, and lse[t, s].
 
-    k~_j for j < c_t comes from `gkeys` [batch, NBmax, Hkv, h]; the current block uses the
-    prefix key (R7). Entries j > c_t are -inf. `rows` (packed token indices) restricts the
-    rows computed; returns (s [n, Hkv, NBmax], lse [n, Hkv], rows).
+    k~_j for j < c_t comes from `gkeys` [batch, NBmax, Hkv, h] (of the gate head's KV head);
+    the current block uses the prefix key (R7). Entries j > c_t are -inf. `rows` (packed
+    token indices) restricts the rows computed; returns (s [n, Hs, NBmax], lse [n, Hs], rows).
     """
     q = as64(q_nope)
     k = as64(k_nope)
@@ -182,17 +187,19 @@ def gate_scores(q_nope, k_nope, gkeys, wq, qnorm_w, wk, knorm_w, cu_seqlens, blo
     T = q.shape[0]
     rows = np.arange(T) if rows is None else np.asarray(rows)
     nbm, Hkv, h = gk.shape[1], gk.shape[2], gk.shape[3]
-    s = np.full((len(rows), Hkv, nbm), NEG_INF, dtype=F64)
-    lse = np.empty((len(rows), Hkv), dtype=F64)
+    Hs = wq_.shape[0]                       # gate heads: Hkv (per KV group) or Hq (per query head)
+    kv_of = np.arange(Hs) // (Hs // Hkv)    # KV head whose block keys gate head s scores against
+    s = np.full((len(rows), Hs, nbm), NEG_INF, dtype=F64)
+    lse = np.empty((len(rows), Hs), dtype=F64)
     starts = np.array([a for a, _ in seqs])
     for r, tg in enumerate(rows):
         b = int(np.searchsorted(starts, tg, side="right") - 1)
         s0 = seqs[b][0]
         t = int(tg - s0)
         c = t // block
-        qt = gate_query(q[tg:tg + 1], wq_, qw, eps, [t], base)[0]                # [Hkv, h]
+        qt = gate_query(q[tg:tg + 1], wq_, qw, eps, [t], base)[0]                # [Hs, h]
         kc = current_block_key(k[s0:seqs[b][1]], t, block, wk_, kw, eps, base)   # [Hkv, h]
-        keys = np.concatenate([gk[b, :c], kc[None]], axis=0)                    # [c+1, Hkv, h]
+        keys = np.concatenate([gk[b, :c], kc[None]], axis=0)[:, kv_of]          # [c+1, Hs, h]
         s[r, :, : c + 1] = np.einsum("kh,jkh->kj", qt, keys) / np.sqrt(h)
         m = s[r, :, : c + 1].max(axis=1, keepdims=True)
         lse[r] = (m + np.log(np.exp(s[r, :, : c + 1] - m).sum(axis=1, keepdims=True)))[:, 0]
@@ -261,7 +268,8 @@ def logit_bias(idx_seq: np.ndarray, logg_seq: np.ndarray, block: int, rows) -> n
 def attention_fwd(q, k, v, idx, logg, cu_seqlens, block: int, rows=None):
     """O and LSE of gated sparse causal attention.
 
-    q [T, Hq, d], k/v [T, Hkv, d] (rotated), idx/logg [T, Hkv, K+1]. For head hq (kv = hq//G)
+    q [T, Hq, d], k/v [T, Hkv, d] (rotated), idx/logg [T, Hs, K+1] (Hs gate heads: Hkv, or
+    Hq for one gate per query head). For head hq (gate head hq // (Hq/Hs), kv = hq // G)
     and token t: z_i = q_t . k_i / sqrt(d) + bias(t, i); O_t = softmax(z) V; LSE natural log.
     `rows` (packed token indices) restricts the rows computed. Returns (O [n, Hq, d],
     LSE [n, Hq], rows).
@@ -272,6 +280,8 @@ def attention_fwd(q, k, v, idx, logg, cu_seqlens, block: int, rows=None):
     T, Hq, d = q.shape
     Hkv = k.shape[1]
     G = Hq // Hkv
+    Hs = idx.shape[1]
+    Gs = Hq // Hs
     rows = np.arange(T) if rows is None else np.asarray(rows)
     O = np.zeros((len(rows), Hq, d), dtype=F64)
     LSE = np.zeros((len(rows), Hq), dtype=F64)
@@ -280,10 +290,11 @@ def attention_fwd(q, k, v, idx, logg, cu_seqlens, block: int, rows=None):
         if len(sel) == 0:
             continue
         loc = rows[sel] - s0
-        for kv in range(Hkv):
-            bias = logit_bias(idx[s0:s1, kv], logg[s0:s1, kv], block, loc)
-            for g in range(G):
-                hq = kv * G + g
+        for sh in range(Hs):
+            bias = logit_bias(idx[s0:s1, sh], logg[s0:s1, sh], block, loc)
+            for g in range(Gs):
+                hq = sh * Gs + g
+                kv = hq // G
                 z = q[s0 + loc, hq] @ k[s0:s1, kv].T / np.sqrt(d) + bias
                 m = z.max(axis=1, keepdims=True)
                 p = np.exp(z - m)
@@ -298,8 +309,9 @@ def attention_bwd(q, k, v, dout, idx, logg, cu_seqlens, block: int):
 
     With P = softmax(z): D_t = sum_i P_ti dP_ti = dO_t . O_t, dP = dO V^T,
     dS = P (dP - D), dQ = dS K / sqrt(d), dK = dS^T Q / sqrt(d), dV = P^T dO,
-    dlogg[t, kv, slot] = sum over the G heads and the keys of block idx[t, kv, slot] of dS.
-    Returns dq [T, Hq, d], dk, dv [T, Hkv, d], dlogg [T, Hkv, K+1].
+    dlogg[t, s, slot] = sum over the query heads of gate head s and the keys of block
+    idx[t, s, slot] of dS.
+    Returns dq [T, Hq, d], dk, dv [T, Hkv, d], dlogg [T, Hs, K+1].
     """
     q, k, v, do = as64(q), as64(k), as64(v), as64(dout)
     idx = np.asarray(idx)
@@ -307,16 +319,19 @@ def attention_bwd(q, k, v, dout, idx, logg, cu_seqlens, block: int):
     T, Hq, d = q.shape
     Hkv = k.shape[1]
     G = Hq // Hkv
+    Hs = idx.shape[1]
+    Gs = Hq // Hs
     dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
     dlogg = np.zeros(logg.shape, dtype=F64)
     for (s0, s1) in seq_ranges(cu_seqlens):
         L = s1 - s0
         loc = np.arange(L)
-        for kv in range(Hkv):
-            bias = logit_bias(idx[s0:s1, kv], logg[s0:s1, kv], block, loc)
+        for sh in range(Hs):
+            bias = logit_bias(idx[s0:s1, sh], logg[s0:s1, sh], block, loc)
             dbias = np.zeros((L, L), dtype=F64)
-            for g in range(G):
-                hq = kv * G + g
+            for g in range(Gs):
+                hq = sh * Gs + g
+                kv = hq // G
                 z = q[s0:s1, hq] @ k[s0:s1, kv].T / np.sqrt(d) + bias
                 m = z.max(axis=1, keepdims=True)
                 p = np.exp(z - m)
@@ -330,9 +345,9 @@ def attention_bwd(q, k, v, dout, idx, logg, cu_seqlens, block: int):
                 dv[s0:s1, kv] += p.T @ do[s0:s1, hq]
                 dbias += ds
             for t in range(L):
-                for slot, j in enumerate(idx[s0 + t, kv]):
+                for slot, j in enumerate(idx[s0 + t, sh]):
                     if j >= 0:
-                        dlogg[s0 + t, kv, slot] = dbias[t, j * block: min((j + 1) * block, t + 1)].sum()
+                        dlogg[s0 + t, sh, slot] = dbias[t, j * block: min((j + 1) * block, t + 1)].sum()
     return dq, dk, dv, dlogg
 
 
@@ -344,19 +359,22 @@ def attention_bwd_rows(q, k, v, dout, idx, logg, cu_seqlens, block: int, rows):
     T, Hq, d = q.shape
     Hkv = k.shape[1]
     G = Hq // Hkv
+    Hs = idx.shape[1]
+    Gs = Hq // Hs
     rows = np.asarray(rows)
     dq = np.zeros((len(rows), Hq, d), dtype=F64)
-    dlogg = np.zeros((len(rows), Hkv, idx.shape[2]), dtype=F64)
+    dlogg = np.zeros((len(rows), Hs, idx.shape[2]), dtype=F64)
     for (s0, s1) in seq_ranges(cu_seqlens):
         sel = np.nonzero((rows >= s0) & (rows < s1))[0]
         if len(sel) == 0:
             continue
         loc = rows[sel] - s0
-        for kv in range(Hkv):
-            bias = logit_bias(idx[s0:s1, kv], logg[s0:s1, kv], block, loc)
+        for sh in range(Hs):
+            bias = logit_bias(idx[s0:s1, sh], logg[s0:s1, sh], block, loc)
             dbias = np.zeros_like(bias)
-            for g in range(G):
-                hq = kv * G + g
+            for g in range(Gs):
+                hq = sh * Gs + g
+                kv = hq // G
                 z = q[s0 + loc, hq] @ k[s0:s1, kv].T / np.sqrt(d) + bias
                 m = z.max(axis=1, keepdims=True)
                 p = np.exp(z - m)
@@ -368,9 +386,9 @@ def attention_bwd_rows(q, k, v, dout, idx, logg, cu_seqlens, block: int, rows):
                 dq[sel, hq] = ds @ k[s0:s1, kv] / np.sqrt(d)
                 dbias += ds
             for r, t in enumerate(loc):
-                for slot, j in enumerate(idx[s0 + t, kv]):
+                for slot, j in enumerate(idx[s0 + t, sh]):
                     if j >= 0:
-                        dlogg[sel[r], kv, slot] = dbias[r, j * block: min((j + 1) * block, t + 1)].sum()
+                        dlogg[sel[r], sh, slot] = dbias[r, j * block: min((j + 1) * block, t + 1)].sum()
     return dq, dlogg
 
 
@@ -387,19 +405,34 @@ def attention_bwd_keys(q, k, v, dout, idx, logg, cu_seqlens, block: int, seq: in
     Hq, d = q.shape[1], q.shape[2]
     Hkv = k.shape[1]
     G = Hq // Hkv
+    Hs = idx.shape[1]
+    Gs = Hq // Hs
     s0, s1 = seq_ranges(cu_seqlens)[seq]
     L = s1 - s0
     jlo, jhi = key_lo // block, (key_hi - 1) // block
-    cand = np.arange(key_lo, L)
-    hit = np.any((idx[s0 + cand, kv, :, None] >= jlo) & (idx[s0 + cand, kv, :, None] <= jhi), axis=(1, 2))
-    loc = cand[hit]
     dk = np.zeros((key_hi - key_lo, d), dtype=F64)
     dv = np.zeros((key_hi - key_lo, d), dtype=F64)
-    if len(loc) == 0:
-        return dk, dv
-    bias = logit_bias(idx[s0:s1, kv], logg[s0:s1, kv], block, loc)
-    for g in range(G):
-        hq = kv * G + g
+    cand = np.arange(key_lo, L)
+    for sh in range(Hs):
+        if (sh * Gs) // G != kv:          # gate heads whose query heads read this KV head
+            continue
+        hit = np.any((idx[s0 + cand, sh, :, None] >= jlo) & (idx[s0 + cand, sh, :, None] <= jhi),
+                     axis=(1, 2))
+        loc = cand[hit]
+        if len(loc) == 0:
+            continue
+        _keys_grad_one_gate_head(q, k, v, do, idx, logg, block, s0, s1, sh, Gs, kv, key_lo,
+                                 key_hi, loc, dk, dv)
+    return dk, dv
+
+
+def _keys_grad_one_gate_head(q, k, v, do, idx, logg, block, s0, s1, sh, Gs, kv, key_lo, key_hi,
+                             loc, dk, dv):
+    """Adds to dk, dv the contribution of the query heads of gate head sh (rows `loc`)."""
+    d = q.shape[2]
+    bias = logit_bias(idx[s0:s1, sh], logg[s0:s1, sh], block, loc)
+    for g in range(Gs):
+        hq = sh * Gs + g
         z = q[s0 + loc, hq] @ k[s0:s1, kv].T / np.sqrt(d) + bias
         m = z.max(axis=1, keepdims=True)
         p = np.exp(z - m)
@@ -410,7 +443,6 @@ def attention_bwd_keys(q, k, v, dout, idx, logg, cu_seqlens, block: int, seq: in
         ds = p * (dp - D)
         dk += ds[:, key_lo:key_hi].T @ q[s0 + loc, hq] / np.sqrt(d)
         dv += p[:, key_lo:key_hi].T @ do[s0 + loc, hq]
-    return dk, dv
 
 
 # ------------------------------------------------------------------------------------------
@@ -472,6 +504,8 @@ def gate_backward(q_nope, k_nope, wq, qnorm_w, wk, knorm_w, idx, dlogg, cu_seqle
     dl = as64(dlogg)
     T, Hq, d = q.shape
     Hkv, h = wq_.shape[0], wq_.shape[1]
+    if wk_.shape[0] != Hkv:
+        raise NotImplementedError("router backward: one gate per KV group only")
     G = Hq // Hkv
     cu = np.asarray(cu_seqlens, dtype=np.int64)
     seqs = seq_ranges(cu)
@@ -552,44 +586,46 @@ def decode(q, q_nope, k_cache, v_cache, lengths, gate_key_cache, cur_pool, wq, q
     wq_, wk_, qw, kw = as64(wq), as64(wk), as64(qnorm_w), as64(knorm_w)
     lengths = np.asarray(lengths, dtype=np.int64)
     nb_all, Hq, d = q.shape
-    Hkv, h = wq_.shape[0], wq_.shape[1]
-    G = Hq // Hkv
+    Hs, h = wq_.shape[0], wq_.shape[1]          # gate heads: Hkv, or Hq (one per query head)
+    Hkv = wk_.shape[0]
+    G, Gs = Hq // Hkv, Hq // Hs
     rows = np.arange(nb_all) if rows is None else np.asarray(rows)
     O = np.zeros((len(rows), Hq, d))
-    idx = np.full((len(rows), Hkv, K + 1), -1, dtype=np.int32)
-    logg = np.zeros((len(rows), Hkv, K + 1))
-    margin = np.zeros((len(rows), Hkv))
+    idx = np.full((len(rows), Hs, K + 1), -1, dtype=np.int32)
+    logg = np.zeros((len(rows), Hs, K + 1))
+    margin = np.zeros((len(rows), Hs))
     for r, b in enumerate(rows):
         L = int(lengths[b])
         t = L - 1
         c = t // block
         n = L - c * block
-        qt = gate_query(qn[b:b + 1], wq_, qw, eps, [t], base)[0]                   # [Hkv, h]
+        qt = gate_query(qn[b:b + 1], wq_, qw, eps, [t], base)[0]                   # [Hs, h]
         P = np.concatenate([cp[b, :, 0], cp[b, :, 1], cp[b, :, 2] / n], axis=-1)   # [Hkv, 3d]
         kc = project_key(P, wk_, kw, eps, float(c * block), base)                   # [Hkv, h]
         kcache = as64(k_cache[b]) if not isinstance(k_cache, np.ndarray) else k_cache[b]
         vcache = as64(v_cache[b]) if not isinstance(v_cache, np.ndarray) else v_cache[b]
-        for kv in range(Hkv):
+        for sh in range(Hs):
+            kv = (sh * Gs) // G
             keys = np.concatenate([as64(gkc[b, kv, :c]), kc[kv][None]], axis=0)    # [c+1, h]
-            s = keys @ qt[kv] / np.sqrt(h)
+            s = keys @ qt[sh] / np.sqrt(h)
             m = s.max()
             lse = m + np.log(np.exp(s - m).sum())
             ids, mg = select_row(s, c, K)
-            idx[r, kv, : len(ids)] = ids
-            logg[r, kv, : len(ids)] = s[ids] - lse
-            margin[r, kv] = mg
+            idx[r, sh, : len(ids)] = ids
+            logg[r, sh, : len(ids)] = s[ids] - lse
+            margin[r, sh] = mg
             if selection is None:
                 use_ids, use_lg = ids, s[ids] - lse
             else:
-                keep = np.asarray(selection[0][r, kv]) >= 0
-                use_ids = np.asarray(selection[0][r, kv])[keep]
-                use_lg = as64(selection[1][r, kv])[keep]
+                keep = np.asarray(selection[0][r, sh]) >= 0
+                use_ids = np.asarray(selection[0][r, sh])[keep]
+                use_lg = as64(selection[1][r, sh])[keep]
             bias = np.full(L, NEG_INF)
             for j, lg in zip(use_ids, use_lg):
                 bias[j * block: min((j + 1) * block, L)] = lg if gated else 0.0
             kk, vv = kcache[kv, :L], vcache[kv, :L]
-            for g in range(G):
-                hq = kv * G + g
+            for g in range(Gs):
+                hq = sh * Gs + g
                 z = kk @ q[b, hq] / np.sqrt(d) + bias
                 zm = z.max()
                 p = np.exp(z - zm)

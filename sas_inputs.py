@@ -186,10 +186,20 @@ class Shape:
     rms_eps: float = 1e-6
     gate_rope_base: float = 1e6
     attn_rope_base: float = 1e6
+    gate_heads: int | None = None   # gate (selection) heads: None/Hkv per KV group, Hq per query head
 
     @property
     def group(self) -> int:
         return self.num_q_heads // self.num_kv_heads
+
+    @property
+    def sel_heads(self) -> int:
+        return self.gate_heads or self.num_kv_heads
+
+    @property
+    def sel_group(self) -> int:
+        """query heads per gate head"""
+        return self.num_q_heads // self.sel_heads
 
     @property
     def batch(self) -> int:
@@ -257,8 +267,8 @@ def prefill_inputs(shape: Shape, device="cpu", *, with_dout: bool = False,
     `sequence` = b draws only sequence b's tokens (the same values as in the packed draw)
     and returns them as a one-sequence problem (see `sequence_shape`).
     """
-    Hq, Hkv, d, h, G = (shape.num_q_heads, shape.num_kv_heads, shape.head_dim,
-                        shape.gate_hidden, shape.group)
+    Hq, Hkv, d, h = shape.num_q_heads, shape.num_kv_heads, shape.head_dim, shape.gate_hidden
+    Hs, Gs = shape.sel_heads, shape.sel_group
     dt, s = shape.torch_dtype, shape.seed
     if sequence is None:
         T, t0, pos, cu = shape.total_tokens, 0, shape.positions(), shape.cu_seqlens
@@ -272,7 +282,7 @@ def prefill_inputs(shape: Shape, device="cpu", *, with_dout: bool = False,
         "q_nope": q_nope.to(dt),
         "k_nope": k_nope.to(dt),
         "v": draw(s, "v", (T, Hkv, d), dtype=dt, device=device, offset=t0 * Hkv * d),
-        "wq": draw(s, "wq", (Hkv, h, G * d), dtype=dt, device=device, scale=1.0 / math.sqrt(G * d)),
+        "wq": draw(s, "wq", (Hs, h, Gs * d), dtype=dt, device=device, scale=1.0 / math.sqrt(Gs * d)),
         "wk": draw(s, "wk", (Hkv, h, 3 * d), dtype=dt, device=device, scale=1.0 / math.sqrt(3 * d)),
         "qnorm_w": norm_weight(s, "qnorm_w", h, device),
         "knorm_w": norm_weight(s, "knorm_w", h, device),
@@ -295,14 +305,15 @@ def sequence_shape(shape: Shape, b: int) -> Shape:
 def random_selection(shape: Shape, seed: int | None = None):
     """A valid selection input for the attention alone, drawn independently of any gate.
 
-    Per (token, kv head): min(K, c_t) distinct historical blocks chosen uniformly
+    Per (token, gate head -- the kv head, or the query head with one gate per query head):
+    min(K, c_t) distinct historical blocks chosen uniformly
     (c_t = in-sequence block of the token), ascending, then the current block,
     then -1 padding. Log-gates are -(1 + 2|z|), z ~ N(0,1); padding slots hold 0.
-    Returns int32 idx [T, Hkv, K+1] and fp32 logg [T, Hkv, K+1] (numpy).
+    Returns int32 idx [T, Hs, K+1] and fp32 logg [T, Hs, K+1] (numpy).
     """
     seed = shape.seed if seed is None else seed
     g = np.random.Generator(np.random.PCG64(seed * 7919 + 13))
-    T, Hkv, B, K = shape.total_tokens, shape.num_kv_heads, shape.block, shape.topk
+    T, Hkv, B, K = shape.total_tokens, shape.sel_heads, shape.block, shape.topk
     idx = np.full((T, Hkv, K + 1), -1, dtype=np.int32)
     base = 0
     for L in shape.lengths:
@@ -345,6 +356,7 @@ class DecodeShape:
     rms_eps: float = 1e-6
     gate_rope_base: float = 1e6
     attn_rope_base: float = 1e6
+    gate_heads: int | None = None   # gate (selection) heads: None/Hkv per KV group, Hq per query head
 
     @property
     def batch(self) -> int:
@@ -353,6 +365,14 @@ class DecodeShape:
     @property
     def group(self) -> int:
         return self.num_q_heads // self.num_kv_heads
+
+    @property
+    def sel_heads(self) -> int:
+        return self.gate_heads or self.num_kv_heads
+
+    @property
+    def sel_group(self) -> int:
+        return self.num_q_heads // self.sel_heads
 
     @property
     def max_blocks(self) -> int:
@@ -417,7 +437,8 @@ def decode_inputs(shape: DecodeShape, device="cpu", *, batch_rows=None) -> dict:
         "v_cache": per_seq("v_cache", (Hkv, C, d)),
         "gate_key_cache": per_seq("gate_key_cache", (Hkv, NBm, h), torch.bfloat16),
         "cur_pool": cur_pool,
-        "wq": draw(s, "wq", (Hkv, h, G * d), dtype=dt, device=device, scale=1.0 / math.sqrt(G * d)),
+        "wq": draw(s, "wq", (shape.sel_heads, h, shape.sel_group * d), dtype=dt, device=device,
+                   scale=1.0 / math.sqrt(shape.sel_group * d)),
         "wk": draw(s, "wk", (Hkv, h, 3 * d), dtype=dt, device=device, scale=1.0 / math.sqrt(3 * d)),
         "qnorm_w": norm_weight(s, "qnorm_w", h, device),
         "knorm_w": norm_weight(s, "knorm_w", h, device),

@@ -52,8 +52,10 @@ class SecondGate:
         self.lengths = list(lengths)
         self.starts = [int(x) for x in np.concatenate([[0], np.cumsum(lengths)[:-1]])]
         self.B, self.eps, self.base = block, eps, base
-        self.Hkv, self.h = self.wq.shape[0], self.wq.shape[1]
-        self.G = self.q.shape[1] // self.Hkv
+        self.Hs, self.h = self.wq.shape[0], self.wq.shape[1]      # gate heads
+        self.Hkv = self.wk.shape[0]
+        self.Gs = self.q.shape[1] // self.Hs                     # query heads per gate head
+        self.G = self.q.shape[1] // self.Hkv                     # query heads per KV head
         self.mut = mutation
         self._block_keys = {}
 
@@ -87,13 +89,17 @@ class SecondGate:
     def key(self, pooled, kv, pos):
         return self.normalise_and_rotate(self.wk[kv] @ pooled, self.kw, pos)
 
-    def query(self, tg, kv, pos):
-        parts = [self.q[tg, kv * self.G + g] for g in range(self.G)]
+    def query(self, tg, sh, pos):
+        parts = [self.q[tg, sh * self.Gs + g] for g in range(self.Gs)]
         if self.mut == "concat_interleaved":
             qcat = torch.stack(parts, dim=1).reshape(-1)
         else:
             qcat = torch.cat(parts)
-        return self.normalise_and_rotate(self.wq[kv] @ qcat, self.qw, pos)
+        return self.normalise_and_rotate(self.wq[sh] @ qcat, self.qw, pos)
+
+    def kv_of(self, sh):
+        """the KV head whose keys gate head sh's query heads read"""
+        return (sh * self.Gs) // self.G
 
     def block_key(self, b, j, kv):
         if (b, j, kv) not in self._block_keys:
@@ -103,13 +109,14 @@ class SecondGate:
         return self._block_keys[(b, j, kv)]
 
     # -- one row ---------------------------------------------------------------------------
-    def row(self, b, t, kv, K):
+    def row(self, b, t, sh, K):
         """Scores over blocks 0..c, logsumexp, kept ids and their log-gates for token t
-        (in-sequence) of sequence b and kv head kv."""
+        (in-sequence) of sequence b and gate head sh."""
         s0 = self.starts[b]
         c = t // self.B
         qpos = s0 + t if self.mut == "packed_positions" else t
-        qt = self.query(s0 + t, kv, qpos)
+        qt = self.query(s0 + t, sh, qpos)
+        kv = self.kv_of(sh)
         keys = [self.block_key(b, j, kv) for j in range(c)]
         if self.mut == "full_block_current":
             keys.append(self.block_key(b, c, kv))
@@ -124,8 +131,8 @@ class SecondGate:
         return s, lse, ids, [float(s[j] - lse) for j in ids]
 
 
-def _problem(lengths, Hq, Hkv, d, B, K, h, dtype, seed):
-    shape = si.Shape(list(lengths), Hq, Hkv, d, B, K, h, dtype, seed=seed)
+def _problem(lengths, Hq, Hkv, d, B, K, h, dtype, seed, gate_heads=None):
+    shape = si.Shape(list(lengths), Hq, Hkv, d, B, K, h, dtype, seed=seed, gate_heads=gate_heads)
     return shape, si.prefill_inputs(shape)
 
 
@@ -133,13 +140,17 @@ CASES = {
     # several sequences (in-sequence positions), non-unit norm weights, G 2 and 5
     "fp32-G2-3seq": (([70, 33, 129], 4, 2, 8, 16, 3, 16, "fp32"), 11),
     "bf16-G5-2seq": (([90, 51], 10, 2, 16, 16, 2, 32, "bf16"), 12),
+    # one gate per query head (gate_heads = Hq)
+    "fp32-G2-per-head": (([70, 33], 4, 2, 8, 16, 3, 16, "fp32", 4), 14),
 }
 
 
 @pytest.mark.parametrize("name", list(CASES))
 def test_oracle_gate_matches_second_implementation(name):
-    (lengths, Hq, Hkv, d, B, K, h, dt), seed = CASES[name]
-    shape, inp = _problem(lengths, Hq, Hkv, d, B, K, h, dt, seed)
+    args, seed = CASES[name]
+    lengths, Hq, Hkv, d, B, K, h, dt = args[:8]
+    shape, inp = _problem(lengths, Hq, Hkv, d, B, K, h, dt, seed, *args[8:])
+    Hs = shape.sel_heads
     assert not torch.all(inp["qnorm_w"] == 1) and not torch.all(inp["knorm_w"] == 1)
     ref = orc.prefill_selection(inp["q_nope"], inp["k_nope"], inp["wq"], inp["qnorm_w"], inp["wk"],
                                 inp["knorm_w"], shape.cu_seqlens, B, K, 1e-6, 1e6)
@@ -153,24 +164,26 @@ def test_oracle_gate_matches_second_implementation(name):
                                            rtol=1e-11, atol=1e-12)
         for t in range(L):                           # A3/A4: every row
             c = t // B
-            for kv in range(Hkv):
-                s, lse, ids, lg = two.row(b, t, kv, K)
-                np.testing.assert_allclose(ref["scores"][s0 + t, kv, :c + 1], s.numpy(),
+            for sh in range(Hs):
+                s, lse, ids, lg = two.row(b, t, sh, K)
+                np.testing.assert_allclose(ref["scores"][s0 + t, sh, :c + 1], s.numpy(),
                                            rtol=1e-11, atol=1e-12)
-                assert np.isneginf(ref["scores"][s0 + t, kv, c + 1:]).all()
-                assert abs(ref["lse"][s0 + t, kv] - float(lse)) <= 1e-11
-                kept = ref["idx"][s0 + t, kv]
+                assert np.isneginf(ref["scores"][s0 + t, sh, c + 1:]).all()
+                assert abs(ref["lse"][s0 + t, sh] - float(lse)) <= 1e-11
+                kept = ref["idx"][s0 + t, sh]
                 assert list(kept[kept >= 0]) == ids
-                np.testing.assert_allclose(ref["logg"][s0 + t, kv, :len(ids)], lg, rtol=0, atol=1e-11)
+                np.testing.assert_allclose(ref["logg"][s0 + t, sh, :len(ids)], lg, rtol=0, atol=1e-11)
                 n += 1
-    assert n == shape.total_tokens * Hkv
+    assert n == shape.total_tokens * Hs
 
 
-def test_oracle_decode_gate_matches_second_implementation():
+@pytest.mark.parametrize("gate_heads", [None, 8])
+def test_oracle_decode_gate_matches_second_implementation(gate_heads):
     """The decode gate (cached block keys + a running pool state for the current block) gives
-    the second implementation's selection and log-gates for the newest token."""
+    the second implementation's selection and log-gates for the newest token (gate_heads = 8
+    = Hq: one gate per query head)."""
     lengths, Hq, Hkv, d, B, K, h = [77, 130, 16, 200], 8, 2, 16, 16, 4, 32
-    shape, inp = _problem(lengths, Hq, Hkv, d, B, K, h, "fp32", 13)
+    shape, inp = _problem(lengths, Hq, Hkv, d, B, K, h, "fp32", 13, gate_heads)
     two = SecondGate(inp, lengths, B)
     nbm = shape.max_blocks
     cap = max(lengths)
@@ -192,11 +205,11 @@ def test_oracle_decode_gate_matches_second_implementation():
     _, idx, logg, _ = orc.decode(qn, qn, kc, kc, lengths, gkc, pool, inp["wq"], inp["qnorm_w"],
                                  inp["wk"], inp["knorm_w"], B, K, 1e-6, 1e6)
     for b, L in enumerate(lengths):
-        for kv in range(Hkv):
-            _, _, ids, lg = two.row(b, L - 1, kv, K)
-            kept = idx[b, kv]
+        for sh in range(shape.sel_heads):
+            _, _, ids, lg = two.row(b, L - 1, sh, K)
+            kept = idx[b, sh]
             assert list(kept[kept >= 0]) == ids
-            np.testing.assert_allclose(logg[b, kv, :len(ids)], lg, rtol=0, atol=1e-11)
+            np.testing.assert_allclose(logg[b, sh, :len(ids)], lg, rtol=0, atol=1e-11)
 
 
 @pytest.mark.parametrize("mutation", ["weight_after_rotary", "packed_positions",

@@ -13,8 +13,8 @@ import sas_inputs as si
 from oracle import sas_oracle as orc
 
 
-def _problem(lengths, Hq=4, Hkv=2, d=16, B=8, K=3, seed=5):
-    shape = si.Shape(list(lengths), Hq, Hkv, d, B, K, 8, "fp32", seed=seed)
+def _problem(lengths, Hq=4, Hkv=2, d=16, B=8, K=3, seed=5, gate_heads=None):
+    shape = si.Shape(list(lengths), Hq, Hkv, d, B, K, 8, "fp32", seed=seed, gate_heads=gate_heads)
     inp = si.prefill_inputs(shape, with_dout=True)
     idx, logg = si.random_selection(shape)
     return shape, inp, idx, logg
@@ -35,8 +35,10 @@ def _mask_from_selection(idx_seq, logg_seq, B):
 
 
 def _sdpa_reference(shape, inp, idx, logg):
-    """Per sequence: SDPA (fp64) with the float mask; returns O, and grads incl. d(logg)."""
-    G, B = shape.group, shape.block
+    """Per sequence: SDPA (fp64) with the float mask; returns O, and grads incl. d(logg).
+    The mask is built per gate head (KV head, or query head with one gate per query head)
+    and repeated over that gate head's query heads."""
+    G, B, Gs = shape.group, shape.block, shape.sel_group
     outs, grads = [], []
     for (s0, s1) in orc.seq_ranges(shape.cu_seqlens):
         q = inp["q"][s0:s1].double().transpose(0, 1).requires_grad_(True)          # [Hq, L, d]
@@ -45,16 +47,16 @@ def _sdpa_reference(shape, inp, idx, logg):
         m = torch.from_numpy(_mask_from_selection(idx[s0:s1], logg[s0:s1], B)).requires_grad_(True)
         kk = k.repeat_interleave(G, 0)
         vv = v.repeat_interleave(G, 0)
-        mm = m.repeat_interleave(G, 0)
+        mm = m.repeat_interleave(Gs, 0)
         o = F.scaled_dot_product_attention(q[None], kk[None], vv[None], attn_mask=mm[None])[0]
         o.backward(inp["dout"][s0:s1].double().transpose(0, 1))
-        # d(logg[t, kv, slot]) = sum of d(mask) over the keys of that block (mask grad is
-        # already summed over the G heads by repeat_interleave's backward)
+        # d(logg[t, s, slot]) = sum of d(mask) over the keys of that block (mask grad is
+        # already summed over the gate head's query heads by repeat_interleave's backward)
         gm = m.grad.numpy()
         L = s1 - s0
         dl = np.zeros((L,) + idx.shape[1:])
         for t in range(L):
-            for kv in range(shape.num_kv_heads):
+            for kv in range(shape.sel_heads):
                 for sl, j in enumerate(idx[s0 + t, kv]):
                     if j >= 0:
                         dl[t, kv, sl] = gm[kv, t, j * B:(j + 1) * B][: max(0, t + 1 - j * B)].sum()
@@ -65,9 +67,12 @@ def _sdpa_reference(shape, inp, idx, logg):
     return np.concatenate(outs), cat(0), cat(1), cat(2), cat(3)
 
 
-@pytest.mark.parametrize("lengths,K", [([50], 2), ([37, 64, 9], 3), ([130], 20)])
-def test_matches_sdpa_with_block_mask(lengths, K):
-    shape, inp, idx, logg = _problem(lengths, K=K)
+@pytest.mark.parametrize("lengths,K,gate_heads", [([50], 2, None), ([37, 64, 9], 3, None),
+                                                  ([130], 20, None), ([37, 64, 9], 3, 4),
+                                                  ([90], 5, 4)])
+def test_matches_sdpa_with_block_mask(lengths, K, gate_heads):
+    """gate_heads = 4 = Hq: one gate, and so one selection, per query head."""
+    shape, inp, idx, logg = _problem(lengths, K=K, gate_heads=gate_heads)
     O, LSE, _ = orc.attention_fwd(inp["q"], inp["k"], inp["v"], idx, logg, shape.cu_seqlens, shape.block)
     dq, dk, dv, dl = orc.attention_bwd(inp["q"], inp["k"], inp["v"], inp["dout"], idx, logg,
                                        shape.cu_seqlens, shape.block)
@@ -109,9 +114,12 @@ def test_log_gate_shift_invariance_and_gradient_sum():
     np.testing.assert_allclose(O0, O1, rtol=1e-12, atol=1e-13)
 
 
-def test_finite_differences():
-    """Central differences of L = sum(O * W) against the analytic gradients (selection fixed)."""
-    shape, inp, idx, logg = _problem([21], Hq=2, Hkv=1, d=4, B=4, K=2, seed=11)
+@pytest.mark.parametrize("gate_heads", [None, 2])
+def test_finite_differences(gate_heads):
+    """Central differences of L = sum(O * W) against the analytic gradients (selection fixed);
+    gate_heads = 2 = Hq: one selection per query head."""
+    shape, inp, idx, logg = _problem([21], Hq=2, Hkv=1, d=4, B=4, K=2, seed=11,
+                                     gate_heads=gate_heads)
     q, k, v = (orc.as64(inp[n]) for n in ("q", "k", "v"))
     w = orc.as64(inp["dout"])
     lg = logg.astype(np.float64)
@@ -137,8 +145,9 @@ def test_finite_differences():
             assert abs(fd - grad.flat[e]) < 1e-6 * max(1.0, abs(fd)), (name, e, fd, grad.flat[e])
 
 
-def test_row_and_key_subsets_match_full():
-    shape, inp, idx, logg = _problem([45, 33], K=2)
+@pytest.mark.parametrize("gate_heads", [None, 4])
+def test_row_and_key_subsets_match_full(gate_heads):
+    shape, inp, idx, logg = _problem([45, 33], K=2, gate_heads=gate_heads)
     args = (inp["q"], inp["k"], inp["v"])
     O, LSE, _ = orc.attention_fwd(*args, idx, logg, shape.cu_seqlens, 8)
     rows = np.array([0, 7, 44, 45, 60, 77])

@@ -7,11 +7,14 @@ import sas_inputs as si
 from oracle import sas_oracle as orc
 
 
-@pytest.mark.parametrize("L,K", [(1, 3), (16, 3), (17, 3), (63, 3), (100, 3), (128, 3),
-                                 (300, 15), (290, 7)])
-def test_decode_equals_prefill_last_row(L, K):
+@pytest.mark.parametrize("L,K,gate_heads", [(1, 3, None), (16, 3, None), (17, 3, None),
+                                            (63, 3, None), (100, 3, None), (128, 3, None),
+                                            (300, 15, None), (290, 7, None), (100, 3, 4),
+                                            (290, 7, 4)])
+def test_decode_equals_prefill_last_row(L, K, gate_heads):
+    """gate_heads = 4 = Hq: one gate per query head."""
     B, h = 16, 16
-    shape = si.Shape([L], 4, 2, 8, B, K, h, "fp32", seed=20 + L)
+    shape = si.Shape([L], 4, 2, 8, B, K, h, "fp32", seed=20 + L, gate_heads=gate_heads)
     inp = si.prefill_inputs(shape)
     sel = orc.prefill_selection(inp["q_nope"], inp["k_nope"], inp["wq"], inp["qnorm_w"], inp["wk"],
                                 inp["knorm_w"], shape.cu_seqlens, B, K, 1e-6, 1e6)
