@@ -32,7 +32,7 @@ class SasProblem(ctypes.Structure):
                 ("num_q_heads", _i32), ("num_kv_heads", _i32), ("head_dim", _i32),
                 ("block", _i32), ("topk", _i32), ("gate_hidden", _i32), ("rms_eps", _f32),
                 ("dtype", ctypes.c_int), ("cu_seqlens", _vp), ("gate_rope_cos", _vp),
-                ("gate_rope_sin", _vp)]
+                ("gate_rope_sin", _vp), ("gate_heads", _i32)]
 
 
 class SasDecodeProblem(ctypes.Structure):
@@ -40,7 +40,7 @@ class SasDecodeProblem(ctypes.Structure):
                 ("num_kv_heads", _i32), ("head_dim", _i32), ("block", _i32), ("topk", _i32),
                 ("gate_hidden", _i32), ("rms_eps", _f32), ("dtype", ctypes.c_int),
                 ("seqlens", _vp), ("gate_rope_cos", _vp), ("gate_rope_sin", _vp),
-                ("ungated", _i32)]
+                ("ungated", _i32), ("gate_heads", _i32)]
 
 
 _P = ctypes.POINTER(SasProblem)
@@ -193,6 +193,7 @@ class Problem:
     gate_rope_base: float = 1e6
     rope_cos: torch.Tensor | None = None
     rope_sin: torch.Tensor | None = None
+    gate_heads: int = 0             # 0 / num_kv_heads: one gate per KV group; num_q_heads: per query head
 
     def __post_init__(self):
         if self.rope_cos is None:
@@ -203,7 +204,13 @@ class Problem:
         self._c = SasProblem(len(self.cu_seqlens) - 1, self.total_tokens, self.max_seqlen,
                              self.num_q_heads, self.num_kv_heads, self.head_dim, self.block,
                              self.topk, self.gate_hidden, self.rms_eps, _dtype_code(self.dtype),
-                             _ptr(self.cu_seqlens), _ptr(self.rope_cos), _ptr(self.rope_sin))
+                             _ptr(self.cu_seqlens), _ptr(self.rope_cos), _ptr(self.rope_sin),
+                             int(self.gate_heads or 0))
+
+    @property
+    def sel_heads(self) -> int:
+        """gate (selection) heads Hs: the second axis of idx / logg / dlogg / scores"""
+        return self.gate_heads or self.num_kv_heads
 
     @property
     def batch(self) -> int:
@@ -253,10 +260,10 @@ def gate_scores_workspace(p: Problem):
 def sas_gate_scores(p: Problem, q_nope, k_nope, gate_keys, wq, qnorm_w, wk, knorm_w,
                     scores=None, lse=None, workspace=None, stream=None):
     if scores is None:
-        scores = torch.empty((p.total_tokens, p.num_kv_heads, p.max_blocks), dtype=torch.float32,
+        scores = torch.empty((p.total_tokens, p.sel_heads, p.max_blocks), dtype=torch.float32,
                              device=p.device)
     if lse is None:
-        lse = torch.empty((p.total_tokens, p.num_kv_heads), dtype=torch.float32, device=p.device)
+        lse = torch.empty((p.total_tokens, p.sel_heads), dtype=torch.float32, device=p.device)
     ws = workspace if workspace is not None else gate_scores_workspace(p)
     _check(_lib.sas_gate_scores(p.ref, _ptr(q_nope), _ptr(k_nope), _ptr(gate_keys), _ptr(wq),
                                 _ptr(qnorm_w), _ptr(wk), _ptr(knorm_w), _ptr(scores), _ptr(lse),
@@ -286,7 +293,7 @@ def sas_gate_bwd(p: Problem, q_nope, k_nope, pooled, wq, qnorm_w, wk, knorm_w, i
 
 
 def sas_topk(p: Problem, scores, lse, idx=None, logg=None, stream=None):
-    shape = (p.total_tokens, p.num_kv_heads, p.topk + 1)
+    shape = (p.total_tokens, p.sel_heads, p.topk + 1)
     if idx is None:
         idx = torch.empty(shape, dtype=torch.int32, device=p.device)
     if logg is None:
@@ -336,7 +343,7 @@ def sas_attn_bwd(p: Problem, q, k, v, o, dout, lse, idx, logg, dq=None, dk=None,
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
     if dlogg is None:
-        dlogg = torch.empty((p.total_tokens, p.num_kv_heads, p.topk + 1), dtype=torch.float32,
+        dlogg = torch.empty((p.total_tokens, p.sel_heads, p.topk + 1), dtype=torch.float32,
                             device=p.device)
     ws = workspace if workspace is not None else _workspace(_lib.sas_attn_bwd_workspace_size, p.ref, p.device)
     _check(_lib.sas_attn_bwd(p.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
@@ -356,13 +363,13 @@ def sas_gate_select(p: Problem, q_nope, k_nope, gate_keys, wq, qnorm_w, wk, knor
                     logg=None, lse=None, workspace=None, stream=None, want_lse: bool = False):
     """Gate scores + Top-K in one pass (scores never written for the fused shapes).
     Returns (idx, logg), or (idx, logg, lse) with want_lse."""
-    shape = (p.total_tokens, p.num_kv_heads, p.topk + 1)
+    shape = (p.total_tokens, p.sel_heads, p.topk + 1)
     if idx is None:
         idx = torch.empty(shape, dtype=torch.int32, device=p.device)
     if logg is None:
         logg = torch.empty(shape, dtype=torch.float32, device=p.device)
     if want_lse and lse is None:
-        lse = torch.empty((p.total_tokens, p.num_kv_heads), dtype=torch.float32, device=p.device)
+        lse = torch.empty((p.total_tokens, p.sel_heads), dtype=torch.float32, device=p.device)
     ws = workspace if workspace is not None else gate_select_workspace(p)
     _check(_lib.sas_gate_select(p.ref, _ptr(q_nope), _ptr(k_nope), _ptr(gate_keys), _ptr(wq),
                                 _ptr(qnorm_w), _ptr(wk), _ptr(knorm_w), _ptr(idx), _ptr(logg),
@@ -398,6 +405,7 @@ class DecodeProblem:
     rope_cos: torch.Tensor | None = None
     rope_sin: torch.Tensor | None = None
     gated: bool = True              # False: hard selection, no log-gate in the attention logits
+    gate_heads: int = 0             # 0 / num_kv_heads: one gate per KV group; num_q_heads: per query head
 
     def __post_init__(self):
         if self.rope_cos is None:
@@ -409,7 +417,11 @@ class DecodeProblem:
                                    self.num_kv_heads, self.head_dim, self.block, self.topk,
                                    self.gate_hidden, self.rms_eps, _dtype_code(self.dtype),
                                    _ptr(self.seqlens), _ptr(self.rope_cos), _ptr(self.rope_sin),
-                                   0 if self.gated else 1)
+                                   0 if self.gated else 1, int(self.gate_heads or 0))
+
+    @property
+    def sel_heads(self) -> int:
+        return self.gate_heads or self.num_kv_heads
 
     @property
     def batch(self) -> int:
@@ -432,9 +444,9 @@ def sas_decode(p: DecodeProblem, q, q_nope, k_cache, v_cache, gate_key_cache, cu
     if o is None:
         o = torch.empty((p.batch, p.num_q_heads, p.head_dim), dtype=p.dtype, device=p.device)
     if want_selection and idx_out is None:
-        idx_out = torch.empty((p.batch, p.num_kv_heads, p.topk + 1), dtype=torch.int32,
+        idx_out = torch.empty((p.batch, p.sel_heads, p.topk + 1), dtype=torch.int32,
                               device=p.device)
-        logg_out = torch.empty((p.batch, p.num_kv_heads, p.topk + 1), dtype=torch.float32,
+        logg_out = torch.empty((p.batch, p.sel_heads, p.topk + 1), dtype=torch.float32,
                                device=p.device)
     ws = workspace if workspace is not None else _workspace(_lib.sas_decode_workspace_size, p.ref, p.device)
     _check(_lib.sas_decode(p.ref, _ptr(q), _ptr(q_nope), _ptr(k_cache), _ptr(v_cache),
@@ -455,9 +467,9 @@ def sas_decode_paged(p: DecodeProblem, page_table, num_pages: int, q, q_nope, k_
     if o is None:
         o = torch.empty((p.batch, p.num_q_heads, p.head_dim), dtype=p.dtype, device=p.device)
     if want_selection and idx_out is None:
-        idx_out = torch.empty((p.batch, p.num_kv_heads, p.topk + 1), dtype=torch.int32,
+        idx_out = torch.empty((p.batch, p.sel_heads, p.topk + 1), dtype=torch.int32,
                               device=p.device)
-        logg_out = torch.empty((p.batch, p.num_kv_heads, p.topk + 1), dtype=torch.float32,
+        logg_out = torch.empty((p.batch, p.sel_heads, p.topk + 1), dtype=torch.float32,
                                device=p.device)
     ws = workspace if workspace is not None else _workspace(_lib.sas_decode_workspace_size, p.ref, p.device)
     _check(_lib.sas_decode_paged(p.ref, _ptr(page_table), int(num_pages), _ptr(q), _ptr(q_nope),

@@ -70,6 +70,10 @@ static sas_status check_problem(const sas_problem* p, bool needs_rope) {
   SAS_CHECK_ARG(p->topk >= 1 && p->topk + 1 <= 128, "topk must be in 1..127 (got %d)", p->topk);
   SAS_CHECK_ARG(p->dtype == SAS_BF16 || p->dtype == SAS_FP32, "unknown dtype %d", (int)p->dtype);
   SAS_CHECK_ARG(p->rms_eps >= 0.f && isfinite(p->rms_eps), "rms_eps must be finite and >= 0");
+  SAS_CHECK_ARG(p->gate_heads == 0 || p->gate_heads == p->num_kv_heads ||
+                    p->gate_heads == p->num_q_heads,
+                "gate_heads must be 0, num_kv_heads (%d) or num_q_heads (%d) (got %d)",
+                p->num_kv_heads, p->num_q_heads, p->gate_heads);
   if (max_blocks(*p) > 2048) {
     set_error("max_seqlen / block must be <= 2048 blocks (got %d)", max_blocks(*p));
     return SAS_ERR_UNSUPPORTED;
@@ -215,7 +219,7 @@ sas_status sas_gate_bwd_workspace_size(const sas_problem* p, size_t* bytes) {
   SAS_TRY(check_problem(p, true));
   SAS_CHECK_ARG(bytes != nullptr, "bytes is NULL");
   if (!gate_bwd_supported(*p)) {
-    set_error("gate_bwd: supported for bf16, head_dim 128, gate_hidden 128, block <= 128");
+    set_error("gate_bwd: supported for bf16, head_dim 128, gate_hidden 128, block <= 128, one gate per KV group");
     return SAS_ERR_UNSUPPORTED;
   }
   *bytes = gate_bwd_workspace_bytes(*p);
@@ -242,7 +246,7 @@ sas_status sas_gate_bwd(const sas_problem* p, const void* q_nope, const void* k_
   SAS_PTR(dwk);
   SAS_PTR(dknorm_w);
   if (!gate_bwd_supported(*p)) {
-    set_error("gate_bwd: supported for bf16, head_dim 128, gate_hidden 128, block <= 128");
+    set_error("gate_bwd: supported for bf16, head_dim 128, gate_hidden 128, block <= 128, one gate per KV group");
     return SAS_ERR_UNSUPPORTED;
   }
   if (p->total_tokens == 0) {   // no rows: every gradient is zero
@@ -395,6 +399,10 @@ static sas_status check_decode(const sas_decode_problem* p) {
   SAS_CHECK_ARG(p->gate_rope_cos != nullptr && p->gate_rope_sin != nullptr,
                 "gate rotary tables are NULL");
   SAS_CHECK_ARG(p->ungated == 0 || p->ungated == 1, "ungated must be 0 or 1 (got %d)", p->ungated);
+  SAS_CHECK_ARG(p->gate_heads == 0 || p->gate_heads == p->num_kv_heads ||
+                    p->gate_heads == p->num_q_heads,
+                "gate_heads must be 0, num_kv_heads (%d) or num_q_heads (%d) (got %d)",
+                p->num_kv_heads, p->num_q_heads, p->gate_heads);
   return SAS_OK;
 }
 

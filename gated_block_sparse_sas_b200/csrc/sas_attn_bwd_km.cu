@@ -95,6 +95,7 @@ struct KmBwdArgs {
   float* dlogg;      // [T][Hkv][K+1]
   int* err;
   int batch, Hq, Hkv, G, Mq, P, K1;
+  int Hs, R;         // gate heads, gate heads per KV head (1, or G with one gate per query head)
   float scale_log2, scale;
 };
 
@@ -196,7 +197,7 @@ __global__ void __launch_bounds__(kmb::kThreads, 1)
           ok = false;
         } else {
           desc[ds * 2] = key0;
-          desc[ds * 2 + 1] = kv;
+          desc[ds * 2 + 1] = kv / a.R;   // the KV head the item's gate head reads
           mbar_arrive(item_full + ds);
         }
       }
@@ -246,12 +247,12 @@ __global__ void __launch_bounds__(kmb::kThreads, 1)
         rcf[rc_slot(rs, 1) + r] = d_v;
         rci[rc_slot(rs, 2) + r] = valid ? min(kB - 1, tg - key0) : -1;
         rci[rc_slot(rs, 3) + r] = valid ? (int)qrow : -1;
-        rci[rc_slot(rs, 4) + r] = valid ? (tg * a.Hkv + kv) * a.K1 + slot : -1;
+        rci[rc_slot(rs, 4) + r] = valid ? (tg * a.Hs + kv) * a.K1 + slot : -1;
         if (r == 0) {
           hdr[rs * 4] = (m == 0 ? kFlagFirst : 0) | (m == ntile - 1 ? kFlagLast : 0);
           hdr[rs * 4 + 1] = key0;
           hdr[rs * 4 + 2] = min(kB, L - j * kB);
-          hdr[rs * 4 + 3] = kv;
+          hdr[rs * 4 + 3] = kv / a.R;
         }
         cp_async_wait_all();
         fence_async_smem();
@@ -610,7 +611,8 @@ sas_status launch_attn_bwd_km(const sas_problem& p, const void* q, const void* k
   float* dk_acc = reinterpret_cast<float*>(ws + L.dk);
   float* dv_acc = reinterpret_cast<float*>(ws + L.dv);
   const KmLists lists = km_lists_carve(p, ws + L.lists);
-  const int G = p.num_q_heads / p.num_kv_heads;
+  const int Hs = gate_heads(p);
+  const int G = p.num_q_heads / Hs;   // query heads per gate head (the rows of a token)
   const int Hkv = p.num_kv_heads;
   const int T = p.total_tokens;
 
@@ -623,7 +625,7 @@ sas_status launch_attn_bwd_km(const sas_problem& p, const void* q, const void* k
     return SAS_ERR_CUDA;
   }
   if (cudaMemsetAsync(dq_acc, 0, L.lists - L.dq, st) != cudaSuccess ||
-      cudaMemsetAsync(dlogg, 0, (size_t)T * Hkv * (p.topk + 1) * 4, st) != cudaSuccess) {
+      cudaMemsetAsync(dlogg, 0, (size_t)T * Hs * (p.topk + 1) * 4, st) != cudaSuccess) {
     set_error("attn_bwd: clearing the accumulators failed");
     return SAS_ERR_CUDA;
   }
@@ -651,6 +653,8 @@ sas_status launch_attn_bwd_km(const sas_problem& p, const void* q, const void* k
   a.Hq = p.num_q_heads;
   a.Hkv = Hkv;
   a.G = G;
+  a.Hs = Hs;
+  a.R = Hs / Hkv;
   a.Mq = tc_rows_per_tile(G);
   a.P = lists.P;
   a.K1 = p.topk + 1;

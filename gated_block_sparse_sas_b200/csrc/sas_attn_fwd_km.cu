@@ -90,21 +90,24 @@ struct KmFwdArgs {
   float* lacc;             // [T][Hq]
   int* err;
   int batch, Hq, Hkv, G, Mq, P;
+  int R;                   // gate heads per KV head (1, or G with one gate per query head)
   float scale_log2;
 };
 
 // ---------------------------------------------------------------------------------------
 // preparation
 // ---------------------------------------------------------------------------------------
-// m_row = (q_t,h . k_t,kv / sqrt(d) + log g_current) log2e + 32; one warp per (token, kv head)
+// m_row = (q_t,h . k_t,kv / sqrt(d) + log g_current) log2e + 32; one warp per (token, gate
+// head): the gate head's G query heads (G = Hq / Hs here), keys of KV head kv / R
 __global__ void km_rowref_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                                  const int32_t* __restrict__ idx, const float* __restrict__ logg,
                                  const int32_t* __restrict__ cu, int batch, int T, int Hq, int Hkv,
-                                 int G, int K, float scale_log2, float* __restrict__ mref) {
+                                 int R, int G, int K, float scale_log2, float* __restrict__ mref) {
   const int lane = threadIdx.x & 31;
   const int gw = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5);
   if (gw >= T * Hkv) return;
-  const int tg = gw / Hkv, kv = gw - tg * Hkv;
+  const int tg = gw / Hkv, kv = gw - tg * Hkv;   // Hkv counts gate heads here
+  const int Hk = Hkv / R, kh = kv / R;
   const int b = seq_of(cu, batch, tg);
   const int c = (tg - cu[b]) / kmf::kB;
   const size_t irow = (size_t)gw * (K + 1);
@@ -120,7 +123,7 @@ __global__ void km_rowref_kernel(const __nv_bfloat16* __restrict__ q, const __nv
       break;
     }
   }
-  const uint2 kr = *reinterpret_cast<const uint2*>(k + ((size_t)tg * Hkv + kv) * kmf::kD + lane * 4);
+  const uint2 kr = *reinterpret_cast<const uint2*>(k + ((size_t)tg * Hk + kh) * kmf::kD + lane * 4);
   const float2 k01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&kr.x));
   const float2 k23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&kr.y));
   for (int g = 0; g < G; ++g) {
@@ -250,10 +253,11 @@ __global__ void __launch_bounds__(kmf::kThreads, 1)
           uint8_t* stg = sm + OFF_KV + kvs * kKVStage;
           const int row = s0 + j * kB;
           mbar_arrive_expect_tx(kv_full + kvs, kKVStage);
-          tma_load_3d(stg, &tmK, kv_full + kvs, 0, kv, row);
-          tma_load_3d(stg + kKVHalf, &tmK, kv_full + kvs, 64, kv, row);
-          tma_load_3d(stg + 2 * kKVHalf, &tmV, kv_full + kvs, 0, kv, row);
-          tma_load_3d(stg + 3 * kKVHalf, &tmV, kv_full + kvs, 64, kv, row);
+          const int kh = kv / a.R;   // the item's gate head reads KV head kh
+          tma_load_3d(stg, &tmK, kv_full + kvs, 0, kh, row);
+          tma_load_3d(stg + kKVHalf, &tmK, kv_full + kvs, 64, kh, row);
+          tma_load_3d(stg + 2 * kKVHalf, &tmV, kv_full + kvs, 0, kh, row);
+          tma_load_3d(stg + 3 * kKVHalf, &tmV, kv_full + kvs, 64, kh, row);
         }
       }
       ++item_seq;
@@ -507,8 +511,10 @@ sas_status launch_attn_fwd_km(const sas_problem& p, const void* q, const void* k
   float* oacc = reinterpret_cast<float*>(ws + L.oacc);
   float* lacc = reinterpret_cast<float*>(ws + L.lacc);
   const KmLists lists = km_lists_carve(p, ws + L.lists);
-  const int G = p.num_q_heads / p.num_kv_heads;
+  const int Hs = gate_heads(p);
+  const int G = p.num_q_heads / Hs;   // query heads per gate head (the rows of a token)
   const int Hkv = p.num_kv_heads;
+  const int R = Hs / Hkv;
   const int T = p.total_tokens;
   const float scale_log2 = kLog2e / sqrtf(128.f);
 
@@ -523,10 +529,10 @@ sas_status launch_attn_fwd_km(const sas_problem& p, const void* q, const void* k
     set_error("attn_fwd: clearing the accumulators failed");
     return SAS_ERR_CUDA;
   }
-  const int wpr = T * Hkv;
+  const int wpr = T * Hs;
   km_rowref_kernel<<<(wpr + 7) / 8, 256, 0, st>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
                                                   idx, logg, p.cu_seqlens, p.batch, T,
-                                                  p.num_q_heads, Hkv, G, p.topk, scale_log2, mref);
+                                                  p.num_q_heads, Hs, R, G, p.topk, scale_log2, mref);
   SAS_TRY(launch_km_lists(p, idx, logg, lists, st));
 
   KmFwdArgs a;
@@ -546,6 +552,7 @@ sas_status launch_attn_fwd_km(const sas_problem& p, const void* q, const void* k
   a.Hq = p.num_q_heads;
   a.Hkv = Hkv;
   a.G = G;
+  a.R = R;
   a.Mq = tc_rows_per_tile(G);
   a.P = lists.P;
   a.scale_log2 = scale_log2;

@@ -2,9 +2,12 @@
 //
 // These kernels serve the shapes the tensor-core path does not take (fp32 inputs,
 // head_dim 64) and give a second, independent GPU implementation. One warp owns one
-// (token, kv head) row: the G query heads of the KV group share the row's selection
+// (token, gate head) row: the G query heads of the gate head share the row's selection
 // (README (b): per-query Top-K blocks with a continuous gate; abstract: the gate enters
-// the attention softmax in log form), each lane holds d/32 channels of every head.
+// the attention softmax in log form), each lane holds d/32 channels of every head. A gate
+// head is a KV head (one gate per KV group: Hs = Hkv, R = 1) or a query head (one gate per
+// query head: Hs = Hq, G = 1 here, R = Hq / Hkv); its keys and values are those of KV head
+// s / R.
 #include <math.h>
 
 #include "sas_common.cuh"
@@ -31,16 +34,17 @@ template <typename T, int D, int G>
 __global__ void __launch_bounds__(128) attn_fwd_simt_kernel(
     const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
     const int32_t* __restrict__ idx, const float* __restrict__ logg, const int32_t* __restrict__ cu,
-    int batch, int T_total, int Hkv, int B, int K, float scale_log2, T* __restrict__ o,
+    int batch, int T_total, int Hkv, int R, int B, int K, float scale_log2, T* __restrict__ o,
     float* __restrict__ lse) {
   constexpr int E = D / 32;
   const int row = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= T_total * Hkv) return;
-  const int tg = row / Hkv, kv = row - tg * Hkv;
+  const int tg = row / Hkv, kv = row - tg * Hkv;   // kv: gate head; its K/V head is kv / R
   const int b = seq_of(cu, batch, tg);
   const int s0 = cu[b], t = tg - s0;
   const int Hq = Hkv * G;
+  const int Hk = Hkv / R, kh = kv / R;
   float qr[G][E], acc[G][E], m[G], l[G];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
@@ -59,7 +63,7 @@ __global__ void __launch_bounds__(128) attn_fwd_simt_kernel(
     const int i0 = j * B, i1 = min(i0 + B, t + 1);
     for (int i = i0; i < i1; ++i) {
       float kk[E], vv[E];
-      const size_t off = ((size_t)(s0 + i) * Hkv + kv) * D + lane * E;
+      const size_t off = ((size_t)(s0 + i) * Hk + kh) * D + lane * E;
       load_vec<T, E>(k + off, kk);
       load_vec<T, E>(v + off, vv);
 #pragma unroll
@@ -119,16 +123,17 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_simt_kernel(
     const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
     const T* __restrict__ dout, const float* __restrict__ lse, const float* __restrict__ drow,
     const int32_t* __restrict__ idx, const float* __restrict__ logg, const int32_t* __restrict__ cu,
-    int batch, int T_total, int Hkv, int B, int K, float scale, T* __restrict__ dq,
+    int batch, int T_total, int Hkv, int R, int B, int K, float scale, T* __restrict__ dq,
     float* __restrict__ dlogg) {
   constexpr int E = D / 32;
   const int row = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= T_total * Hkv) return;
-  const int tg = row / Hkv, kv = row - tg * Hkv;
+  const int tg = row / Hkv, kv = row - tg * Hkv;   // kv: gate head; its K/V head is kv / R
   const int b = seq_of(cu, batch, tg);
   const int s0 = cu[b], t = tg - s0;
   const int Hq = Hkv * G;
+  const int Hk = Hkv / R, kh = kv / R;
   const float scale_log2 = scale * kLog2e;
   float qr[G][E], dor[G][E], acc[G][E], l2[G], dd[G];
 #pragma unroll
@@ -155,7 +160,7 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_simt_kernel(
     float dsum = 0.f;
     for (int i = i0; i < i1; ++i) {
       float kk[E], vv[E];
-      const size_t off = ((size_t)(s0 + i) * Hkv + kv) * D + lane * E;
+      const size_t off = ((size_t)(s0 + i) * Hk + kh) * D + lane * E;
       load_vec<T, E>(k + off, kk);
       load_vec<T, E>(v + off, vv);
 #pragma unroll
@@ -200,19 +205,21 @@ __global__ void __launch_bounds__(kDkvThreads) attn_bwd_dkdv_simt_kernel(
     const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
     const T* __restrict__ dout, const float* __restrict__ lse, const float* __restrict__ drow,
     const int32_t* __restrict__ idx, const float* __restrict__ logg, const int32_t* __restrict__ cu,
-    int Hkv, int B, int K, float scale, T* __restrict__ dk, T* __restrict__ dv) {
+    int Hkv, int R, int B, int K, float scale, T* __restrict__ dk, T* __restrict__ dv) {
+  // Hkv here counts gate heads; the CTA's KV head kh is read by gate heads kh*R .. kh*R+R-1
   constexpr int E = D / 32;
   __shared__ int list_t[kDkvChunk];
   __shared__ int list_s[kDkvChunk];
   __shared__ int warp_cnt[kDkvWarps];
   __shared__ int n_list;
-  const int j = blockIdx.x, b = blockIdx.y, kv = blockIdx.z;
+  const int j = blockIdx.x, b = blockIdx.y, kh = blockIdx.z;
   const int s0 = cu[b], L = cu[b + 1] - s0;
   const int i0 = j * B;
   if (i0 >= L) return;
   const int nkeys = min(B, L - i0);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int Hq = Hkv * G;
+  const int Hk = Hkv / R;
   const float scale_log2 = scale * kLog2e;
 
   // this warp's keys: local key index kk = warp + r * kDkvWarps
@@ -223,12 +230,13 @@ __global__ void __launch_bounds__(kDkvThreads) attn_bwd_dkdv_simt_kernel(
 #pragma unroll
     for (int e = 0; e < E; ++e) { kr[r][e] = vr[r][e] = dkr[r][e] = dvr[r][e] = 0.f; }
     if (kl < nkeys) {
-      const size_t off = ((size_t)(s0 + i0 + kl) * Hkv + kv) * D + lane * E;
+      const size_t off = ((size_t)(s0 + i0 + kl) * Hk + kh) * D + lane * E;
       load_vec<T, E>(k + off, kr[r]);
       load_vec<T, E>(v + off, vr[r]);
     }
   }
 
+  for (int kv = kh * R; kv < kh * R + R; ++kv)   // the gate heads reading this KV head
   for (int c0 = i0; c0 < L; c0 += kDkvChunk) {
     // ---- ordered compaction of the rows in [c0, c0 + chunk) that selected block j ----
     const int t = c0 + threadIdx.x;
@@ -298,7 +306,7 @@ __global__ void __launch_bounds__(kDkvThreads) attn_bwd_dkdv_simt_kernel(
   for (int r = 0; r < KPW; ++r) {
     const int kl = warp + r * kDkvWarps;
     if (kl >= nkeys) continue;
-    const size_t off = ((size_t)(s0 + i0 + kl) * Hkv + kv) * D + lane * E;
+    const size_t off = ((size_t)(s0 + i0 + kl) * Hk + kh) * D + lane * E;
     float a[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) a[e] = dkr[r][e] * scale;
@@ -314,12 +322,13 @@ template <typename T, int D, int G>
 static void fwd_simt_launch(const sas_problem& p, const void* q, const void* k, const void* v,
                             const int32_t* idx, const float* logg, void* o, float* lse,
                             cudaStream_t st) {
-  const int rows = p.total_tokens * p.num_kv_heads;
+  const int Hs = gate_heads(p), R = Hs / p.num_kv_heads;
+  const int rows = p.total_tokens * Hs;
   const int grid = (int)(((size_t)rows * 32 + 127) / 128);
   const float scale_log2 = kLog2e / sqrtf((float)D);
   attn_fwd_simt_kernel<T, D, G><<<grid, 128, 0, st>>>(
       (const T*)q, (const T*)k, (const T*)v, idx, logg, p.cu_seqlens, p.batch, p.total_tokens,
-      p.num_kv_heads, p.block, p.topk, scale_log2, (T*)o, lse);
+      Hs, R, p.block, p.topk, scale_log2, (T*)o, lse);
 }
 
 template <typename T, int D, int G>
@@ -330,17 +339,18 @@ static void bwd_simt_launch(const sas_problem& p, const void* q, const void* k, 
   const int rows_q = p.total_tokens * p.num_q_heads;
   attn_bwd_rowdot_kernel<T, D><<<(int)(((size_t)rows_q * 32 + 255) / 256), 256, 0, st>>>(
       (const T*)o, (const T*)dout, rows_q, drow);
-  const int rows = p.total_tokens * p.num_kv_heads;
+  const int Hs = gate_heads(p), R = Hs / p.num_kv_heads;
+  const int rows = p.total_tokens * Hs;
   const float scale = 1.0f / sqrtf((float)D);
   attn_bwd_dq_simt_kernel<T, D, G><<<(int)(((size_t)rows * 32 + 127) / 128), 128, 0, st>>>(
       (const T*)q, (const T*)k, (const T*)v, (const T*)dout, lse, drow, idx, logg, p.cu_seqlens,
-      p.batch, p.total_tokens, p.num_kv_heads, p.block, p.topk, scale, (T*)dq, dlogg);
+      p.batch, p.total_tokens, Hs, R, p.block, p.topk, scale, (T*)dq, dlogg);
   const int NBmax = (p.max_seqlen + p.block - 1) / p.block;
   dim3 grid(NBmax, p.batch, p.num_kv_heads);
 #define SAS_DKV(KPW)                                                                          \
   attn_bwd_dkdv_simt_kernel<T, D, G, KPW><<<grid, kDkvThreads, 0, st>>>(                       \
       (const T*)q, (const T*)k, (const T*)v, (const T*)dout, lse, drow, idx, logg,              \
-      p.cu_seqlens, p.num_kv_heads, p.block, p.topk, scale, (T*)dk, (T*)dv)
+      p.cu_seqlens, Hs, R, p.block, p.topk, scale, (T*)dk, (T*)dv)
   if (p.block <= 16) SAS_DKV(2);
   else if (p.block <= 32) SAS_DKV(4);
   else if (p.block <= 64) SAS_DKV(8);
@@ -349,7 +359,7 @@ static void bwd_simt_launch(const sas_problem& p, const void* q, const void* k, 
 }
 
 #define SAS_FOR_G(MACRO, T, D)           \
-  switch (p.num_q_heads / p.num_kv_heads) { \
+  switch (p.num_q_heads / gate_heads(p)) { \
     case 1: MACRO(T, D, 1); break;       \
     case 2: MACRO(T, D, 2); break;       \
     case 4: MACRO(T, D, 4); break;       \

@@ -51,12 +51,12 @@ __global__ void __launch_bounds__(kDecThreads) decode_gate_kernel(
     const T* __restrict__ q_nope, const __nv_bfloat16* __restrict__ gkc,
     const float* __restrict__ cur_pool, const T* __restrict__ wq, const float* __restrict__ qnorm_w,
     const T* __restrict__ wk, const float* __restrict__ knorm_w, const int32_t* __restrict__ seqlens,
-    const float* __restrict__ rc, const float* __restrict__ rs, int Hq, int Hkv, int d, int B, int K,
+    const float* __restrict__ rc, const float* __restrict__ rs, int Hq, int Hkv, int Hs, int d, int B, int K,
     int NBmax, int capacity, float eps, int ungated, int32_t* __restrict__ sel_idx,
     float* __restrict__ sel_logg, int32_t* __restrict__ idx_out, float* __restrict__ logg_out,
     const int32_t* __restrict__ pt, int num_pages, int* __restrict__ err) {
   extern __shared__ float smem[];
-  const int G = Hq / Hkv, GD = G * d, C = 3 * d;
+  const int G = Hq / Hs, GD = G * d, C = 3 * d;   // G: query heads of the gate head
   float* qcat = smem;                  // [GD]
   float* P = qcat + GD;                // [C]
   float* xq = P + C;                   // [H]
@@ -68,11 +68,14 @@ __global__ void __launch_bounds__(kDecThreads) decode_gate_kernel(
   int* hist = misc + 4;                                     // [256] radix histogram
   int* pages = hist + 256;                                  // [NBmax] paged caches: page of block j
 
-  const int kv = blockIdx.x, b = blockIdx.y;
+  // gate head sh (a KV head, or a query head with one gate per query head); its block keys,
+  // pool state and Kproj are KV head kv's
+  const int sh = blockIdx.x, b = blockIdx.y;
+  const int kv = sh / (Hs / Hkv);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int L = seqlens[b];
   const int t = L - 1, c = t / B, n = L - c * B;
-  const size_t orow = ((size_t)b * Hkv + kv) * (K + 1);
+  const size_t orow = ((size_t)b * Hs + sh) * (K + 1);
   bool empty = L < 1 || L > capacity;   // invalid length: empty selection, the merge writes 0
   if (!empty && pt != nullptr) {   // paged caches: the pages of blocks 0..c, range-checked
     int bad = 0;
@@ -106,7 +109,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_gate_kernel(
     }
   }
   for (int e = tid; e < GD; e += kDecThreads)
-    qcat[e] = to_f(q_nope[((size_t)b * Hq + (size_t)kv * G) * d + e]);
+    qcat[e] = to_f(q_nope[((size_t)b * Hq + (size_t)sh * G) * d + e]);
   for (int e = tid; e < C; e += kDecThreads) {
     const int part = e / d, ch = e - part * d;
     const float x = cur_pool[(((size_t)b * Hkv + kv) * 3 + part) * d + ch];
@@ -119,7 +122,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_gate_kernel(
     for (int job = warp; job < 2 * H; job += kDecWarps) {
       const bool isq = job < H;
       const int i = isq ? job : job - H;
-      const T* w = isq ? wq + ((size_t)kv * H + i) * GD : wk + ((size_t)kv * H + i) * C;
+      const T* w = isq ? wq + ((size_t)sh * H + i) * GD : wk + ((size_t)kv * H + i) * C;
       const float* x = isq ? qcat : P;
       const int n_in = isq ? GD : C;
       float acc = 0.f;
@@ -137,7 +140,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_gate_kernel(
     for (int job0 = warp * R; job0 < 2 * H; job0 += kDecWarps * R) {
       const bool isq = job0 < H;   // H is a multiple of 8: a step never mixes q and k rows
       const int i0 = isq ? job0 : job0 - H;
-      const T* w = isq ? wq + ((size_t)kv * H + i0) * GD : wk + ((size_t)kv * H + i0) * C;
+      const T* w = isq ? wq + ((size_t)sh * H + i0) * GD : wk + ((size_t)kv * H + i0) * C;
       const int n_in = isq ? GD : C;
       const float* x = isq ? qcat : P;
       const int nv = n_in / 8;   // 16-byte vectors per row
@@ -392,8 +395,9 @@ template <typename T, int D, int G>
 __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(
     const T* __restrict__ q, const T* __restrict__ kc, const T* __restrict__ vc,
     const int32_t* __restrict__ seqlens, const int32_t* __restrict__ sel_idx,
-    const float* __restrict__ sel_logg, int Hkv, int capacity, int B, int K, int nsplit,
+    const float* __restrict__ sel_logg, int Hkv, int R, int capacity, int B, int K, int nsplit,
     float scale_log2, float* __restrict__ part_ml, float* __restrict__ part_acc) {
+  // Hkv counts gate heads here; gate head kv reads the keys/values of KV head kv / R
   constexpr int E = D / 32;
   __shared__ float sm_m[kDecWarps][G], sm_l[kDecWarps][G];
   __shared__ float sm_acc[kDecWarps][G][D];
@@ -416,8 +420,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(
     m[g] = -INFINITY;
     l[g] = 0.f;
   }
-  const T* kbase = kc + ((size_t)b * Hkv + kv) * (size_t)capacity * D + lane * E;
-  const T* vbase = vc + ((size_t)b * Hkv + kv) * (size_t)capacity * D + lane * E;
+  const T* kbase = kc + ((size_t)b * (Hkv / R) + kv / R) * (size_t)capacity * D + lane * E;
+  const T* vbase = vc + ((size_t)b * (Hkv / R) + kv / R) * (size_t)capacity * D + lane * E;
   for (int sl = sl0; sl < sl1; ++sl) {
     const int j = sel_idx[srow + sl];
     if (j < 0) continue;
@@ -496,9 +500,10 @@ template <int G>
 __global__ void __launch_bounds__(kDecThreads, 2) decode_attn_bulk_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kc,
     const __nv_bfloat16* __restrict__ vc, const int32_t* __restrict__ seqlens,
-    const int32_t* __restrict__ sel_idx, const float* __restrict__ sel_logg, int Hkv, int capacity,
-    int B, int K, int nsplit, float scale_log2, float* __restrict__ part_ml,
+    const int32_t* __restrict__ sel_idx, const float* __restrict__ sel_logg, int Hkv, int R,
+    int capacity, int B, int K, int nsplit, float scale_log2, float* __restrict__ part_ml,
     float* __restrict__ part_acc, int* __restrict__ err) {
+  // Hkv counts gate heads here; gate head kv reads the keys/values of KV head kv / R
   using namespace sm100;
   constexpr int D = 128;
   constexpr int NP = (G * 64 + kDecThreads - 1) / kDecThreads;   // (head, 2-channel) pairs per thread
@@ -556,8 +561,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_attn_bulk_kernel(
   }
   __syncthreads();
   const int nblk = *nblk_s;
-  const __nv_bfloat16* kbase = kc + ((size_t)b * Hkv + kv) * (size_t)capacity * D;
-  const __nv_bfloat16* vbase = vc + ((size_t)b * Hkv + kv) * (size_t)capacity * D;
+  const __nv_bfloat16* kbase = kc + ((size_t)b * (Hkv / R) + kv / R) * (size_t)capacity * D;
+  const __nv_bfloat16* vbase = vc + ((size_t)b * (Hkv / R) + kv / R) * (size_t)capacity * D;
   auto issue = [&](int n) {   // thread 0: copy block n's K and V rows into stage n % kAttStages
     const int st = n % kAttStages;
     const int i0 = blk_j[n] * B;
@@ -735,7 +740,7 @@ __global__ void decode_merge_kernel(const float* __restrict__ part_ml, const flo
 
 // ---------------------------------------------------------------------------------------
 int decode_nsplit(const sas_decode_problem& p) {
-  const int pairs = p.batch * p.num_kv_heads;
+  const int pairs = p.batch * gate_heads(p);
   int ns = (4 * 148 + pairs - 1) / pairs;   // about 4 CTAs per SM, each a long stream
   if (ns < 1) ns = 1;
   if (ns > p.topk + 1) ns = p.topk + 1;
@@ -743,8 +748,8 @@ int decode_nsplit(const sas_decode_problem& p) {
 }
 
 size_t decode_workspace_bytes(const sas_decode_problem& p) {
-  const int G = p.num_q_heads / p.num_kv_heads;
-  const size_t pairs = (size_t)p.batch * p.num_kv_heads;
+  const int G = p.num_q_heads / gate_heads(p);
+  const size_t pairs = (size_t)p.batch * gate_heads(p);
   const size_t ns = decode_nsplit(p);
   auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
   return 256 /* error word */ + al(pairs * (p.topk + 1) * 4) * 2 + al(pairs * ns * G * 2 * 4) +
@@ -762,12 +767,13 @@ static void decode_attn_launch(const sas_decode_problem& p, const void* q, const
                                const void* vc, int32_t* sel_idx, float* sel_logg, float* part_ml,
                                float* part_acc, int* err, void* o, int ns,
                                const DecodePaging& pg, cudaStream_t st) {
-  dim3 grid(p.num_kv_heads, p.batch, ns);
+  const int Hs = gate_heads(p), R = Hs / p.num_kv_heads;   // G: query heads per gate head
+  dim3 grid(Hs, p.batch, ns);
   if constexpr (std::is_same<T, __nv_bfloat16>::value && D == 128) {
     if (decode_attn_tc_supported(p)) {   // tensor-core path (sas_decode_tc.cu)
       launch_decode_attn_tc(p, q, kc, vc, sel_idx, sel_logg, part_ml, part_acc, err, ns, pg, st);
-      decode_merge_kernel<T, D, G><<<dim3(p.num_kv_heads, p.batch), 256, 0, st>>>(
-          part_ml, part_acc, p.num_kv_heads, ns, (T*)o);
+      decode_merge_kernel<T, D, G><<<dim3(Hs, p.batch), 256, 0, st>>>(part_ml, part_acc, Hs, ns,
+                                                                     (T*)o);
       return;
     }
     if (p.block <= 64) {   // bulk-copy streaming path
@@ -776,18 +782,18 @@ static void decode_attn_launch(const sas_decode_problem& p, const void* q, const
                            (int)smem);
       decode_attn_bulk_kernel<G><<<grid, kDecThreads, smem, st>>>(
           (const __nv_bfloat16*)q, (const __nv_bfloat16*)kc, (const __nv_bfloat16*)vc, p.seqlens,
-          sel_idx, sel_logg, p.num_kv_heads, p.capacity, p.block, p.topk, ns,
+          sel_idx, sel_logg, Hs, R, p.capacity, p.block, p.topk, ns,
           kLog2e / sqrtf((float)D), part_ml, part_acc, err);
-      decode_merge_kernel<T, D, G><<<dim3(p.num_kv_heads, p.batch), 256, 0, st>>>(
-          part_ml, part_acc, p.num_kv_heads, ns, (T*)o);
+      decode_merge_kernel<T, D, G><<<dim3(Hs, p.batch), 256, 0, st>>>(part_ml, part_acc, Hs, ns,
+                                                                     (T*)o);
       return;
     }
   }
   decode_attn_kernel<T, D, G><<<grid, kDecThreads, 0, st>>>(
-      (const T*)q, (const T*)kc, (const T*)vc, p.seqlens, sel_idx, sel_logg, p.num_kv_heads,
+      (const T*)q, (const T*)kc, (const T*)vc, p.seqlens, sel_idx, sel_logg, Hs, R,
       p.capacity, p.block, p.topk, ns, kLog2e / sqrtf((float)D), part_ml, part_acc);
-  decode_merge_kernel<T, D, G><<<dim3(p.num_kv_heads, p.batch), 256, 0, st>>>(
-      part_ml, part_acc, p.num_kv_heads, ns, (T*)o);
+  decode_merge_kernel<T, D, G><<<dim3(Hs, p.batch), 256, 0, st>>>(part_ml, part_acc, Hs, ns,
+                                                                 (T*)o);
 }
 
 template <typename T>
@@ -797,10 +803,10 @@ static void decode_gate_launch(const sas_decode_problem& p, const void* q_nope, 
                                float* sel_logg, int32_t* idx_out, float* logg_out,
                                const DecodePaging& pg, int* err, cudaStream_t st) {
   const int NBmax = (p.capacity + p.block - 1) / p.block;
-  const int G = p.num_q_heads / p.num_kv_heads;
+  const int G = p.num_q_heads / gate_heads(p);
   const size_t smem = (size_t)(G * p.head_dim + 3 * p.head_dim + 2 * p.gate_hidden + NBmax + 1 +
                                3 * kDecWarps + 4 + 256 + NBmax) * sizeof(float);
-  dim3 grid(p.num_kv_heads, p.batch);
+  dim3 grid(gate_heads(p), p.batch);
 #define SAS_DG(H, NPT)                                                                           \
   {                                                                                              \
     cudaFuncSetAttribute(decode_gate_kernel<T, H, NPT>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
@@ -808,6 +814,7 @@ static void decode_gate_launch(const sas_decode_problem& p, const void* q_nope, 
     decode_gate_kernel<T, H, NPT><<<grid, kDecThreads, smem, st>>>(                              \
         (const T*)q_nope, (const __nv_bfloat16*)gkc, cur_pool, (const T*)wq, qnorm_w, (const T*)wk, \
         knorm_w, p.seqlens, p.gate_rope_cos, p.gate_rope_sin, p.num_q_heads, p.num_kv_heads,      \
+        gate_heads(p),                                                                           \
         p.head_dim, p.block, p.topk, NBmax, p.capacity, p.rms_eps, p.ungated, sel_idx, sel_logg, \
         idx_out, logg_out, pg.pt, pg.num_pages, err);                                           \
   }
@@ -830,8 +837,8 @@ sas_status launch_decode(const sas_decode_problem& p, const void* q, const void*
                          const float* cur_pool, const void* wq, const float* qnorm_w,
                          const void* wk, const float* knorm_w, void* o, int32_t* idx_out,
                          float* logg_out, void* ws, const DecodePaging& pg, cudaStream_t st) {
-  const int G = p.num_q_heads / p.num_kv_heads;
-  const size_t pairs = (size_t)p.batch * p.num_kv_heads;
+  const int G = p.num_q_heads / gate_heads(p);   // query heads per gate head
+  const size_t pairs = (size_t)p.batch * gate_heads(p);
   const int ns = decode_nsplit(p);
   auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
   char* w = (char*)ws;

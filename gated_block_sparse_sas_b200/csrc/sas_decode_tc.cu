@@ -65,6 +65,8 @@ struct DecTcArgs {
   float scale_log2;
   const int32_t* pt;            // paged caches: page of block j of sequence b ([batch][NBmax]); or null
   int nbmax, num_pages;
+  int R;                        // gate heads per KV head: Hkv above counts gate heads, and gate
+                                // head kv reads the K/V of KV head kv / R (of Hkv / R)
 };
 
 __global__ void __launch_bounds__(dtc::kThreads, 2)
@@ -80,7 +82,7 @@ __global__ void __launch_bounds__(dtc::kThreads, 2)
   bool len_ok = Lraw >= 1 && Lraw <= a.capacity;
   int own_page = 0;   // paged caches: the page of the newest token's block, range-checked
   if (len_ok && a.pt != nullptr) {
-    own_page = a.pt[(size_t)b * a.nbmax + (Lraw - 1) / kB];
+    own_page = a.pt[(size_t)b * a.nbmax + (Lraw - 1) / kB];   // pt rows are per sequence
     len_ok = own_page >= 0 && own_page < a.num_pages;
   }
   const bool seq_ok = len_ok;
@@ -173,9 +175,10 @@ __global__ void __launch_bounds__(dtc::kThreads, 2)
     for (int h = w4; h < G; h += 4) {
       float dot = 0.f;
       if (seq_ok) {
+        const int Hk = a.Hkv / a.R, kh = kv / a.R;
         const size_t own = a.pt != nullptr
-                               ? ((size_t)own_page * a.Hkv + kv) * kB + (L - 1) % kB
-                               : ((size_t)b * a.Hkv + kv) * a.capacity + (L - 1);
+                               ? ((size_t)own_page * Hk + kh) * kB + (L - 1) % kB
+                               : ((size_t)b * Hk + kh) * a.capacity + (L - 1);
         const uint2 kr = *reinterpret_cast<const uint2*>(a.kc + own * kD + lane * 4);
         const uint2 qr = *reinterpret_cast<const uint2*>(a.q + ((size_t)b * Hq + kv * G + h) * kD + lane * 4);
         const float2 k01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&kr.x));
@@ -201,7 +204,8 @@ __global__ void __launch_bounds__(dtc::kThreads, 2)
     if (lane == 0) {
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
-      const int z = b * a.Hkv + kv;
+      const int Hk = a.Hkv / a.R, kh = kv / a.R;   // K/V of the gate head's KV head
+      const int z = b * Hk + kh;
       int issued = 0;   // ring loads issued: load i = K (i even) or V (i odd) of pair i / 2
       for (int i = 0; i < 2 * npairs; ++i) {
         const int slot = i % kSlots;
@@ -220,8 +224,8 @@ __global__ void __launch_bounds__(dtc::kThreads, 2)
         int ya = ja * kB, yb = jb * kB, za = z, zb = z;
         if (a.pt != nullptr) {
           ya = yb = 0;
-          za = a.pt[(size_t)b * a.nbmax + ja] * a.Hkv + kv;
-          zb = a.pt[(size_t)b * a.nbmax + jb] * a.Hkv + kv;
+          za = a.pt[(size_t)b * a.nbmax + ja] * Hk + kh;
+          zb = a.pt[(size_t)b * a.nbmax + jb] * Hk + kh;
         }
         mbar_arrive_expect_tx(full + slot, kKV);
 #pragma unroll
@@ -364,7 +368,7 @@ __global__ void __launch_bounds__(dtc::kThreads, 2)
 
 // ---------------------------------------------------------------------------------------
 bool decode_attn_tc_supported(const sas_decode_problem& p) {
-  const int G = p.num_q_heads / p.num_kv_heads;
+  const int G = p.num_q_heads / gate_heads(p);
   return tma_available() && p.dtype == SAS_BF16 && p.head_dim == 128 && p.block == 64 && G <= 8 &&
          p.topk + 1 <= 128;
 }
@@ -392,8 +396,9 @@ sas_status launch_decode_attn_tc(const sas_decode_problem& p, const void* q, con
   a.part_ml = part_ml;
   a.part_acc = part_acc;
   a.err = err;
-  a.Hkv = p.num_kv_heads;
-  a.G = p.num_q_heads / p.num_kv_heads;
+  a.Hkv = gate_heads(p);                       // gate heads: CTAs, selections, partials
+  a.G = p.num_q_heads / gate_heads(p);         // query heads per gate head
+  a.R = gate_heads(p) / p.num_kv_heads;
   a.capacity = p.capacity;
   a.K = p.topk;
   a.nsplit = ns;
@@ -406,7 +411,7 @@ sas_status launch_decode_attn_tc(const sas_decode_problem& p, const void* q, con
     cudaFuncSetAttribute(decode_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          dtc::kSmemBytes);
   });
-  decode_attn_tc_kernel<<<dim3(p.num_kv_heads, p.batch, ns), dtc::kThreads, dtc::kSmemBytes, st>>>(
+  decode_attn_tc_kernel<<<dim3(gate_heads(p), p.batch, ns), dtc::kThreads, dtc::kSmemBytes, st>>>(
       tk, tv, a);
   return SAS_OK;
 }

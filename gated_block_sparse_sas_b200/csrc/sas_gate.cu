@@ -181,14 +181,15 @@ struct GsSmem {
 };
 
 // PROJ: the two projections come precomputed (tensor-core GEMMs, sas_gate_tc.cu) as
-// qproj / kproj [T, Hkv, H] fp32, so phases 1 and 2 only load, normalise and rotate them.
+// qproj [T, Hs, H] / kproj [T, Hkv, H] fp32, so phases 1 and 2 only load, normalise and
+// rotate them.
 template <typename T, int H, bool PROJ>
 __global__ void __launch_bounds__(kGsThreads) gate_scores_kernel(
     const T* __restrict__ q_nope, const T* __restrict__ k_nope, const float* __restrict__ gkeys,
     const T* __restrict__ wq, const float* __restrict__ qnorm_w, const T* __restrict__ wk,
     const float* __restrict__ knorm_w, const int32_t* __restrict__ cu,
-    const float* __restrict__ rc, const float* __restrict__ rs, int Hq, int Hkv, int d, int B,
-    int NBmax, float eps, const float* __restrict__ qproj, const float* __restrict__ kproj,
+    const float* __restrict__ rc, const float* __restrict__ rs, int Hq, int Hkv, int Hs, int d,
+    int B, int NBmax, float eps, const float* __restrict__ qproj, const float* __restrict__ kproj,
     float* __restrict__ scores, float* __restrict__ lse) {
   extern __shared__ float smem[];
   using S = GsSmem<H, PROJ>;
@@ -197,12 +198,14 @@ __global__ void __launch_bounds__(kGsThreads) gate_scores_kernel(
   float* R = smem + S::QT;     // phase-dependent region
   float* scur = R + S::RMAX;   // [64]
 
-  const int tile = blockIdx.x, b = blockIdx.y, kv = blockIdx.z;
+  // gate head sh: its Gs query heads feed the query projection; its keys are KV head kv's
+  const int tile = blockIdx.x, b = blockIdx.y, sh = blockIdx.z;
+  const int kv = sh / (Hs / Hkv);
   const int s0 = cu[b], L = cu[b + 1] - s0;
   const int t0 = tile * kTQ;
   if (t0 >= L) return;
   const int nt = min(kTQ, L - t0);
-  const int G = Hq / Hkv, GD = G * d;
+  const int G = Hq / Hs, GD = G * d;
   const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
   const int warp = tid >> 5, lane = tid & 31;
 
@@ -211,7 +214,7 @@ __global__ void __launch_bounds__(kGsThreads) gate_scores_kernel(
     float* X = R;  // [64][H+1]
     for (int e = tid; e < kTQ * H; e += kGsThreads) {
       const int t = e / H, c = e - t * H;
-      X[t * (H + 1) + c] = (t < nt) ? qproj[((size_t)(s0 + t0 + t) * Hkv + kv) * H + c] : 0.f;
+      X[t * (H + 1) + c] = (t < nt) ? qproj[((size_t)(s0 + t0 + t) * Hs + sh) * H + c] : 0.f;
     }
     __syncthreads();
     for (int t = warp; t < kTQ; t += kGsThreads / 32) {
@@ -235,7 +238,7 @@ __global__ void __launch_bounds__(kGsThreads) gate_scores_kernel(
         const int t = tid >> 2, part = tid & 3;
         float v[8];
         if (t < nt) {
-          load8<T>(q_nope + ((size_t)(s0 + t0 + t) * Hq + (size_t)kv * G) * d + k0 + part * 8, v);
+          load8<T>(q_nope + ((size_t)(s0 + t0 + t) * Hq + (size_t)sh * G) * d + k0 + part * 8, v);
         } else {
 #pragma unroll
           for (int u = 0; u < 8; ++u) v[u] = 0.f;
@@ -246,7 +249,7 @@ __global__ void __launch_bounds__(kGsThreads) gate_scores_kernel(
       for (int e = tid; e < H * (kKC / 8); e += kGsThreads) {  // B: H x 32
         const int i = e / (kKC / 8), part = e - i * (kKC / 8);
         float v[8];
-        load8<T>(wq + ((size_t)kv * H + i) * GD + k0 + part * 8, v);
+        load8<T>(wq + ((size_t)sh * H + i) * GD + k0 + part * 8, v);
 #pragma unroll
         for (int u = 0; u < 8; ++u) Bs[(part * 8 + u) * (H + 4) + i] = v[u];
       }
@@ -414,7 +417,7 @@ __global__ void __launch_bounds__(kGsThreads) gate_scores_kernel(
         const int t = ty * 4 + aa;
         if (t >= nt) continue;
         const int ct = (t0 + t) / B;
-        float* srow = scores + ((size_t)(s0 + t0 + t) * Hkv + kv) * NBmax;
+        float* srow = scores + ((size_t)(s0 + t0 + t) * Hs + sh) * NBmax;
 #pragma unroll
         for (int o = 0; o < 4; ++o) {
           const int j = j0 + tx * 4 + o;
@@ -445,7 +448,7 @@ __global__ void __launch_bounds__(kGsThreads) gate_scores_kernel(
         mm = M;
       }
       const int t = ty * 4 + aa;
-      if (tx == 0 && t < nt) lse[(size_t)(s0 + t0 + t) * Hkv + kv] = mm + logf(ll);
+      if (tx == 0 && t < nt) lse[(size_t)(s0 + t0 + t) * Hs + sh] = mm + logf(ll);
     }
   }
 }
@@ -456,7 +459,8 @@ static sas_status gate_scores_dispatch(const sas_problem& p, const void* q_nope,
                                        const void* wk, const float* knorm_w, float* scores,
                                        float* lse, void* workspace, cudaStream_t st) {
   const int NBmax = (p.max_seqlen + p.block - 1) / p.block;
-  dim3 grid((p.max_seqlen + kTQ - 1) / kTQ, p.batch, p.num_kv_heads);
+  const int Hs = gate_heads(p);
+  dim3 grid((p.max_seqlen + kTQ - 1) / kTQ, p.batch, Hs);
   if (gate_tc_supported(p)) {   // projections on the tensor cores, then norms, rotary, scores
     float *qproj = nullptr, *kproj = nullptr;
     SAS_TRY(launch_gate_proj_tc(p, q_nope, k_nope, wq, wk, workspace, &qproj, &kproj, st));
@@ -468,7 +472,7 @@ static sas_status gate_scores_dispatch(const sas_problem& p, const void* q_nope,
     });
     gate_scores_kernel<T, 128, true><<<grid, kGsThreads, smem, st>>>(
         (const T*)q_nope, (const T*)k_nope, gkeys, (const T*)wq, qnorm_w, (const T*)wk, knorm_w,
-        p.cu_seqlens, p.gate_rope_cos, p.gate_rope_sin, p.num_q_heads, p.num_kv_heads,
+        p.cu_seqlens, p.gate_rope_cos, p.gate_rope_sin, p.num_q_heads, p.num_kv_heads, Hs,
         p.head_dim, p.block, NBmax, p.rms_eps, qproj, kproj, scores, lse);
     return launch_status("gate_scores (tensor-core projections)", 4);
   }
@@ -480,7 +484,8 @@ static sas_status gate_scores_dispatch(const sas_problem& p, const void* q_nope,
     gate_scores_kernel<T, H, false><<<grid, kGsThreads, smem, st>>>(                          \
         (const T*)q_nope, (const T*)k_nope, gkeys, (const T*)wq, qnorm_w, (const T*)wk,        \
         knorm_w, p.cu_seqlens, p.gate_rope_cos, p.gate_rope_sin, p.num_q_heads,               \
-        p.num_kv_heads, p.head_dim, p.block, NBmax, p.rms_eps, nullptr, nullptr, scores, lse); \
+        p.num_kv_heads, Hs, p.head_dim, p.block, NBmax, p.rms_eps, nullptr, nullptr, scores,   \
+        lse);                                                                                  \
   }
   switch (p.gate_hidden) {
     case 32: SAS_GS(32); break;
@@ -552,12 +557,12 @@ __global__ void topk_kernel(const float* __restrict__ scores, const float* __res
 sas_status launch_topk(const sas_problem& p, const float* scores, const float* lse, int32_t* idx,
                        float* logg, cudaStream_t st) {
   const int NBmax = (p.max_seqlen + p.block - 1) / p.block;
-  const int rows = p.total_tokens * p.num_kv_heads;
+  const int rows = p.total_tokens * gate_heads(p);
   const int threads = 256;
   const int grid = (int)(((size_t)rows * 32 + threads - 1) / threads);
 #define SAS_TK(N)                                                                              \
   topk_kernel<N><<<grid, threads, 0, st>>>(scores, lse, p.cu_seqlens, p.batch, p.total_tokens,  \
-                                           p.num_kv_heads, NBmax, p.block, p.topk, idx, logg)
+                                           gate_heads(p), NBmax, p.block, p.topk, idx, logg)
   if (NBmax <= 64) SAS_TK(2);
   else if (NBmax <= 256) SAS_TK(8);
   else if (NBmax <= 512) SAS_TK(16);

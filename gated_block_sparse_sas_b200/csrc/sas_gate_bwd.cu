@@ -472,7 +472,8 @@ GbwLayout gbw_layout(const sas_problem& p) {
 }  // namespace
 
 bool gate_bwd_supported(const sas_problem& p) {
-  return gate_tc_supported(p) && p.gate_hidden == gbw::H && p.head_dim == 128;
+  return gate_tc_supported(p) && p.gate_hidden == gbw::H && p.head_dim == 128 &&
+         gate_heads(p) == p.num_kv_heads;
 }
 
 size_t gate_bwd_workspace_bytes(const sas_problem& p) { return gbw_layout(p).total; }

@@ -54,8 +54,8 @@ __global__ void __launch_bounds__(kThreads) gate_select_kernel(
     const float* __restrict__ qproj, const float* __restrict__ kproj,
     const float* __restrict__ gkeys, const float* __restrict__ qnorm_w,
     const float* __restrict__ knorm_w, const int32_t* __restrict__ cu,
-    const float* __restrict__ rc, const float* __restrict__ rs, int Hkv, int B, int NBmax, int SS,
-    int K, float eps, int32_t* __restrict__ idx, float* __restrict__ logg,
+    const float* __restrict__ rc, const float* __restrict__ rs, int Hkv, int Hs, int B, int NBmax,
+    int SS, int K, float eps, int32_t* __restrict__ idx, float* __restrict__ logg,
     float* __restrict__ lse_out) {
   using C = Cfg<TQ>;
   extern __shared__ float4 smem4[];
@@ -65,7 +65,10 @@ __global__ void __launch_bounds__(kThreads) gate_select_kernel(
   float* scur = R + C::RB;            // [TQ]
   float* S = scur + TQ;               // [TQ][SS]  score rows
 
-  const int tile = blockIdx.x, b = blockIdx.y, kv = blockIdx.z;
+  // gate head sh (a KV head, or a query head with one gate per query head); its block keys
+  // and current-block key are KV head kv's
+  const int tile = blockIdx.x, b = blockIdx.y, sh = blockIdx.z;
+  const int kv = sh / (Hs / Hkv);
   const int s0 = cu[b], L = cu[b + 1] - s0;
   const int t0 = tile * TQ;
   if (t0 >= L) return;
@@ -78,7 +81,7 @@ __global__ void __launch_bounds__(kThreads) gate_select_kernel(
     float* X = R;   // [TQ][H+1]
     for (int e = tid; e < TQ * kH; e += kThreads) {
       const int t = e / kH, c = e - t * kH;
-      X[t * (kH + 1) + c] = (t < nt) ? qproj[((size_t)(s0 + t0 + t) * Hkv + kv) * kH + c] : 0.f;
+      X[t * (kH + 1) + c] = (t < nt) ? qproj[((size_t)(s0 + t0 + t) * Hs + sh) * kH + c] : 0.f;
     }
     __syncthreads();
     for (int t = warp; t < TQ; t += kThreads / 32) {
@@ -165,7 +168,7 @@ __global__ void __launch_bounds__(kThreads) gate_select_kernel(
     for (int j = lane; j <= c; j += 32) l += expf(srow[j] - m);
     l = warp_sum(l);
     const float lse = m + logf(l);
-    const size_t row = (size_t)(s0 + t0 + t) * Hkv + kv;
+    const size_t row = (size_t)(s0 + t0 + t) * Hs + sh;
     int32_t* irow = idx + row * (K + 1);
     float* grow = logg + row * (K + 1);
     if (lse_out != nullptr && lane == 0) lse_out[row] = lse;
@@ -201,7 +204,7 @@ size_t gate_select_workspace_bytes(const sas_problem& p) {
   if (gate_select_fused(p)) return gate_tc_workspace_bytes(p);
   // other shapes: sas_gate_scores' own workspace, then the scores and their logsumexp
   const int NBmax = (p.max_seqlen + p.block - 1) / p.block;
-  const size_t rows = (size_t)p.total_tokens * p.num_kv_heads;
+  const size_t rows = (size_t)p.total_tokens * gate_heads(p);
   return al256s(gate_scores_workspace_bytes(p)) + al256s(rows * NBmax * 4) + al256s(rows * 4);
 }
 
@@ -211,7 +214,7 @@ sas_status launch_gate_select(const sas_problem& p, const void* q_nope, const vo
                               float* lse, void* workspace, cudaStream_t st) {
   const int NBmax = (p.max_seqlen + p.block - 1) / p.block;
   if (!gate_select_fused(p)) {
-    const size_t rows = (size_t)p.total_tokens * p.num_kv_heads;
+    const size_t rows = (size_t)p.total_tokens * gate_heads(p);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     float* scores = reinterpret_cast<float*>(ws + al256s(gate_scores_workspace_bytes(p)));
     float* slse = lse != nullptr
@@ -230,10 +233,10 @@ sas_status launch_gate_select(const sas_problem& p, const void* q_nope, const vo
     const size_t smem = gsel::smem_bytes<TQ>(NBmax);                                          \
     cudaFuncSetAttribute(gsel::gate_select_kernel<TQ>,                                        \
                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);             \
-    const dim3 grid((p.max_seqlen + TQ - 1) / TQ, p.batch, p.num_kv_heads);                  \
+    const dim3 grid((p.max_seqlen + TQ - 1) / TQ, p.batch, gate_heads(p));                   \
     gsel::gate_select_kernel<TQ><<<grid, gsel::kThreads, smem, st>>>(                         \
         qproj, kproj, gkeys, qnorm_w, knorm_w, p.cu_seqlens, p.gate_rope_cos, p.gate_rope_sin, \
-        p.num_kv_heads, p.block, NBmax, SS, p.topk, p.rms_eps, idx, logg, lse);               \
+        p.num_kv_heads, gate_heads(p), p.block, NBmax, SS, p.topk, p.rms_eps, idx, logg, lse);\
   }
   if (NBmax <= 512) SAS_GSEL(64)
   else SAS_GSEL(32)

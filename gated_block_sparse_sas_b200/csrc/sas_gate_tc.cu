@@ -183,33 +183,35 @@ __global__ void __launch_bounds__(128) gate_prefix_kernel(const __nv_bfloat16* _
 // ---------------------------------------------------------------------------------------
 bool gate_tc_supported(const sas_problem& p) {
   return tma_available() && p.dtype == SAS_BF16 && p.head_dim == 128 && p.gate_hidden == 128 &&
-         p.block <= 128 && ((p.num_q_heads / p.num_kv_heads) * 128) % gtc::kBK == 0;
+         p.block <= 128 && ((p.num_q_heads / gate_heads(p)) * 128) % gtc::kBK == 0;
 }
 
 static size_t al256g(size_t x) { return (x + 255) & ~(size_t)255; }
 
 size_t gate_tc_workspace_bytes(const sas_problem& p) {
   const size_t rows = (size_t)p.total_tokens * p.num_kv_heads;
-  return 256 + al256g(rows * gtc::kKCols * 2) + 2 * al256g(rows * 128 * 4);
+  const size_t qrows = (size_t)p.total_tokens * gate_heads(p);
+  return 256 + al256g(rows * gtc::kKCols * 2) + al256g(qrows * 128 * 4) + al256g(rows * 128 * 4);
 }
 
 sas_status launch_gate_proj_tc(const sas_problem& p, const void* q_nope, const void* k_nope,
                                const void* wq, const void* wk, void* workspace, float** qproj,
                                float** kproj, cudaStream_t st) {
-  const int T = p.total_tokens, Hkv = p.num_kv_heads, Hq = p.num_q_heads;
-  const int G = Hq / Hkv;
+  // qproj per gate head s (Hs of them; Gs query heads each), kproj per KV head
+  const int T = p.total_tokens, Hkv = p.num_kv_heads, Hq = p.num_q_heads, Hs = gate_heads(p);
+  const int G = Hq / Hs;
   const size_t rows = (size_t)T * Hkv;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   int* err = reinterpret_cast<int*>(ws);
   __nv_bfloat16* ak = reinterpret_cast<__nv_bfloat16*>(ws + 256);
   *qproj = reinterpret_cast<float*>(ws + 256 + al256g(rows * gtc::kKCols * 2));
-  *kproj = *qproj + al256g(rows * 128 * 4) / 4;
+  *kproj = *qproj + al256g((size_t)T * Hs * 128 * 4) / 4;
   const int NBmax = (p.max_seqlen + p.block - 1) / p.block;
   gate_prefix_kernel<<<dim3(NBmax, p.batch, Hkv), 128, 0, st>>>((const __nv_bfloat16*)k_nope,
                                                                 p.cu_seqlens, Hkv, p.block, ak);
   CUtensorMap tAq, tBq, tAk, tBk;
   if (!make_tmap_bf16_2d(&tAq, q_nope, (uint64_t)Hq * 128, T, (uint64_t)Hq * 128 * 2, 64, 128) ||
-      !make_tmap_bf16_2d(&tBq, wq, (uint64_t)G * 128, (uint64_t)Hkv * 128, (uint64_t)G * 128 * 2,
+      !make_tmap_bf16_2d(&tBq, wq, (uint64_t)G * 128, (uint64_t)Hs * 128, (uint64_t)G * 128 * 2,
                          64, 128) ||
       !make_tmap_bf16_2d(&tAk, ak, (uint64_t)Hkv * gtc::kKCols, T, (uint64_t)Hkv * gtc::kKCols * 2,
                          64, 128) ||
@@ -222,11 +224,11 @@ sas_status launch_gate_proj_tc(const sas_problem& p, const void* q_nope, const v
     cudaFuncSetAttribute(gemm_bf16_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          gtc::kSmemBytes);
   });
-  const dim3 grid((T + gtc::kM - 1) / gtc::kM, Hkv);
-  GemmArgs aq{T, G * 128, G * 128, 0, *qproj, Hkv * 128, err};
-  gemm_bf16_tc_kernel<<<grid, gtc::kThreads, gtc::kSmemBytes, st>>>(tAq, tBq, aq);
+  const dim3 qgrid((T + gtc::kM - 1) / gtc::kM, Hs), kgrid((T + gtc::kM - 1) / gtc::kM, Hkv);
+  GemmArgs aq{T, G * 128, G * 128, 0, *qproj, Hs * 128, err};
+  gemm_bf16_tc_kernel<<<qgrid, gtc::kThreads, gtc::kSmemBytes, st>>>(tAq, tBq, aq);
   GemmArgs ak_args{T, gtc::kKCols, gtc::kKCols, 1, *kproj, Hkv * 128, err};
-  gemm_bf16_tc_kernel<<<grid, gtc::kThreads, gtc::kSmemBytes, st>>>(tAk, tBk, ak_args);
+  gemm_bf16_tc_kernel<<<kgrid, gtc::kThreads, gtc::kSmemBytes, st>>>(tAk, tBk, ak_args);
   return SAS_OK;
 }
 

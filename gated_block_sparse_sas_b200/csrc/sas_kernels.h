@@ -11,6 +11,14 @@
 
 namespace sas {
 
+// Gate (selection) heads: one gate per KV head (default) or one per query head.
+inline int gate_heads(const sas_problem& p) {
+  return p.gate_heads > 0 ? p.gate_heads : p.num_kv_heads;
+}
+inline int gate_heads(const sas_decode_problem& p) {
+  return p.gate_heads > 0 ? p.gate_heads : p.num_kv_heads;
+}
+
 sas_status launch_pool_keys(const sas_problem& p, const void* k_nope, float* pooled, cudaStream_t st);
 sas_status launch_gate_keys(const sas_problem& p, const float* pooled, const void* wk,
                             const float* knorm_w, float* gkeys, cudaStream_t st);

@@ -131,7 +131,7 @@ static size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
 static void km_dims(const sas_problem& p, int* nW, int* P, int* E) {
   *nW = (p.max_seqlen + km::kW - 1) / km::kW;
   *P = km::kWB * (*nW * (*nW + 1) / 2);
-  *E = p.num_kv_heads * p.batch * *P;
+  *E = gate_heads(p) * p.batch * *P;   // entries per gate head
 }
 
 bool km_supported(const sas_problem& p) {
@@ -144,7 +144,7 @@ size_t km_lists_bytes(const sas_problem& p) {
   int nW, P, E;
   km_dims(p, &nW, &P, &E);
   return 3 * al256((size_t)E * 4) + al256((size_t)E * kQuarters * 4) + 256 +
-         al256((size_t)p.total_tokens * p.num_kv_heads * (p.topk + 1) * 8);
+         al256((size_t)p.total_tokens * gate_heads(p) * (p.topk + 1) * 8);
 }
 
 KmLists km_lists_carve(const sas_problem& p, uint8_t* base) {
@@ -162,15 +162,15 @@ KmLists km_lists_carve(const sas_problem& p, uint8_t* base) {
 
 sas_status launch_km_lists(const sas_problem& p, const int32_t* idx, const float* logg,
                            const KmLists& L, cudaStream_t st) {
-  const dim3 wgrid(L.nW * kQuarters, p.batch, p.num_kv_heads);
+  const dim3 wgrid(L.nW * kQuarters, p.batch, gate_heads(p));
   if (cudaMemsetAsync(L.cnt, 0, (size_t)L.E * 4, st) != cudaSuccess) {
     set_error("key-major lists: clearing the counts failed");
     return SAS_ERR_CUDA;
   }
-  km_count_kernel<<<wgrid, 512, 0, st>>>(idx, p.cu_seqlens, p.batch, p.num_kv_heads, p.topk, L.P,
+  km_count_kernel<<<wgrid, 512, 0, st>>>(idx, p.cu_seqlens, p.batch, gate_heads(p), p.topk, L.P,
                                          L.cnt, L.cnt_q);
   km_scan_kernel<<<1, 1024, 0, st>>>(L.cnt, L.E, L.off, L.items, L.ctl);
-  km_fill_kernel<<<wgrid, 512, 0, st>>>(idx, logg, p.cu_seqlens, p.batch, p.num_kv_heads, p.topk,
+  km_fill_kernel<<<wgrid, 512, 0, st>>>(idx, logg, p.cu_seqlens, p.batch, gate_heads(p), p.topk,
                                         L.P, L.off, L.cnt_q, L.list);
   return launch_status("key-major selection lists", 3);
 }

@@ -95,6 +95,13 @@ typedef struct sas_problem {
   const int32_t* cu_seqlens;   /* device [batch+1], cu_seqlens[0] = 0              */
   const float* gate_rope_cos;  /* device [max_seqlen, h/2] (sas_rope_tables)        */
   const float* gate_rope_sin;  /* device [max_seqlen, h/2]                          */
+  /* Gate heads Hs. 0 or num_kv_heads: one gate per (token, KV head), shared by the G query
+   * heads of the KV group (the default reading). num_q_heads: one gate per (token, query
+   * head) -- the query projection reads that head alone (wq [Hq, h, d]), scores it against
+   * its KV head's block keys, and every query head keeps its own blocks. Either way the
+   * gate has Hq*d*h + Hkv*3d*h + 2h parameters. Tensors marked Hs below follow it; Gs =
+   * Hq/Hs query heads share a selection. */
+  int32_t gate_heads;
 } sas_problem;
 
 /* One decode step over a batch of contiguous KV caches. */
@@ -119,6 +126,9 @@ typedef struct sas_decode_problem {
    * would compute it (Hugging Face card "tencent/Simple-Attention-Sparsification", SGLang
    * seer_attn backend section). */
   int32_t ungated;
+  /* Gate heads Hs as in sas_problem (0 or num_kv_heads: per KV group; num_q_heads: per query
+   * head, wq [Hq, h, d], selections [batch, Hq, K+1]). */
+  int32_t gate_heads;
 } sas_decode_problem;
 
 /* Reason for the last non-OK status returned on this thread ("" if none). */
@@ -152,13 +162,14 @@ sas_status sas_gate_keys(const sas_problem* p, const float* pooled, const void* 
 
 /* A3 -- gate scores (model card: Query projection Qproj; abstract: normalised
  * softmax gates calibrated against the always-retained current block).
- * q~_t = rope(RMSNorm(Wq . concat_g q_nope[t, kv*G+g]) * qnorm_w, pos = t);
- * s[t, kv, j] = q~_t . k~_j / sqrt(h) for j < c_t from gate_keys, and for j = c_t
- * with the current block's key pooled over its tokens c_t*B..t (computed here from
- * k_nope, wk, knorm_w); s = -inf for j > c_t. lse[t, kv] = logsumexp_{j<=c_t} s.
+ * q~_t,s = rope(RMSNorm(Wq[s] . concat_g q_nope[t, s*Gs+g]) * qnorm_w, pos = t) for gate
+ * head s; s[t, s, j] = q~_t,s . k~_j / sqrt(h) with the block keys of KV head
+ * kv = s*Gs/G: for j < c_t from gate_keys, and for j = c_t the current block's key pooled
+ * over its tokens c_t*B..t (computed here from k_nope, wk, knorm_w); s = -inf for j > c_t.
+ * lse[t, s] = logsumexp_{j<=c_t} s.
  * q_nope dtype [T, Hq, d]; k_nope dtype [T, Hkv, d]; gate_keys fp32 [batch, NBmax,
- * Hkv, h]; wq dtype [Hkv, h, G*d]; wk dtype [Hkv, h, 3d]; qnorm_w, knorm_w fp32 [h];
- * scores fp32 [T, Hkv, NBmax]; lse fp32 [T, Hkv].
+ * Hkv, h]; wq dtype [Hs, h, Gs*d]; wk dtype [Hkv, h, 3d]; qnorm_w, knorm_w fp32 [h];
+ * scores fp32 [T, Hs, NBmax]; lse fp32 [T, Hs].
  * Workspace (size from sas_gate_scores_workspace_size): for bf16, d = 128, h = 128 the two
  * projections run as tensor-core GEMMs and the workspace holds their inputs and outputs
  * (per token and kv head: the current block's prefix max, min and mean as exact bf16 parts,
@@ -172,8 +183,8 @@ sas_status sas_gate_scores(const sas_problem* p, const void* q_nope, const void*
 /* A3 + A4 fused -- gate scores and Top-K selection in one pass (paper abstract: Top-K keeps
  * the computation sparse; model card: Qproj, Q/K normalisation, gate RoPE, Top-K).
  * Same inputs as sas_gate_scores, same results as sas_gate_scores followed by sas_topk:
- * idx int32 / logg fp32 [T, Hkv, K+1] (ids ascending, current block last, -1 padding),
- * and, if lse is not NULL, the gate logsumexp fp32 [T, Hkv]. For bf16, d = 128, h = 128
+ * idx int32 / logg fp32 [T, Hs, K+1] (ids ascending, current block last, -1 padding),
+ * and, if lse is not NULL, the gate logsumexp fp32 [T, Hs]. For bf16, d = 128, h = 128
  * and NBmax <= 1024 the scores live only in shared memory (one kernel holds a tile's score
  * rows, selects and writes the kept ids); the scores are bit-identical to sas_gate_scores',
  * so the ids are too, and the log-gates agree to fp32 rounding (the logsumexp is summed in
@@ -200,7 +211,7 @@ sas_status sas_gate_select(const sas_problem* p, const void* q_nope, const void*
  * idx int32 / dlogg fp32 [T, Hkv, K+1]. Outputs (overwritten, fp32): dwq [Hkv, h, G*d],
  * dqnorm_w [h], dwk [Hkv, h, 3d], dknorm_w [h]; sums of floating-point atomics, so their low
  * bits can change from run to run. Supported: bf16, head_dim 128, gate_hidden 128,
- * block <= 128 (SAS_ERR_UNSUPPORTED otherwise). Workspace (sas_gate_bwd_workspace_size):
+ * block <= 128, one gate per KV group (SAS_ERR_UNSUPPORTED otherwise). Workspace (sas_gate_bwd_workspace_size):
  * word 0 is the call's error word (the tensor-core projections' codes 91-93; 0 = none). */
 sas_status sas_gate_bwd_workspace_size(const sas_problem* p, size_t* bytes);
 sas_status sas_gate_bwd(const sas_problem* p, const void* q_nope, const void* k_nope,
@@ -210,16 +221,17 @@ sas_status sas_gate_bwd(const sas_problem* p, const void* q_nope, const void* k_
                         size_t workspace_bytes, cudaStream_t stream);
 
 /* A4 -- Top-K selection (README (b); model card: Training Top-K 31 historical blocks).
- * Per (t, kv): the min(K, c_t) historical blocks with the highest score (ties to
+ * Per (t, gate head s): the min(K, c_t) historical blocks with the highest score (ties to
  * the lower index), ascending, then the current block c_t, then -1 padding.
- * idx int32 [T, Hkv, K+1]; logg fp32 [T, Hkv, K+1] = s - lse on kept slots, 0 on
+ * idx int32 [T, Hs, K+1]; logg fp32 [T, Hs, K+1] = s - lse on kept slots, 0 on
  * padding. Bit-exact given the scores. */
 sas_status sas_topk(const sas_problem* p, const float* scores, const float* lse,
                     int32_t* idx, float* logg, cudaStream_t stream);
 
 /* A5 -- gated sparse attention forward (README (b); abstract: gate in the softmax in
- * log form, FlashAttention-style). For query head hq (kv = hq / G), token t:
- * z_i = q_t.k_i/sqrt(d) + logg[t, kv, slot] for keys i <= t of block idx[t, kv, slot];
+ * log form, FlashAttention-style). For query head hq (KV head kv = hq / G, gate head
+ * s = hq / Gs), token t:
+ * z_i = q_t.k_i/sqrt(d) + logg[t, s, slot] for keys i <= t of block idx[t, s, slot];
  * O_t = softmax(z) V; lse_attn = natural-log logsumexp of z.
  * q dtype [T, Hq, d]; k, v dtype [T, Hkv, d] (rotated); idx/logg as from sas_topk
  * (any valid selection: ascending historical, current block, -1 padding);
@@ -239,8 +251,8 @@ sas_status sas_attn_fwd(const sas_problem* p, const void* q, const void* k, cons
 /* A6 -- backward of A5 with the selection held fixed (abstract: the loss reaches the
  * selector through standard backpropagation). Inputs as A5 plus o, dout (dtype
  * [T, Hq, d]) and lse_attn. Outputs dq dtype [T, Hq, d]; dk, dv dtype [T, Hkv, d];
- * dlogg fp32 [T, Hkv, K+1] = sum over the G heads and the keys of block
- * idx[t, kv, slot] of P (dP - D), 0 on padding. */
+ * dlogg fp32 [T, Hs, K+1] = sum over the gate head's Gs query heads and the keys of block
+ * idx[t, s, slot] of P (dP - D), 0 on padding. */
 sas_status sas_attn_bwd_workspace_size(const sas_problem* p, size_t* bytes);
 sas_status sas_attn_bwd(const sas_problem* p, const void* q, const void* k, const void* v,
                         const void* o, const void* dout, const float* lse_attn,
@@ -253,12 +265,13 @@ sas_status sas_attn_bwd(const sas_problem* p, const void* q, const void* k, cons
  * cached tokens (newest at L_b-1, c = (L_b-1)/B): gate query at position L_b-1;
  * historical block keys read from gate_key_cache; the current block's key from the
  * running pool state (max, min, sum/n, n = L_b - c*B) at position c*B; softmax
- * gates, Top-K, then the gated attention of the G query heads over the kept blocks.
+ * gates, Top-K, then the gated attention of the gate head's query heads over its kept
+ * blocks (gate heads as sas_problem's: per KV group, or per query head).
  * q dtype [batch, Hq, d] (rotated); q_nope dtype [batch, Hq, d];
  * k_cache, v_cache dtype [batch, Hkv, capacity, d]; gate_key_cache bf16
  * [batch, Hkv, NBmax, h] (entries j < c read); cur_pool fp32 [batch, Hkv, 3, d]
  * (max, min, sum over tokens c*B..L_b-1); wq, wk, qnorm_w, knorm_w as A3;
- * o dtype [batch, Hq, d]; idx_out int32 / logg_out fp32 [batch, Hkv, K+1] may be NULL.
+ * o dtype [batch, Hq, d]; idx_out int32 / logg_out fp32 [batch, Hs, K+1] may be NULL.
  * Workspace (sas_decode_workspace_size): word 0 is the call's error word (cleared by the
  * call; 41 / 81-83 a bounded wait gave up, 61 a row outside the fixed reference's range). */
 sas_status sas_decode_workspace_size(const sas_decode_problem* p, size_t* bytes);

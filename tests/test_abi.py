@@ -73,6 +73,7 @@ def _call_pool(sas, prob, k=0x10000, out=0x20000):
     ("batch", 0, -1, "batch"),
     ("cu_seqlens", None, -1, "cu_seqlens"),
     ("max_seqlen", 64 * 4096, -2, "blocks"),
+    ("gate_heads", 3, -1, "gate_heads"),
 ])
 def test_invalid_problem_rejected(sas, field, value, status, frag):
     p = _prob(sas, **{field: value})

@@ -451,3 +451,120 @@ def test_decode_paged_equals_contiguous(sas, name):
     assert sas.error_code(ws) == 62
     assert torch.count_nonzero(o_b[0]).item() == 0
     assert torch.equal(o_b[1:], o_c[1:])
+
+
+PER_HEAD_CASES = {
+    # one gate per query head (gate_heads = Hq): tensor-core paths (gate projections, fused
+    # selection, key-major attention with 128 single-head rows per tile, tensor-core decode)
+    "bf16-d128-B64-G4": ([4200, 300, 65], 8, 2, 128, 64, 15, 128, "bf16"),
+    # CUDA-core paths (fp32, d 64)
+    "fp32-d64-B16-G2": ([300, 77], 4, 2, 64, 16, 5, 32, "fp32"),
+}
+
+
+def _per_head(sas, name, seed):
+    lengths, Hq, Hkv, d, B, K, h, dt = PER_HEAD_CASES[name]
+    shape = si.Shape(list(lengths), Hq, Hkv, d, B, K, h, dt, seed=seed, gate_heads=Hq)
+    inp = si.prefill_inputs(shape, with_dout=True)
+    dev = torch.device("cuda:0")
+    g = {k: v.to(dev) for k, v in inp.items()}
+    prob = sas.Problem.from_lengths(shape.lengths, dev, num_q_heads=Hq, num_kv_heads=Hkv,
+                                    head_dim=d, block=B, topk=K, gate_hidden=h,
+                                    dtype=shape.torch_dtype, gate_heads=Hq)
+    return shape, inp, g, prob
+
+
+def _edge_rows(shape, n_random, seed):
+    rows = set()
+    for s0, s1 in zip(shape.cu_seqlens[:-1], shape.cu_seqlens[1:]):
+        L = int(s1 - s0)
+        for t in (0, 15, 16, 63, 64, 4095, 4096, L - 1):
+            if 0 <= t < L:
+                rows.add(int(s0) + t)
+    rng = np.random.default_rng(seed)
+    rows |= set(rng.choice(shape.total_tokens, n_random, replace=False).tolist())
+    return np.array(sorted(rows))
+
+
+@pytest.mark.parametrize("name", list(PER_HEAD_CASES))
+def test_per_head_gate_selection(sas, name):
+    """One gate per query head: the fused and the unfused selection agree bit for bit, and
+    match the oracle (per-query-head Qproj, scored against the KV head's block keys)."""
+    shape, inp, g, prob = _per_head(sas, name, 800)
+    idx, logg = sas.prefill_selection(prob, g["q_nope"], g["k_nope"], g["wq"], g["qnorm_w"],
+                                      g["wk"], g["knorm_w"])
+    idx_u, logg_u = sas.prefill_selection(prob, g["q_nope"], g["k_nope"], g["wq"], g["qnorm_w"],
+                                          g["wk"], g["knorm_w"], fused=False)
+    torch.cuda.synchronize()
+    assert idx.shape == (shape.total_tokens, shape.num_q_heads, shape.topk + 1)
+    assert torch.equal(idx, idx_u)
+    assert (logg - logg_u).abs().max().item() <= 2e-6
+    rows = _edge_rows(shape, 60, 801)
+    ref = orc.prefill_selection(inp["q_nope"], inp["k_nope"], inp["wq"], inp["qnorm_w"], inp["wk"],
+                                inp["knorm_w"], shape.cu_seqlens, shape.block, shape.topk, 1e-6,
+                                1e6, rows)
+    compare_selection(idx.cpu().numpy()[rows], logg.cpu().numpy()[rows], ref["idx"], ref["logg"],
+                      ref["margin"])
+
+
+@pytest.mark.parametrize("name", list(PER_HEAD_CASES))
+def test_per_head_attention(sas, name):
+    """Every query head on its own selection: forward rows, dQ / dlogg rows and dK / dV of
+    first, middle and last blocks against the oracle."""
+    shape, inp, g, prob = _per_head(sas, name, 810)
+    idx, logg = si.random_selection(shape)
+    ti, tl = torch.from_numpy(idx).cuda(), torch.from_numpy(logg).cuda()
+    wsf, wsb = sas.attn_fwd_workspace(prob), sas.attn_bwd_workspace(prob)
+    o, lse = sas.sas_attn_fwd(prob, g["q"], g["k"], g["v"], ti, tl, workspace=wsf)
+    dq, dk, dv, dl = sas.sas_attn_bwd(prob, g["q"], g["k"], g["v"], o, g["dout"], lse, ti, tl,
+                                      workspace=wsb)
+    torch.cuda.synchronize()
+    assert sas.error_code(wsf) == 0 and sas.error_code(wsb) == 0
+    fp32 = shape.dtype == "fp32"
+    cu = shape.cu_seqlens
+    rows = _edge_rows(shape, 40, 811)
+    O, LSE, _ = orc.attention_fwd(inp["q"], inp["k"], inp["v"], idx, logg, cu, shape.block,
+                                  rows=rows)
+    assert_out_close(o[torch.from_numpy(rows).cuda()], O, fp32, "O")
+    assert np.abs(to64(lse)[rows] - LSE).max() <= (1e-4 if fp32 else 2e-3)
+    dq_r, dl_r = orc.attention_bwd_rows(inp["q"], inp["k"], inp["v"], inp["dout"], idx, logg, cu,
+                                        shape.block, rows)
+    assert_grad_close(dq.cpu()[rows], dq_r, fp32, "dQ rows")
+    assert_grad_close(dl.cpu()[rows], dl_r, fp32, "dlogg rows")
+    assert (to64(dl)[idx < 0] == 0).all()
+    B = shape.block
+    for b, (s0, s1) in enumerate(zip(cu[:-1], cu[1:])):
+        L = int(s1 - s0)
+        nb = (L + B - 1) // B
+        for j, kv in sorted({(0, 0), (nb // 2, shape.num_kv_heads - 1), (nb - 1, 0)}):
+            lo, hi = j * B, min((j + 1) * B, L)
+            dk_r, dv_r = orc.attention_bwd_keys(inp["q"], inp["k"], inp["v"], inp["dout"], idx,
+                                                logg, cu, B, b, kv, lo, hi)
+            if np.linalg.norm(dk_r) > 1e-9:
+                assert_grad_close(dk.cpu()[int(s0) + lo:int(s0) + hi, kv], dk_r, fp32,
+                                  f"dK seq {b} block {j}")
+            assert_grad_close(dv.cpu()[int(s0) + lo:int(s0) + hi, kv], dv_r, fp32,
+                              f"dV seq {b} block {j}")
+
+
+@pytest.mark.parametrize("d,B,h,dt", [(128, 64, 128, "bf16"), (64, 16, 32, "bf16")])
+def test_per_head_decode(sas, d, B, h, dt):
+    """Decode with one gate per query head against the oracle (selection per query head)."""
+    shp = si.DecodeShape([3000, 65, 1, 1777], 4096, 8, 2, d, B, 15, h, seed=820, dtype=dt,
+                         gate_heads=8)
+    inp = si.decode_inputs(shp)
+    g = {k: v.cuda() for k, v in inp.items()}
+    prob = sas.DecodeProblem(seqlens=g["lengths"], capacity=shp.capacity, num_q_heads=8,
+                             num_kv_heads=2, head_dim=d, block=B, topk=15, gate_hidden=h,
+                             dtype=torch.bfloat16, gate_heads=8)
+    o, idx, logg = sas.sas_decode(prob, g["q"], g["q_nope"], g["k_cache"], g["v_cache"],
+                                  g["gate_key_cache"], g["cur_pool"], g["wq"], g["qnorm_w"], g["wk"],
+                                  g["knorm_w"], want_selection=True, check=True)
+    torch.cuda.synchronize()
+    assert idx.shape == (4, 8, 16)
+    O, ridx, rlogg, margin = orc.decode(inp["q"], inp["q_nope"], inp["k_cache"], inp["v_cache"],
+                                        shp.lengths, inp["gate_key_cache"], inp["cur_pool"],
+                                        inp["wq"], inp["qnorm_w"], inp["wk"], inp["knorm_w"], B, 15,
+                                        1e-6, 1e6, selection=(idx.cpu().numpy(), logg.cpu().numpy()))
+    compare_selection(idx.cpu().numpy(), logg, ridx, rlogg, margin)
+    assert_out_close(o, O, False, "O")
