@@ -292,6 +292,42 @@ def alloc_outputs(sas, prob, g, backward):
         g["_wsb"] = torch.empty(max(256, n.value), dtype=torch.uint8, device=dev)
 
 
+def bench_gate_paths(sas, prob, g, flush, steps):
+    """Gate scores + Top-K two ways on the step's inputs: the fused pass (score rows kept on
+    chip) and the two separate kernels (the [T, Hs, NBmax] scores written to and read back
+    from HBM). Both give the same selection; timed after the step, not part of it."""
+    scores = torch.empty((prob.total_tokens, prob.sel_heads, prob.max_blocks), dtype=torch.float32,
+                         device=prob.device)
+    lse = torch.empty((prob.total_tokens, prob.sel_heads), dtype=torch.float32, device=prob.device)
+    wsu = sas.gate_scores_workspace(prob)
+    args = (prob, g["q_nope"], g["k_nope"], g["_gk"], g["wq"], g["qnorm_w"], g["wk"], g["knorm_w"])
+
+    def fused():
+        sas.sas_gate_select(*args, idx=g["_idx"], logg=g["_logg"], workspace=g["_wsg"])
+
+    def unfused():
+        sas.sas_gate_scores(*args, scores=scores, lse=lse, workspace=wsu)
+        sas.sas_topk(prob, scores, lse, idx=g["_idx"], logg=g["_logg"])
+
+    out = {}
+    for name, fn in (("fused_ms", fused), ("unfused_ms", unfused)):
+        for _ in range(2):
+            fn()
+        ev = []
+        for _ in range(steps):
+            flush.zero_()
+            a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a_.record()
+            fn()
+            b_.record()
+            ev.append((a_, b_))
+        torch.cuda.synchronize()
+        out[name] = sum(x.elapsed_time(y) for x, y in ev) / len(ev)
+    out["score_bytes_avoided"] = 2 * scores.numel() * 4
+    del scores
+    return out
+
+
 def bench_router_bwd(sas, prob, g, flush, steps):
     """The router backward (gate parameter gradients from the step's own dlogg), timed on its
     own after the step: it is not part of the timed step."""
@@ -463,9 +499,12 @@ def time_workload(sas, name, shape, backward, g, prob, steps, warmup, flush, ws,
     G, d = shape.group, shape.head_dim
     fwd_flops = 4.0 * pairs * G * d
     bwd_flops = 2.5 * fwd_flops if backward else 0.0
-    Mq = 25 if G == 5 else 128 // G
-    tiles, kept = km_stats(out[2], prob.cu_seqlens, shape.lengths, Mq, shape.num_kv_heads,
-                           prob.max_blocks)
+    # tokens per gathered 128-row tile: forward 25 (G = 5) or 128 / G; backward whole tokens
+    # per warp, 4 floor(32 / G)
+    tiles, kept = km_stats(out[2], prob.cu_seqlens, shape.lengths, 25 if G == 5 else 128 // G,
+                           shape.num_kv_heads, prob.max_blocks)
+    tiles_bwd, _ = km_stats(out[2], prob.cu_seqlens, shape.lengths, 4 * (32 // G),
+                            shape.num_kv_heads, prob.max_blocks)
     timer = Timer()
     evs = []
     barrier(ws)
@@ -487,7 +526,7 @@ def time_workload(sas, name, shape, backward, g, prob, steps, warmup, flush, ws,
     ms = sum(x.elapsed_time(y) for x, y in evs) / len(evs)
     ms = max_over_ranks(ms, ws, dev)
     return dict(ms=ms, ops=timer.mean_ms(), pairs=pairs, fwd_flops=fwd_flops, bwd_flops=bwd_flops,
-                tiles=tiles, kept=kept, launches=launches)
+                tiles=tiles, tiles_bwd=tiles_bwd, kept=kept, launches=launches)
 
 
 class _Null:
@@ -515,7 +554,7 @@ def summarise(name, shape, backward, r, peak, peak_note, ws):
     work = r["fwd_flops"] + r["bwd_flops"]
     mma = 2.0 * 128 * 64 * d                           # one 128-row x 64-key x d product
     comp_fwd = r["tiles"] * 2 * mma                    # S = Q K^T, O = P V per gathered tile
-    comp_bwd = r["tiles"] * 5 * mma if backward else 0.0   # S, dP, dV^T, dK^T, dQ
+    comp_bwd = r["tiles_bwd"] * 5 * mma if backward else 0.0   # S, dP, dV^T, dK^T, dQ
     red_bytes = r["kept"] * G * d * 4                  # fp32 partial rows reduced into L2
     dom = max(("sas_attn_fwd", "sas_attn_bwd") if backward else ("sas_attn_fwd",),
               key=lambda k: ops[k])
@@ -534,7 +573,7 @@ def summarise(name, shape, backward, r, peak, peak_note, ws):
                      "dense_causal_fraction": r["pairs"] / (shape.num_kv_heads * sum(
                          L * (L + 1) / 2 for L in shape.lengths))},
         "computed": {"fwd_tflop": comp_fwd / 1e12, "bwd_tflop": comp_bwd / 1e12,
-                     "gathered_tiles": r["tiles"],
+                     "gathered_tiles": r["tiles"], "gathered_tiles_bwd": r["tiles_bwd"],
                      "attended_over_computed": work / max(1.0, comp_fwd + comp_bwd),
                      "fwd_tflops": comp_fwd / (ops["sas_attn_fwd"] * 1e-3) / 1e12,
                      "bwd_tflops": (comp_bwd / (ops["sas_attn_bwd"] * 1e-3) / 1e12) if backward else None,
@@ -595,6 +634,7 @@ def main():
         line["e2e"] = e2e(sas, prob, g, backward, r["fwd_flops"] + r["bwd_flops"], dev, a, ws)
     if backward:   # after the timed step and e2e legs, so it cannot perturb them
         line["router_bwd"] = bench_router_bwd(sas, prob, g, flush, max(3, a.steps))
+    line["gate_paths"] = bench_gate_paths(sas, prob, g, flush, max(3, a.steps))
     if rank == 0 and ws == 1 and not a.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(g, shape, backward, a)
     del g, prob
@@ -625,7 +665,8 @@ def main():
             line["decode"] = {"error": f"out of memory: {ex}"[:200]}
 
     line["extra_keys"] = [k for k in line if k in ("train_32k", "prefill_32k", "decode",
-                                                   "router_bwd", "computed", "attended", "ops_ms")]
+                                                   "router_bwd", "gate_paths", "computed",
+                                                   "attended", "ops_ms")]
     if rank == 0:
         print(json.dumps(line), flush=True)
     if ws > 1:

@@ -32,7 +32,8 @@
 //               buffer [32 rows][32 columns] (each lane's 16-byte pieces rotated by lane so the
 //               stores hit distinct banks), then one TMA tensor reduction (cp.reduce.async.bulk
 //               .tensor .add, fp32) per token: the G rows of a token are its G adjacent query
-//               heads in dQ_acc (a Q/dO stage is free as soon as the tile's gradient MMAs are
+//               heads in dQ_acc and G adjacent lanes of one warp (a warp holds floor(32 / G)
+//               whole tokens; G = 5: 24 tokens per tile) (a Q/dO stage is free as soon as the tile's gradient MMAs are
 //               done); at an item's end dK/dV from TMEM (lane = d, column = key) into the
 //               accumulators.
 // Every wait is bounded; a timeout records an error code in the workspace and all roles
@@ -172,9 +173,13 @@ __global__ void __launch_bounds__(kmb::kThreads, 1)
 
   if (warp < 4) {
     // ------------------------------ gather ------------------------------
+    // a token's G rows never straddle two warps: a warp holds floor(32 / G) whole tokens
+    // (G = 5: six tokens in lanes 0..29, lanes 30 and 31 idle), so the dS and epilogue warps
+    // can sum and reduce a token's rows together (Mq = 4 floor(32 / G) tokens per tile)
     const int r = tid;
-    const int tl = r / G, g = r - tl * G;
-    const bool row_ok = r < G * Mq;
+    const int tpw = 32 / G, lr = r & 31;
+    const int tl = (r >> 5) * tpw + lr / G, g = lr % G;
+    const bool row_ok = lr < tpw * G;
     bool ok = true;
     int n = 0, item_seq = 0;
     while (true) {
@@ -203,17 +208,25 @@ __global__ void __launch_bounds__(kmb::kThreads, 1)
       }
       ++item_seq;
       const int ntile = (cnt + Mq - 1) / Mq;
+      // the row's list entry and its LSE and D are loaded one tile ahead, so a tile's gather
+      // waits for one L2 round trip (the Q / dO rows) instead of three dependent ones
       int2 nxt = make_int2(0, 0);
-      if (row_ok && tl < cnt) nxt = a.list[off + tl];
+      float nxt_lse = 0.f, nxt_d = 0.f;
+      if (row_ok && tl < cnt) {
+        nxt = a.list[off + tl];
+        const size_t qr0 = (size_t)(nxt.x & 0xFFFFFF) * a.Hq + kv * G + g;
+        nxt_lse = a.lse[qr0];
+        nxt_d = a.drow[qr0];
+      }
       for (int m = 0; m < ntile; ++m, ++n) {
         const int rank = m * Mq + tl;
         const bool valid = row_ok && rank < cnt;
         const int2 ent = nxt;
-        if (row_ok && rank + Mq < cnt) nxt = a.list[off + rank + Mq];   // next tile's entry
+        const float lse_v = nxt_lse, d_v = nxt_d;
+        const bool more = row_ok && rank + Mq < cnt;
+        if (more) nxt = a.list[off + rank + Mq];   // next tile's entry
         const int tg = ent.x & 0xFFFFFF, slot = ent.x >> 24;
         const size_t qrow = (size_t)tg * a.Hq + kv * G + g;
-        const float lse_v = valid ? a.lse[qrow] : 0.f;
-        const float d_v = valid ? a.drow[qrow] : 0.f;
         const int qs = n & 1, rs = n & 3;
         if (ok && n >= 2 && !mbar_wait(qd_empty + qs, ((n >> 1) - 1) & 1, abort_flag)) {
           tc_fail(a.err, 72, abort_flag);
@@ -243,8 +256,13 @@ __global__ void __launch_bounds__(kmb::kThreads, 1)
             st_shared_v4(do_dst + o, 0u, 0u, 0u, 0u);
           }
         }
+        if (more) {   // the next tile's LSE and D (its list entry has arrived by now)
+          const size_t nq = (size_t)(nxt.x & 0xFFFFFF) * a.Hq + kv * G + g;
+          nxt_lse = a.lse[nq];
+          nxt_d = a.drow[nq];
+        }
         rcf[rc_slot(rs, 0) + r] = valid ? (__int_as_float(ent.y) - lse_v) * kLog2e : -INFINITY;
-        rcf[rc_slot(rs, 1) + r] = d_v;
+        rcf[rc_slot(rs, 1) + r] = valid ? d_v : 0.f;
         rci[rc_slot(rs, 2) + r] = valid ? min(kB - 1, tg - key0) : -1;
         rci[rc_slot(rs, 3) + r] = valid ? (int)qrow : -1;
         rci[rc_slot(rs, 4) + r] = valid ? (tg * a.Hs + kv) * a.K1 + slot : -1;
@@ -456,13 +474,16 @@ __global__ void __launch_bounds__(kmb::kThreads, 1)
         st_shared_v4(ds_row + o, pd[4 * c], pd[4 * c + 1], pd[4 * c + 2], pd[4 * c + 3]);
       }
       fence_async_smem();
-      // dlogg of (token, slot) = sum over the token's G rows (tile rows G*i .. G*i+G-1)
-      if ((32 % G) == 0) {   // the G rows share a warp: butterfly over the G lanes
+      // dlogg of (token, slot) = sum over the token's G rows: G adjacent lanes of this warp,
+      // the first at a multiple of G
+      if ((G & (G - 1)) == 0) {   // a power of two: butterfly over the G lanes
         for (int o = 1; o < G; o <<= 1) dlsum += __shfl_xor_sync(0xffffffffu, dlsum, o);
-        if (dli >= 0 && (r % G) == 0) a.dlogg[dli] = dlsum;
-      } else if (dli >= 0) {  // G = 5: the rows of a token can straddle two warps
-        atomicAdd(a.dlogg + dli, dlsum);
+      } else {                    // G = 5: the token's first lane adds its next G - 1 lanes
+        float sum = dlsum;
+        for (int o = 1; o < G; ++o) sum += __shfl_down_sync(0xffffffffu, dlsum, o);
+        dlsum = sum;
       }
+      if (dli >= 0 && ((r & 31) % G) == 0) a.dlogg[dli] = dlsum;
       mbar_arrive(ps_full);
     }
     if (!ok) tc_fail(a.err, 76, abort_flag);
@@ -470,10 +491,8 @@ __global__ void __launch_bounds__(kmb::kThreads, 1)
     // ------------------------------ epilogue ------------------------------
     const int r = tid - 384, ew = warp - 12;
     const uint32_t lane_addr = (uint32_t)(ew * 32) << 16;
-    // one reduction box per token (its G rows) when G divides 32, so no token straddles two
-    // warps; otherwise one box per row
-    const int Gb = (32 % G) == 0 ? G : 1;
-    const bool issuer = (lane % Gb) == 0;
+    // one reduction box per token: its G rows, adjacent lanes of one warp (see the gather)
+    const bool issuer = (lane % G) == 0;
     const int rot = lane & 7;
     const uint32_t my_row = smem_u32(sm + OFF_EPI) + (uint32_t)(ew * kEpiBytes + lane * 128);
     if (lane == 0) prefetch_tmap(&tmDQ);
@@ -617,7 +636,7 @@ sas_status launch_attn_bwd_km(const sas_problem& p, const void* q, const void* k
   const int T = p.total_tokens;
 
   CUtensorMap tk, tv, tdq;
-  const uint32_t box_rows = (32 % G) == 0 ? (uint32_t)G : 1u;   // the epilogue's box per token
+  const uint32_t box_rows = (uint32_t)G;   // the epilogue's box: one token's G rows
   if (!make_tmap_bf16_3d(&tk, k, 128, Hkv, T, 64, 1, 64) ||
       !make_tmap_bf16_3d(&tv, v, 128, Hkv, T, 64, 1, 64) ||
       !make_tmap_f32_3d(&tdq, dq_acc, 128, p.num_q_heads, T, 32, box_rows, 1)) {
@@ -655,7 +674,7 @@ sas_status launch_attn_bwd_km(const sas_problem& p, const void* q, const void* k
   a.G = G;
   a.Hs = Hs;
   a.R = Hs / Hkv;
-  a.Mq = tc_rows_per_tile(G);
+  a.Mq = 4 * (32 / G);   // whole tokens per warp (G = 5: 24 tokens, 120 of the 128 rows)
   a.P = lists.P;
   a.K1 = p.topk + 1;
   a.scale = 1.f / sqrtf(128.f);

@@ -4,7 +4,8 @@
 // normalisation, gate RoPE, Top-K 31 historical blocks); paper abstract (softmax gates over
 // the history plus the always-retained current block; Top-K keeps the computation sparse).
 //
-// CTA = (TQ-token tile of one sequence, kv head), 256 threads:
+// CTA = (TQ-token tile of one sequence, gate head), 512 threads (one CTA per SM: the score
+// rows fill most of the shared memory, so the CTA brings its own warps to hide latency):
 //   1. q~_t: the tensor-core query projection of each token (sas_gate_tc.cu), RMSNorm with
 //      its weight, rotary at t; kept transposed in shared memory.
 //   2. the current block's key from the tensor-core projection of its visible prefix,
@@ -26,12 +27,13 @@
 namespace sas {
 namespace gsel {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 constexpr int kH = 128;   // gate hidden size of the fused path
+constexpr int kRT = 2;    // tokens per thread in the score GEMM (x 4 blocks)
 
 template <int TQ>
 struct Cfg {
-  static constexpr int NTY = TQ / 4;           // groups of 4 tokens
+  static constexpr int NTY = TQ / kRT;         // groups of kRT tokens
   static constexpr int NTX = kThreads / NTY;   // groups of 4 blocks
   static constexpr int CHUNK = NTX * 4;        // cached block keys staged per step
   static constexpr int QS = TQ + 4;            // row stride of the transposed q~ tile
@@ -50,7 +52,7 @@ size_t smem_bytes(int NBmax) {
 }
 
 template <int TQ>
-__global__ void __launch_bounds__(kThreads) gate_select_kernel(
+__global__ void __launch_bounds__(kThreads, 1) gate_select_kernel(
     const float* __restrict__ qproj, const float* __restrict__ kproj,
     const float* __restrict__ gkeys, const float* __restrict__ qnorm_w,
     const float* __restrict__ knorm_w, const int32_t* __restrict__ cu,
@@ -125,25 +127,25 @@ __global__ void __launch_bounds__(kThreads) gate_select_kernel(
         Bs[i * C::BS + jj] = (j < cmax) ? gkeys[(((size_t)b * NBmax + j) * Hkv + kv) * kH + i] : 0.f;
       }
       __syncthreads();
-      float acc[4][4];
+      float acc[kRT][4];
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
+      for (int a = 0; a < kRT; ++a)
 #pragma unroll
         for (int o = 0; o < 4; ++o) acc[a][o] = 0.f;
 #pragma unroll 8
       for (int k = 0; k < kH; ++k) {
-        const float4 a = *reinterpret_cast<const float4*>(Qt + k * C::QS + ty * 4);
+        const float2 a = *reinterpret_cast<const float2*>(Qt + k * C::QS + ty * kRT);
         const float4 bb = *reinterpret_cast<const float4*>(Bs + k * C::BS + tx * 4);
-        const float av[4] = {a.x, a.y, a.z, a.w};
+        const float av[kRT] = {a.x, a.y};
         const float bv[4] = {bb.x, bb.y, bb.z, bb.w};
 #pragma unroll
-        for (int aa = 0; aa < 4; ++aa)
+        for (int aa = 0; aa < kRT; ++aa)
 #pragma unroll
           for (int o = 0; o < 4; ++o) acc[aa][o] = fmaf(av[aa], bv[o], acc[aa][o]);
       }
 #pragma unroll
-      for (int aa = 0; aa < 4; ++aa) {
-        const int t = ty * 4 + aa;
+      for (int aa = 0; aa < kRT; ++aa) {
+        const int t = ty * kRT + aa;
         const int ct = (t0 + t) / B;
         float* srow = S + (size_t)t * SS;
 #pragma unroll
