@@ -2,8 +2,8 @@
 """Benchmark of the SAS gated block-sparse attention hot path on B200.
 
 One step = one pass of the whole prefill/training path over the workload's inputs
-(already resident in HBM): key pooling -> gate keys -> gate scores + Top-K (one fused pass)
--> gated attention forward -> gated attention backward. The headline workload is the largest
+(already resident in HBM): key pooling -> gate keys -> gate scores -> Top-K -> gated
+attention forward -> gated attention backward. The headline workload is the largest
 single-GPU configuration, the Qwen3-14B-shaped varlen training step (4 packed sequences of
 8k..64k tokens, 40 query / 8 KV heads, Top-K 63). The Qwen3-4B 32k training step, the 32k
 forward-only prefill and the batch-64 decode step are measured beside it and reported under
@@ -251,9 +251,13 @@ def train_step(sas, prob, g, backward: bool, timer: Timer | None = None):
     pooled = run("sas_pool_keys", lambda: sas.sas_pool_keys(prob, g["k_nope"], pooled=g["_pooled"]))
     gk = run("sas_gate_keys", lambda: sas.sas_gate_keys(prob, pooled, g["wk"], g["knorm_w"],
                                                         gate_keys=g["_gk"]))
-    idx, logg = run("sas_gate_select", lambda: sas.sas_gate_select(
+    # gate scores + Top-K: the two kernels through an HBM score matrix, the faster path on
+    # B200 today (the fused pass that keeps the scores on chip is timed beside it, gate_paths)
+    scores, lse = run("sas_gate_scores", lambda: sas.sas_gate_scores(
         prob, g["q_nope"], g["k_nope"], gk, g["wq"], g["qnorm_w"], g["wk"], g["knorm_w"],
-        idx=g["_idx"], logg=g["_logg"], workspace=g["_wsg"]))
+        scores=g["_scores"], lse=g["_glse"], workspace=g["_wsgs"]))
+    idx, logg = run("sas_topk", lambda: sas.sas_topk(prob, scores, lse, idx=g["_idx"],
+                                                     logg=g["_logg"]))
     o, alse = run("sas_attn_fwd", lambda: sas.sas_attn_fwd(prob, g["q"], g["k"], g["v"], idx, logg,
                                                            o=g["_o"], lse=g["_alse"],
                                                            workspace=g["_wsf"]))
@@ -273,6 +277,8 @@ def alloc_outputs(sas, prob, g, backward):
                                prob.head_dim, prob.topk, prob.max_blocks, prob.gate_hidden)
     g["_pooled"] = torch.empty((prob.batch, NB, Hkv, 3 * d), dtype=torch.float32, device=dev)
     g["_gk"] = torch.empty((prob.batch, NB, Hkv, h), dtype=torch.float32, device=dev)
+    g["_scores"] = torch.empty((T, prob.sel_heads, NB), dtype=torch.float32, device=dev)
+    g["_glse"] = torch.empty((T, prob.sel_heads), dtype=torch.float32, device=dev)
     g["_idx"] = torch.empty((T, Hkv, K + 1), dtype=torch.int32, device=dev)
     g["_logg"] = torch.empty((T, Hkv, K + 1), dtype=torch.float32, device=dev)
     g["_o"] = torch.empty((T, Hq, d), dtype=prob.dtype, device=dev)
@@ -281,6 +287,8 @@ def alloc_outputs(sas, prob, g, backward):
     n = ctypes.c_size_t(0)
     lib.sas_gate_select_workspace_size(prob.ref, ctypes.byref(n))
     g["_wsg"] = torch.empty(max(256, n.value), dtype=torch.uint8, device=dev)
+    lib.sas_gate_scores_workspace_size(prob.ref, ctypes.byref(n))
+    g["_wsgs"] = torch.empty(max(256, n.value), dtype=torch.uint8, device=dev)
     lib.sas_attn_fwd_workspace_size(prob.ref, ctypes.byref(n))
     g["_wsf"] = torch.empty(max(256, n.value), dtype=torch.uint8, device=dev)
     if backward:
@@ -296,10 +304,7 @@ def bench_gate_paths(sas, prob, g, flush, steps):
     """Gate scores + Top-K two ways on the step's inputs: the fused pass (score rows kept on
     chip) and the two separate kernels (the [T, Hs, NBmax] scores written to and read back
     from HBM). Both give the same selection; timed after the step, not part of it."""
-    scores = torch.empty((prob.total_tokens, prob.sel_heads, prob.max_blocks), dtype=torch.float32,
-                         device=prob.device)
-    lse = torch.empty((prob.total_tokens, prob.sel_heads), dtype=torch.float32, device=prob.device)
-    wsu = sas.gate_scores_workspace(prob)
+    scores, lse, wsu = g["_scores"], g["_glse"], g["_wsgs"]
     args = (prob, g["q_nope"], g["k_nope"], g["_gk"], g["wq"], g["qnorm_w"], g["wk"], g["knorm_w"])
 
     def fused():
@@ -324,7 +329,7 @@ def bench_gate_paths(sas, prob, g, flush, steps):
         torch.cuda.synchronize()
         out[name] = sum(x.elapsed_time(y) for x, y in ev) / len(ev)
     out["score_bytes_avoided"] = 2 * scores.numel() * 4
-    del scores
+    sas.check_workspace(g["_wsg"], "sas_gate_select")
     return out
 
 
@@ -482,7 +487,7 @@ def setup_workload(sas, name, dev):
 
 def check_error_words(sas, g, backward):
     """The device-side error words of the step's last calls (0 = none); raises otherwise."""
-    sas.check_workspace(g["_wsg"], "sas_gate_select")
+    sas.check_workspace(g["_wsgs"], "sas_gate_scores")
     sas.check_workspace(g["_wsf"], "sas_attn_fwd")
     if backward:
         sas.check_workspace(g["_wsb"], "sas_attn_bwd")

@@ -208,25 +208,17 @@ __global__ void __launch_bounds__(kmb::kThreads, 1)
       }
       ++item_seq;
       const int ntile = (cnt + Mq - 1) / Mq;
-      // the row's list entry and its LSE and D are loaded one tile ahead, so a tile's gather
-      // waits for one L2 round trip (the Q / dO rows) instead of three dependent ones
       int2 nxt = make_int2(0, 0);
-      float nxt_lse = 0.f, nxt_d = 0.f;
-      if (row_ok && tl < cnt) {
-        nxt = a.list[off + tl];
-        const size_t qr0 = (size_t)(nxt.x & 0xFFFFFF) * a.Hq + kv * G + g;
-        nxt_lse = a.lse[qr0];
-        nxt_d = a.drow[qr0];
-      }
+      if (row_ok && tl < cnt) nxt = a.list[off + tl];
       for (int m = 0; m < ntile; ++m, ++n) {
         const int rank = m * Mq + tl;
         const bool valid = row_ok && rank < cnt;
         const int2 ent = nxt;
-        const float lse_v = nxt_lse, d_v = nxt_d;
-        const bool more = row_ok && rank + Mq < cnt;
-        if (more) nxt = a.list[off + rank + Mq];   // next tile's entry
+        if (row_ok && rank + Mq < cnt) nxt = a.list[off + rank + Mq];   // next tile's entry
         const int tg = ent.x & 0xFFFFFF, slot = ent.x >> 24;
         const size_t qrow = (size_t)tg * a.Hq + kv * G + g;
+        const float lse_v = valid ? a.lse[qrow] : 0.f;
+        const float d_v = valid ? a.drow[qrow] : 0.f;
         const int qs = n & 1, rs = n & 3;
         if (ok && n >= 2 && !mbar_wait(qd_empty + qs, ((n >> 1) - 1) & 1, abort_flag)) {
           tc_fail(a.err, 72, abort_flag);
@@ -256,13 +248,8 @@ __global__ void __launch_bounds__(kmb::kThreads, 1)
             st_shared_v4(do_dst + o, 0u, 0u, 0u, 0u);
           }
         }
-        if (more) {   // the next tile's LSE and D (its list entry has arrived by now)
-          const size_t nq = (size_t)(nxt.x & 0xFFFFFF) * a.Hq + kv * G + g;
-          nxt_lse = a.lse[nq];
-          nxt_d = a.drow[nq];
-        }
         rcf[rc_slot(rs, 0) + r] = valid ? (__int_as_float(ent.y) - lse_v) * kLog2e : -INFINITY;
-        rcf[rc_slot(rs, 1) + r] = valid ? d_v : 0.f;
+        rcf[rc_slot(rs, 1) + r] = d_v;
         rci[rc_slot(rs, 2) + r] = valid ? min(kB - 1, tg - key0) : -1;
         rci[rc_slot(rs, 3) + r] = valid ? (int)qrow : -1;
         rci[rc_slot(rs, 4) + r] = valid ? (tg * a.Hs + kv) * a.K1 + slot : -1;

@@ -263,23 +263,16 @@ __global__ void __launch_bounds__(kmf::kThreads, 1)
       ++item_seq;
       const int ntile = (cnt + Mq - 1) / Mq;
       const int jk0 = j * kB;
-      // the row's list entry and reference logit are loaded one tile ahead, so a tile's
-      // gather waits for one L2 round trip (the Q row) instead of two dependent ones
       int2 nxt = make_int2(0, 0);
-      float nxt_mr = 0.f;
-      if (row_ok && tl < cnt) {
-        nxt = a.list[off + tl];
-        nxt_mr = a.mref[(size_t)(nxt.x & 0xFFFFFF) * a.Hq + kv * G + g];
-      }
+      if (row_ok && tl < cnt) nxt = a.list[off + tl];
       for (int m = 0; m < ntile; ++m, ++n) {
         const int rank = m * Mq + tl;
         const bool valid = row_ok && rank < cnt;
         const int2 ent = nxt;
-        const float mr = valid ? nxt_mr : 0.f;
-        const bool more = row_ok && rank + Mq < cnt;
-        if (more) nxt = a.list[off + rank + Mq];   // next tile's entry
+        if (row_ok && rank + Mq < cnt) nxt = a.list[off + rank + Mq];   // next tile's entry
         const int tg = ent.x & 0xFFFFFF;
         const size_t qrow = (size_t)tg * a.Hq + kv * G + g;
+        const float mr = valid ? a.mref[qrow] : 0.f;
         const int qs = n & 1, rs = n & 3;
         if (ok && n >= 2 && !mbar_wait(q_empty + qs, ((n >> 1) - 1) & 1, abort_flag)) {
           tc_fail(a.err, 52, abort_flag);
@@ -301,8 +294,6 @@ __global__ void __launch_bounds__(kmf::kThreads, 1)
           for (int c = 0; c < 16; ++c)
             st_shared_v4(q_dst + (uint32_t)((c >> 3) * kQHalf + (c & 7) * 16), 0u, 0u, 0u, 0u);
         }
-        if (more)   // the next tile's reference (its list entry has arrived by now)
-          nxt_mr = a.mref[(size_t)(nxt.x & 0xFFFFFF) * a.Hq + kv * G + g];
         float* rcb = rcf + rs * 3 * kM;
         rcb[r] = valid ? __int_as_float(ent.y) * kLog2e - mr : -INFINITY;
         // last visible key column of block j for this row (all 64 unless j is its current block)

@@ -47,7 +47,7 @@ __device__ __forceinline__ float block_reduce_max(float v, float* red) {
 // at c*B), scores against the cached block keys, logsumexp over j <= c, Top-K over j < c.
 // ---------------------------------------------------------------------------------------
 template <typename T, int H, int NPT>
-__global__ void __launch_bounds__(kDecThreads, 3) decode_gate_kernel(
+__global__ void __launch_bounds__(kDecThreads) decode_gate_kernel(
     const T* __restrict__ q_nope, const __nv_bfloat16* __restrict__ gkc,
     const float* __restrict__ cur_pool, const T* __restrict__ wq, const float* __restrict__ qnorm_w,
     const T* __restrict__ wk, const float* __restrict__ knorm_w, const int32_t* __restrict__ seqlens,
@@ -116,9 +116,8 @@ __global__ void __launch_bounds__(kDecThreads, 3) decode_gate_kernel(
     P[e] = (part == 2) ? x / (float)n : x;
   }
   __syncthreads();
-  // projections: warp-coalesced weight rows (lanes across the input, 16-byte loads), four
-  // output channels per warp step with all their loads issued before any arithmetic (three
-  // CTAs per SM keep enough of these steps in flight)
+  // projections: warp-coalesced weight rows (lanes across the input, 16-byte loads), eight
+  // output channels per warp step with all their loads issued before any arithmetic
   if constexpr (!std::is_same<T, __nv_bfloat16>::value) {   // fp32 weights: one row per step
     for (int job = warp; job < 2 * H; job += kDecWarps) {
       const bool isq = job < H;
@@ -137,7 +136,7 @@ __global__ void __launch_bounds__(kDecThreads, 3) decode_gate_kernel(
       if (lane == 0) (isq ? xq : xk)[i] = acc;
     }
   } else {
-    constexpr int R = 4;
+    constexpr int R = 8;
     for (int job0 = warp * R; job0 < 2 * H; job0 += kDecWarps * R) {
       const bool isq = job0 < H;   // H is a multiple of 8: a step never mixes q and k rows
       const int i0 = isq ? job0 : job0 - H;
