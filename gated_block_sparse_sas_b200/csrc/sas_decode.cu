@@ -756,9 +756,20 @@ int decode_nsplit(const sas_decode_problem& p) {
 // one's latency hides behind the other's streaming. Each chunk is an independent sub-problem
 // (its sequences' rows of every batch-indexed tensor) with its own workspace region.
 // ---------------------------------------------------------------------------------------
+#ifndef SAS_DECODE_CHUNKS
+#define SAS_DECODE_CHUNKS 4        // most chunks a batch is split into (1: no chunks)
+#endif
+#ifndef SAS_DECODE_CHUNK_NS_LOCAL
+#define SAS_DECODE_CHUNK_NS_LOCAL 0   // 1: each chunk's split count from its own pairs
+#endif
+
 static int decode_chunks(const sas_decode_problem& p) {
-  if ((size_t)p.batch * gate_heads(p) < 256 || p.batch < 8) return 1;
-  return p.batch >= 32 ? 4 : 2;
+  if (SAS_DECODE_CHUNKS <= 1 || (size_t)p.batch * gate_heads(p) < 256 || p.batch < 8) return 1;
+  return p.batch >= 32 ? std::min(8, SAS_DECODE_CHUNKS) : std::min(2, SAS_DECODE_CHUNKS);
+}
+
+static int decode_chunk_nsplit(const sas_decode_problem& whole, const sas_decode_problem& chunk) {
+  return SAS_DECODE_CHUNK_NS_LOCAL ? decode_nsplit(chunk) : decode_nsplit(whole);
 }
 
 static sas_decode_problem decode_chunk(const sas_decode_problem& p, int c, int nc, int* b0) {
@@ -787,7 +798,8 @@ size_t decode_workspace_bytes(const sas_decode_problem& p) {
   const int nc = decode_chunks(p);
   for (int c = 0; c < nc; ++c) {
     int b0 = 0;
-    total += decode_chunk_bytes(decode_chunk(p, c, nc, &b0), decode_nsplit(p));
+    const sas_decode_problem ch = decode_chunk(p, c, nc, &b0);
+    total += decode_chunk_bytes(ch, nc == 1 ? decode_nsplit(p) : decode_chunk_nsplit(p, ch));
   }
   return total;
 }
@@ -920,7 +932,7 @@ static sas_status launch_decode_part(const sas_decode_problem& p, const void* q,
 namespace {
 struct DecodeSide {
   cudaStream_t stream = nullptr;
-  cudaEvent_t ev[4] = {};
+  cudaEvent_t ev[8] = {};
 };
 std::mutex g_side_mu;
 DecodeSide g_side[64];
@@ -983,7 +995,8 @@ sas_status launch_decode(const sas_decode_problem& p, const void* q, const void*
     float* lg;
     char* w;
     DecodePaging pg;
-  } part[4];
+    int ns;
+  } part[8];
   for (int c = 0; c < nc; ++c) {   // chunk c: its sequences' rows of every batch-indexed tensor
     int b0 = 0;
     Part& x = part[c];
@@ -1005,14 +1018,15 @@ sas_status launch_decode(const sas_decode_problem& p, const void* q, const void*
       x.vc = (const char*)v_cache + (size_t)b0 * Hkv * p.capacity * d * esz;
       x.gk = (const char*)gkc + (size_t)b0 * Hkv * NBmax * p.gate_hidden * 2;
     }
+    x.ns = decode_chunk_nsplit(p, x.p);
     x.w = w;
-    w += decode_chunk_bytes(x.p, ns);
+    w += decode_chunk_bytes(x.p, x.ns);
   }
   auto run = [&](int c, bool gate, bool attn, cudaStream_t s) {
     const Part& x = part[c];
     if (x.p.batch <= 0) return SAS_OK;
     return launch_decode_part(x.p, x.q, x.qn, x.kc, x.vc, x.gk, x.pool, wq, qnorm_w, wk, knorm_w,
-                              x.o, x.idx, x.lg, x.w, err, x.pg, ns, gate, attn, s);
+                              x.o, x.idx, x.lg, x.w, err, x.pg, x.ns, gate, attn, s);
   };
   // caller's stream: gate 0, attention 0, then attention c once the side stream's gate c is done;
   // side stream: gates 1 .. nc-1 in order, starting when gate 0 is done

@@ -447,7 +447,7 @@ def test_decode_paged_equals_contiguous(sas, name):
     assert torch.equal(o_p, o_c)
     # a bad page id in sequence 0's history
     bad = pt.clone()
-    bad[0, 3] = n_pages + 5
+    bad[0, 0] = n_pages + 5   # block 0 is read by every sequence
     ws = sas._workspace(sas.lib_handle().sas_decode_workspace_size, prob.ref, prob.device)
     o_b = sas.sas_decode_paged(prob, bad, n_pages, g["q"], g["q_nope"], kp, vp, gp, *common,
                                workspace=ws)
