@@ -228,24 +228,29 @@ __global__ void __launch_bounds__(kmb::kThreads, 1)
           tc_fail(a.err, 73, abort_flag);
           ok = false;
         }
+        ok = __all_sync(0xffffffffu, ok);   // warp-uniform: the copies below are cooperative
         if (!ok) continue;   // keep the loop shape: the item fetch barriers stay matched
-        const uint32_t q_dst = smem_u32(sm + OFF_QD + qs * kStage) + r * 128;
-        const uint32_t do_dst = q_dst + kTile;
-        if (valid) {
-          const __nv_bfloat16* qsrc = a.q + qrow * kD;
-          const __nv_bfloat16* dsrc = a.dout + qrow * kD;
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const uint32_t o = (uint32_t)((c >> 3) * kHalf + (((c & 7) ^ (r & 7)) << 4));
-            cp_async16(q_dst + o, qsrc + c * 8);
-            cp_async16(do_dst + o, dsrc + c * 8);
-          }
-        } else {   // rows past the list: finite zeros (0 * garbage could be NaN in the MMAs)
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const uint32_t o = (uint32_t)((c >> 3) * kHalf + (c & 7) * 16);
-            st_shared_v4(q_dst + o, 0u, 0u, 0u, 0u);
-            st_shared_v4(do_dst + o, 0u, 0u, 0u, 0u);
+        // the warp's 32 rows, two rows per step: lane l copies 16-byte piece l & 15 of row
+        // 2 i + (l >> 4), so each copy instruction reads two whole 256-byte rows (coalesced)
+        // instead of one 16-byte piece of 32 rows; rows past the list become zeros (0 times
+        // garbage could be NaN in the MMAs)
+        {
+          const uint32_t stage = smem_u32(sm + OFF_QD + qs * kStage);
+          const long long my_row = valid ? (long long)qrow : -1ll;
+          const int c = lane & 15;
+#pragma unroll 4
+          for (int i = 0; i < 16; ++i) {
+            const int rr = 2 * i + (lane >> 4);
+            const long long row = __shfl_sync(0xffffffffu, my_row, rr);
+            const int R = (r & ~31) + rr;   // tile row
+            const uint32_t o = (uint32_t)(R * 128 + (c >> 3) * kHalf + (((c & 7) ^ (R & 7)) << 4));
+            if (row >= 0) {
+              cp_async16(stage + o, a.q + row * kD + c * 8);
+              cp_async16(stage + kTile + o, a.dout + row * kD + c * 8);
+            } else {
+              st_shared_v4(stage + o, 0u, 0u, 0u, 0u);
+              st_shared_v4(stage + kTile + o, 0u, 0u, 0u, 0u);
+            }
           }
         }
         rcf[rc_slot(rs, 0) + r] = valid ? (__int_as_float(ent.y) - lse_v) * kLog2e : -INFINITY;
@@ -336,12 +341,13 @@ __global__ void __launch_bounds__(kmb::kThreads, 1)
           mma_bf16_ss(tmem + kColDK, sdesc_sw128(q_addr + kk * 2048, kHalf, 1024),
                       sdesc_sw128(ds_addr + kk * 2048, kHalf, 1024), kIdKV,
                       (!first || kk > 0) ? 1u : 0u);
+        // the tile's Q/dO stage is read by no later MMA: release it to the gather before dQ
+        tc_commit(qd_empty + (m & 1));
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)   // dQ = dS K: A = dS (K-major), B = K (MN-major)
           mma_bf16_ss(tmem + kColDQ + (m & 1) * kD, sdesc_sw128(ds_addr + kk * 32, 16, 1024),
                       sdesc_sw128(k_addr + kk * 2048, kKVHalf, 1024), kIdQ, kk > 0 ? 1u : 0u);
         tc_commit(ps_empty);
-        tc_commit(qd_empty + (m & 1));   // the tile's Q/dO stage is read by no later MMA
         tc_commit(dq_full + (m & 1));
         if (flags & kFlagLast) tc_commit(kv_empty);
       };

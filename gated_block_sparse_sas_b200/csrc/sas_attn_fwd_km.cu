@@ -282,17 +282,24 @@ __global__ void __launch_bounds__(kmf::kThreads, 1)
           tc_fail(a.err, 53, abort_flag);
           ok = false;
         }
+        ok = __all_sync(0xffffffffu, ok);   // warp-uniform: the copies below are cooperative
         if (!ok) continue;   // keep the loop shape: the item fetch barriers stay matched
-        const uint32_t q_dst = q_row_dst + qs * kQStage;
-        if (valid) {
-          const __nv_bfloat16* src = a.q + qrow * kD;
-#pragma unroll
-          for (int c = 0; c < 16; ++c)
-            cp_async16(q_dst + (uint32_t)((c >> 3) * kQHalf + (((c & 7) ^ (r & 7)) << 4)), src + c * 8);
-        } else {   // rows past the list: finite zeros (0 * garbage could be NaN in the MMA)
-#pragma unroll
-          for (int c = 0; c < 16; ++c)
-            st_shared_v4(q_dst + (uint32_t)((c >> 3) * kQHalf + (c & 7) * 16), 0u, 0u, 0u, 0u);
+        // the warp's 32 rows, two rows per step: lane l copies 16-byte piece l & 15 of row
+        // 2 i + (l >> 4) (two whole 256-byte rows per copy instruction); rows past the list
+        // become finite zeros (0 times garbage could be NaN in the MMA)
+        {
+          const uint32_t stage = smem_u32(sm + OFF_Q) + qs * kQStage;
+          const long long my_row = valid ? (long long)qrow : -1ll;
+          const int c = lane & 15;
+#pragma unroll 4
+          for (int i = 0; i < 16; ++i) {
+            const int rr = 2 * i + (lane >> 4);
+            const long long row = __shfl_sync(0xffffffffu, my_row, rr);
+            const int R = (r & ~31) + rr;   // tile row
+            const uint32_t o = (uint32_t)(R * 128 + (c >> 3) * kQHalf + (((c & 7) ^ (R & 7)) << 4));
+            if (row >= 0) cp_async16(stage + o, a.q + row * kD + c * 8);
+            else st_shared_v4(stage + o, 0u, 0u, 0u, 0u);
+          }
         }
         float* rcb = rcf + rs * 3 * kM;
         rcb[r] = valid ? __int_as_float(ent.y) * kLog2e - mr : -INFINITY;

@@ -8,8 +8,6 @@
 // (3) merge of the splits -> O. The attention only ever reads the selected blocks.
 #include <math.h>
 
-#include <algorithm>
-#include <mutex>
 #include <type_traits>
 
 #include "sas_common.cuh"
@@ -749,59 +747,13 @@ int decode_nsplit(const sas_decode_problem& p) {
   return ns;
 }
 
-// ---------------------------------------------------------------------------------------
-// Batch chunks. The gate of a (sequence, gate head) is a chain of dependent latency-bound
-// steps; the attention streams K/V from HBM. A large batch is split into chunks: the gate of
-// chunk c + 1 runs on a side stream while chunk c's attention runs on the caller's stream, so
-// one's latency hides behind the other's streaming. Each chunk is an independent sub-problem
-// (its sequences' rows of every batch-indexed tensor) with its own workspace region.
-// ---------------------------------------------------------------------------------------
-#ifndef SAS_DECODE_CHUNKS
-#define SAS_DECODE_CHUNKS 4        // most chunks a batch is split into (1: no chunks)
-#endif
-#ifndef SAS_DECODE_CHUNK_NS_LOCAL
-#define SAS_DECODE_CHUNK_NS_LOCAL 0   // 1: each chunk's split count from its own pairs
-#endif
-
-static int decode_chunks(const sas_decode_problem& p) {
-  if (SAS_DECODE_CHUNKS <= 1 || (size_t)p.batch * gate_heads(p) < 256 || p.batch < 8) return 1;
-  return p.batch >= 32 ? std::min(8, SAS_DECODE_CHUNKS) : std::min(2, SAS_DECODE_CHUNKS);
-}
-
-static int decode_chunk_nsplit(const sas_decode_problem& whole, const sas_decode_problem& chunk) {
-  return SAS_DECODE_CHUNK_NS_LOCAL ? decode_nsplit(chunk) : decode_nsplit(whole);
-}
-
-static sas_decode_problem decode_chunk(const sas_decode_problem& p, int c, int nc, int* b0) {
-  const int per = (p.batch + nc - 1) / nc;
-  *b0 = std::min(p.batch, c * per);
-  sas_decode_problem s = p;
-  s.batch = std::min(per, p.batch - *b0);
-  s.seqlens = p.seqlens + *b0;
-  return s;
-}
-
-static size_t al256d(size_t x) { return (x + 255) & ~(size_t)255; }
-
-// per chunk: selection (ids, log-gates) and the split-K partials (m, l; acc) for ns splits
-// (the whole batch's split count: a chunk's attention is as wide per pair as the whole one's)
-static size_t decode_chunk_bytes(const sas_decode_problem& s, int ns) {
-  if (s.batch <= 0) return 0;
-  const int G = s.num_q_heads / gate_heads(s);
-  const size_t pairs = (size_t)s.batch * gate_heads(s);
-  return al256d(pairs * (s.topk + 1) * 4) * 2 + al256d(pairs * ns * G * 2 * 4) +
-         al256d(pairs * ns * G * s.head_dim * 4);
-}
-
 size_t decode_workspace_bytes(const sas_decode_problem& p) {
-  size_t total = 256;   // error word
-  const int nc = decode_chunks(p);
-  for (int c = 0; c < nc; ++c) {
-    int b0 = 0;
-    const sas_decode_problem ch = decode_chunk(p, c, nc, &b0);
-    total += decode_chunk_bytes(ch, nc == 1 ? decode_nsplit(p) : decode_chunk_nsplit(p, ch));
-  }
-  return total;
+  const int G = p.num_q_heads / gate_heads(p);
+  const size_t pairs = (size_t)p.batch * gate_heads(p);
+  const size_t ns = decode_nsplit(p);
+  auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  return 256 /* error word */ + al(pairs * (p.topk + 1) * 4) * 2 + al(pairs * ns * G * 2 * 4) +
+         al(pairs * ns * G * p.head_dim * 4);
 }
 
 template <int G>
@@ -880,33 +832,39 @@ static void decode_gate_launch(const sas_decode_problem& p, const void* q_nope, 
 #undef SAS_DG
 }
 
-// One chunk (or the whole batch): gate + Top-K, then split-K attention and merge, on `st`.
-static sas_status launch_decode_part(const sas_decode_problem& p, const void* q,
-                                     const void* q_nope, const void* k_cache, const void* v_cache,
-                                     const void* gkc, const float* cur_pool, const void* wq,
-                                     const float* qnorm_w, const void* wk, const float* knorm_w,
-                                     void* o, int32_t* idx_out, float* logg_out, char* w, int* err,
-                                     const DecodePaging& pg, int ns, bool gate, bool attn,
-                                     cudaStream_t st) {
+sas_status launch_decode(const sas_decode_problem& p, const void* q, const void* q_nope,
+                         const void* k_cache, const void* v_cache, const void* gkc,
+                         const float* cur_pool, const void* wq, const float* qnorm_w,
+                         const void* wk, const float* knorm_w, void* o, int32_t* idx_out,
+                         float* logg_out, void* ws, const DecodePaging& pg, cudaStream_t st) {
   const int G = p.num_q_heads / gate_heads(p);   // query heads per gate head
   const size_t pairs = (size_t)p.batch * gate_heads(p);
-  int32_t* sel_idx = (int32_t*)w;
-  w += al256d(pairs * (p.topk + 1) * 4);
-  float* sel_logg = (float*)w;
-  w += al256d(pairs * (p.topk + 1) * 4);
-  float* part_ml = (float*)w;
-  w += al256d(pairs * ns * G * 2 * 4);
-  float* part_acc = (float*)w;
-  if (gate) {
-    if (p.dtype == SAS_BF16)
-      decode_gate_launch<__nv_bfloat16>(p, q_nope, gkc, cur_pool, wq, qnorm_w, wk, knorm_w,
-                                        sel_idx, sel_logg, idx_out, logg_out, pg, err, st);
-    else
-      decode_gate_launch<float>(p, q_nope, gkc, cur_pool, wq, qnorm_w, wk, knorm_w, sel_idx,
-                                sel_logg, idx_out, logg_out, pg, err, st);
-    SAS_TRY(launch_status("decode gate", 1));
+  const int ns = decode_nsplit(p);
+  auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  char* w = (char*)ws;
+  // word 0: this call's error code (0 = none), cleared first so it never reports an earlier call
+  int* err = (int*)w;
+  if (cudaMemsetAsync(err, 0, sizeof(int), st) != cudaSuccess) {
+    set_error("decode: clearing the error word failed");
+    return SAS_ERR_CUDA;
   }
-  if (!attn) return SAS_OK;
+  w += 256;
+  int32_t* sel_idx = (int32_t*)w;
+  w += al(pairs * (p.topk + 1) * 4);
+  float* sel_logg = (float*)w;
+  w += al(pairs * (p.topk + 1) * 4);
+  float* part_ml = (float*)w;
+  w += al(pairs * ns * G * 2 * 4);
+  float* part_acc = (float*)w;
+  w += al(pairs * ns * G * p.head_dim * 4);
+  if (p.dtype == SAS_BF16)
+    decode_gate_launch<__nv_bfloat16>(p, q_nope, gkc, cur_pool, wq, qnorm_w, wk, knorm_w, sel_idx,
+                                      sel_logg, idx_out, logg_out, pg, err, st);
+  else
+    decode_gate_launch<float>(p, q_nope, gkc, cur_pool, wq, qnorm_w, wk, knorm_w, sel_idx, sel_logg,
+                              idx_out, logg_out, pg, err, st);
+  sas_status s = launch_status("decode gate", 1);
+  if (s != SAS_OK) return s;
 #define SAS_DA(T, D, G)                                                                      \
   decode_attn_launch<T, D, G>(p, q, k_cache, v_cache, sel_idx, sel_logg, part_ml, part_acc, err, \
                               o, ns, pg, st)
@@ -926,131 +884,6 @@ static sas_status launch_decode_part(const sas_decode_problem& p, const void* q,
 #undef SAS_DA_G
 #undef SAS_DA
   return launch_status("decode attention", 2);
-}
-
-// The side stream and events of the batch chunks, one set per device, made on first use.
-namespace {
-struct DecodeSide {
-  cudaStream_t stream = nullptr;
-  cudaEvent_t ev[8] = {};
-};
-std::mutex g_side_mu;
-DecodeSide g_side[64];
-}  // namespace
-
-static sas_status decode_side(DecodeSide** out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
-    set_error("decode: no usable current device");
-    return SAS_ERR_CUDA;
-  }
-  std::lock_guard<std::mutex> lock(g_side_mu);
-  DecodeSide& d = g_side[dev];
-  if (d.stream == nullptr) {
-    int lo = 0, hi = 0;   // the gates get the higher priority: their CTAs start first
-    cudaDeviceGetStreamPriorityRange(&lo, &hi);
-    if (cudaStreamCreateWithPriority(&d.stream, cudaStreamNonBlocking, hi) != cudaSuccess) {
-      set_error("decode: creating the side stream failed");
-      return SAS_ERR_CUDA;
-    }
-    for (auto& e : d.ev)
-      if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) {
-        set_error("decode: creating the chunk events failed");
-        return SAS_ERR_CUDA;
-      }
-  }
-  *out = &d;
-  return SAS_OK;
-}
-
-sas_status launch_decode(const sas_decode_problem& p, const void* q, const void* q_nope,
-                         const void* k_cache, const void* v_cache, const void* gkc,
-                         const float* cur_pool, const void* wq, const float* qnorm_w,
-                         const void* wk, const float* knorm_w, void* o, int32_t* idx_out,
-                         float* logg_out, void* ws, const DecodePaging& pg, cudaStream_t st) {
-  char* w = (char*)ws;
-  // word 0: this call's error code (0 = none), cleared first so it never reports an earlier call
-  int* err = (int*)w;
-  if (cudaMemsetAsync(err, 0, sizeof(int), st) != cudaSuccess) {
-    set_error("decode: clearing the error word failed");
-    return SAS_ERR_CUDA;
-  }
-  w += 256;
-  const int nc = decode_chunks(p);
-  const int ns = decode_nsplit(p);
-  if (nc == 1)
-    return launch_decode_part(p, q, q_nope, k_cache, v_cache, gkc, cur_pool, wq, qnorm_w, wk,
-                              knorm_w, o, idx_out, logg_out, w, err, pg, ns, true, true, st);
-  DecodeSide* side = nullptr;
-  SAS_TRY(decode_side(&side));
-  const size_t esz = p.dtype == SAS_BF16 ? 2 : 4;
-  const int Hs = gate_heads(p), Hkv = p.num_kv_heads, d = p.head_dim;
-  const int NBmax = (p.capacity + p.block - 1) / p.block;
-  struct Part {
-    sas_decode_problem p;
-    const char *q, *qn, *kc, *vc, *gk;
-    const float* pool;
-    char* o;
-    int32_t* idx;
-    float* lg;
-    char* w;
-    DecodePaging pg;
-    int ns;
-  } part[8];
-  for (int c = 0; c < nc; ++c) {   // chunk c: its sequences' rows of every batch-indexed tensor
-    int b0 = 0;
-    Part& x = part[c];
-    x.p = decode_chunk(p, c, nc, &b0);
-    x.q = (const char*)q + (size_t)b0 * p.num_q_heads * d * esz;
-    x.qn = (const char*)q_nope + (size_t)b0 * p.num_q_heads * d * esz;
-    x.o = (char*)o + (size_t)b0 * p.num_q_heads * d * esz;
-    x.pool = cur_pool + (size_t)b0 * Hkv * 3 * d;
-    x.idx = idx_out ? idx_out + (size_t)b0 * Hs * (p.topk + 1) : nullptr;
-    x.lg = logg_out ? logg_out + (size_t)b0 * Hs * (p.topk + 1) : nullptr;
-    x.pg = pg;
-    if (pg.pt != nullptr) {   // page pools are shared; the page table has a row per sequence
-      x.kc = (const char*)k_cache;
-      x.vc = (const char*)v_cache;
-      x.gk = (const char*)gkc;
-      x.pg.pt = pg.pt + (size_t)b0 * NBmax;
-    } else {
-      x.kc = (const char*)k_cache + (size_t)b0 * Hkv * p.capacity * d * esz;
-      x.vc = (const char*)v_cache + (size_t)b0 * Hkv * p.capacity * d * esz;
-      x.gk = (const char*)gkc + (size_t)b0 * Hkv * NBmax * p.gate_hidden * 2;
-    }
-    x.ns = decode_chunk_nsplit(p, x.p);
-    x.w = w;
-    w += decode_chunk_bytes(x.p, x.ns);
-  }
-  auto run = [&](int c, bool gate, bool attn, cudaStream_t s) {
-    const Part& x = part[c];
-    if (x.p.batch <= 0) return SAS_OK;
-    return launch_decode_part(x.p, x.q, x.qn, x.kc, x.vc, x.gk, x.pool, wq, qnorm_w, wk, knorm_w,
-                              x.o, x.idx, x.lg, x.w, err, x.pg, x.ns, gate, attn, s);
-  };
-  // caller's stream: gate 0, attention 0, then attention c once the side stream's gate c is done;
-  // side stream: gates 1 .. nc-1 in order, starting when gate 0 is done
-  SAS_TRY(run(0, true, false, st));
-  if (cudaEventRecord(side->ev[0], st) != cudaSuccess ||
-      cudaStreamWaitEvent(side->stream, side->ev[0], 0) != cudaSuccess) {
-    set_error("decode: ordering the chunk streams failed");
-    return SAS_ERR_CUDA;
-  }
-  for (int c = 1; c < nc; ++c) {
-    SAS_TRY(run(c, true, false, side->stream));
-    if (cudaEventRecord(side->ev[c], side->stream) != cudaSuccess) {
-      set_error("decode: ordering the chunk streams failed");
-      return SAS_ERR_CUDA;
-    }
-  }
-  for (int c = 0; c < nc; ++c) {
-    if (c > 0 && cudaStreamWaitEvent(st, side->ev[c], 0) != cudaSuccess) {
-      set_error("decode: ordering the chunk streams failed");
-      return SAS_ERR_CUDA;
-    }
-    SAS_TRY(run(c, false, true, st));
-  }
-  return SAS_OK;
 }
 
 }  // namespace sas

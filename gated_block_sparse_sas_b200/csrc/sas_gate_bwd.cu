@@ -22,6 +22,8 @@
 //   4. weight gradients as sums of outer products over rows, register-tiled 64 x 64 tiles:
 //      dWq += dxq (x) q_nope group, dWk += dxk (x) P_j + dxc (x) P_cur(t) (the prefix pools
 //      rebuilt per block by a running max / min / sum).
+#include <mutex>
+
 #include "sas_common.cuh"
 #include "sas_kernels.h"
 #include "sas_sm100.cuh"
@@ -446,11 +448,173 @@ __global__ void __launch_bounds__(64) gbw_outer_kernel(
 }
 
 // ---------------------------------------------------------------------------------------
+// (4') the two token-row outer products on the tensor cores. dW[kv] (+)= X^T Y summed over
+// the token rows t, with X = dx[t, kv, :] (fp32, split into bf16 hi + lo parts: their sum
+// carries 16 significant bits, so the products keep fp32-like accuracy) and Y the projection's
+// bf16 input row (the G query heads for dWq; the prefix pools [max | min | mean hi | mid | lo]
+// of the forward's tensor-core gate for dWk, whose three mean parts add into the same mean
+// columns of dWk). CTA = (128 columns of W, kv head, split of the rows), 128 threads:
+// warp 0 lane 0 loads 64-row chunks of X hi, X lo and Y by TMA into a 4-stage ring, warp 1
+// lane 0 issues two MMAs per 16 rows (M = 128 W rows, N = 128 W columns; both operands
+// MN-major: the rows of the chunk are the reduction dimension) into a TMEM accumulator, and
+// all four warps add the 128 x 128 fp32 result into dW with vector atomics.
+// ---------------------------------------------------------------------------------------
+namespace gwt {
+constexpr int kM = 128, kN = 128, kK = 64;   // W rows, W columns, token rows per stage
+constexpr int kStages = 4;
+constexpr int kBox = kK * 128;               // [64 rows][64 bf16]: 8 KB, 128B-swizzled
+constexpr int kStage = 6 * kBox;             // X hi (2 halves), X lo (2 halves), Y (2 halves)
+constexpr int kThreads = 128;
+constexpr int OFF_BAR = kStages * kStage;
+constexpr int OFF_MISC = OFF_BAR + (2 * kStages + 1) * 8;
+constexpr int kSmemBytes = OFF_MISC + 64 + 1024;
+}  // namespace gwt
+
+struct WgradArgs {
+  int T;             // token rows
+  int rows_per;      // rows per split (a multiple of gwt::kK)
+  int y_col0;        // Y column of W column 0 for kv head 0
+  int y_col_kv;      // Y columns between kv heads
+  float* dW;         // [Hkv][128][C]
+  int C;             // W columns
+  int mean_cols;     // > 0: W columns >= 2 * mean_cols fold onto [2 mean_cols, 3 mean_cols)
+  int* err;
+};
+
+__global__ void __launch_bounds__(gwt::kThreads)
+    gbw_wgrad_tc_kernel(const __grid_constant__ CUtensorMap tXh, const __grid_constant__ CUtensorMap tXl,
+                        const __grid_constant__ CUtensorMap tY, const WgradArgs a) {
+  using namespace gwt;
+  using namespace sm100;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = align1024(smem_raw);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n0 = blockIdx.x * kN, kv = blockIdx.y, split = blockIdx.z;
+  const int r0 = split * a.rows_per, r1 = min(a.T, r0 + a.rows_per);
+  const int nk = r1 > r0 ? (r1 - r0 + kK - 1) / kK : 0;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
+  uint64_t* empty = full + kStages;
+  uint64_t* done = empty + kStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + OFF_MISC + 4);
+  if (tid == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(full + i, 1);
+      mbar_init(empty + i, 1);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {   // TMA producer: X hi, X lo (W rows 0-63, 64-127), Y (2 halves)
+    prefetch_tmap(&tXh);
+    prefetch_tmap(&tXl);
+    prefetch_tmap(&tY);
+    const int xc = kv * kM, yc = a.y_col0 + kv * a.y_col_kv + n0;
+    int issued = 0;
+    for (int ks = 0; ks < nk; ++ks) {
+      const int st = ks % kStages;
+      if (ks >= kStages && !mbar_wait(empty + st, ((ks / kStages) - 1) & 1, abort_flag)) {
+        tc_fail(a.err, 94, abort_flag);
+        break;
+      }
+      const int row = r0 + ks * kK;   // rows past T are filled with zeros by the TMA unit
+      uint8_t* stg = sm + st * kStage;
+      mbar_arrive_expect_tx(full + st, kStage);
+      tma_load_2d(stg, &tXh, full + st, xc, row);
+      tma_load_2d(stg + kBox, &tXh, full + st, xc + 64, row);
+      tma_load_2d(stg + 2 * kBox, &tXl, full + st, xc, row);
+      tma_load_2d(stg + 3 * kBox, &tXl, full + st, xc + 64, row);
+      tma_load_2d(stg + 4 * kBox, &tY, full + st, yc, row);
+      tma_load_2d(stg + 5 * kBox, &tY, full + st, yc + 64, row);
+      issued = ks + 1;
+    }
+    for (int ks = max(0, issued - kStages); ks < issued; ++ks)
+      mbar_wait_drain(full + ks % kStages, (ks / kStages) & 1);
+  } else if (warp == 1 && lane == 0) {   // MMA issue
+    // A = X^T (M = W rows, K = token rows), B = Y (N = W columns, K = token rows): both
+    // MN-major in the chunk ([64 rows][64 elements] halves, 8 KB apart)
+    constexpr uint32_t kId = idesc_bf16_f32(kM, kN, true, true);
+    bool ok = true;
+    for (int ks = 0; ks < nk; ++ks) {
+      const int st = ks % kStages;
+      if (!mbar_wait(full + st, (ks / kStages) & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t base = smem_u32(sm + st * kStage);
+#pragma unroll
+      for (int kk = 0; kk < kK / 16; ++kk) {   // 16 token rows per MMA
+        const uint64_t bdesc = sdesc_sw128(base + 4 * kBox + kk * 2048, kBox, 1024);
+        mma_bf16_ss(tmem, sdesc_sw128(base + kk * 2048, kBox, 1024), bdesc, kId,
+                    (ks > 0 || kk > 0) ? 1u : 0u);
+        mma_bf16_ss(tmem, sdesc_sw128(base + 2 * kBox + kk * 2048, kBox, 1024), bdesc, kId, 1u);
+      }
+      tc_commit(empty + st);
+    }
+    if (!ok) tc_fail(a.err, 95, abort_flag);
+    tc_commit(done);
+    mbar_wait_drain(done, 0);
+  }
+  __syncwarp();
+  // epilogue: thread r = TMEM lane r = W row r; 128 fp32 W columns
+  const bool have = warp_wait(done, 0, abort_flag) && nk > 0;
+  if (have) {
+    tc_fence_after();
+    int col = n0;
+    if (a.mean_cols > 0 && n0 >= 2 * a.mean_cols) col = 2 * a.mean_cols;   // mean parts
+    float* drow = a.dW + ((size_t)kv * kM + tid) * a.C + col;
+    const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
+#pragma unroll 1
+    for (int c0 = 0; c0 < kN; c0 += 32) {
+      float v[32];
+      tmem_ld32(tmem + lane_addr + c0, v);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        red_add_v4(drow + c0 + 4 * i, make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]));
+    }
+  } else if (nk > 0) {
+    tc_fail(a.err, 96, abort_flag);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kN);
+  }
+}
+
+// dx fp32 -> bf16 hi + lo (hi = round(x), lo = round(x - hi))
+__global__ void gbw_split_kernel(const float4* __restrict__ x, size_t n4, uint2* __restrict__ hi,
+                                 uint2* __restrict__ lo) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const float4 v = x[i];
+    const __nv_bfloat16 h0 = __float2bfloat16_rn(v.x), h1 = __float2bfloat16_rn(v.y);
+    const __nv_bfloat16 h2 = __float2bfloat16_rn(v.z), h3 = __float2bfloat16_rn(v.w);
+    uint2 H, L;
+    H.x = sm100::pack_bf16x2(__bfloat162float(h0), __bfloat162float(h1));
+    H.y = sm100::pack_bf16x2(__bfloat162float(h2), __bfloat162float(h3));
+    L.x = sm100::pack_bf16x2(v.x - __bfloat162float(h0), v.y - __bfloat162float(h1));
+    L.y = sm100::pack_bf16x2(v.z - __bfloat162float(h2), v.w - __bfloat162float(h3));
+    hi[i] = H;
+    lo[i] = L;
+  }
+}
+
+// ---------------------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------------------
 namespace {
 struct GbwLayout {
-  size_t tc, xk, kt, dkt, dxk, dxq, dxc, total;
+  size_t tc, xk, kt, dkt, dxk, dxq, dxc, xh, xl, total;
 };
 size_t al256w(size_t x) { return (x + 255) & ~(size_t)255; }
 GbwLayout gbw_layout(const sas_problem& p) {
@@ -466,6 +630,8 @@ GbwLayout gbw_layout(const sas_problem& p) {
   L.dxk = o; o += al256w(brow);
   L.dxq = o; o += al256w(trow);
   L.dxc = o; o += al256w(trow);
+  L.xh = o;  o += al256w(trow / 2);   // dx as bf16 hi / lo parts for the tensor-core products
+  L.xl = o;  o += al256w(trow / 2);
   L.total = o;
   return L;
 }
@@ -504,7 +670,9 @@ sas_status launch_gate_bwd(const sas_problem& p, const void* q_nope, const void*
     return SAS_ERR_CUDA;
   }
   float *xq_all = nullptr, *xc_all = nullptr;
-  SAS_TRY(launch_gate_proj_tc(p, q_nope, k_nope, wq, wk, ws + L.tc, &xq_all, &xc_all, st));
+  const void* prefix_rows = nullptr;
+  SAS_TRY(launch_gate_proj_tc(p, q_nope, k_nope, wq, wk, ws + L.tc, &xq_all, &xc_all, st,
+                              &prefix_rows));
   const int nsm = sm_count();
   const __nv_bfloat16* qn = static_cast<const __nv_bfloat16*>(q_nope);
   const __nv_bfloat16* kn = static_cast<const __nv_bfloat16*>(k_nope);
@@ -518,18 +686,47 @@ sas_status launch_gate_bwd(const sas_problem& p, const void* q_nope, const void*
   gbw_block_bwd_kernel<<<2 * nsm, gbw::kRowThreads, 0, st>>>(
       xk, dkt, knorm_w, p.cu_seqlens, p.gate_rope_cos, p.gate_rope_sin, p.batch, NBmax, Hkv, B,
       p.rms_eps, dxk, dknorm_w);
-  // outer products: enough row splits that the grid covers every SM a few times
+  // block-row outer products (few rows) on CUDA cores
   const int CQ = G * d, CK = 3 * d;
-  const int tq = (CQ / gbw::kTile) * (gbw::H / gbw::kTile) * Hkv;
   const int tk = (CK / gbw::kTile) * (gbw::H / gbw::kTile) * Hkv;
-  const int sq = max(1, min(64, 16 * nsm / tq)), sk = max(1, min(64, 16 * nsm / tk));
-  gbw_outer_kernel<0><<<dim3(CQ / gbw::kTile, gbw::H / gbw::kTile, Hkv * sq), 64, 0, st>>>(
-      dxq, qn, pooled, kn, p.cu_seqlens, p.batch, T, Hq, Hkv, d, B, NBmax, CQ, sq, dwq);
+  const int sk = max(1, min(64, 16 * nsm / tk));
   gbw_outer_kernel<1><<<dim3(CK / gbw::kTile, gbw::H / gbw::kTile, Hkv * sk), 64, 0, st>>>(
       dxk, qn, pooled, kn, p.cu_seqlens, p.batch, T, Hq, Hkv, d, B, NBmax, CK, sk, dwk);
-  gbw_outer_kernel<2><<<dim3(CK / gbw::kTile, gbw::H / gbw::kTile, Hkv * sk), 64, 0, st>>>(
-      dxc, qn, pooled, kn, p.cu_seqlens, p.batch, T, Hq, Hkv, d, B, NBmax, CK, sk, dwk);
-  return launch_status("gate backward", 9);   // + the prefix pass and two projection GEMMs
+  // token-row outer products on the tensor cores: dWq from dxq and the query heads, the
+  // token part of dWk from dxc and the forward gate's prefix-pool rows
+  __nv_bfloat16* xh = reinterpret_cast<__nv_bfloat16*>(ws + L.xh);
+  __nv_bfloat16* xl = reinterpret_cast<__nv_bfloat16*>(ws + L.xl);
+  CUtensorMap tXh, tXl, tQ, tP;
+  if (!make_tmap_bf16_2d(&tXh, xh, (uint64_t)Hkv * gbw::H, T, (uint64_t)Hkv * gbw::H * 2, 64, 64) ||
+      !make_tmap_bf16_2d(&tXl, xl, (uint64_t)Hkv * gbw::H, T, (uint64_t)Hkv * gbw::H * 2, 64, 64) ||
+      !make_tmap_bf16_2d(&tQ, q_nope, (uint64_t)Hq * d, T, (uint64_t)Hq * d * 2, 64, 64) ||
+      !make_tmap_bf16_2d(&tP, prefix_rows, (uint64_t)Hkv * 5 * d, T, (uint64_t)Hkv * 5 * d * 2,
+                         64, 64)) {
+    set_error("gate_bwd: TMA descriptor creation failed");
+    return SAS_ERR_CUDA;
+  }
+  static std::once_flag attr_once;
+  std::call_once(attr_once, [] {
+    cudaFuncSetAttribute(gbw_wgrad_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         gwt::kSmemBytes);
+  });
+  const int chunks = (T + gwt::kK - 1) / gwt::kK;
+  auto wgrad = [&](const float* dx, const CUtensorMap& tY, int y_col_kv, int ncol_tiles, float* dW,
+                   int C, int mean_cols) {
+    const size_t n4 = (size_t)T * Hkv * gbw::H / 4;
+    gbw_split_kernel<<<4 * nsm, 256, 0, st>>>(reinterpret_cast<const float4*>(dx), n4,
+                                              reinterpret_cast<uint2*>(xh),
+                                              reinterpret_cast<uint2*>(xl));
+    const int ctas = ncol_tiles * Hkv;
+    const int nsplit = max(1, min(chunks, (2 * nsm + ctas - 1) / ctas));
+    WgradArgs wa{T, ((chunks + nsplit - 1) / nsplit) * gwt::kK, 0, y_col_kv, dW, C, mean_cols,
+                 reinterpret_cast<int*>(ws)};
+    gbw_wgrad_tc_kernel<<<dim3(ncol_tiles, Hkv, nsplit), gwt::kThreads, gwt::kSmemBytes, st>>>(
+        tXh, tXl, tY, wa);
+  };
+  wgrad(dxq, tQ, G * d, CQ / gwt::kN, dwq, CQ, 0);
+  wgrad(dxc, tP, 5 * d, 5 * d / gwt::kN, dwk, CK, d);
+  return launch_status("gate backward", 11);   // + the prefix pass and two projection GEMMs
 }
 
 }  // namespace sas

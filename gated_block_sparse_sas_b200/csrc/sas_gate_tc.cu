@@ -196,7 +196,7 @@ size_t gate_tc_workspace_bytes(const sas_problem& p) {
 
 sas_status launch_gate_proj_tc(const sas_problem& p, const void* q_nope, const void* k_nope,
                                const void* wq, const void* wk, void* workspace, float** qproj,
-                               float** kproj, cudaStream_t st) {
+                               float** kproj, cudaStream_t st, const void** prefix_rows) {
   // qproj per gate head s (Hs of them; Gs query heads each), kproj per KV head
   const int T = p.total_tokens, Hkv = p.num_kv_heads, Hq = p.num_q_heads, Hs = gate_heads(p);
   const int G = Hq / Hs;
@@ -204,6 +204,7 @@ sas_status launch_gate_proj_tc(const sas_problem& p, const void* q_nope, const v
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   int* err = reinterpret_cast<int*>(ws);
   __nv_bfloat16* ak = reinterpret_cast<__nv_bfloat16*>(ws + 256);
+  if (prefix_rows != nullptr) *prefix_rows = ak;   // [T, Hkv, 640]: max | min | mean hi, mid, lo
   *qproj = reinterpret_cast<float*>(ws + 256 + al256g(rows * gtc::kKCols * 2));
   *kproj = *qproj + al256g((size_t)T * Hs * 128 * 4) / 4;
   const int NBmax = (p.max_seqlen + p.block - 1) / p.block;

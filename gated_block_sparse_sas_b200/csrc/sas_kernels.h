@@ -97,7 +97,8 @@ bool gate_tc_supported(const sas_problem& p);
 size_t gate_tc_workspace_bytes(const sas_problem& p);
 sas_status launch_gate_proj_tc(const sas_problem& p, const void* q_nope, const void* k_nope,
                                const void* wq, const void* wk, void* workspace, float** qproj,
-                               float** kproj, cudaStream_t st);
+                               float** kproj, cudaStream_t st,
+                               const void** prefix_rows = nullptr);
 // Paged decode caches: pt = page table [batch, ceil(capacity / B)] (page of block j of
 // sequence b), pages of [Hkv, B, d] keys / values and [Hkv, h] gate keys; pt == nullptr for
 // the contiguous [batch, Hkv, capacity, d] layout.

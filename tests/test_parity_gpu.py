@@ -231,9 +231,8 @@ DEC_CASES = {
     # the card's other decode budgets: 1,024 tokens (K 15) and 4,096 tokens (K 63)
     "bf16-budget1024-K15": ([3000, 1100, 70, 2048], 4096, 32, 8, 128, 64, 15, 128),
     "bf16-budget4096-K63": ([6000, 4200, 130, 5000], 8192, 16, 4, 128, 64, 63, 128),
-    # 40 sequences x 8 KV heads: the batch runs in four chunks, each chunk's gate on a side
-    # stream while the previous chunk's attention streams
-    "bf16-batch40-chunks": (si.draw_lengths(41, 40, 1, 2500), 2560, 32, 8, 128, 64, 15, 128),
+    # 40 sequences x 8 KV heads of mixed lengths
+    "bf16-batch40-mixed": (si.draw_lengths(41, 40, 1, 2500), 2560, 32, 8, 128, 64, 15, 128),
 }
 
 
@@ -419,7 +418,7 @@ def _paged_from_contiguous(inp, shp, seed, spare=17):
 PAGED_CASES = {
     "budget2048-K31": ([3000, 65, 1, 1777, 4096], 4096, 16, 4, 128, 64, 31, 128),
     "budget4096-K63-G5": ([6000, 4200, 130, 64], 8192, 20, 4, 128, 64, 63, 128),
-    "chunks-batch32": (si.draw_lengths(42, 32, 1, 1024), 1024, 32, 8, 128, 64, 7, 128),
+    "batch32-mixed": (si.draw_lengths(42, 32, 1, 1024), 1024, 32, 8, 128, 64, 7, 128),
 }
 
 
