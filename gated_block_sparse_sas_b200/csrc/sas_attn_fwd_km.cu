@@ -225,7 +225,6 @@ __global__ void __launch_bounds__(kmf::kThreads, 1)
     const int r = tid;
     const int tl = r / G, g = r - tl * G;
     const bool row_ok = r < G * Mq;
-    const uint32_t q_row_dst = smem_u32(sm + OFF_Q) + r * 128;
     bool ok = true;
     int n = 0, item_seq = 0;
     if (r == 0) {
