@@ -59,6 +59,9 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=256, help="oracle rows per CPU-baseline sample")
+    ap.add_argument("--step-only", action="store_true",
+                    help="the headline step alone: no e2e, side legs, other workloads, decode or "
+                         "CPU baseline (profiling)")
     return ap.parse_args()
 
 
@@ -359,8 +362,9 @@ def bench_router_bwd(sas, prob, g, flush, steps):
     G = prob.num_q_heads // Hkv
     outer = 2.0 * T * Hkv * h * (G * d + 3 * d) + 2.0 * prob.batch * prob.max_blocks * Hkv * h * 3 * d
     return {"ms": ms, "outer_product_gflop": outer / 1e9, "achieved_tflops": outer / (ms * 1e-3) / 1e12,
-            "note": "dWq, dWk, norm-weight gradients from the step's dlogg; fp32 CUDA-core outer "
-                    "products; timed separately, not part of the step"}
+            "note": "dWq, dWk, norm-weight gradients from the step's dlogg; the token-row outer "
+                    "products as tcgen05 GEMMs (dx split into bf16 hi + lo), the block-row ones on "
+                    "CUDA cores; timed separately, not part of the step"}
 
 
 # ------------------------------------------------------------------------------------------
@@ -603,6 +607,8 @@ def summarise(name, shape, backward, r, peak, peak_note, ws):
 
 def main():
     a = parse()
+    if a.step_only:
+        a.no_e2e = a.no_extra = a.no_decode = a.no_cpu_baseline = True
     ws, rank, local = dist_setup()
     if a.impl == "reference":
         return reference_arm(a, ws, rank)
@@ -637,9 +643,10 @@ def main():
         line["clocks"] = cs
     if not a.no_e2e:
         line["e2e"] = e2e(sas, prob, g, backward, r["fwd_flops"] + r["bwd_flops"], dev, a, ws)
-    if backward:   # after the timed step and e2e legs, so it cannot perturb them
+    if backward and not a.step_only:   # after the timed step and e2e, so they cannot perturb them
         line["router_bwd"] = bench_router_bwd(sas, prob, g, flush, max(3, a.steps))
-    line["gate_paths"] = bench_gate_paths(sas, prob, g, flush, max(3, a.steps))
+    if not a.step_only:
+        line["gate_paths"] = bench_gate_paths(sas, prob, g, flush, max(3, a.steps))
     if rank == 0 and ws == 1 and not a.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(g, shape, backward, a)
     del g, prob

@@ -245,6 +245,8 @@ def workload(name: str) -> Shape:
                      seed=1 if name.endswith("prefill-32k") else 2)
     if name == "qwen3-4b-train-16k":      # same layer, half length: profiling captures
         return Shape([16384], 32, 8, 128, 64, 31, 128, "bf16", seed=5)
+    if name == "qwen3-14b-train-16k":     # the 14B layer shape on one 16k sequence: captures
+        return Shape([16384], 40, 8, 128, 64, 63, 128, "bf16", seed=7)
     if name == "qwen3-14b-varlen-4seq":
         return Shape(draw_lengths(4, 4, 8192, 65536), 40, 8, 128, 64, 63, 128, "bf16", seed=4)
     raise KeyError(name)
