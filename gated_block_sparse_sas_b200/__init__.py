@@ -67,6 +67,7 @@ _SIGS = {
     "sas_decode_paged": ([_DP, _vp, _i32] + [_vp] * 14 + [_sz, _vp], ctypes.c_int),
     "sas_decode_noalloc": ([_DP] + [_vp] * 13 + [_vp], ctypes.c_int),
     "sas_decode_noalloc_error_word": ([ctypes.POINTER(_vp)], ctypes.c_int),
+    "sas_decode_set_fused": ([_i32], ctypes.c_int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -102,6 +103,9 @@ ERROR_CODES = {
     79: "attn_bwd: a bounded wait gave up",
     81: "decode attention: a bounded wait gave up", 82: "decode attention: a bounded wait gave up",
     83: "decode attention: a bounded wait gave up",
+    84: "fused decode: a selection waited too long for its gate projections",
+    85: "fused decode: an attention split waited too long for its selection",
+    86: "fused decode: a bounded wait for cached gate keys gave up",
     91: "gate projections: a bounded wait gave up", 92: "gate projections: a bounded wait gave up",
     93: "gate projections: a bounded wait gave up",
 }
@@ -127,6 +131,12 @@ def check_workspace(workspace, where: str = "sas"):
     code = error_code(workspace)
     if code != 0:
         raise SasDeviceError(code, where)
+
+
+def sas_decode_set_fused(enable: bool) -> None:
+    """Process-wide choice of decode implementation: the single persistent launch (True, the
+    default, where the shapes allow it) or the three-launch decode (False)."""
+    _check(_lib.sas_decode_set_fused(1 if enable else 0), "sas_decode_set_fused")
 
 
 def decode_noalloc_error_code() -> int:

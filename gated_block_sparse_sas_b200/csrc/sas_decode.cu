@@ -11,35 +11,11 @@
 #include <type_traits>
 
 #include "sas_common.cuh"
+#include "sas_decode_select.cuh"
 #include "sas_kernels.h"
 #include "sas_sm100.cuh"
 
 namespace sas {
-
-constexpr int kDecThreads = 256;
-constexpr int kDecWarps = kDecThreads / 32;
-
-__device__ __forceinline__ float block_reduce_sum(float v, float* red) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  v = warp_sum(v);
-  __syncthreads();
-  if (lane == 0) red[warp] = v;
-  __syncthreads();
-  float r = 0.f;
-  for (int w = 0; w < kDecWarps; ++w) r += red[w];
-  return r;
-}
-
-__device__ __forceinline__ float block_reduce_max(float v, float* red) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  v = warp_max(v);
-  __syncthreads();
-  if (lane == 0) red[warp] = v;
-  __syncthreads();
-  float r = -INFINITY;
-  for (int w = 0; w < kDecWarps; ++w) r = fmaxf(r, red[w]);
-  return r;
-}
 
 // ---------------------------------------------------------------------------------------
 // (1) gate: q~ (Qproj over the G concatenated pre-rotary heads, RMSNorm, rotary at L-1),
@@ -90,12 +66,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_gate_kernel(
     }
   }
   if (empty) {
-    for (int sl = tid; sl <= K; sl += kDecThreads) {
-      sel_idx[orow + sl] = -1;
-      sel_logg[orow + sl] = 0.f;
-      if (idx_out) idx_out[orow + sl] = -1;
-      if (logg_out) logg_out[orow + sl] = 0.f;
-    }
+    decode_select_empty(K, orow, sel_idx, sel_logg, idx_out, logg_out);
     return;
   }
 
@@ -254,136 +225,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_gate_kernel(
     }
   }
   __syncthreads();
-  // logsumexp over j <= c
-  float mx = -INFINITY;
-  for (int j = tid; j <= c; j += kDecThreads) mx = fmaxf(mx, s[j]);
-  mx = block_reduce_max(mx, red);
-  float se = 0.f;
-  for (int j = tid; j <= c; j += kDecThreads) se += expf(s[j] - mx);
-  se = block_reduce_sum(se, red);
-  const float lse = mx + logf(se);
-  if (c <= K) {
-    for (int sl = tid; sl <= K; sl += kDecThreads) {
-      const int jj = sl <= c ? sl : -1;
-      const float lg = sl <= c ? s[sl] - lse : 0.f;
-      sel_idx[orow + sl] = jj;
-      sel_logg[orow + sl] = ungated ? 0.f : lg;   // the attention's bias
-      if (idx_out) idx_out[orow + sl] = jj;
-      if (logg_out) logg_out[orow + sl] = lg;
-    }
-    return;
-  }
-  // exact K-th largest of s[0..c-1] over order-preserving keys, by a radix select: four
-  // rounds of an 8-bit digit histogram; `need` is the wanted rank among the keys that share the
-  // digits chosen so far (padding keys are 0, below every real key, and c > K)
-  uint32_t key[NPT];
-#pragma unroll
-  for (int r = 0; r < NPT; ++r) {
-    const int j = tid + r * kDecThreads;
-    key[r] = (j < c) ? order_key(s[j]) : 0u;
-  }
-  uint32_t thr = 0, pmask = 0;
-  int need = K;
-#pragma unroll 1
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = tid; i < 256; i += kDecThreads) hist[i] = 0;
-    __syncthreads();
-#pragma unroll
-    for (int r = 0; r < NPT; ++r) {   // one shared atomic per distinct digit in the warp
-      const bool in = (key[r] & pmask) == thr;
-      const int bin = in ? (int)((key[r] >> shift) & 255u) : 256;
-      const unsigned peers = __match_any_sync(0xffffffffu, bin);
-      if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
-    }
-    __syncthreads();
-    if (warp == 0) {   // lane owns digits 8 lane .. 8 lane + 7; find the digit where the
-                       // count of keys with a larger-or-equal digit first reaches `need`
-      int hv[8], loc = 0;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        hv[k] = hist[8 * lane + k];
-        loc += hv[k];
-      }
-      int incl = loc;   // keys in this lane's digits and all larger ones
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_down_sync(0xffffffffu, incl, o);
-        if (lane + o < 32) incl += v;
-      }
-      int acc = incl - loc, found = -1, rest = 0;
-#pragma unroll
-      for (int k = 7; k >= 0; --k) {
-        if (found < 0 && acc < need && acc + hv[k] >= need) {
-          found = 8 * lane + k;
-          rest = need - acc;
-        }
-        acc += hv[k];
-      }
-      const unsigned who = __ballot_sync(0xffffffffu, found >= 0);   // exactly one lane
-      const int src = who ? __ffs(who) - 1 : 0;
-      const int dsel = __shfl_sync(0xffffffffu, found, src);
-      const int nrest = __shfl_sync(0xffffffffu, rest, src);
-      if (lane == 0) {
-        misc[1] = dsel;
-        misc[2] = nrest;
-      }
-    }
-    __syncthreads();
-    thr |= (uint32_t)misc[1] << shift;
-    pmask |= 255u << shift;
-    need = misc[2];
-  }
-  const int need_eq = need;   // keys equal to thr to take, lowest block indices first
-  // ordered emission: warp w takes a contiguous range of blocks; a first pass counts its keys
-  // above and equal to thr, a second writes its selected blocks at their global positions
-  const int per = (c + kDecWarps - 1) / kDecWarps;
-  const int wj0 = min(c, warp * per), wj1 = min(c, wj0 + per);
-  const unsigned below = (1u << lane) - 1u;
-  int n_gt = 0, n_eq = 0;
-  for (int j0 = wj0; j0 < wj1; j0 += 32) {
-    const int j = j0 + lane;
-    const uint32_t kk = j < wj1 ? order_key(s[j]) : 0u;
-    n_gt += __popc(__ballot_sync(0xffffffffu, j < wj1 && kk > thr));
-    n_eq += __popc(__ballot_sync(0xffffffffu, j < wj1 && kk == thr));
-  }
-  if (lane == 0) {
-    cnt_red[warp] = n_gt;
-    cnt_red[kDecWarps + warp] = n_eq;
-  }
-  __syncthreads();
-  int gt_before = 0, eq_seen = 0;
-  for (int w = 0; w < warp; ++w) {
-    gt_before += cnt_red[w];
-    eq_seen += cnt_red[kDecWarps + w];
-  }
-  int out = gt_before + min(eq_seen, need_eq);
-  for (int j0 = wj0; j0 < wj1; j0 += 32) {
-    const int j = j0 + lane;
-    const bool valid = j < wj1;
-    const uint32_t kk = valid ? order_key(s[j]) : 0u;
-    const bool is_gt = valid && kk > thr, is_eq = valid && kk == thr;
-    const unsigned eqm = __ballot_sync(0xffffffffu, is_eq);
-    const int eq_rank = eq_seen + __popc(eqm & below);
-    const bool sel = is_gt || (is_eq && eq_rank < need_eq);
-    const unsigned selm = __ballot_sync(0xffffffffu, sel);
-    if (sel) {
-      const int pos = out + __popc(selm & below);
-      const float lg = s[j] - lse;
-      sel_idx[orow + pos] = j;
-      sel_logg[orow + pos] = ungated ? 0.f : lg;
-      if (idx_out) idx_out[orow + pos] = j;
-      if (logg_out) logg_out[orow + pos] = lg;
-    }
-    out += __popc(selm);
-    eq_seen += __popc(eqm);
-  }
-  if (tid == 0) {
-    const float lg = s[c] - lse;
-    sel_idx[orow + K] = c;
-    sel_logg[orow + K] = ungated ? 0.f : lg;
-    if (idx_out) idx_out[orow + K] = c;
-    if (logg_out) logg_out[orow + K] = lg;
-  }
+  decode_select_row<NPT>(s, c, K, ungated, orow, sel_idx, sel_logg, idx_out, logg_out,
+                         DecSelScratch{red, cnt_red, misc, hist});
 }
 
 // ---------------------------------------------------------------------------------------
@@ -752,9 +595,18 @@ size_t decode_workspace_bytes(const sas_decode_problem& p) {
   const size_t pairs = (size_t)p.batch * gate_heads(p);
   const size_t ns = decode_nsplit(p);
   auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
-  return 256 /* error word */ + al(pairs * (p.topk + 1) * 4) * 2 + al(pairs * ns * G * 2 * 4) +
-         al(pairs * ns * G * p.head_dim * 4);
+  const size_t three = 256 /* error word */ + al(pairs * (p.topk + 1) * 4) * 2 +
+                       al(pairs * ns * G * 2 * 4) + al(pairs * ns * G * p.head_dim * 4);
+  // either path may run (the choice is process-wide and may change between calls)
+  if (!decode_fused_supported(p)) return three;
+  const size_t fused = decode_fused_workspace_bytes(p);
+  return fused > three ? fused : three;
 }
+
+namespace {
+bool g_decode_fused = true;
+}
+bool decode_fused_enabled() { return g_decode_fused; }
 
 template <int G>
 static size_t decode_bulk_smem() {
@@ -837,6 +689,11 @@ sas_status launch_decode(const sas_decode_problem& p, const void* q, const void*
                          const float* cur_pool, const void* wq, const float* qnorm_w,
                          const void* wk, const float* knorm_w, void* o, int32_t* idx_out,
                          float* logg_out, void* ws, const DecodePaging& pg, cudaStream_t st) {
+  if (decode_fused_enabled() && decode_fused_supported(p)) {
+    SAS_TRY(launch_decode_fused(p, q, q_nope, k_cache, v_cache, gkc, cur_pool, wq, qnorm_w, wk,
+                                knorm_w, o, idx_out, logg_out, ws, pg, st));
+    return launch_status("decode (fused)", 1);
+  }
   const int G = p.num_q_heads / gate_heads(p);   // query heads per gate head
   const size_t pairs = (size_t)p.batch * gate_heads(p);
   const int ns = decode_nsplit(p);
@@ -887,3 +744,8 @@ sas_status launch_decode(const sas_decode_problem& p, const void* q, const void*
 }
 
 }  // namespace sas
+
+extern "C" sas_status sas_decode_set_fused(int enable) {
+  sas::g_decode_fused = enable != 0;
+  return SAS_OK;
+}

@@ -30,6 +30,12 @@ __device__ __forceinline__ void norm_rope_row(const float* x, const float* __res
   }
 }
 
+// Nearest tf32 value of a finite x (rounded, low 13 mantissa bits cleared): the hi part of the
+// split x = hi + lo used by the tensor-core historical scores.
+__device__ __forceinline__ float tf32_hi(float x) {
+  return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u);
+}
+
 // One row with c > K historical candidates held as NPL keys per lane (c <= 32 NPL).
 template <int NPL>
 __device__ __forceinline__ void topk_row(const float* __restrict__ srow, float l, int c, int K,

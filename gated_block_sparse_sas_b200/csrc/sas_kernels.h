@@ -93,8 +93,17 @@ sas_status launch_attn_bwd_km(const sas_problem& p, const void* q, const void* k
 bool tma_available();
 bool make_tmap_bf16_2d(CUtensorMap* m, const void* base, uint64_t n0, uint64_t n1,
                        uint64_t row_bytes, uint32_t b0, uint32_t b1);
+bool make_tmap_f32_sw128(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
+                         const uint32_t* box);
 bool gate_tc_supported(const sas_problem& p);
 size_t gate_tc_workspace_bytes(const sas_problem& p);
+// Historical gate scores on the tensor cores (sas_gate_hist_tc.cu): q~ and the block keys split
+// into tf32 hi + lo parts, three tf32 products per element (hi.hi + hi.lo + lo.hi).
+bool gate_hist_tc_supported(const sas_problem& p);
+size_t gate_hist_tc_workspace_bytes(const sas_problem& p);   // key splits (ghi, glo)
+sas_status launch_gate_hist_tc(const sas_problem& p, const float* gkeys, const float* qhi,
+                               const float* qlo, void* key_ws, float* scores, float* lse, int* err,
+                               cudaStream_t st);
 sas_status launch_gate_proj_tc(const sas_problem& p, const void* q_nope, const void* k_nope,
                                const void* wq, const void* wk, void* workspace, float** qproj,
                                float** kproj, cudaStream_t st,
@@ -111,6 +120,18 @@ sas_status launch_decode_attn_tc(const sas_decode_problem& p, const void* q, con
                                  const void* vc, const int32_t* sel_idx, const float* sel_logg,
                                  float* part_ml, float* part_acc, int* err, int ns,
                                  const DecodePaging& pg, cudaStream_t st);
+
+// Fused persistent decode (sas_decode_fused.cu): gate, Top-K, attention and merge in one launch.
+bool decode_fused_supported(const sas_decode_problem& p);
+size_t decode_fused_workspace_bytes(const sas_decode_problem& p);
+sas_status launch_decode_fused(const sas_decode_problem& p, const void* q, const void* q_nope,
+                               const void* k_cache, const void* v_cache, const void* gkc,
+                               const float* cur_pool, const void* wq, const float* qnorm_w,
+                               const void* wk, const float* knorm_w, void* o, int32_t* idx_out,
+                               float* logg_out, void* ws, const DecodePaging& pg, cudaStream_t st);
+// Process-wide choice between the fused decode and the three-launch decode (default: fused
+// where supported).
+bool decode_fused_enabled();
 
 int decode_nsplit(const sas_decode_problem& p);
 size_t decode_workspace_bytes(const sas_decode_problem& p);

@@ -68,6 +68,27 @@ bool make_tmap_f32_3d(CUtensorMap* m, const void* base, uint64_t n0, uint64_t n1
             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// fp32 map of rank 2..5 over a contiguous array (dims[0] contiguous) with the given box, 128B
+// swizzle (box[0] * 4 must be 128 bytes).
+bool make_tmap_f32_sw128(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
+                         const uint32_t* box) {
+  PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+  if (!fn || rank < 2 || rank > 5) return false;
+  cuuint64_t d[5], str[4];
+  cuuint32_t bx[5], estr[5];
+  uint64_t stride = 4;
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    bx[i] = box[i];
+    estr[i] = 1;
+    if (i > 0) str[i - 1] = stride;
+    stride *= dims[i];
+  }
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, rank, const_cast<void*>(base), d, str, bx, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool tma_available() { return encode_fn() != nullptr; }
 
 // Tokens per 128-row tile: Mq tokens x G heads <= 128 (G = 5: 25 tokens, 125 rows).

@@ -46,8 +46,8 @@
  *     int32 (word 0) as the call's error word. The call clears it on `stream`
  *     before its kernels run, and a kernel that meets a device-side failure
  *     writes a nonzero code there; read it once the stream has completed
- *     (0 = none). Codes: 41, 81-83 decode waits that gave up (bounded mbarrier
- *     waits, about one second); 51-57 forward, 71-79 backward, 91-93 gate
+ *     (0 = none). Codes: 41, 81-86 decode waits that gave up (bounded mbarrier
+ *     or flag waits, about one second); 51-57 forward, 71-79 backward, 91-93 gate
  *     projection waits that gave up; 60 forward / 61 decode: a row whose largest
  *     logit exceeds its own key's logit by more than ~97 nats (outside the fixed
  *     per-row reference's fp32 range; that row's output is 0 and its lse -inf);
@@ -273,7 +273,10 @@ sas_status sas_attn_bwd(const sas_problem* p, const void* q, const void* k, cons
  * (max, min, sum over tokens c*B..L_b-1); wq, wk, qnorm_w, knorm_w as A3;
  * o dtype [batch, Hq, d]; idx_out int32 / logg_out fp32 [batch, Hs, K+1] may be NULL.
  * Workspace (sas_decode_workspace_size): word 0 is the call's error word (cleared by the
- * call; 41 / 81-83 a bounded wait gave up, 61 a row outside the fixed reference's range). */
+ * call; 41 / 81-86 a bounded wait gave up, 61 a row outside the fixed reference's range).
+ * Implementation: where supported (bf16, d 128, B 64, G <= 8, h in {64, 128},
+ * ceil(capacity / B) <= 2048) one persistent launch runs the gate, Top-K, attention and the
+ * merge of the attention's splits (sas_decode_set_fused); otherwise three launches. */
 sas_status sas_decode_workspace_size(const sas_decode_problem* p, size_t* bytes);
 sas_status sas_decode(const sas_decode_problem* p, const void* q, const void* q_nope,
                       const void* k_cache, const void* v_cache, const void* gate_key_cache,
@@ -281,6 +284,15 @@ sas_status sas_decode(const sas_decode_problem* p, const void* q, const void* q_
                       const void* wk, const float* knorm_w, void* o, int32_t* idx_out,
                       float* logg_out, void* workspace, size_t workspace_bytes,
                       cudaStream_t stream);
+
+/* Decode implementation switch (no counterpart in the SAS pages; a tuning and diagnostic
+ * control). enable != 0 (the default): sas_decode, sas_decode_paged and sas_decode_noalloc use
+ * the single persistent launch where it supports the shapes; 0: they always use the
+ * three-launch decode (gate + Top-K; split-K attention; merge). Both select the same blocks
+ * (the gate arithmetic is the same, in the same order); O agrees up to fp32 summation order
+ * when the two choose different split counts. Process-wide: set it between calls, not while
+ * another thread is issuing decode calls. Always returns SAS_OK. */
+sas_status sas_decode_set_fused(int enable);
 
 /* A7 over paged caches -- the decode step of sas_decode with the KV cache in fixed-size pages
  * (one KV block per page), as a paged serving backend holds it (README "Acknowledgements":

@@ -266,6 +266,59 @@ def test_decode(sas, name, gated):
         assert_out_close(o[torch.from_numpy(~same)], Og[~same], False, "O (near-tie rows)")
 
 
+FUSED_CASES = {
+    # (lengths, capacity, Hq, Hkv, d, B, K, h, gate_heads or None, gated, paged)
+    "K31-G4": ([4000, 129, 2500, 1, 64, 65], 4096, 16, 4, 128, 64, 31, 128, None, True, False),
+    "K63-G5": ([6000, 4200, 130, 5000], 8192, 20, 4, 128, 64, 63, 128, None, True, False),
+    "K15-batch40": (si.draw_lengths(43, 40, 1, 2500), 2560, 32, 8, 128, 64, 15, 128, None, True, False),
+    "K31-h64-ungated": ([3000, 700, 64], 4096, 16, 4, 128, 64, 31, 64, None, False, False),
+    "K15-per-head": ([4200, 300, 65], 4224, 8, 2, 128, 64, 15, 128, 8, True, False),
+    "K31-paged": ([3000, 65, 1, 1777, 4096], 4096, 16, 4, 128, 64, 31, 128, None, True, True),
+}
+
+
+@pytest.mark.parametrize("name", list(FUSED_CASES))
+def test_decode_fused_equals_three_launch(sas, name):
+    """The single persistent decode launch and the three-launch decode select the same blocks
+    with the same log-gates (the gate arithmetic is the same, in the same order) and give the
+    same O up to the split merge's summation order; both agree with the oracle."""
+    lengths, cap, Hq, Hkv, d, B, K, h, gh, gated, paged = FUSED_CASES[name]
+    shp = si.DecodeShape(list(lengths), cap, Hq, Hkv, d, B, K, h, seed=420,
+                         **({} if gh is None else {"gate_heads": gh}))
+    inp = si.decode_inputs(shp)
+    g = {k: v.cuda() for k, v in inp.items()}
+    prob = sas.DecodeProblem(seqlens=g["lengths"], capacity=cap, num_q_heads=Hq, num_kv_heads=Hkv,
+                             head_dim=d, block=B, topk=K, gate_hidden=h, dtype=torch.bfloat16,
+                             gated=gated, **({} if gh is None else {"gate_heads": gh}))
+    common = (g["cur_pool"], g["wq"], g["qnorm_w"], g["wk"], g["knorm_w"])
+    if paged:
+        pt, n_pages, kp, vp, gp = _paged_from_contiguous(inp, shp, 421)
+        pt, kp, vp, gp = pt.cuda(), kp.cuda(), vp.cuda(), gp.cuda()
+        run = lambda: sas.sas_decode_paged(prob, pt, n_pages, g["q"], g["q_nope"], kp, vp, gp,
+                                           *common, want_selection=True, check=True)
+    else:
+        run = lambda: sas.sas_decode(prob, g["q"], g["q_nope"], g["k_cache"], g["v_cache"],
+                                     g["gate_key_cache"], *common, want_selection=True, check=True)
+    try:
+        sas.sas_decode_set_fused(False)
+        o3, i3, l3 = run()
+        sas.sas_decode_set_fused(True)
+        of, i_f, lf = run()
+    finally:
+        sas.sas_decode_set_fused(True)
+    torch.cuda.synchronize()
+    assert torch.equal(i_f, i3)
+    assert torch.equal(lf, l3)
+    assert_out_close(of, o3.float().cpu().numpy(), False, "O fused vs three-launch")
+    O, ridx, rlogg, margin = orc.decode(inp["q"], inp["q_nope"], inp["k_cache"], inp["v_cache"],
+                                        lengths, inp["gate_key_cache"], inp["cur_pool"], inp["wq"],
+                                        inp["qnorm_w"], inp["wk"], inp["knorm_w"], B, K, 1e-6, 1e6,
+                                        gated=gated)
+    compare_selection(i_f.cpu().numpy(), lf, ridx, rlogg, margin)
+    same = (i_f.cpu().numpy() == ridx).all(axis=-1).all(axis=-1)
+    assert_out_close(of[torch.from_numpy(same)], O[same], False, "O")
+
+
 def test_decode_equals_prefill_row(sas):
     """A decode step over caches written from a prefill equals that prefill's last row."""
     L, B, K, h = 777, 64, 5, 128
