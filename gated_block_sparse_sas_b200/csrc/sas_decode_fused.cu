@@ -860,6 +860,9 @@ static sas_status launch_fused_hn(const CUtensorMap& tk, const CUtensorMap& tv, 
   std::call_once(once, [] {
     cudaFuncSetAttribute(decode_fused_kernel<H, NPT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          dfz::kSmemBytes);
+    // two CTAs per SM need nearly all of the SM's shared memory: ask for the largest carveout
+    cudaFuncSetAttribute(decode_fused_kernel<H, NPT>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                         100);
     int dev = 0, sms = 0, per_sm = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

@@ -557,19 +557,24 @@ sas_status launch_gate_scores(const sas_problem& p, const void* q_nope, const vo
 
 // ---------------------------------------------------------------------------------------
 // A4: Top-K. One warp per (token, kv) row. The K-th largest score is found exactly by a
-// 32-step bitwise search over order-preserving uint32 keys held in registers; then the
-// row is emitted in ascending block order with ballots: every key above the threshold,
-// plus the lowest-index ties at the threshold until K are kept.
+// radix select over order-preserving uint32 keys held in registers (four 8-bit digit rounds,
+// warp-private shared counters); then the row is emitted in ascending block order with
+// ballots: every key above the threshold, plus the lowest-index ties at the threshold until K
+// are kept.
 // ---------------------------------------------------------------------------------------
 // The key count per lane follows the row's own candidate count c_t (warp-uniform), so the
 // work of a row scales with its visible blocks, not with the longest sequence. MAXNPL bounds
 // the instantiated sizes (and so the registers) by the problem's NBmax.
+constexpr int kTopkThreads = 256;
+
 template <int MAXNPL>
-__global__ void topk_kernel(const float* __restrict__ scores, const float* __restrict__ lse,
+__global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float* __restrict__ scores, const float* __restrict__ lse,
                             const int32_t* __restrict__ cu, int batch, int T, int Hkv, int NBmax,
                             int B, int K, int32_t* __restrict__ idx, float* __restrict__ logg) {
+  __shared__ int hist_s[kTopkThreads / 32][256];   // per-warp radix counters
   const int row = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5);
   const int lane = threadIdx.x & 31;
+  int* hist = hist_s[threadIdx.x >> 5];
   if (row >= T * Hkv) return;
   const int tg = row / Hkv;
   const int b = seq_of(cu, batch, tg);
@@ -586,12 +591,12 @@ __global__ void topk_kernel(const float* __restrict__ scores, const float* __res
     }
     return;
   }
-  if (MAXNPL <= 2 || c <= 64) topk_row<2>(srow, l, c, K, lane, irow, grow);
-  else if (MAXNPL <= 4 || c <= 128) topk_row<(MAXNPL < 4 ? MAXNPL : 4)>(srow, l, c, K, lane, irow, grow);
-  else if (MAXNPL <= 8 || c <= 256) topk_row<(MAXNPL < 8 ? MAXNPL : 8)>(srow, l, c, K, lane, irow, grow);
-  else if (MAXNPL <= 16 || c <= 512) topk_row<(MAXNPL < 16 ? MAXNPL : 16)>(srow, l, c, K, lane, irow, grow);
-  else if (MAXNPL <= 32 || c <= 1024) topk_row<(MAXNPL < 32 ? MAXNPL : 32)>(srow, l, c, K, lane, irow, grow);
-  else topk_row<MAXNPL>(srow, l, c, K, lane, irow, grow);
+  if (MAXNPL <= 2 || c <= 64) topk_row_radix<2>(srow, l, c, K, lane, hist, irow, grow);
+  else if (MAXNPL <= 4 || c <= 128) topk_row_radix<(MAXNPL < 4 ? MAXNPL : 4)>(srow, l, c, K, lane, hist, irow, grow);
+  else if (MAXNPL <= 8 || c <= 256) topk_row_radix<(MAXNPL < 8 ? MAXNPL : 8)>(srow, l, c, K, lane, hist, irow, grow);
+  else if (MAXNPL <= 16 || c <= 512) topk_row_radix<(MAXNPL < 16 ? MAXNPL : 16)>(srow, l, c, K, lane, hist, irow, grow);
+  else if (MAXNPL <= 32 || c <= 1024) topk_row_radix<(MAXNPL < 32 ? MAXNPL : 32)>(srow, l, c, K, lane, hist, irow, grow);
+  else topk_row_radix<MAXNPL>(srow, l, c, K, lane, hist, irow, grow);
   if (lane == 0) {
     irow[K] = c;
     grow[K] = srow[c] - l;
@@ -602,7 +607,7 @@ sas_status launch_topk(const sas_problem& p, const float* scores, const float* l
                        float* logg, cudaStream_t st) {
   const int NBmax = (p.max_seqlen + p.block - 1) / p.block;
   const int rows = p.total_tokens * gate_heads(p);
-  const int threads = 256;
+  const int threads = kTopkThreads;
   const int grid = (int)(((size_t)rows * 32 + threads - 1) / threads);
 #define SAS_TK(N)                                                                              \
   topk_kernel<N><<<grid, threads, 0, st>>>(scores, lse, p.cu_seqlens, p.batch, p.total_tokens,  \

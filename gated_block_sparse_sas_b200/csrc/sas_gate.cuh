@@ -82,4 +82,82 @@ __device__ __forceinline__ void topk_row(const float* __restrict__ srow, float l
   }
 }
 
+// The same row selection as topk_row (exact K-th largest key, ties to the lower block index,
+// ascending emission), with the threshold found by a radix select: four rounds over the 8-bit
+// digits of the order-preserving keys, each a histogram in the warp's own 256 shared counters
+// (`hist`) over the keys that share the digits chosen so far. Padding keys are 0, below every
+// real key, and c > K, so the K-th largest is a real key.
+template <int NPL>
+__device__ __forceinline__ void topk_row_radix(const float* __restrict__ srow, float l, int c, int K,
+                                               int lane, int* hist, int32_t* __restrict__ irow,
+                                               float* __restrict__ grow) {
+  uint32_t key[NPL];
+#pragma unroll
+  for (int r = 0; r < NPL; ++r) {
+    const int j = r * 32 + lane;
+    key[r] = (j < c) ? order_key(srow[j]) : 0u;
+  }
+  uint32_t thr = 0, pmask = 0;
+  int need = K;   // rank wanted among the keys that share the digits chosen so far
+#pragma unroll 1
+  for (int shift = 24; shift >= 0; shift -= 8) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) hist[i * 32 + lane] = 0;
+    __syncwarp();
+#pragma unroll
+    for (int r = 0; r < NPL; ++r)
+      if ((key[r] & pmask) == thr) atomicAdd(&hist[(key[r] >> shift) & 255u], 1);
+    __syncwarp();
+    // lane owns digits 8 lane .. 8 lane + 7: the digit where the count of keys with a larger or
+    // equal digit first reaches `need`
+    int hv[8], loc = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      hv[k] = hist[8 * lane + k];
+      loc += hv[k];
+    }
+    int incl = loc;   // keys in this lane's digits and all larger ones
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_down_sync(0xffffffffu, incl, o);
+      if (lane + o < 32) incl += v;
+    }
+    int acc = incl - loc, found = -1, rest = 0;
+#pragma unroll
+    for (int k = 7; k >= 0; --k) {
+      if (found < 0 && acc < need && acc + hv[k] >= need) {
+        found = 8 * lane + k;
+        rest = need - acc;
+      }
+      acc += hv[k];
+    }
+    const unsigned who = __ballot_sync(0xffffffffu, found >= 0);   // exactly one lane
+    const int src = who ? __ffs(who) - 1 : 0;
+    const int dsel = __shfl_sync(0xffffffffu, found, src);
+    need = __shfl_sync(0xffffffffu, rest, src);
+    thr |= (uint32_t)dsel << shift;
+    pmask |= 255u << shift;
+    __syncwarp();   // every lane has read the counters before the next round clears them
+  }
+  const int need_eq = need;   // keys equal to thr to take, lowest block indices first
+  const unsigned below = (1u << lane) - 1u;
+  int out = 0, eq_seen = 0;
+#pragma unroll
+  for (int r = 0; r < NPL; ++r) {
+    const bool is_gt = key[r] > thr, is_eq = key[r] == thr;
+    const unsigned eqm = __ballot_sync(0xffffffffu, is_eq);
+    const int eq_rank = eq_seen + __popc(eqm & below);
+    const bool sel = is_gt || (is_eq && eq_rank < need_eq);
+    const unsigned selm = __ballot_sync(0xffffffffu, sel);
+    if (sel) {
+      const int pos = out + __popc(selm & below);
+      const int j = r * 32 + lane;
+      irow[pos] = j;
+      grow[pos] = srow[j] - l;
+    }
+    out += __popc(selm);
+    eq_seen += __popc(eqm);
+  }
+}
+
 }  // namespace sas

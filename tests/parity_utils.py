@@ -54,6 +54,30 @@ def assert_grad_close(gpu, ref, fp32: bool, what: str):
     return e
 
 
+# Two GPU selection paths (fused scores + Top-K against the separate kernels): the historical
+# scores come from different arithmetic (tf32 hi/lo products on the tensor cores, fp32 FMA on
+# the CUDA cores), each within GATE_ABS of the oracle, so their log-gates and logsumexps agree
+# to a few fp32 roundings of the row's score range; 2e-5 bounds that with room.
+PATHS_GATE_ABS = 2e-5
+
+
+def assert_paths_agree(idx_a, idx_b, scores, K):
+    """Selections of two GPU paths: identical ids except at rows whose K-th and (K+1)-th largest
+    historical scores (from `scores` [T, Hs, NBmax], the unfused path's) are a near-tie, where
+    both selections are correct. Returns the number of such rows."""
+    a, b = np.asarray(idx_a), np.asarray(idx_b)
+    diff = ~(a == b).all(axis=-1)
+    if not diff.any():
+        return 0
+    s = to64(scores)
+    for r, h in np.argwhere(diff):
+        c = int(a[r, h, K])   # the current block, always in the last slot when c > K
+        row = np.sort(s[r, h, :c])[::-1]
+        assert c > K and row[K - 1] - row[K] < NEAR_TIE, \
+            f"row {r} head {h}: selections differ with margin {row[K - 1] - row[K]:.3e}"
+    return int(diff.sum())
+
+
 def compare_selection(idx_gpu, logg_gpu, idx_ref, logg_ref, margin_ref):
     """Top-K parity: exact ids except near-ties; log-gates within GATE_ABS where ids agree.
     Returns (n_rows, n_near_tie, n_mismatch_near_tie)."""
