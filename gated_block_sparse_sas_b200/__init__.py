@@ -108,6 +108,12 @@ ERROR_CODES = {
     86: "fused decode: a bounded wait for cached gate keys gave up",
     91: "gate projections: a bounded wait gave up", 92: "gate projections: a bounded wait gave up",
     93: "gate projections: a bounded wait gave up",
+    94: "router weight gradients: a bounded wait gave up",
+    95: "router weight gradients: a bounded wait gave up",
+    96: "router weight gradients: a bounded wait gave up",
+    97: "tensor-core gate scores: a bounded wait gave up",
+    98: "tensor-core gate scores: a bounded wait gave up",
+    99: "tensor-core gate scores: a bounded wait gave up",
 }
 
 

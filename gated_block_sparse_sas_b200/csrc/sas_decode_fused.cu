@@ -742,8 +742,10 @@ __device__ void attn_item(const FzArgs& a, const CUtensorMap* tmK, const CUtenso
 
 }  // namespace
 
+// 120 registers per thread: two 256-thread CTAs per SM (at 128 the occupancy calculation admits
+// one, and the persistent grid would run at half the planned concurrency)
 template <int H, int NPT>
-__global__ void __launch_bounds__(dfz::kThreads, 2)
+__global__ void __maxnreg__(120)
     decode_fused_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                         const FzArgs a) {
   using namespace dfz;
@@ -863,11 +865,19 @@ static sas_status launch_fused_hn(const CUtensorMap& tk, const CUtensorMap& tv, 
     // two CTAs per SM need nearly all of the SM's shared memory: ask for the largest carveout
     cudaFuncSetAttribute(decode_fused_kernel<H, NPT>, cudaFuncAttributePreferredSharedMemoryCarveout,
                          100);
-    int dev = 0, sms = 0, per_sm = 0;
+    // CTAs per SM from the SM's shared memory and registers (the occupancy query returns one
+    // for this kernel, while two run side by side and halve the step time)
+    int dev = 0, sms = 0, sm_smem = 0, reserved = 0, sm_regs = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_fused_kernel<H, NPT>, dfz::kThreads,
-                                                  dfz::kSmemBytes);
+    cudaDeviceGetAttribute(&sm_smem, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+    cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+    cudaDeviceGetAttribute(&sm_regs, cudaDevAttrMaxRegistersPerMultiprocessor, dev);
+    cudaFuncAttributes fa;
+    cudaFuncGetAttributes(&fa, decode_fused_kernel<H, NPT>);
+    const int by_smem = sm_smem / (dfz::kSmemBytes + reserved);
+    const int by_regs = sm_regs / (fa.numRegs * dfz::kThreads);
+    const int per_sm = by_smem < by_regs ? by_smem : by_regs;   // 2 (shared memory)
     grid = sms * (per_sm > 0 ? per_sm : 1);
   });
   const int total = a.nP + a.nS + a.nA;

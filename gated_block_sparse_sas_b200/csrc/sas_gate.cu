@@ -183,18 +183,14 @@ struct GsSmem {
 // PROJ: the two projections come precomputed (tensor-core GEMMs, sas_gate_tc.cu) as
 // qproj [T, Hs, H] / kproj [T, Hkv, H] fp32, so phases 1 and 2 only load, normalise and
 // rotate them.
-// HTC (with PROJ): the historical scores and the logsumexp are left to the tensor-core kernel
-// (sas_gate_hist_tc.cu); this kernel writes q~ split into tf32 hi + lo ([T, Hs, H] each) and
-// the current block's score s[t, c_t].
-template <typename T, int H, bool PROJ, bool HTC = false>
+template <typename T, int H, bool PROJ>
 __global__ void __launch_bounds__(kGsThreads) gate_scores_kernel(
     const T* __restrict__ q_nope, const T* __restrict__ k_nope, const float* __restrict__ gkeys,
     const T* __restrict__ wq, const float* __restrict__ qnorm_w, const T* __restrict__ wk,
     const float* __restrict__ knorm_w, const int32_t* __restrict__ cu,
     const float* __restrict__ rc, const float* __restrict__ rs, int Hq, int Hkv, int Hs, int d,
     int B, int NBmax, float eps, const float* __restrict__ qproj, const float* __restrict__ kproj,
-    float* __restrict__ scores, float* __restrict__ lse, float* __restrict__ qhi = nullptr,
-    float* __restrict__ qlo = nullptr) {
+    float* __restrict__ scores, float* __restrict__ lse) {
   extern __shared__ float smem[];
   using S = GsSmem<H, PROJ>;
   constexpr int NO = H / 16;   // outputs per thread in the 64 x H GEMMs
@@ -227,16 +223,6 @@ __global__ void __launch_bounds__(kGsThreads) gate_scores_kernel(
       }
       __syncwarp();
       for (int e = lane; e < H; e += 32) Qt[e * kAP + t] = (t < nt) ? X[t * (H + 1) + e] : 0.f;
-      if constexpr (HTC) {
-        if (t < nt) {
-          const size_t o = ((size_t)(s0 + t0 + t) * Hs + sh) * H;
-          for (int e = lane; e < H; e += 32) {
-            const float x = X[t * (H + 1) + e], hi = tf32_hi(x);
-            qhi[o + e] = hi;
-            qlo[o + e] = x - hi;
-          }
-        }
-      }
     }
     __syncthreads();
   } else {
@@ -391,11 +377,6 @@ __global__ void __launch_bounds__(kGsThreads) gate_scores_kernel(
     __syncthreads();
   }
 
-  if constexpr (HTC) {   // the current block's score; the rest comes from the tensor cores
-    for (int t = tid; t < nt; t += kGsThreads)
-      scores[((size_t)(s0 + t0 + t) * Hs + sh) * NBmax + (t0 + t) / B] = scur[t];
-    return;
-  }
   // ---------------- phase 3: historical scores + logsumexp ----------------
   {
     float* Bs = R;  // [H][kAP] block keys of a 64-block chunk, transposed
@@ -488,17 +469,8 @@ static sas_status gate_scores_dispatch(const sas_problem& p, const void* q_nope,
     float* qhi = (float*)extra;
     float* qlo = (float*)(extra + qbytes);
     void* key_ws = extra + 2 * qbytes;
-    const size_t smem = (size_t)GsSmem<128, true>::TOTAL * sizeof(float);
-    static std::once_flag once_h;
-    std::call_once(once_h, [smem] {
-      cudaFuncSetAttribute(gate_scores_kernel<T, 128, true, true>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    });
-    gate_scores_kernel<T, 128, true, true><<<grid, kGsThreads, smem, st>>>(
-        (const T*)q_nope, (const T*)k_nope, gkeys, (const T*)wq, qnorm_w, (const T*)wk, knorm_w,
-        p.cu_seqlens, p.gate_rope_cos, p.gate_rope_sin, p.num_q_heads, p.num_kv_heads, Hs,
-        p.head_dim, p.block, NBmax, p.rms_eps, qproj, kproj, scores, lse, qhi, qlo);
-    SAS_TRY(launch_gate_hist_tc(p, gkeys, qhi, qlo, key_ws, scores, lse, (int*)workspace, st));
+    SAS_TRY(launch_gate_hist_tc(p, gkeys, qproj, kproj, qnorm_w, knorm_w, qhi, qlo, key_ws, scores,
+                                lse, (int*)workspace, st));
     return launch_status("gate_scores (tensor-core projections and historical scores)", 6);
   }
   if (gate_tc_supported(p)) {   // projections on the tensor cores, then norms, rotary, scores

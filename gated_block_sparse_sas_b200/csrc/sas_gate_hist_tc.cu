@@ -1,7 +1,8 @@
-// Historical gate scores on the tensor cores (A3): s[t, j] = q~_t . k~_j / sqrt(h) for every
-// block j before the token's current block c_t, the -inf padding past c_t, and the logsumexp
-// over j <= c_t (the current block's score s[t, c_t] is written beforehand by the gate-score
-// kernel). Model card "tencent/Simple-Attention-Sparsification", "Checkpoint configuration"
+// Gate scores with the historical part on the tensor cores (A3), after the two projections:
+// gate_qk_split_kernel normalises and rotates q~ and the current block's key, writes q~ split
+// into tf32 hi + lo and the current block's score s[t, c_t]; gate_hist_tc_kernel computes
+// s[t, j] = q~_t . k~_j / sqrt(h) for every block j before c_t, the -inf padding past c_t, and
+// the logsumexp over j <= c_t. Model card "tencent/Simple-Attention-Sparsification", "Checkpoint configuration"
 // (gate hidden 128); paper abstract (softmax over history plus the current block).
 //
 // The selection must agree with an exact evaluation except at near-ties, so the products keep
@@ -64,6 +65,63 @@ __global__ void split_tf32_kernel(const float* __restrict__ x, float* __restrict
     hi[i] = h;
     lo[i] = v - h;
   }
+}
+
+// q~ and the current block's score for the tensor-core path: one warp per (token, gate head).
+// The two projected rows (Qproj of the gate head, Kproj of the current block's prefix pool) are
+// held as four elements per lane (channels lane + 32 u), so the rotate-half pairs (e, e + 64)
+// sit in the same lane; RMSNorm (weight after the normalisation), rotary at t (query) and at
+// c_t B (current block), then q~ split into tf32 hi + lo, and s[t, c_t] = q~ . k~cur / sqrt(h).
+// The sums run in the same order as the shared-memory kernels' (lane partials over e = lane,
+// lane + 32, ..., then the warp tree).
+__global__ void __launch_bounds__(256) gate_qk_split_kernel(
+    const float* __restrict__ qproj, const float* __restrict__ kproj, const float* __restrict__ qnorm_w,
+    const float* __restrict__ knorm_w, const int32_t* __restrict__ cu, const float* __restrict__ rc,
+    const float* __restrict__ rs, int batch, int T, int Hs, int Hkv, int B, int NBmax, float eps,
+    float* __restrict__ qhi, float* __restrict__ qlo, float* __restrict__ scores) {
+  constexpr int H = ghc::kH;
+  const int lane = threadIdx.x & 31;
+  const long long gw = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5;
+  if (gw >= (long long)T * Hs) return;
+  const int tg = (int)(gw / Hs), sh = (int)(gw - (long long)tg * Hs);
+  const int kv = sh / (Hs / Hkv);
+  const int b = seq_of(cu, batch, tg);
+  const int t = tg - cu[b], c = t / B;
+  auto norm_rope = [&](float* x, const float* __restrict__ w, int pos) {
+    float ss = 0.f;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) ss += x[u] * x[u];
+    ss = warp_sum(ss);
+    const float rn = sqrtf(ss / (float)H + eps);
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {   // pairs (lane + 32 u, lane + 32 u + 64)
+      const int e = lane + 32 * u;
+      const float a = x[u] / rn * w[e], bb = x[u + 2] / rn * w[e + H / 2];
+      const float cs = rc[(size_t)pos * (H / 2) + e], sn = rs[(size_t)pos * (H / 2) + e];
+      x[u] = a * cs - bb * sn;
+      x[u + 2] = bb * cs + a * sn;
+    }
+  };
+  float q[4], k[4];
+  const float* qr = qproj + (size_t)gw * H;
+  const float* kr = kproj + ((size_t)tg * Hkv + kv) * H;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    q[u] = qr[lane + 32 * u];
+    k[u] = kr[lane + 32 * u];
+  }
+  norm_rope(q, qnorm_w, t);
+  norm_rope(k, knorm_w, c * B);
+  float dot = 0.f;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const float hi = tf32_hi(q[u]);
+    qhi[(size_t)gw * H + lane + 32 * u] = hi;
+    qlo[(size_t)gw * H + lane + 32 * u] = q[u] - hi;
+    dot += q[u] * k[u];
+  }
+  dot = warp_sum(dot);
+  if (lane == 0) scores[(size_t)gw * NBmax + c] = dot / sqrtf((float)H);
 }
 
 __global__ void __launch_bounds__(ghc::kThreads, 1)
@@ -244,7 +302,7 @@ __global__ void __launch_bounds__(ghc::kThreads, 1)
       }
     }
     if (!ok) tc_fail(a.err, 99, abort_flag);
-    if (valid) {   // the current block's score (written by the gate-score kernel) closes the sum
+    if (valid) {   // the current block's score (written by gate_qk_split_kernel) closes the sum
       const size_t row = (size_t)(s0 + t0 + r) * a.Hs + sh;
       const float y = a.scores[row * a.NBmax + c_t] * kLog2e;
       const float M = fmaxf(m2, y);
@@ -274,11 +332,18 @@ size_t gate_hist_tc_workspace_bytes(const sas_problem& p) {
   return 2 * al256h(keys * 4);
 }
 
-sas_status launch_gate_hist_tc(const sas_problem& p, const float* gkeys, const float* qhi,
-                               const float* qlo, void* key_ws, float* scores, float* lse, int* err,
-                               cudaStream_t st) {
+sas_status launch_gate_hist_tc(const sas_problem& p, const float* gkeys, const float* qproj,
+                               const float* kproj, const float* qnorm_w, const float* knorm_w,
+                               float* qhi, float* qlo, void* key_ws, float* scores, float* lse,
+                               int* err, cudaStream_t st) {
   const int NBmax = (p.max_seqlen + p.block - 1) / p.block;
   const int Hs = gate_heads(p), Hkv = p.num_kv_heads;
+  {
+    const long long warps = (long long)p.total_tokens * Hs;
+    gate_qk_split_kernel<<<(int)((warps * 32 + 255) / 256), 256, 0, st>>>(
+        qproj, kproj, qnorm_w, knorm_w, p.cu_seqlens, p.gate_rope_cos, p.gate_rope_sin, p.batch,
+        p.total_tokens, Hs, Hkv, p.block, NBmax, p.rms_eps, qhi, qlo, scores);
+  }
   const size_t keys = (size_t)p.batch * NBmax * Hkv * ghc::kH;
   float* ghi = (float*)key_ws;
   float* glo = (float*)((char*)key_ws + al256h(keys * 4));

@@ -101,9 +101,10 @@ size_t gate_tc_workspace_bytes(const sas_problem& p);
 // into tf32 hi + lo parts, three tf32 products per element (hi.hi + hi.lo + lo.hi).
 bool gate_hist_tc_supported(const sas_problem& p);
 size_t gate_hist_tc_workspace_bytes(const sas_problem& p);   // key splits (ghi, glo)
-sas_status launch_gate_hist_tc(const sas_problem& p, const float* gkeys, const float* qhi,
-                               const float* qlo, void* key_ws, float* scores, float* lse, int* err,
-                               cudaStream_t st);
+sas_status launch_gate_hist_tc(const sas_problem& p, const float* gkeys, const float* qproj,
+                               const float* kproj, const float* qnorm_w, const float* knorm_w,
+                               float* qhi, float* qlo, void* key_ws, float* scores, float* lse,
+                               int* err, cudaStream_t st);
 sas_status launch_gate_proj_tc(const sas_problem& p, const void* q_nope, const void* k_nope,
                                const void* wq, const void* wk, void* workspace, float** qproj,
                                float** kproj, cudaStream_t st,

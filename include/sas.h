@@ -48,7 +48,8 @@
  *     writes a nonzero code there; read it once the stream has completed
  *     (0 = none). Codes: 41, 81-86 decode waits that gave up (bounded mbarrier
  *     or flag waits, about one second); 51-57 forward, 71-79 backward, 91-93 gate
- *     projection waits that gave up; 60 forward / 61 decode: a row whose largest
+ *     projection, 94-96 router weight-gradient, 97-99 tensor-core gate score waits
+ *     that gave up; 60 forward / 61 decode: a row whose largest
  *     logit exceeds its own key's logit by more than ~97 nats (outside the fixed
  *     per-row reference's fp32 range; that row's output is 0 and its lse -inf);
  *     62 paged decode: a page id out of range.
@@ -173,7 +174,12 @@ sas_status sas_gate_keys(const sas_problem* p, const float* pooled, const void* 
  * Workspace (size from sas_gate_scores_workspace_size): for bf16, d = 128, h = 128 the two
  * projections run as tensor-core GEMMs and the workspace holds their inputs and outputs
  * (per token and kv head: the current block's prefix max, min and mean as exact bf16 parts,
- * 1280 B, and the two projections, 1024 B); otherwise 256 B suffice. */
+ * 1280 B, and the two projections, 1024 B); the historical scores then also run on the
+ * tensor cores, from q~ and the block keys split into tf32 hi + lo parts (three tf32
+ * products per element, hi.hi + hi.lo + lo.hi, fp32 accumulation: within a few fp32
+ * roundings of the exact dot product), and the workspace holds the splits (per token and
+ * gate head 1024 B, per cached block key 1024 B). Otherwise 256 B suffice. Word 0 is the
+ * call's error word (codes 91-93, 97-99). */
 sas_status sas_gate_scores_workspace_size(const sas_problem* p, size_t* bytes);
 sas_status sas_gate_scores(const sas_problem* p, const void* q_nope, const void* k_nope,
                            const float* gate_keys, const void* wq, const float* qnorm_w,
@@ -186,9 +192,10 @@ sas_status sas_gate_scores(const sas_problem* p, const void* q_nope, const void*
  * idx int32 / logg fp32 [T, Hs, K+1] (ids ascending, current block last, -1 padding),
  * and, if lse is not NULL, the gate logsumexp fp32 [T, Hs]. For bf16, d = 128, h = 128
  * and NBmax <= 1024 the scores live only in shared memory (one kernel holds a tile's score
- * rows, selects and writes the kept ids); the scores are bit-identical to sas_gate_scores',
- * so the ids are too, and the log-gates agree to fp32 rounding (the logsumexp is summed in
- * another order). Other shapes run the two unfused kernels through the workspace, which
+ * rows, selects and writes the kept ids). Its historical products are fp32 FMA chains, where
+ * sas_gate_scores uses tf32 hi/lo products on the tensor cores; both are within a few fp32
+ * roundings of the exact scores, so the ids agree except at near-ties (both are then a
+ * correct Top-K) and the log-gates to about 1e-5. Other shapes run the two unfused kernels through the workspace, which
  * then also holds the scores. Workspace (sas_gate_select_workspace_size): word 0 is the
  * call's error word (codes 91-93). */
 sas_status sas_gate_select_workspace_size(const sas_problem* p, size_t* bytes);
