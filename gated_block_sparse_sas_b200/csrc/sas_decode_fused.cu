@@ -26,6 +26,9 @@
 // finishes it. Every wait is bounded anyway: a wait that gives up records an error code and
 // raises the workspace's abort word, which ends every other wait and stops every CTA.
 //
+// (Interleaving the queue so that a row's A items follow its S item a few sequences later was
+// slower: A items then wait for selections still running.)
+//
 // Shared memory is reused between item kinds: P items keep their inputs in the K/V ring, S items
 // stream key chunks through the ring and keep the score row in the Q/P region. mbarrier phases
 // are counted across items (every thread of the CTA keeps the same counters).
@@ -476,6 +479,33 @@ __device__ void attn_item(const FzArgs& a, const CUtensorMap* tmK, const CUtenso
   __syncthreads();
   if (*abort_flag) return;
 
+  // K/V load i of this item (i even: K of pair i / 2, odd: V) into ring slot (ring + i) % 3,
+  // once the slot's previous use has been released; warp 0 lane 0 only
+  const int Hk = a.Hkv, kh = sh / a.R;
+  auto load_kv = [&](int i, int nblk) -> bool {
+    const uint32_t gi = rc.ring + i, slot = gi % kSlots;
+    if (gi >= kSlots && !mbar_wait(empty + slot, ((gi / kSlots) - 1) & 1, abort_flag)) return false;
+    const int n = i >> 1;
+    const CUtensorMap* map = (i & 1) ? tmV : tmK;
+    uint8_t* dst = sm + OFF_STAGE + slot * kKV;
+    const int ja = blk_j[2 * n];
+    const int jb = (2 * n + 1 < nblk) ? blk_j[2 * n + 1] : ja;   // odd count: masked copy
+    int ya = ja * kB, yb = jb * kB, za = b * Hk + kh, zb = za;
+    if (a.pt != nullptr) {   // pages range-checked by the S item (a bad one empties the row)
+      ya = yb = 0;
+      za = a.pt[(size_t)b * a.nbmax + ja] * Hk + kh;
+      zb = a.pt[(size_t)b * a.nbmax + jb] * Hk + kh;
+    }
+    mbar_arrive_expect_tx(full + slot, kKV);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      tma_load_3d(dst + h * kHalfPair, map, full + slot, 64 * h, ya, za);
+      tma_load_3d(dst + h * kHalfPair + kHalfBlk, map, full + slot, 64 * h, yb, zb);
+    }
+    return true;
+  };
+  int issued = 0;   // warp 0 lane 0: K/V loads issued so far
+
   // ---------------- setup ----------------
   if (warp == 0) {   // this split's kept blocks in slot order (valid ones only)
     int n = 0;
@@ -496,7 +526,17 @@ __device__ void attn_item(const FzArgs& a, const CUtensorMap* tmK, const CUtenso
       }
       n += __popc(m);
     }
-    if (lane == 0) *nblk_s = n;
+    __syncwarp();
+    if (lane == 0) {
+      *nblk_s = n;
+      // the first loads go out now, while the other warps set up Q and the references
+      const int first = min(2 * ((n + 1) >> 1), kSlots);
+      for (; issued < first; ++issued)
+        if (!load_kv(issued, n)) {
+          fz_fail(a, 81, abort_flag);
+          break;
+        }
+    }
   } else if (warp == 2 || warp == 3) {   // Q tile: rows h < G = q heads, rows >= G zero; P^T zero
     const int t = tid - 64;
     for (int e = t; e < kN * 16; e += 64) {
@@ -553,34 +593,11 @@ __device__ void attn_item(const FzArgs& a, const CUtensorMap* tmK, const CUtenso
   if (warp == 0) {
     // ---------------- K/V loads ----------------
     if (lane == 0) {
-      const int Hk = a.Hkv, kh = sh / a.R;
-      const int z = b * Hk + kh;
-      int issued = 0;
-      for (int i = 0; i < 2 * npairs; ++i) {
-        const uint32_t gi = rc.ring + i, slot = gi % kSlots;
-        if (gi >= kSlots && !mbar_wait(empty + slot, ((gi / kSlots) - 1) & 1, abort_flag)) {
+      for (; issued < 2 * npairs && !*abort_flag; ++issued)
+        if (!load_kv(issued, nblk)) {
           fz_fail(a, 81, abort_flag);
           break;
         }
-        const int n = i >> 1;
-        const CUtensorMap* map = (i & 1) ? tmV : tmK;
-        uint8_t* dst = sm + OFF_STAGE + slot * kKV;
-        const int ja = blk_j[2 * n];
-        const int jb = (2 * n + 1 < nblk) ? blk_j[2 * n + 1] : ja;   // odd count: masked copy
-        int ya = ja * kB, yb = jb * kB, za = z, zb = z;
-        if (a.pt != nullptr) {   // pages range-checked by the S item (a bad one empties the row)
-          ya = yb = 0;
-          za = a.pt[(size_t)b * a.nbmax + ja] * Hk + kh;
-          zb = a.pt[(size_t)b * a.nbmax + jb] * Hk + kh;
-        }
-        mbar_arrive_expect_tx(full + slot, kKV);
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          tma_load_3d(dst + h * kHalfPair, map, full + slot, 64 * h, ya, za);
-          tma_load_3d(dst + h * kHalfPair + kHalfBlk, map, full + slot, 64 * h, yb, zb);
-        }
-        issued = i + 1;
-      }
       for (int i = max(0, issued - kSlots); i < issued; ++i) {   // none in flight at exit
         const uint32_t gi = rc.ring + i;
         mbar_wait_drain(full + gi % kSlots, (gi / kSlots) & 1);
@@ -781,7 +798,7 @@ __global__ void __maxnreg__(120)
     const int it = *item_s;
     __syncthreads();
     if (it >= total || *abort_flag) break;
-    if (it < a.nP) {
+    if (it < a.nP) {   // (4-sequence chunk, gate head, part)
       const int part = it & 1, rest = it >> 1;
       proj_item<H>(a, sm, rest % a.Hs, part, rest / a.Hs);
     } else if (it < a.nP + a.nS) {
