@@ -67,6 +67,7 @@ struct KmLists {
   int* items;
   int* cnt_q;    // per entry and window quarter
   int* ctl;      // [0] non-empty entries, [1] work counter
+  int2* chunk;   // scan scratch: per-chunk totals, then offsets
   int2* list;
   int nW, P, E;
 };

@@ -1,8 +1,9 @@
 // Construction of the inverted selection lists of the key-major attention passes (layout in
-// sas_km.cuh). Three launches and a clear, no host synchronisation:
+// sas_km.cuh). Five launches and a clear, no host synchronisation:
 //   count  CTA per (window quarter, sequence, kv head): shared-memory histogram of the kept
 //          blocks of 1024 tokens; per-quarter counts, entry totals by global atomics
-//   scan   one CTA: exclusive scan of the entry totals, ascending list of non-empty entries
+//   scan   exclusive scan of the entry totals (per-chunk totals, a scan of those, per-chunk
+//          writes), ascending list of non-empty entries
 //   fill   CTA per (window quarter, sequence, kv head): every kept (token, block) pair placed
 //          at its entry's offset + the counts of the window's earlier quarters + a shared
 //          atomic cursor (order inside an entry arbitrary)
@@ -45,51 +46,100 @@ __global__ void km_count_kernel(const int32_t* __restrict__ idx, const int32_t* 
   }
 }
 
-// Exclusive scan of the E counts (one CTA of 1024 threads); ascending list of the non-empty
-// entries; ctl[0] = their number; ctl[1] (the work counter of the main kernels) = 0.
-__global__ void __launch_bounds__(1024) km_scan_kernel(const int* __restrict__ cnt, int E,
-                                                       int* __restrict__ off, int* __restrict__ items,
-                                                       int* __restrict__ ctl) {
-  __shared__ int ws_c[32], ws_n[32];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int per = (E + 1023) / 1024;
-  const int e0 = min(E, tid * per), e1 = min(E, e0 + per);
+// Exclusive scan of the E entry counts in three launches (chunks of kScanChunk entries per CTA):
+// per-chunk totals of the pairs and of the non-empty entries; one CTA scans the chunk totals;
+// every chunk writes its entries' offsets and its non-empty entries, ascending, into `items`.
+// ctl[0] = the number of non-empty entries; ctl[1] (the work counter of the main kernels) = 0.
+constexpr int kScanThreads = 1024, kScanPer = 4, kScanChunk = kScanThreads * kScanPer;
+
+// block-wide inclusive scan of (a, b) over kScanThreads threads; returns the block totals
+__device__ __forceinline__ int2 block_scan2(int& a, int& b, int2* ws) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int x = __shfl_up_sync(0xffffffffu, a, o), y = __shfl_up_sync(0xffffffffu, b, o);
+    if (lane >= o) { a += x; b += y; }
+  }
+  if (lane == 31) ws[warp] = make_int2(a, b);
+  __syncthreads();
+  if (warp == 0) {
+    int2 v = ws[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int x = __shfl_up_sync(0xffffffffu, v.x, o), y = __shfl_up_sync(0xffffffffu, v.y, o);
+      if (lane >= o) { v.x += x; v.y += y; }
+    }
+    ws[lane] = v;   // inclusive over warps
+  }
+  __syncthreads();
+  if (warp > 0) { a += ws[warp - 1].x; b += ws[warp - 1].y; }
+  const int2 tot = ws[31];
+  __syncthreads();   // ws is reused by the caller's next scan
+  return tot;
+}
+
+__global__ void __launch_bounds__(kScanThreads) km_scan_chunks_kernel(const int* __restrict__ cnt, int E,
+                                                                     int2* __restrict__ chunk_tot) {
+  __shared__ int2 ws[32];
+  const int e0 = blockIdx.x * kScanChunk + threadIdx.x * kScanPer;
   int sc = 0, sn = 0;
-  for (int e = e0; e < e1; ++e) {
-    const int c = cnt[e];
+#pragma unroll
+  for (int u = 0; u < kScanPer; ++u) {
+    const int c = e0 + u < E ? cnt[e0 + u] : 0;
     sc += c;
     sn += c > 0;
   }
-  int ic = sc, in = sn;   // inclusive warp scans
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int a = __shfl_up_sync(0xffffffffu, ic, o), bb = __shfl_up_sync(0xffffffffu, in, o);
-    if (lane >= o) { ic += a; in += bb; }
+  const int2 tot = block_scan2(sc, sn, ws);
+  if (threadIdx.x == 0) chunk_tot[blockIdx.x] = tot;
+}
+
+// exclusive scan of the nchunk chunk totals in place (one CTA)
+__global__ void __launch_bounds__(kScanThreads) km_scan_top_kernel(int2* __restrict__ chunk_tot, int nchunk,
+                                                                  int* __restrict__ ctl) {
+  __shared__ int2 ws[32];
+  const int per = (nchunk + kScanThreads - 1) / kScanThreads;
+  const int c0 = min(nchunk, (int)threadIdx.x * per), c1 = min(nchunk, c0 + per);
+  int sc = 0, sn = 0;
+  for (int c = c0; c < c1; ++c) { sc += chunk_tot[c].x; sn += chunk_tot[c].y; }
+  int ic = sc, in = sn;
+  const int2 tot = block_scan2(ic, in, ws);
+  int rc = ic - sc, rn = in - sn;
+  for (int c = c0; c < c1; ++c) {
+    const int2 t = chunk_tot[c];
+    chunk_tot[c] = make_int2(rc, rn);
+    rc += t.x;
+    rn += t.y;
   }
-  if (lane == 31) { ws_c[warp] = ic; ws_n[warp] = in; }
-  __syncthreads();
-  if (warp == 0) {
-    int vc = ws_c[lane], vn = ws_n[lane];
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int a = __shfl_up_sync(0xffffffffu, vc, o), bb = __shfl_up_sync(0xffffffffu, vn, o);
-      if (lane >= o) { vc += a; vn += bb; }
-    }
-    ws_c[lane] = vc;   // inclusive over warps
-    ws_n[lane] = vn;
-  }
-  __syncthreads();
-  int rc = ic - sc + (warp ? ws_c[warp - 1] : 0);
-  int rn = in - sn + (warp ? ws_n[warp - 1] : 0);
-  for (int e = e0; e < e1; ++e) {
-    const int c = cnt[e];
-    off[e] = rc;
-    rc += c;
-    if (c > 0) items[rn++] = e;
-  }
-  if (tid == 1023) {
-    ctl[0] = ws_n[31];
+  if (threadIdx.x == 0) {
+    ctl[0] = tot.y;
     ctl[1] = 0;
+  }
+}
+
+__global__ void __launch_bounds__(kScanThreads) km_scan_write_kernel(const int* __restrict__ cnt, int E,
+                                                                    const int2* __restrict__ chunk_off,
+                                                                    int* __restrict__ off,
+                                                                    int* __restrict__ items) {
+  __shared__ int2 ws[32];
+  const int e0 = blockIdx.x * kScanChunk + threadIdx.x * kScanPer;
+  int c[kScanPer], sc = 0, sn = 0;
+#pragma unroll
+  for (int u = 0; u < kScanPer; ++u) {
+    c[u] = e0 + u < E ? cnt[e0 + u] : 0;
+    sc += c[u];
+    sn += c[u] > 0;
+  }
+  int ic = sc, in = sn;
+  block_scan2(ic, in, ws);
+  const int2 base = chunk_off[blockIdx.x];
+  int rc = base.x + ic - sc, rn = base.y + in - sn;
+#pragma unroll
+  for (int u = 0; u < kScanPer; ++u) {
+    if (e0 + u < E) {
+      off[e0 + u] = rc;
+      if (c[u] > 0) items[rn++] = e0 + u;
+    }
+    rc += c[u];
   }
 }
 
@@ -143,7 +193,8 @@ bool km_supported(const sas_problem& p) {
 size_t km_lists_bytes(const sas_problem& p) {
   int nW, P, E;
   km_dims(p, &nW, &P, &E);
-  return 3 * al256((size_t)E * 4) + al256((size_t)E * kQuarters * 4) + 256 +
+  const size_t nchunk = ((size_t)E + kScanChunk - 1) / kScanChunk;
+  return 3 * al256((size_t)E * 4) + al256((size_t)E * kQuarters * 4) + 256 + al256(nchunk * 8) +
          al256((size_t)p.total_tokens * gate_heads(p) * (p.topk + 1) * 8);
 }
 
@@ -156,6 +207,8 @@ KmLists km_lists_carve(const sas_problem& p, uint8_t* base) {
   L.items = reinterpret_cast<int*>(base + o); o += al256((size_t)L.E * 4);
   L.cnt_q = reinterpret_cast<int*>(base + o); o += al256((size_t)L.E * kQuarters * 4);
   L.ctl = reinterpret_cast<int*>(base + o);   o += 256;
+  L.chunk = reinterpret_cast<int2*>(base + o);
+  o += al256((((size_t)L.E + kScanChunk - 1) / kScanChunk) * 8);
   L.list = reinterpret_cast<int2*>(base + o);
   return L;
 }
@@ -169,10 +222,13 @@ sas_status launch_km_lists(const sas_problem& p, const int32_t* idx, const float
   }
   km_count_kernel<<<wgrid, 512, 0, st>>>(idx, p.cu_seqlens, p.batch, gate_heads(p), p.topk, L.P,
                                          L.cnt, L.cnt_q);
-  km_scan_kernel<<<1, 1024, 0, st>>>(L.cnt, L.E, L.off, L.items, L.ctl);
+  const int nchunk = (L.E + kScanChunk - 1) / kScanChunk;
+  km_scan_chunks_kernel<<<nchunk, kScanThreads, 0, st>>>(L.cnt, L.E, L.chunk);
+  km_scan_top_kernel<<<1, kScanThreads, 0, st>>>(L.chunk, nchunk, L.ctl);
+  km_scan_write_kernel<<<nchunk, kScanThreads, 0, st>>>(L.cnt, L.E, L.chunk, L.off, L.items);
   km_fill_kernel<<<wgrid, 512, 0, st>>>(idx, logg, p.cu_seqlens, p.batch, gate_heads(p), p.topk,
                                         L.P, L.off, L.cnt_q, L.list);
-  return launch_status("key-major selection lists", 3);
+  return launch_status("key-major selection lists", 5);
 }
 
 int sm_count() {
