@@ -82,6 +82,11 @@ __device__ __forceinline__ void topk_row(const float* __restrict__ srow, float l
   }
 }
 
+// Inverse of order_key: the float whose key is k (bit for bit).
+__device__ __forceinline__ float key_float(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
 // The same row selection as topk_row (exact K-th largest key, ties to the lower block index,
 // ascending emission), with the threshold found by a radix select: four rounds over the 8-bit
 // digits of the order-preserving keys, each a histogram in the warp's own 256 shared counters
@@ -149,11 +154,10 @@ __device__ __forceinline__ void topk_row_radix(const float* __restrict__ srow, f
     const int eq_rank = eq_seen + __popc(eqm & below);
     const bool sel = is_gt || (is_eq && eq_rank < need_eq);
     const unsigned selm = __ballot_sync(0xffffffffu, sel);
-    if (sel) {
+    if (sel) {   // the score comes back from its key, exactly (no reload)
       const int pos = out + __popc(selm & below);
-      const int j = r * 32 + lane;
-      irow[pos] = j;
-      grow[pos] = srow[j] - l;
+      irow[pos] = r * 32 + lane;
+      grow[pos] = key_float(key[r]) - l;
     }
     out += __popc(selm);
     eq_seen += __popc(eqm);

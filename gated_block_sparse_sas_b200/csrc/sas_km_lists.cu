@@ -5,8 +5,9 @@
 //   scan   exclusive scan of the entry totals (per-chunk totals, a scan of those, per-chunk
 //          writes), ascending list of non-empty entries
 //   fill   CTA per (window quarter, sequence, kv head): every kept (token, block) pair placed
-//          at its entry's offset + the counts of the window's earlier quarters + a shared
-//          atomic cursor (order inside an entry arbitrary)
+//          at its entry's offset + the counts of the window's earlier quarters + a per-entry
+//          cursor, 64 tokens at a time staged in shared memory by block (order inside an
+//          entry arbitrary)
 #include <mutex>
 
 #include "sas_common.cuh"
@@ -144,34 +145,108 @@ __global__ void __launch_bounds__(kScanThreads) km_scan_write_kernel(const int* 
 }
 
 // Place every kept (token, block) pair of quarter q of window w at its entry's next free
-// position: entry offset + the earlier quarters' counts + a shared atomic cursor.
-__global__ void km_fill_kernel(const int32_t* __restrict__ idx, const float* __restrict__ logg,
-                               const int32_t* __restrict__ cu, int batch, int Hkv, int K, int P,
-                               const int* __restrict__ off, const int* __restrict__ cnt_q,
-                               int2* __restrict__ list) {
-  __shared__ int cur[km::kMaxBins];
+// position: entry offset + the earlier quarters' counts + a cursor per entry. The quarter is
+// taken 64 tokens at a time: the pairs are counted per block (their shared-atomic return value is
+// their rank in the block), the counts scanned, the pairs staged in shared memory grouped by
+// block and then written out in that order, so each block's pairs of the 64 tokens land in one
+// contiguous run of the list instead of as scattered 8-byte stores.
+constexpr int kFillThreads = 512;
+constexpr int kFillTok = 64;                        // tokens per staging round
+constexpr int kFillPer = kFillTok * 128 / kFillThreads;   // pairs per thread per round (K + 1 <= 128)
+// shared memory: three per-block arrays, the staged pairs and their list positions (K + 1 per
+// token), scan partials
+static size_t fill_smem(int K1) { return (size_t)3 * km::kMaxBins * 4 + (size_t)kFillTok * K1 * 12 + 64; }
+
+__global__ void __launch_bounds__(kFillThreads) km_fill_kernel(
+    const int32_t* __restrict__ idx, const float* __restrict__ logg, const int32_t* __restrict__ cu,
+    int batch, int Hkv, int K, int P, const int* __restrict__ off, const int* __restrict__ cnt_q,
+    int2* __restrict__ list) {
+  extern __shared__ int fsm[];
+  int* cur = fsm;                          // [kMaxBins] next list position of each block
+  int* lcnt = cur + km::kMaxBins;          // [kMaxBins] this round's pairs per block
+  int* loff = lcnt + km::kMaxBins;         // [kMaxBins] their start in the staging buffer
+  const int K1 = K + 1, cap = kFillTok * K1;
+  int2* stage = reinterpret_cast<int2*>(loff + km::kMaxBins);   // [cap]
+  int* gpos = reinterpret_cast<int*>(stage + cap);                // [cap] list position
+  int* wsum = gpos + cap;                                         // [16] scan partials
   const int w = blockIdx.x / kQuarters, qt = blockIdx.x - w * kQuarters;
   const int b = blockIdx.y, kv = blockIdx.z;
   const int s0 = cu[b], L = cu[b + 1] - s0;
   const int t0 = w * km::kW + qt * kQTok, t1 = min(L, t0 + kQTok);
   if (t0 >= L) return;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nbins = km::kWB * (w + 1);
   const int base = km::entry(kv, b, w, 0, batch, P);
-  for (int j = threadIdx.x; j < nbins; j += blockDim.x) {
+  for (int j = tid; j < nbins; j += kFillThreads) {
     int o = off[base + j];
     for (int q = 0; q < qt; ++q) o += cnt_q[(size_t)(base + j) * kQuarters + q];
     cur[j] = o;
   }
-  __syncthreads();
-  const int K1 = K + 1;
-  for (int e = threadIdx.x; e < (t1 - t0) * K1; e += blockDim.x) {
-    const int tl = t0 + e / K1, s = e - (e / K1) * K1;
-    const size_t gi = ((size_t)(s0 + tl) * Hkv + kv) * K1 + s;
-    const int j = idx[gi];
-    if (j >= 0 && j < nbins) {
-      const int pos = atomicAdd(&cur[j], 1);
-      list[pos] = make_int2((s0 + tl) | (s << 24), __float_as_int(logg[gi]));
+  for (int r0 = t0; r0 < t1; r0 += kFillTok) {
+    const int npair = (min(t1, r0 + kFillTok) - r0) * K1;
+    for (int j = tid; j < nbins; j += kFillThreads) lcnt[j] = 0;
+    __syncthreads();
+    int jj[kFillPer], rk[kFillPer];
+#pragma unroll
+    for (int u = 0; u < kFillPer; ++u) {   // count, and the pair's rank within its block
+      const int e = tid + u * kFillThreads;
+      jj[u] = -1;
+      if (e < npair) {
+        const int tl = r0 + e / K1, sl = e - (e / K1) * K1;
+        const int j = idx[((size_t)(s0 + tl) * Hkv + kv) * K1 + sl];
+        if (j >= 0 && j < nbins) {
+          jj[u] = j;
+          rk[u] = atomicAdd(&lcnt[j], 1);
+        }
+      }
     }
+    __syncthreads();
+    {   // exclusive scan of lcnt[0..nbins) into loff (each thread 4 consecutive blocks)
+      constexpr int kPerT = km::kMaxBins / kFillThreads;
+      int v[kPerT], sum = 0;
+#pragma unroll
+      for (int u = 0; u < kPerT; ++u) {
+        const int j = tid * kPerT + u;
+        v[u] = j < nbins ? lcnt[j] : 0;
+        sum += v[u];
+      }
+      int inc = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int x = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += x;
+      }
+      if (lane == 31) wsum[warp] = inc;
+      __syncthreads();
+      int wbase = 0;
+      for (int q = 0; q < warp; ++q) wbase += wsum[q];
+      int run = wbase + inc - sum;
+#pragma unroll
+      for (int u = 0; u < kPerT; ++u) {
+        const int j = tid * kPerT + u;
+        if (j < nbins) loff[j] = run;
+        run += v[u];
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < kFillPer; ++u) {   // stage grouped by block
+      if (jj[u] >= 0) {
+        const int e = tid + u * kFillThreads;
+        const int tl = r0 + e / K1, sl = e - (e / K1) * K1;
+        const size_t gi = ((size_t)(s0 + tl) * Hkv + kv) * K1 + sl;
+        const int slot = loff[jj[u]] + rk[u];
+        stage[slot] = make_int2((s0 + tl) | (sl << 24), __float_as_int(logg[gi]));
+        gpos[slot] = cur[jj[u]] + rk[u];
+      }
+    }
+    __syncthreads();
+    int nvalid = 0;   // = sum of lcnt: the last block's offset plus its count
+    if (nbins > 0) nvalid = loff[nbins - 1] + lcnt[nbins - 1];
+    for (int i = tid; i < nvalid; i += kFillThreads) list[gpos[i]] = stage[i];
+    __syncthreads();
+    for (int j = tid; j < nbins; j += kFillThreads) cur[j] += lcnt[j];
+    __syncthreads();
   }
 }
 
@@ -226,8 +301,12 @@ sas_status launch_km_lists(const sas_problem& p, const int32_t* idx, const float
   km_scan_chunks_kernel<<<nchunk, kScanThreads, 0, st>>>(L.cnt, L.E, L.chunk);
   km_scan_top_kernel<<<1, kScanThreads, 0, st>>>(L.chunk, nchunk, L.ctl);
   km_scan_write_kernel<<<nchunk, kScanThreads, 0, st>>>(L.cnt, L.E, L.chunk, L.off, L.items);
-  km_fill_kernel<<<wgrid, 512, 0, st>>>(idx, logg, p.cu_seqlens, p.batch, gate_heads(p), p.topk,
-                                        L.P, L.off, L.cnt_q, L.list);
+  static std::once_flag fill_once;
+  std::call_once(fill_once, [] {
+    cudaFuncSetAttribute(km_fill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fill_smem(128));
+  });
+  km_fill_kernel<<<wgrid, kFillThreads, fill_smem(p.topk + 1), st>>>(idx, logg, p.cu_seqlens, p.batch, gate_heads(p),
+                                                         p.topk, L.P, L.off, L.cnt_q, L.list);
   return launch_status("key-major selection lists", 5);
 }
 
