@@ -334,9 +334,9 @@ __device__ void select_item(const FzArgs& a, uint8_t* sm, uint64_t* gfull, uint3
   float* xk = xq + H;
   float* red = reinterpret_cast<float*>(sm + OFF_RED);
   int* cnt_red = reinterpret_cast<int*>(red + kDecWarps);
-  int* misc = cnt_red + 2 * kDecWarps;   // misc[3]: a page id out of range
+  int* misc = cnt_red + 2 * kDecWarps;   // [4], decode_select_row's; misc[4]: a page id out of range
   int* hist = reinterpret_cast<int*>(sm + OFF_BLK);
-  volatile bool* bad = reinterpret_cast<volatile bool*>(misc + 3);
+  volatile bool* bad = reinterpret_cast<volatile bool*>(misc + 4);
   if (seq_len_ok(L, a.capacity)) {
     const int c = (L - 1) / kB;
     const int nchunk = (c + CK - 1) / CK;

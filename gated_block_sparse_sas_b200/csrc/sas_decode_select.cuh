@@ -74,9 +74,10 @@ __device__ void decode_select_row(const float* s, int c, int K, int ungated, siz
     }
     return;
   }
-  // exact K-th largest of s[0..c-1] over order-preserving keys, by a radix select: four
+  // exact K-th largest of s[0..c-1] over order-preserving keys, by a radix select: up to four
   // rounds of an 8-bit digit histogram; `need` is the wanted rank among the keys that share the
-  // digits chosen so far (padding keys are 0, below every real key, and c > K)
+  // digits chosen so far (padding keys are 0, below every real key, and c > K); once at most 32
+  // keys share them, warp 0 ranks those directly
   uint32_t key[NPT];
 #pragma unroll
   for (int r = 0; r < NPT; ++r) {
@@ -111,12 +112,13 @@ __device__ void decode_select_row(const float* s, int c, int K, int ungated, siz
         const int v = __shfl_down_sync(0xffffffffu, incl, o);
         if (lane + o < 32) incl += v;
       }
-      int acc = incl - loc, found = -1, rest = 0;
+      int acc = incl - loc, found = -1, rest = 0, fcnt = 0;
 #pragma unroll
       for (int k = 7; k >= 0; --k) {
         if (found < 0 && acc < need && acc + hv[k] >= need) {
           found = 8 * lane + k;
           rest = need - acc;
+          fcnt = hv[k];
         }
         acc += hv[k];
       }
@@ -124,15 +126,49 @@ __device__ void decode_select_row(const float* s, int c, int K, int ungated, siz
       const int src = who ? __ffs(who) - 1 : 0;
       const int dsel = __shfl_sync(0xffffffffu, found, src);
       const int nrest = __shfl_sync(0xffffffffu, rest, src);
+      const int ncand = __shfl_sync(0xffffffffu, fcnt, src);
       if (lane == 0) {
+        w.misc[0] = ncand;   // keys sharing the new prefix
         w.misc[1] = dsel;
         w.misc[2] = nrest;
+        w.misc[3] = 0;       // gather cursor of the direct finish
       }
     }
     __syncthreads();
     thr |= (uint32_t)w.misc[1] << shift;
     pmask |= 255u << shift;
     need = w.misc[2];
+    const int ncand = w.misc[0];
+    if (shift > 0 && ncand <= 32) {
+      // few candidates left: gather them and let warp 0 rank them against each other (the
+      // need-th largest), instead of more histogram rounds
+      uint32_t* cand = reinterpret_cast<uint32_t*>(w.hist);
+#pragma unroll
+      for (int r = 0; r < NPT; ++r)
+        if ((key[r] & pmask) == thr) cand[atomicAdd(&w.misc[3], 1)] = key[r];
+      __syncthreads();
+      if (warp == 0) {
+        const uint32_t x = lane < ncand ? cand[lane] : 0u;
+        int gt = 0, eq = 0;
+        for (int i = 0; i < ncand; ++i) {
+          const uint32_t y = cand[i];
+          gt += y > x ? 1 : 0;
+          eq += y == x ? 1 : 0;
+        }
+        const unsigned hit = __ballot_sync(0xffffffffu, lane < ncand && gt < need && need <= gt + eq);
+        const int hs = hit ? __ffs(hit) - 1 : 0;
+        const uint32_t xs = __shfl_sync(0xffffffffu, x, hs);
+        const int gs = __shfl_sync(0xffffffffu, gt, hs);
+        if (lane == 0) {
+          w.misc[1] = (int)xs;
+          w.misc[2] = need - gs;
+        }
+      }
+      __syncthreads();
+      thr = (uint32_t)w.misc[1];
+      need = w.misc[2];
+      break;
+    }
   }
   const int need_eq = need;   // keys equal to thr to take, lowest block indices first
   // ordered emission: warp w takes a contiguous range of blocks; a first pass counts its keys

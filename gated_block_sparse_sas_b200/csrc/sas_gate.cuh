@@ -91,7 +91,8 @@ __device__ __forceinline__ float key_float(uint32_t k) {
 // ascending emission), with the threshold found by a radix select: four rounds over the 8-bit
 // digits of the order-preserving keys, each a histogram in the warp's own 256 shared counters
 // (`hist`) over the keys that share the digits chosen so far. Padding keys are 0, below every
-// real key, and c > K, so the K-th largest is a real key.
+// real key, and c > K, so the K-th largest is a real key. Once at most 32 keys share the digits
+// chosen so far (usually after two rounds), they are ranked directly in the warp.
 template <int NPL>
 __device__ __forceinline__ void topk_row_radix(const float* __restrict__ srow, float l, int c, int K,
                                                int lane, int* hist, int32_t* __restrict__ irow,
@@ -127,12 +128,13 @@ __device__ __forceinline__ void topk_row_radix(const float* __restrict__ srow, f
       const int v = __shfl_down_sync(0xffffffffu, incl, o);
       if (lane + o < 32) incl += v;
     }
-    int acc = incl - loc, found = -1, rest = 0;
+    int acc = incl - loc, found = -1, rest = 0, fcnt = 0;
 #pragma unroll
     for (int k = 7; k >= 0; --k) {
       if (found < 0 && acc < need && acc + hv[k] >= need) {
         found = 8 * lane + k;
         rest = need - acc;
+        fcnt = hv[k];
       }
       acc += hv[k];
     }
@@ -140,9 +142,37 @@ __device__ __forceinline__ void topk_row_radix(const float* __restrict__ srow, f
     const int src = who ? __ffs(who) - 1 : 0;
     const int dsel = __shfl_sync(0xffffffffu, found, src);
     need = __shfl_sync(0xffffffffu, rest, src);
+    const int ncand = __shfl_sync(0xffffffffu, fcnt, src);   // keys sharing the new prefix
     thr |= (uint32_t)dsel << shift;
     pmask |= 255u << shift;
-    __syncwarp();   // every lane has read the counters before the next round clears them
+    __syncwarp();   // every lane has read the counters before they are reused
+    if (shift > 0 && ncand <= 32) {
+      // few candidates left: gather them (one per lane) and take the need-th largest by
+      // ranking them against each other, instead of more histogram rounds
+      uint32_t* cand = reinterpret_cast<uint32_t*>(hist);
+      int at = 0;
+#pragma unroll
+      for (int r = 0; r < NPL; ++r) {
+        const bool m = (key[r] & pmask) == thr;
+        const unsigned bal = __ballot_sync(0xffffffffu, m);
+        if (m) cand[at + __popc(bal & ((1u << lane) - 1u))] = key[r];
+        at += __popc(bal);
+      }
+      __syncwarp();
+      const uint32_t x = lane < ncand ? cand[lane] : 0u;
+      int gt = 0, eq = 0;
+      for (int i = 0; i < ncand; ++i) {
+        const uint32_t y = cand[i];
+        gt += y > x ? 1 : 0;
+        eq += y == x ? 1 : 0;
+      }
+      const unsigned hit = __ballot_sync(0xffffffffu, lane < ncand && gt < need && need <= gt + eq);
+      const int hs = hit ? __ffs(hit) - 1 : 0;
+      thr = __shfl_sync(0xffffffffu, x, hs);
+      need -= __shfl_sync(0xffffffffu, gt, hs);
+      __syncwarp();
+      break;
+    }
   }
   const int need_eq = need;   // keys equal to thr to take, lowest block indices first
   const unsigned below = (1u << lane) - 1u;
