@@ -708,6 +708,44 @@ def cpu_baseline(g, shape, backward, a):
                       ") at full sequence length, fp64 numpy"}
 
 
+def link_probe(dev, nbytes=1 << 30):
+    """Pinned host <-> device copy bandwidth (GB/s): each direction alone and both at once
+    (two streams), best of 3, CUDA events. The end-to-end step moves its inputs and results over
+    this link, so it bounds that step from below."""
+    h_in = torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
+    h_out = torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
+    d_in = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    d_out = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def run(h2d, d2h):   # best (ms) of 3 trials per direction; 0 for a direction not run
+        th, td = [], []
+        for _ in range(3):
+            torch.cuda.synchronize()
+            a0, a1, b0, b1 = ev(), ev(), ev(), ev()
+            with torch.cuda.stream(s1):
+                a0.record(s1)
+                if h2d:
+                    d_in.copy_(h_in, non_blocking=True)
+                a1.record(s1)
+            with torch.cuda.stream(s2):
+                b0.record(s2)
+                if d2h:
+                    h_out.copy_(d_out, non_blocking=True)
+                b1.record(s2)
+            torch.cuda.synchronize()
+            th.append(a0.elapsed_time(a1))
+            td.append(b0.elapsed_time(b1))
+        return (min(th) if h2d else 0.0), (min(td) if d2h else 0.0)
+
+    h, _ = run(True, False)
+    _, d = run(False, True)
+    hb, db = run(True, True)
+    gbs = lambda ms: nbytes / (ms * 1e-3) / 1e9 if ms > 0 else None
+    return {"h2d_gbs": gbs(h), "d2h_gbs": gbs(d), "h2d_gbs_duplex": gbs(hb), "d2h_gbs_duplex": gbs(db)}
+
+
 def e2e(sas, prob, g, backward, work, dev, a, ws):
     """Same step through the public API with host buffers: every step copies all its inputs
     in from pinned host memory, runs, and copies every result back. The three stages run on
@@ -726,8 +764,10 @@ def e2e(sas, prob, g, backward, work, dev, a, ws):
         sets.append((dg, [torch.empty(dg[k].shape, dtype=dg[k].dtype, pin_memory=True)
                           for k in outs]))
     s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    # the window carries one pipeline fill (the first step's input copy) and one drain (the last
+    # result copy); 16 timed steps spread them, and the steady-state period is reported beside
     warm = 2
-    steps = max(2, min(a.steps, 4))
+    steps = max(4, min(2 * a.steps, 16))
     total = warm + steps
     ev = lambda: torch.cuda.Event(enable_timing=True)
     in_done, comp_done, out_done = [ev() for _ in range(total)], [ev() for _ in range(total)], \
@@ -758,11 +798,20 @@ def e2e(sas, prob, g, backward, work, dev, a, ws):
     torch.cuda.synchronize()
     ms = start.elapsed_time(out_done[total - 1]) / steps
     ms = max_over_ranks(ms, ws, dev)
+    period = out_done[warm].elapsed_time(out_done[total - 1]) / (steps - 1)   # result to result
+    period = max_over_ranks(period, ws, dev)
     h2d = sum(host[k].numel() * host[k].element_size() for k in names)
     d2h = sum(h.numel() * h.element_size() for h in sets[0][1])
+    del sets, host
+    torch.cuda.empty_cache()
+    link = link_probe(dev)
+    # the step time the host link alone allows (inputs in and results out at the same time)
+    bound = max(h2d / (link["h2d_gbs_duplex"] * 1e9), d2h / (link["d2h_gbs_duplex"] * 1e9)) * 1e3
     return {"value": work * ws / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "pipelined": "two buffer sets; H2D, step and D2H on separate streams"}
+            "pipelined": "two buffer sets; H2D, step and D2H on separate streams",
+            "timed_steps": steps, "steady_ms_per_step": period,
+            "link": link, "link_bound_ms": bound}
 
 
 def reference_arm(a, ws, rank):
