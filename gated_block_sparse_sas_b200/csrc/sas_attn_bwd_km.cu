@@ -12,8 +12,9 @@
 //   dV_j^T += dO^T P,  dK_j^T += Q^T dS / sqrt(d)     (M=128 d, N=64 keys, K=128 rows)
 //   dQ_rows = dS K_j / sqrt(d)                         (M=128 rows, N=128 d, K=64 keys)
 // dV^T and dK^T stay in TMEM over the item and are added to fp32 dK/dV accumulators at its
-// end; dQ of every tile is added to an fp32 accumulator with L2 vector reductions;
-// a last pass rounds the three accumulators to bf16. dlogg needs no reduction: each kept
+// end; dQ of every tile is added to an fp32 accumulator with L2 reductions; a last pass
+// rounds the three accumulators to bf16, applying the 1/sqrt(d) of dK and dQ there (the MMAs
+// take the unscaled dS). dlogg needs no reduction: each kept
 // (token, block) pair lives in exactly one tile. Summation order of the reductions is not
 // fixed, so gradients can differ in the last fp32 bits from run to run.
 //
@@ -26,8 +27,9 @@
 //               once the previous item's gradient MMAs have released it.
 //   warp 4      TMEM allocation; lane 0 issues the MMAs, event-driven: S/dP of the next tile
 //               and the gradient MMAs of the oldest pending tile, each once its inputs are ready.
-//   warps 8-11  dS: TMEM lane r = row r: P and dS/sqrt(d) as bf16 into shared tiles (operands
-//               of the gradient MMAs); dlogg summed over the token's G rows.
+//   warps 8-11  dS: TMEM lane r = row r: P and dS as bf16 into shared tiles (operands of the
+//               gradient MMAs), in packed f32x2 arithmetic (the pass is issue-bound); the causal
+//               mask only in tiles that need it; dlogg summed over the token's G rows.
 //   warps 12-15 epilogue: dQ of the tile from TMEM, 32 columns at a time, into a dense per-warp
 //               buffer [32 rows][32 columns] (each lane's 16-byte pieces rotated by lane so the
 //               stores hit distinct banks), then one TMA tensor reduction (cp.reduce.async.bulk
@@ -77,6 +79,34 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kColS = 0, kColDP = 64, kColDQ = 128, kColDV = 384, kColDK = 448;
 constexpr int kFlagFirst = 1, kFlagLast = 2, kFlagStop = 4;
 }  // namespace kmb
+
+// Two fp32 lanes at once (sm_100 packed f32x2 arithmetic): d = a * b + c, d = a - b, d = a * b,
+// d = a + b on the pairs (a0, a1), (b0, b1), (c0, c1).
+__device__ __forceinline__ void fma_x2(float& d0, float& d1, float a0, float a1, float b0, float b1,
+                                       float c0, float c1) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+__device__ __forceinline__ void sub_x2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ void mul_x2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ void add_x2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
 
 struct KmBwdArgs {
   const int32_t* cu;
@@ -434,7 +464,11 @@ __global__ void __launch_bounds__(kmb::kThreads, 1)
       if (!warp_wait(s_full, n & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
       uint32_t pp[kB / 2], pd[kB / 2];
-      float dlsum = 0.f;
+      // keys past the row's limit are masked only in the current block's tiles; rows past the
+      // list have c1 = -inf, so their P is 0 without a mask
+      const bool masked = !__all_sync(0xffffffffu, limit >= kB - 1 || limit < 0);
+      const float sl = a.scale_log2;
+      float dl0 = 0.f, dl1 = 0.f;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         float sv[32], dv[32];
@@ -442,20 +476,23 @@ __global__ void __launch_bounds__(kmb::kThreads, 1)
         tmem_ld32(tmem + lane_addr + kColDP + h * 32, dv);
 #pragma unroll
         for (int c = 0; c < 32; c += 2) {
-          float p2[2], d2[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int key = h * 32 + c + u;
-            const float p = key <= limit ? ex2_approx(fmaf(sv[c + u], a.scale_log2, c1)) : 0.f;
-            const float ds = p * (dv[c + u] - dd);
-            dlsum += ds;
-            p2[u] = p;
-            d2[u] = ds * a.scale;
+          float x0, x1, p0, p1, t0, t1, s0, s1;
+          fma_x2(x0, x1, sv[c], sv[c + 1], sl, sl, c1, c1);
+          p0 = ex2_approx(x0);
+          p1 = ex2_approx(x1);
+          if (masked) {
+            const int key = h * 32 + c;
+            p0 = key <= limit ? p0 : 0.f;
+            p1 = key + 1 <= limit ? p1 : 0.f;
           }
-          pp[(h * 32 + c) >> 1] = pack_bf16x2(p2[0], p2[1]);
-          pd[(h * 32 + c) >> 1] = pack_bf16x2(d2[0], d2[1]);
+          sub_x2(t0, t1, dv[c], dv[c + 1], dd, dd);
+          mul_x2(s0, s1, p0, p1, t0, t1);   // dS (the 1/sqrt(d) of dK and dQ is applied at the end)
+          add_x2(dl0, dl1, dl0, dl1, s0, s1);
+          pp[(h * 32 + c) >> 1] = pack_bf16x2(p0, p1);
+          pd[(h * 32 + c) >> 1] = pack_bf16x2(s0, s1);
         }
       }
+      float dlsum = dl0 + dl1;
       tc_fence_before();
       mbar_arrive(s_free);   // S and dP read: the next tile's MMAs may overwrite them
       // the gradient MMAs of tile n-1 have read the previous P and dS
@@ -574,11 +611,11 @@ __global__ void __launch_bounds__(kmb::kThreads, 1)
 
 // fp32 accumulators -> bf16 gradients (n4 groups of 4 values)
 __global__ void km_bwd_finalize_kernel(const float4* __restrict__ acc, size_t n4,
-                                       uint2* __restrict__ out) {
+                                       uint2* __restrict__ out, float scale) {
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4;
        i += (size_t)gridDim.x * blockDim.x) {
     const float4 x = acc[i];
-    out[i] = make_uint2(pack_bf16x2(x.x, x.y), pack_bf16x2(x.z, x.w));
+    out[i] = make_uint2(pack_bf16x2(x.x * scale, x.y * scale), pack_bf16x2(x.z * scale, x.w * scale));
   }
 }
 
@@ -680,9 +717,9 @@ sas_status launch_attn_bwd_km(const sas_problem& p, const void* q, const void* k
   attn_bwd_km_kernel<<<sm_count(), kmb::kThreads, kmb::kSmemBytes, st>>>(tk, tv, tdq, a);
   const size_t nq4 = (size_t)T * p.num_q_heads * kmb::kD / 4;
   const size_t nk4 = (size_t)T * Hkv * kmb::kD / 4;
-  km_bwd_finalize_kernel<<<4 * sm_count(), 256, 0, st>>>((const float4*)dq_acc, nq4, (uint2*)dq);
-  km_bwd_finalize_kernel<<<4 * sm_count(), 256, 0, st>>>((const float4*)dk_acc, nk4, (uint2*)dk);
-  km_bwd_finalize_kernel<<<4 * sm_count(), 256, 0, st>>>((const float4*)dv_acc, nk4, (uint2*)dv);
+  km_bwd_finalize_kernel<<<4 * sm_count(), 256, 0, st>>>((const float4*)dq_acc, nq4, (uint2*)dq, a.scale);
+  km_bwd_finalize_kernel<<<4 * sm_count(), 256, 0, st>>>((const float4*)dk_acc, nk4, (uint2*)dk, a.scale);
+  km_bwd_finalize_kernel<<<4 * sm_count(), 256, 0, st>>>((const float4*)dv_acc, nk4, (uint2*)dv, 1.f);
   return launch_status("attn_bwd (key-major tensor cores)", 4);
 }
 
